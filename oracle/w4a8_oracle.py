@@ -1,0 +1,337 @@
+"""CPU oracle for the W4A8 MoE expert FFN -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py`` (its CPU-baseline
+and reference legs) may import this module.  The product path (the CUDA library
+and its Python binding) never calls it and shares no code with it.
+
+It is a plain, slow, step-by-step restatement of what the pages define, in
+numpy.  Floating point that only feeds a tolerance comparison is carried in
+fp64; floating point that *decides an integer* (a 4-bit code, a zero point, an
+INT8 activation code) is done in IEEE fp32 exactly as written, because the
+CUDA kernels take the same decisions in fp32 and the codes must agree bit for
+bit.  Integer work (codes, nibble packing, permutation, the per-group INT8 x
+INT4 dot products) is exact.
+
+Sources (cited per function):
+  [P2] «Kimi 2.7 Moe 从 4 bit 存储到 INT8 拆解» (pptc.cn/news/121597)
+  [P1] Kimi 2.7T MoE W4A8 article (hotelren.com/news/5173946)
+  [P3] LLM quantisation primer (hotelren.com/news/5982361)
+  [P4] «MoE部署别把激活参数当成存储需求» (feinterview.poetries.top)
+
+Readings taken where the pages are silent or garbled (each one is listed with
+its reason in the design notes):
+  R1  the integer zero-point form of [P2] §2.2 is used, not the min-offset form of [P1] §2.1;
+  R2  the quantisation range is the group's min and max (not a percentile);
+  R3  the range is widened to contain 0 (mn = min(v, 0), mx = max(v, 0)); an fp16
+      scale that rounds to 0 is replaced by 1;
+  R4  every "round" is round-half-to-even;
+  R5  codes are computed with the fp16-rounded scale, so the stored scale and zero
+      point reproduce them;
+  R6  divisions are correctly rounded fp32 divisions (no reciprocal, no FMA);
+  R7  activation codes are limited to [-127, 127];
+  R9  weights are [N][K] (output channel major), groups of 128 run along K;
+  R10 the up projection's rows are [gate (F rows) | up (F rows)];
+  R11 softmax routing: top-k experts by logit (ties -> lower id), gate weight = the
+      softmax probability over all E experts, not renormalised;
+  R12 tokens inside an expert's segment keep their slot order (t * k + j ascending);
+  R14 h enters the requantisation as fp32.
+
+Parity status: every function below is pinned by tests/test_oracle_pins.py
+against values the pages print, closed forms, brute force or an independent
+formulation; none is "parity unpinned".
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+GROUP = 128  # [P2] §2.1: one scale and one zero point per 128 weights along K
+INT4_MAX = 15  # [P2] §2.2: 2^4 - 1
+INT8_QMAX = 127  # [P3] §2.1: 2^(b-1) - 1 for b = 8 (symmetric)
+
+
+# --------------------------------------------------------------------------- #
+# shapes
+# --------------------------------------------------------------------------- #
+def padded_k(K: int) -> int:
+    """K rounded up to a whole number of groups ([P2] §2.1: pad the matrix to a
+    multiple of the group size at conversion time)."""
+    return ((K + GROUP - 1) // GROUP) * GROUP
+
+
+def pad_k(a: np.ndarray) -> np.ndarray:
+    """Zero-pad the last axis to padded_k ([P2] §2.1)."""
+    K = a.shape[-1]
+    Kp = padded_k(K)
+    if Kp == K:
+        return a
+    pad = [(0, 0)] * (a.ndim - 1) + [(0, Kp - K)]
+    return np.pad(a, pad)
+
+
+# --------------------------------------------------------------------------- #
+# a1: weight quantisation and packing  ([P2] §2.1, §2.2)
+# --------------------------------------------------------------------------- #
+def quantize_weights(w: np.ndarray):
+    """Group-wise asymmetric INT4 of one weight matrix w [N][K] (float32, bf16 values).
+
+    [P2] §2.2, per group of 128 along K:
+        scale      = (max - min) / (2^4 - 1)
+        zero_point = round(-min / scale)
+        index      = clamp(round(weight / scale) + zero_point, 0, 15)
+    with readings R2-R6 (min/max widened to contain 0; fp16 scale used for the
+    codes; round half to even; fp32 correctly rounded division).
+
+    Returns codes uint8 [N][Kp] (values 0..15), scale float16 [N][G], zp float16 [N][G].
+    """
+    w = pad_k(np.asarray(w, dtype=np.float32))
+    N, Kp = w.shape
+    G = Kp // GROUP
+    codes = np.zeros((N, Kp), dtype=np.uint8)
+    scale = np.zeros((N, G), dtype=np.float16)
+    zp = np.zeros((N, G), dtype=np.float16)
+    f15 = np.float32(INT4_MAX)
+    for g in range(G):
+        v = w[:, g * GROUP:(g + 1) * GROUP]  # [N][128]
+        mn = np.minimum(v.min(axis=1), np.float32(0))  # R3
+        mx = np.maximum(v.max(axis=1), np.float32(0))  # R3
+        s32 = (mx - mn) / f15  # fp32 division
+        s16 = s32.astype(np.float16)  # round to nearest even fp16 (R5)
+        s16[s16 == 0] = np.float16(1.0)  # R3: degenerate (all-zero) group
+        sf = s16.astype(np.float32)
+        z = np.clip(np.rint(-mn / sf), 0, INT4_MAX)  # R4, R6
+        q = np.rint(v / sf[:, None]) + z[:, None]
+        codes[:, g * GROUP:(g + 1) * GROUP] = np.clip(q, 0, INT4_MAX).astype(np.uint8)
+        scale[:, g] = s16
+        zp[:, g] = z.astype(np.float16)
+    return codes, scale, zp
+
+
+def dequantize_weights(codes: np.ndarray, scale: np.ndarray, zp: np.ndarray) -> np.ndarray:
+    """weight ~= (index - zero_point) * scale  ([P2] §2.1), in fp64, shape [N][Kp]."""
+    sc = np.repeat(scale.astype(np.float64), GROUP, axis=1)
+    z = np.repeat(zp.astype(np.float64), GROUP, axis=1)
+    return (codes.astype(np.float64) - z) * sc
+
+
+def pack_nibbles(codes: np.ndarray) -> np.ndarray:
+    """Two 4-bit codes per byte, the first in the low 4 bits and the second in the
+    high 4 bits ([P2] §2.2).  codes [..., Kp] -> bytes [..., Kp/2]."""
+    c = np.asarray(codes, dtype=np.uint8)
+    first = c[..., 0::2]
+    second = c[..., 1::2]
+    return (first | (second << 4)).astype(np.uint8)
+
+
+def unpack_nibbles(packed: np.ndarray) -> np.ndarray:
+    """Inverse of pack_nibbles."""
+    p = np.asarray(packed, dtype=np.uint8)
+    out = np.empty(p.shape[:-1] + (p.shape[-1] * 2,), dtype=np.uint8)
+    out[..., 0::2] = p & 0x0F
+    out[..., 1::2] = p >> 4
+    return out
+
+
+# --------------------------------------------------------------------------- #
+# a2 / a6: per-token symmetric INT8 ([P3] §2.1, [P1] §4.3 step 3)
+# --------------------------------------------------------------------------- #
+def quantize_act(x: np.ndarray):
+    """Dynamic per-token symmetric INT8 of x [T][K] (fp32 values).
+
+    [P3] §2.1 symmetric form: scale = max|x| / (2^(b-1) - 1), q = round(x / scale),
+    computed per token at run time ([P1] §4.3).  fp32 arithmetic, round half to even,
+    codes clamped to [-127, 127] (R7).  A row of zeros gets scale 0 and codes 0.
+
+    Returns q int8 [T][Kp] (zero padded) and s float32 [T].
+    """
+    x = np.asarray(x, dtype=np.float32)
+    T = x.shape[0]
+    amax = np.abs(x).max(axis=1) if x.shape[1] else np.zeros(T, np.float32)
+    s = (amax / np.float32(INT8_QMAX)).astype(np.float32)
+    q = np.zeros(x.shape, dtype=np.int8)
+    nz = s > 0
+    if nz.any():
+        r = np.rint(x[nz] / s[nz][:, None])
+        q[nz] = np.clip(r, -INT8_QMAX, INT8_QMAX).astype(np.int8)
+    return pad_k(q), s
+
+
+# --------------------------------------------------------------------------- #
+# a3: routing ([P1] §5.2: the router stays in 16-bit float, never quantised)
+# --------------------------------------------------------------------------- #
+def route_topk(logits: np.ndarray, k: int):
+    """Top-k softmax gating (R11).
+
+    Expert choice: the k largest logits per token, ties broken towards the lower
+    expert id (a stable sort) -- the same set as the k largest softmax probabilities.
+    Gate weight: softmax over all E experts (fp64), not renormalised over the k.
+    Returns ids int32 [T][k], w float64 [T][k].
+    """
+    lg = np.asarray(logits, dtype=np.float64)
+    T, E = lg.shape
+    ids = np.zeros((T, k), dtype=np.int32)
+    for t in range(T):
+        order = sorted(range(E), key=lambda e: (-lg[t, e], e))
+        ids[t] = order[:k]
+    p = np.exp(lg - lg.max(axis=1, keepdims=True))
+    p /= p.sum(axis=1, keepdims=True)
+    w = np.take_along_axis(p, ids.astype(np.int64), axis=1)
+    return ids, w
+
+
+# --------------------------------------------------------------------------- #
+# a4: permutation (grouping tokens by expert)
+# --------------------------------------------------------------------------- #
+def permute(ids: np.ndarray, E: int):
+    """Stable grouping of the T*k routed slots by expert (R12).
+
+    Slot i = t*k + j carries expert ids[t, j].  counts[e] = number of slots routed
+    to e; offs = exclusive prefix sum of counts (length E+1); perm[offs[e] + p] = the
+    p-th slot (in ascending slot order) routed to e; inv[i] = position of slot i in
+    the grouped order.
+    """
+    flat = np.asarray(ids, dtype=np.int64).reshape(-1)
+    counts = np.zeros(E, dtype=np.int64)
+    for e in flat:
+        counts[e] += 1
+    offs = np.zeros(E + 1, dtype=np.int64)
+    for e in range(E):
+        offs[e + 1] = offs[e] + counts[e]
+    fill = offs[:-1].copy()
+    perm = np.zeros(flat.size, dtype=np.int64)
+    inv = np.zeros(flat.size, dtype=np.int64)
+    for i, e in enumerate(flat):
+        perm[fill[e]] = i
+        inv[i] = fill[e]
+        fill[e] += 1
+    return counts, offs, perm, inv
+
+
+def expected_distinct_experts(E: int, B: int) -> float:
+    """Mean number of distinct experts hit by B tokens that each pick one of E
+    experts independently and uniformly: E * (1 - (1 - 1/E)^B)  ([P4], toy model)."""
+    return E * (1.0 - (1.0 - 1.0 / E) ** B)
+
+
+# --------------------------------------------------------------------------- #
+# a5 / a7: W4A8 linear with per-group INT32 partials ([P2] §3.2, [P1] §4.3)
+# --------------------------------------------------------------------------- #
+def group_partials(qa: np.ndarray, codes: np.ndarray, zp: np.ndarray) -> np.ndarray:
+    """acc[m, n, g] = sum over k in group g of qa[m, k] * (codes[n, k] - zp[n, g]).
+
+    INT8 activations times INT4 weights dequantised to integers, accumulated in
+    32 bits per group ([P2] §3.2: INT8 x INT8 accumulates into INT32).  Computed
+    per group with an fp64 matrix product, which is exact here because every
+    partial is an integer of magnitude <= 128 * 127 * 15 < 2^53.
+    Returns int64 [M][N][G].
+    """
+    qa = np.asarray(qa)
+    M, Kp = qa.shape
+    N = codes.shape[0]
+    G = Kp // GROUP
+    acc = np.zeros((M, N, G), dtype=np.int64)
+    for g in range(G):
+        sl = slice(g * GROUP, (g + 1) * GROUP)
+        a = qa[:, sl].astype(np.float64)  # [M][128]
+        wq = codes[:, sl].astype(np.float64) - zp[:, g].astype(np.float64)[:, None]  # [N][128]
+        acc[:, :, g] = np.rint(a @ wq.T).astype(np.int64)
+    return acc
+
+
+def w4a8_linear(qa, sa, codes, scale, zp, acc=None) -> np.ndarray:
+    """y[m, n] = sa[m] * sum_g scale[n, g] * acc[m, n, g]   (fp64).
+
+    [P1] §4.3 steps 2-4: INT8 matrix product, then the INT32 result is scaled back
+    to floating point -- the weight scale of each group times the token's scale.
+    """
+    if acc is None:
+        acc = group_partials(qa, codes, zp)
+    y = np.zeros(acc.shape[:2], dtype=np.float64)
+    for g in range(acc.shape[2]):
+        y += scale[:, g].astype(np.float64)[None, :] * acc[:, :, g].astype(np.float64)
+    return np.asarray(sa, dtype=np.float64)[:, None] * y
+
+
+# --------------------------------------------------------------------------- #
+# a6: SwiGLU between the projections
+# --------------------------------------------------------------------------- #
+def silu(x: np.ndarray) -> np.ndarray:
+    return x / (1.0 + np.exp(-x))
+
+
+def swiglu(y_up: np.ndarray, F: int) -> np.ndarray:
+    """h = silu(gate) * up with gate = columns [0, F) and up = columns [F, 2F) (R10)."""
+    return silu(y_up[:, :F]) * y_up[:, F:2 * F]
+
+
+# --------------------------------------------------------------------------- #
+# a8: weighted combine
+# --------------------------------------------------------------------------- #
+def combine(y2: np.ndarray, w: np.ndarray, inv: np.ndarray, T: int, k: int) -> np.ndarray:
+    """out[t] = sum over j < k of w[t, j] * y2[inv[t*k + j]]  (fp64, j ascending)."""
+    out = np.zeros((T, y2.shape[1]), dtype=np.float64)
+    for j in range(k):
+        out += np.asarray(w, dtype=np.float64)[:, j:j + 1] * y2[inv[np.arange(T) * k + j]]
+    return out
+
+
+# --------------------------------------------------------------------------- #
+# the whole layer
+# --------------------------------------------------------------------------- #
+class QuantExpert:
+    """Quantised weights of one expert: up [2F][Hp] (gate|up rows) and down [H][Fp]."""
+
+    def __init__(self, w_up: np.ndarray, w_down: np.ndarray):
+        self.up = quantize_weights(w_up)
+        self.down = quantize_weights(w_down)
+
+
+def expert_forward(xq, xs, qe: QuantExpert, F: int, stages: dict | None = None):
+    """One expert on its tokens: up GEMM -> SwiGLU -> requantise -> down GEMM.
+
+    xq int8 [M][Hp], xs float32 [M]; returns y2 float64 [M][H].
+    """
+    cu, su, zu = qe.up
+    y_up = w4a8_linear(xq, xs, cu, su, zu)  # [M][2F]
+    h = swiglu(y_up, F).astype(np.float32)  # R14: h enters requant as fp32
+    qh, sh = quantize_act(h)  # [P1] §4.3 step 3: the next op's input is quantised per token
+    cd, sd, zd = qe.down
+    y2 = w4a8_linear(qh, sh, cd, sd, zd)
+    if stages is not None:
+        stages.setdefault("h", []).append(h)
+        stages.setdefault("qh", []).append(qh)
+        stages.setdefault("sh", []).append(sh)
+    return y2
+
+
+def moe_forward(x, ids, w, experts: dict, E: int, F: int, stages: dict | None = None):
+    """Full W4A8 MoE expert FFN (fp64 result, [T][H]).
+
+    x [T][H] float32 (bf16 values); ids [T][k]; w [T][k]; experts[e] = QuantExpert
+    (only experts that receive tokens are needed).
+    """
+    x = np.asarray(x, dtype=np.float32)
+    T, H = x.shape
+    k = ids.shape[1]
+    xq, xs = quantize_act(x)
+    counts, offs, perm, inv = permute(ids, E)
+    y2 = np.zeros((T * k, H), dtype=np.float64)
+    for e in range(E):
+        if counts[e] == 0:
+            continue
+        slots = perm[offs[e]:offs[e + 1]]
+        tok = slots // k
+        y2[offs[e]:offs[e + 1]] = expert_forward(xq[tok], xs[tok], experts[e], F, stages)[:, :H]
+    if stages is not None:
+        stages.update(counts=counts, offs=offs, perm=perm, inv=inv, xq=xq, xs=xs, y2=y2)
+    return combine(y2, w, inv, T, k)
+
+
+def token_forward(t: int, x, ids, w, experts: dict, F: int) -> np.ndarray:
+    """The layer's output for one token only (used to sample large layers)."""
+    xq, xs = quantize_act(np.asarray(x, dtype=np.float32)[t:t + 1])
+    out = 0.0
+    for j in range(ids.shape[1]):
+        y2 = expert_forward(xq, xs, experts[int(ids[t, j])], F)[0]
+        out = out + float(w[t, j]) * y2
+    return out
