@@ -1,0 +1,186 @@
+/*
+ * w4a8.h -- C ABI of libw4a8.so: the W4A8 mixture-of-experts expert FFN on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The method (sources: «Kimi 2.7 Moe 从 4 bit 存储到 INT8 拆解», pptc.cn, sections
+ * 2.1-2.3 and 3.2; the Kimi 2.7T MoE W4A8 article, hotelren.com 5173946, section
+ * 4.3; the LLM quantisation primer, hotelren.com 5982361, section 2.1):
+ *   - weights are group-wise asymmetric INT4, 128 weights per group along K, one
+ *     fp16 scale and one fp16 zero point per group:
+ *       scale = (max - min) / 15, zp = round(-min / scale),
+ *       index = clamp(round(w / scale) + zp, 0, 15),  w ~= (index - zp) * scale;
+ *     two indices per byte, the first in the low nibble;
+ *   - activations are quantised per token to symmetric INT8 at run time:
+ *       s = max|x| / 127, q = clamp(round(x / s), -127, 127);
+ *   - the product is an INT8 x INT8 matrix multiply with INT32 accumulation, one
+ *     INT32 partial per 128-wide K group, scaled back to floating point by
+ *     (weight scale of the group) x (token scale).
+ * "round" is round-half-to-even everywhere; the min/max range of a weight group
+ * is widened to contain 0; an fp16 scale that rounds to 0 is stored as 1.
+ *
+ * Conventions for every entry point:
+ *   - pointers are DEVICE pointers owned by the caller unless a parameter says
+ *     "host"; the library allocates nothing -- scratch memory is the caller's
+ *     workspace `ws`, sized by the matching *_workspace_bytes() function;
+ *   - device pointers must be 16-byte aligned (W4A8_EALIGN otherwise), workspace
+ *     and packed-weight pointers 256-byte aligned;
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream); all work is
+ *     enqueued asynchronously on it and the call returns after launching;
+ *   - the return value reports argument validation and launch errors only
+ *     (w4a8_status).  Faults detected on the device (a bounded wait that ran out,
+ *     an expert id out of range) set a word in the workspace that
+ *     w4a8_last_device_error() reads back;
+ *   - no CUDA context is created or changed, no exception crosses the ABI, and
+ *     there is no CPU fallback: an unsupported shape returns W4A8_EUNSUPPORTED.
+ */
+#ifndef W4A8_H
+#define W4A8_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    W4A8_OK = 0,
+    W4A8_EINVAL = -1,       /* bad argument (null pointer, negative size, k > E, ...) */
+    W4A8_EALIGN = -2,       /* a pointer is not aligned as required */
+    W4A8_ENOSPACE = -3,     /* packed buffer or workspace smaller than required */
+    W4A8_ECUDA = -4,        /* a CUDA runtime call or kernel launch failed */
+    W4A8_EUNSUPPORTED = -5, /* shape outside what the kernels handle */
+    W4A8_ETIMEOUT = -6,     /* (device error word) a bounded wait in a kernel ran out */
+    W4A8_EDEVICE = -7       /* (device error word) bad data seen on the device */
+} w4a8_status;
+
+/* Packed-weight layouts.
+ * W4A8_LAYOUT_PLAIN : rows in order (a plain linear layer, or an expert's down
+ *                     projection [H][F]).
+ * W4A8_LAYOUT_GATEUP: the expert's up projection [2F][H] whose rows [0,F) are the
+ *                     gate projection and rows [F,2F) the up projection; each
+ *                     128-row tile holds 64 gate rows interleaved with the 64
+ *                     matching up rows, so that SwiGLU can be applied in the
+ *                     GEMM's epilogue.                                            */
+enum { W4A8_LAYOUT_PLAIN = 0, W4A8_LAYOUT_GATEUP = 1 };
+
+/* Bytes of a packed weight buffer for E matrices of shape [N][K] in `layout`:
+ * a 256-byte header, then one 8704-byte block per (matrix, 128-row tile, 128-wide
+ * K group): 8192 bytes of 4-bit codes, 128 fp16 scales, 128 fp16 zero points.
+ * K is padded to a multiple of 128 (zero weights).  Returns 0 for invalid shapes
+ * (GATEUP needs an even N). */
+size_t w4a8_packed_bytes(int E, int N, int K, int layout);
+
+/* Quantise and pack E weight matrices  (a1: the offline conversion step).
+ *   w_bf16      : device, bf16 [E][N][K], row-major (nn.Linear orientation).
+ *   packed      : device, w4a8_packed_bytes(E,N,K,layout) bytes (256-B aligned),
+ *                 the tiled layout consumed by w4a8_gemm / w4a8_moe_forward.
+ *   codes_opt   : device or NULL; canonical packed codes uint8 [E][N][Kp/2],
+ *                 byte j of a row = code[2j] | code[2j+1] << 4.
+ *   scale_f16_opt, zp_f16_opt : device or NULL; fp16 bit patterns [E][N][Kp/128].
+ * Returns W4A8_ENOSPACE if packed_bytes is too small. */
+int w4a8_pack_weights(const void* w_bf16, int E, int N, int K, int layout,
+                      void* packed, size_t packed_bytes,
+                      uint8_t* codes_opt, uint16_t* scale_f16_opt, uint16_t* zp_f16_opt,
+                      void* stream);
+
+/* Per-token symmetric INT8 quantisation of activations  (a2).
+ *   x_bf16 : device, bf16 [T][K] row-major.
+ *   q      : device, int8 [T][Kp], Kp = K rounded up to 128 (padding written as 0).
+ *   s      : device, float [T]; s = max|x|/127 (0 for an all-zero row, with q = 0). */
+int w4a8_quant_act(const void* x_bf16, int T, int K, int8_t* q, float* s, void* stream);
+
+/* Top-k softmax routing  (a3; the router stays in 16-bit float).
+ *   logits_bf16 : device, bf16 [T][E];  1 <= k <= min(E, 32), E <= 1024.
+ *   ids         : device, int32 [T][k]: the k largest logits, largest first, ties
+ *                 to the lower expert id.
+ *   w           : device, float [T][k]: softmax probability over all E experts
+ *                 of each chosen expert (not renormalised over the k). */
+int w4a8_route_topk(const void* logits_bf16, int T, int E, int k, int32_t* ids, float* w,
+                    void* stream);
+
+/* Workspace bytes needed by w4a8_moe_forward for this layer shape. */
+size_t w4a8_moe_workspace_bytes(int T, int E, int k, int H, int F);
+
+/* The W4A8 MoE expert FFN  (a4..a8):
+ *   out[t] = sum_j w[t][j] * Down_e( SwiGLU( Up_e( x[t] ) ) ),  e = ids[t][j],
+ * with x quantised per token to INT8, Up/Down W4A8 GEMMs (INT32 per-group
+ * partials), h = silu(gate) * up requantised per token to INT8 before Down.
+ *   packed_up   : from w4a8_pack_weights(E, 2F, H, W4A8_LAYOUT_GATEUP).
+ *   packed_down : from w4a8_pack_weights(E, H, F, W4A8_LAYOUT_PLAIN).
+ *   x_bf16      : device bf16 [T][H].   ids: device int32 [T][k] (0 <= id < E;
+ *                 an id out of range drops that slot and sets W4A8_EDEVICE).
+ *   w           : device float [T][k].  out_bf16: device bf16 [T][H].
+ *   ws          : device, >= w4a8_moe_workspace_bytes(T,E,k,H,F) bytes.
+ * Limits: E <= 1024, k <= 32, T*k < 2^31. */
+int w4a8_moe_forward(const void* packed_up, const void* packed_down, int E, int H, int F,
+                     const void* x_bf16, int T, const int32_t* ids, const float* w, int k,
+                     void* out_bf16, void* ws, size_t ws_bytes, void* stream);
+
+/* Same as w4a8_moe_forward, but x_bf16, ids, w and out_bf16 are HOST buffers
+ * (pinned memory recommended): they are copied to / from the workspace on
+ * `stream` with cudaMemcpyAsync before and after the forward.  Needs
+ * w4a8_moe_host_workspace_bytes() of workspace.  The call returns once the work
+ * is enqueued; out_bf16 is valid after the stream is synchronised. */
+size_t w4a8_moe_host_workspace_bytes(int T, int E, int k, int H, int F);
+int w4a8_moe_forward_host(const void* packed_up, const void* packed_down, int E, int H, int F,
+                          const void* x_bf16_host, int T, const int32_t* ids_host,
+                          const float* w_host, int k, void* out_bf16_host,
+                          void* ws, size_t ws_bytes, void* stream);
+
+/* Workspace bytes needed by w4a8_gemm. */
+size_t w4a8_gemm_workspace_bytes(int M, int N, int K);
+
+/* One dense W4A8 linear layer  (a5 on a single weight matrix):
+ *   y[m][n] = sa[m] * sum_g scale[n][g] * acc[m][n][g],
+ *   acc[m][n][g] = sum_{k in group g} qa[m][k] * (code[n][k] - zp[n][g])   (INT32).
+ *   qa          : device int8 [M][Kp] (as written by w4a8_quant_act), sa: float [M].
+ *   packed      : from w4a8_pack_weights(1, N, K, W4A8_LAYOUT_PLAIN).
+ *   y           : device float [M][N].
+ *   partials_opt: device int32 [M][N][Kp/128] or NULL -- the exact INT32 partials. */
+int w4a8_gemm(const int8_t* qa, const float* sa, int M, const void* packed, int N, int K,
+              float* y, int32_t* partials_opt, void* ws, size_t ws_bytes, void* stream);
+
+/* Intermediate results kept in a w4a8_moe_forward workspace, for stage tests. */
+enum {
+    W4A8_DUMP_COUNTS = 0, /* int32 [E]      tokens routed to each expert             */
+    W4A8_DUMP_OFFS = 1,   /* int32 [E+1]    exclusive prefix sum of counts           */
+    W4A8_DUMP_PERM = 2,   /* int32 [T*k]    slot (t*k+j) at each grouped position     */
+    W4A8_DUMP_INV = 3,    /* int32 [T*k]    padded row of each slot                   */
+    W4A8_DUMP_POFFS = 4,  /* int32 [E+1]    row offsets with every expert padded to 16 */
+    W4A8_DUMP_ACT1 = 5,   /* int8 [Hp/128][R][128] INT8 x rows (tiled, see below)     */
+    W4A8_DUMP_S1 = 6,     /* float [R]      token scale of each padded row            */
+    W4A8_DUMP_H = 7,      /* float [R][Fp]  SwiGLU output h (fp32) per padded row      */
+    W4A8_DUMP_ACT2 = 8,   /* int8 [Fp/128][R][128] requantised h (tiled)              */
+    W4A8_DUMP_S2 = 9,     /* float [R]      scale of the requantised h rows           */
+    W4A8_DUMP_Y2 = 10,    /* float [R][H]   down-projection output per padded row     */
+    W4A8_DUMP_ERR = 11    /* uint32 [1]     device error word                         */
+};
+/* R = w4a8_moe_rows_capacity(T,E,k).  Tiled INT8 planes: plane g holds K columns
+ * [128g, 128g+128); row r's 16-byte chunk c sits at r*128 + ((c ^ (r & 7)) * 16). */
+int w4a8_moe_rows_capacity(int T, int E, int k);
+
+/* Byte offset and size of dump region `what` inside the workspace. */
+int w4a8_debug_region(int T, int E, int k, int H, int F, int what, size_t* offset, size_t* bytes);
+
+/* Copy dump region `what` of workspace `ws` to `dst` (device or host memory,
+ * cudaMemcpyDefault), at most `bytes` bytes, on `stream`. */
+int w4a8_debug_dump(const void* ws, int T, int E, int k, int H, int F, int what, void* dst,
+                    size_t bytes, void* stream);
+
+/* Synchronise `stream`, then return the device error word kept in workspace `ws`
+ * (0 = none; bit 0 = a bounded wait timed out, bit 1 = expert id out of range).
+ * Any workspace from w4a8_moe_forward / w4a8_gemm may be passed. */
+int w4a8_last_device_error(const void* ws, void* stream);
+
+/* Human-readable name of a w4a8_status value. */
+const char* w4a8_status_string(int status);
+
+/* ABI version (major * 100 + minor). */
+int w4a8_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* W4A8_H */

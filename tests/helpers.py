@@ -1,0 +1,100 @@
+"""Test-side helpers: tolerance checks and decoders of the library's tiled layouts.
+
+The decoders restate the layouts documented in include/w4a8.h so that tests can
+compare device buffers with the oracle's canonical arrays; they take no part in
+the product path.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+BLOCK = 8704
+HEADER = 256
+
+
+def rms(a) -> float:
+    a = np.asarray(a, dtype=np.float64)
+    return float(np.sqrt(np.mean(a * a))) if a.size else 0.0
+
+
+def assert_close(gpu, ref, max_rel=1e-2, mae_rel=1e-3, what="output"):
+    """Tolerance of the float results against the oracle.
+
+    max relative error <= max_rel, where the relative error of an element is
+    |gpu - ref| / max(|ref|, rms(ref)) (elements far below the output's rms are
+    judged against the rms), and mean absolute error <= mae_rel * rms(ref).
+    """
+    g = np.asarray(gpu, dtype=np.float64)
+    r = np.asarray(ref, dtype=np.float64)
+    assert g.shape == r.shape, (g.shape, r.shape)
+    if r.size == 0:
+        return
+    s = rms(r)
+    err = np.abs(g - r)
+    assert np.all(np.isfinite(g)), f"{what}: non-finite values"
+    denom = np.maximum(np.abs(r), s if s > 0 else 1.0)
+    worst = float((err / denom).max())
+    mae = float(err.mean())
+    assert worst <= max_rel, f"{what}: max relative error {worst:.3e} > {max_rel}"
+    assert mae <= mae_rel * max(s, 1e-30), f"{what}: mean abs error {mae:.3e} > {mae_rel} * rms {s:.3e}"
+    return worst, mae
+
+
+def packed_tiles(N: int, layout: int) -> int:
+    return -(-(N // 2) // 64) if layout == 1 else -(-N // 128)
+
+
+def decode_packed(buf: np.ndarray, E: int, N: int, K: int, layout: int):
+    """Tiled packed buffer -> (codes uint8 [E][N][Kp], scale f16 [E][N][G], zp f16 [E][N][G])."""
+    G = -(-K // 128)
+    Kp = G * 128
+    NT = packed_tiles(N, layout)
+    blocks = np.asarray(buf, dtype=np.uint8)[HEADER:HEADER + E * NT * G * BLOCK].reshape(E, NT, G, BLOCK)
+    codes = np.zeros((E, N, Kp), np.uint8)
+    scale = np.zeros((E, N, G), np.float16)
+    zp = np.zeros((E, N, G), np.float16)
+    r = np.arange(128)
+    if layout == 1:
+        F = N // 2
+    for t in range(NT):
+        if layout == 1:
+            f = t * 64 + (r >> 1)
+            src = np.where(r & 1, F + f, f)
+            valid = f < F
+        else:
+            src = t * 128 + r
+            valid = src < N
+        for g in range(G):
+            blk = blocks[:, t, g]  # [E][BLOCK]
+            rows = np.zeros((E, 128, 128), np.uint8)
+            for c in range(4):
+                pos = r * 64 + ((c ^ (r >> 1)) & 3) * 16
+                chunk = blk[:, pos[:, None] + np.arange(16)[None, :]]  # [E][128][16]
+                words = chunk.reshape(E, 128, 4, 4).astype(np.uint32)
+                words = words[..., 0] | (words[..., 1] << 8) | (words[..., 2] << 16) | (words[..., 3] << 24)
+                for q in range(4):
+                    i = 4 * c + q
+                    x = words[:, :, q]
+                    for b in range(4):
+                        rows[:, :, 8 * i + b] = (x >> (8 * b)) & 0xF
+                        rows[:, :, 8 * i + 4 + b] = (x >> (8 * b + 4)) & 0xF
+            sc = blk[:, 8192:8448].copy().view(np.float16).reshape(E, 128)
+            z = blk[:, 8448:8704].copy().view(np.float16).reshape(E, 128)
+            codes[:, src[valid], g * 128:(g + 1) * 128] = rows[:, valid]
+            scale[:, src[valid], g] = sc[:, valid]
+            zp[:, src[valid], g] = z[:, valid]
+    return codes, scale, zp
+
+
+def untile_act(planes: np.ndarray, R: int, Kp: int) -> np.ndarray:
+    """Tiled INT8 planes [Kp/128][R][128] (16-byte chunk c of row r at c ^ (r & 7)) -> [R][Kp]."""
+    G = Kp // 128
+    p = np.asarray(planes).reshape(G, R, 8, 16)
+    r = np.arange(R)
+    out = np.zeros((R, Kp), dtype=p.dtype)
+    for c in range(8):
+        phys = (c ^ (r & 7))
+        for g in range(G):
+            out[:, g * 128 + c * 16:g * 128 + (c + 1) * 16] = p[g, r, phys]
+    return out

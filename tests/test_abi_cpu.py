@@ -1,0 +1,107 @@
+"""CPU-only checks of the C ABI: the library loads, exports every symbol the
+header declares, and rejects bad arguments on the host before touching a GPU."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from w4a8_quantized_moe_token_b200 import binding as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "w4a8.h")
+
+EINVAL, EALIGN, ENOSPACE, EUNSUPPORTED = -1, -2, -3, -5
+
+
+def header_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(w4a8_\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(B.LIB_PATH):
+        from w4a8_quantized_moe_token_b200 import build
+        build.build()
+    return B.lib()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = header_functions()
+    assert len(names) >= 15
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(B.exported_symbols())
+
+
+def test_version_and_status_strings(lib):
+    assert lib.w4a8_version() == 100
+    assert lib.w4a8_status_string(0) == b"ok"
+    assert lib.w4a8_status_string(ENOSPACE).startswith(b"buffer")
+
+
+def test_packed_bytes_accounting(lib):
+    # 256-byte header + one 8704-byte block per (matrix, 128-row tile, 128-wide group)
+    assert lib.w4a8_packed_bytes(1, 256, 512, 0) == 256 + 2 * 4 * 8704
+    assert lib.w4a8_packed_bytes(8, 2048, 2048, 1) == 256 + 8 * 16 * 16 * 8704
+    assert lib.w4a8_packed_bytes(1, 100, 200, 0) == 256 + 1 * 1 * 2 * 8704
+    assert lib.w4a8_packed_bytes(1, 3, 128, 1) == 0  # odd N for gate|up
+    assert lib.w4a8_packed_bytes(0, 128, 128, 0) == 0
+    # per weight: 0.5 byte of codes + 4 bytes per 128-group of scale and zero point
+    blk = 8704
+    assert blk == 128 * 128 // 2 + 128 * 4
+
+
+def test_host_validation_without_gpu(lib):
+    vp = ctypes.c_void_p
+    fake = vp(1 << 20)  # aligned, never dereferenced: validation fails first
+    assert lib.w4a8_quant_act(None, 4, 128, None, None, None) == EINVAL
+    assert lib.w4a8_quant_act(fake, -1, 128, fake, fake, None) == EINVAL
+    assert lib.w4a8_quant_act(vp((1 << 20) + 2), 4, 128, fake, fake, None) == EALIGN
+    assert lib.w4a8_quant_act(fake, 0, 128, fake, fake, None) == 0  # nothing to do
+    assert lib.w4a8_pack_weights(fake, 1, 256, 512, 0, fake, 100, None, None, None, None) == ENOSPACE
+    assert lib.w4a8_pack_weights(fake, 1, 256, 512, 7, fake, 1 << 30, None, None, None, None) == EINVAL
+    assert lib.w4a8_route_topk(fake, 4, 2000, 2, fake, fake, None) == EUNSUPPORTED
+    assert lib.w4a8_route_topk(fake, 4, 8, 9, fake, fake, None) == EINVAL
+    ws_small = 16
+    assert lib.w4a8_moe_forward(fake, fake, 8, 256, 128, fake, 4, fake, fake, 2, fake, fake, ws_small, None) == ENOSPACE
+    assert lib.w4a8_moe_forward(fake, vp((1 << 20) + 16), 8, 256, 128, fake, 4, fake, fake, 2, fake, fake, 1 << 40,
+                                None) == EALIGN
+    assert lib.w4a8_moe_forward(fake, fake, 2048, 256, 128, fake, 4, fake, fake, 2, fake, fake, 1 << 40,
+                                None) == EUNSUPPORTED
+    assert lib.w4a8_moe_forward(fake, fake, 8, 256, 128, fake, 4, fake, fake, 9, fake, fake, 1 << 40, None) == EINVAL
+    assert lib.w4a8_gemm(fake, fake, 4, fake, 256, 512, fake, None, fake, 8, None) == ENOSPACE
+    assert lib.w4a8_last_device_error(None, None) == EINVAL
+
+
+def test_moe_workspace_regions(lib):
+    T, E, k, H, F = 64, 64, 6, 4096, 1408
+    R = lib.w4a8_moe_rows_capacity(T, E, k)
+    assert R % 16 == 0 and R >= T * k and R <= T * k + 15 * E + 16
+    total = lib.w4a8_moe_workspace_bytes(T, E, k, H, F)
+    regions = []
+    for what in range(12):
+        off, nb = B.w4a8_debug_region(T, E, k, H, F, what)
+        assert off % 256 == 0 and off + nb <= total
+        regions.append((off, nb))
+    # the documented sizes
+    assert regions[B.DUMP["counts"]][1] == 4 * E
+    assert regions[B.DUMP["act1"]][1] == (4096 // 128) * R * 128
+    assert regions[B.DUMP["h"]][1] == R * 1408 * 4
+    assert regions[B.DUMP["act2"]][1] == (1408 // 128) * R * 128
+    assert regions[B.DUMP["y2"]][1] == R * H * 4
+    s = sorted(r for r in regions if r[1] > 4)
+    for (o1, n1), (o2, _) in zip(s, s[1:]):
+        assert o1 + n1 <= o2  # no overlap
+    assert lib.w4a8_moe_host_workspace_bytes(T, E, k, H, F) >= total + 2 * T * H * 2
+    assert lib.w4a8_moe_workspace_bytes(T, E, 40, H, F) == 0  # k > 32
+    assert lib.w4a8_moe_rows_capacity(0, 8, 2) == 0
+
+
+def test_gemm_workspace(lib):
+    assert lib.w4a8_gemm_workspace_bytes(16, 256, 512) >= 4 * 16 * 128
+    assert lib.w4a8_gemm_workspace_bytes(0, 256, 512) > 0
+    assert lib.w4a8_gemm_workspace_bytes(-1, 256, 512) == 0

@@ -1,0 +1,216 @@
+"""ctypes binding of libw4a8.so (the C ABI declared in include/w4a8.h).
+
+Argument marshalling only: every function checks tensor devices / dtypes /
+shapes, passes raw pointers and the current CUDA stream, and raises W4A8Error
+on a non-zero status.  All computation happens in the CUDA library; if the
+library is missing the first call raises -- there is no fallback.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libw4a8.so")
+
+W4A8_LAYOUT_PLAIN = 0
+W4A8_LAYOUT_GATEUP = 1
+
+DUMP = {
+    "counts": 0, "offs": 1, "perm": 2, "inv": 3, "poffs": 4, "act1": 5, "s1": 6,
+    "h": 7, "act2": 8, "s2": 9, "y2": 10, "err": 11,
+}
+
+_c_int, _c_size, _vp = ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p
+_SIGS = {
+    "w4a8_version": ([], _c_int),
+    "w4a8_status_string": ([_c_int], ctypes.c_char_p),
+    "w4a8_packed_bytes": ([_c_int, _c_int, _c_int, _c_int], _c_size),
+    "w4a8_pack_weights": ([_vp, _c_int, _c_int, _c_int, _c_int, _vp, _c_size, _vp, _vp, _vp, _vp], _c_int),
+    "w4a8_quant_act": ([_vp, _c_int, _c_int, _vp, _vp, _vp], _c_int),
+    "w4a8_route_topk": ([_vp, _c_int, _c_int, _c_int, _vp, _vp, _vp], _c_int),
+    "w4a8_moe_workspace_bytes": ([_c_int] * 5, _c_size),
+    "w4a8_moe_host_workspace_bytes": ([_c_int] * 5, _c_size),
+    "w4a8_moe_rows_capacity": ([_c_int] * 3, _c_int),
+    "w4a8_moe_forward": ([_vp, _vp, _c_int, _c_int, _c_int, _vp, _c_int, _vp, _vp, _c_int, _vp, _vp, _c_size, _vp],
+                         _c_int),
+    "w4a8_moe_forward_host": ([_vp, _vp, _c_int, _c_int, _c_int, _vp, _c_int, _vp, _vp, _c_int, _vp, _vp, _c_size,
+                               _vp], _c_int),
+    "w4a8_gemm_workspace_bytes": ([_c_int] * 3, _c_size),
+    "w4a8_gemm": ([_vp, _vp, _c_int, _vp, _c_int, _c_int, _vp, _vp, _vp, _c_size, _vp], _c_int),
+    "w4a8_debug_region": ([_c_int] * 6 + [ctypes.POINTER(_c_size), ctypes.POINTER(_c_size)], _c_int),
+    "w4a8_debug_dump": ([_vp] + [_c_int] * 6 + [_vp, _c_size, _vp], _c_int),
+    "w4a8_last_device_error": ([_vp, _vp], _c_int),
+}
+
+_lib = None
+
+
+class W4A8Error(RuntimeError):
+    pass
+
+
+def lib() -> ctypes.CDLL:
+    """Load libw4a8.so (built in-tree by w4a8_quantized_moe_token_b200.build)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise W4A8Error(f"{LIB_PATH} is missing: build it with `python -m w4a8_quantized_moe_token_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (args, res) in _SIGS.items():
+            f = getattr(L, name)
+            f.argtypes = args
+            f.restype = res
+        _lib = L
+    return _lib
+
+
+def exported_symbols():
+    return list(_SIGS)
+
+
+def _check(status: int, what: str):
+    if status != 0:
+        msg = lib().w4a8_status_string(status).decode()
+        raise W4A8Error(f"{what}: {msg} ({status})")
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise W4A8Error("tensors passed to libw4a8 must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _dev(t, dtype, name):
+    if not t.is_cuda:
+        raise W4A8Error(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise W4A8Error(f"{name} must be {dtype}, got {t.dtype}")
+
+
+# --------------------------------------------------------------------------- #
+def w4a8_version() -> int:
+    return lib().w4a8_version()
+
+
+def w4a8_packed_bytes(E: int, N: int, K: int, layout: int) -> int:
+    return lib().w4a8_packed_bytes(E, N, K, layout)
+
+
+def w4a8_pack_weights(w: torch.Tensor, layout: int, packed: torch.Tensor, codes=None, scale=None, zp=None):
+    """w: bf16 [E][N][K] (cuda).  packed: uint8 cuda tensor of w4a8_packed_bytes bytes."""
+    _dev(w, torch.bfloat16, "w")
+    if w.dim() == 2:
+        w = w.unsqueeze(0)
+    E, N, K = w.shape
+    _dev(packed, torch.uint8, "packed")
+    for t, dt, nm in ((codes, torch.uint8, "codes"), (scale, torch.float16, "scale"), (zp, torch.float16, "zp")):
+        if t is not None:
+            _dev(t, dt, nm)
+    _check(lib().w4a8_pack_weights(_ptr(w), E, N, K, layout, _ptr(packed), packed.numel(), _ptr(codes),
+                                   _ptr(scale), _ptr(zp), _stream()), "w4a8_pack_weights")
+
+
+def w4a8_quant_act(x: torch.Tensor, q: torch.Tensor, s: torch.Tensor):
+    """x: bf16 [T][K]; q: int8 [T][Kp]; s: float32 [T]."""
+    _dev(x, torch.bfloat16, "x")
+    _dev(q, torch.int8, "q")
+    _dev(s, torch.float32, "s")
+    T, K = x.shape
+    _check(lib().w4a8_quant_act(_ptr(x), T, K, _ptr(q), _ptr(s), _stream()), "w4a8_quant_act")
+
+
+def w4a8_route_topk(logits: torch.Tensor, k: int, ids: torch.Tensor, w: torch.Tensor):
+    _dev(logits, torch.bfloat16, "logits")
+    _dev(ids, torch.int32, "ids")
+    _dev(w, torch.float32, "w")
+    T, E = logits.shape
+    _check(lib().w4a8_route_topk(_ptr(logits), T, E, k, _ptr(ids), _ptr(w), _stream()), "w4a8_route_topk")
+
+
+def w4a8_moe_workspace_bytes(T, E, k, H, F) -> int:
+    return lib().w4a8_moe_workspace_bytes(T, E, k, H, F)
+
+
+def w4a8_moe_host_workspace_bytes(T, E, k, H, F) -> int:
+    return lib().w4a8_moe_host_workspace_bytes(T, E, k, H, F)
+
+
+def w4a8_moe_rows_capacity(T, E, k) -> int:
+    return lib().w4a8_moe_rows_capacity(T, E, k)
+
+
+def w4a8_moe_forward(packed_up, packed_down, E, H, F, x, ids, w, out, ws):
+    """x bf16 [T][H], ids int32 [T][k], w float32 [T][k], out bf16 [T][H], ws uint8 (cuda)."""
+    _dev(x, torch.bfloat16, "x")
+    _dev(ids, torch.int32, "ids")
+    _dev(w, torch.float32, "w")
+    _dev(out, torch.bfloat16, "out")
+    T, k = ids.shape
+    _check(lib().w4a8_moe_forward(_ptr(packed_up), _ptr(packed_down), E, H, F, _ptr(x), T, _ptr(ids), _ptr(w), k,
+                                  _ptr(out), _ptr(ws), ws.numel(), _stream()), "w4a8_moe_forward")
+
+
+def w4a8_moe_forward_host(packed_up, packed_down, E, H, F, x, ids, w, out, ws):
+    """Same as w4a8_moe_forward with x / ids / w / out in (pinned) HOST memory."""
+    for t, nm in ((x, "x"), (ids, "ids"), (w, "w"), (out, "out")):
+        if t.is_cuda:
+            raise W4A8Error(f"{nm} must be a host tensor")
+    T, k = ids.shape
+    _check(lib().w4a8_moe_forward_host(_ptr(packed_up), _ptr(packed_down), E, H, F, _ptr(x), T, _ptr(ids), _ptr(w),
+                                       k, _ptr(out), _ptr(ws), ws.numel(), _stream()), "w4a8_moe_forward_host")
+
+
+def w4a8_gemm_workspace_bytes(M, N, K) -> int:
+    return lib().w4a8_gemm_workspace_bytes(M, N, K)
+
+
+def w4a8_gemm(qa, sa, packed, N, K, y, ws, partials=None):
+    """qa int8 [M][Kp], sa float32 [M], y float32 [M][N], partials int32 [M][N][Kp/128] or None."""
+    _dev(qa, torch.int8, "qa")
+    _dev(sa, torch.float32, "sa")
+    _dev(y, torch.float32, "y")
+    M = qa.shape[0]
+    _check(lib().w4a8_gemm(_ptr(qa), _ptr(sa), M, _ptr(packed), N, K, _ptr(y), _ptr(partials), _ptr(ws), ws.numel(),
+                           _stream()), "w4a8_gemm")
+
+
+def w4a8_debug_region(T, E, k, H, F, what) -> tuple[int, int]:
+    off, nb = ctypes.c_size_t(), ctypes.c_size_t()
+    _check(lib().w4a8_debug_region(T, E, k, H, F, DUMP.get(what, what), ctypes.byref(off), ctypes.byref(nb)),
+           "w4a8_debug_region")
+    return off.value, nb.value
+
+
+def w4a8_debug_dump(ws, T, E, k, H, F, what) -> torch.Tensor:
+    """Copy one workspace region to a new uint8 cuda tensor."""
+    _, nb = w4a8_debug_region(T, E, k, H, F, what)
+    dst = torch.empty(nb, dtype=torch.uint8, device=ws.device)
+    _check(lib().w4a8_debug_dump(_ptr(ws), T, E, k, H, F, DUMP.get(what, what), _ptr(dst), nb, _stream()),
+           "w4a8_debug_dump")
+    return dst
+
+
+def w4a8_last_device_error(ws) -> int:
+    r = lib().w4a8_last_device_error(_ptr(ws), _stream())
+    if r < 0:
+        _check(r, "w4a8_last_device_error")
+    return r
+
+
+def empty_aligned(nbytes: int, device="cuda") -> torch.Tensor:
+    """A uint8 device buffer whose start is 256-byte aligned (torch's caching
+    allocator returns at least 512-byte aligned blocks)."""
+    t = torch.empty(max(int(nbytes), 1), dtype=torch.uint8, device=device)
+    if t.data_ptr() % 256:
+        raise W4A8Error("allocator returned a buffer that is not 256-byte aligned")
+    return t

@@ -1,0 +1,412 @@
+// C ABI of libw4a8.so: argument validation, workspace carve-up and the launch
+// sequence of the W4A8 MoE expert FFN.  Declarations and the contract of every
+// entry point are in include/w4a8.h.
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "../../include/w4a8.h"
+#include "w4a8_common.cuh"
+#include "w4a8_internal.h"
+
+#define W4A8_EXPORT extern "C" __attribute__((visibility("default")))
+
+namespace w4a8 {
+namespace {
+
+constexpr size_t kAlign = 256;
+inline size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int sm_count() {
+    static int counts[64] = {0};
+    static std::mutex mu;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    std::lock_guard<std::mutex> lock(mu);
+    if (counts[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        counts[dev] = n;
+    }
+    return counts[dev];
+}
+
+// Row capacity of the expert-grouped layout: every non-empty expert's segment is
+// padded up to a multiple of 16 rows.
+int rows_capacity(int T, int E, int k) {
+    const long long nslots = (long long)T * k;
+    if (nslots <= 0) return 0;
+    const long long pad = (long long)(kRowPad - 1) * (nslots < E ? nslots : E);
+    return (int)(((nslots + pad + kRowPad - 1) / kRowPad) * kRowPad);
+}
+
+// Workspace of w4a8_moe_forward: regions in the order of the enum below.
+enum Region {
+    R_ERR, R_CHIST, R_COUNTS, R_OFFS, R_POFFS, R_MTSTART, R_PERM, R_INV, R_ROWSRC,
+    R_ACT1, R_S1, R_AMAX, R_H, R_ACT2, R_S2, R_Y2,
+    R_XIN, R_IDSIN, R_WIN, R_OUT,  // host-buffer variant only
+    R_COUNT
+};
+
+struct MoeLayout {
+    size_t off[R_COUNT + 1];
+    size_t bytes[R_COUNT];
+    int nslots, nchunk, R, Hp, Fp, G1, G2;
+};
+
+bool moe_layout(int T, int E, int k, int H, int F, bool host_io, MoeLayout* L) {
+    if (T < 0 || E < 1 || E > kMaxExperts || k < 1 || k > 32 || k > E || H < 1 || F < 1) return false;
+    if ((long long)T * k >= (1ll << 31)) return false;
+    L->nslots = T * k;
+    L->nchunk = ceil_div(L->nslots, kPermChunk);
+    L->R = rows_capacity(T, E, k);
+    L->Hp = round_up(H, kGroup);
+    L->Fp = round_up(F, kGroup);
+    L->G1 = L->Hp / kGroup;
+    L->G2 = L->Fp / kGroup;
+    const size_t R = (size_t)L->R;
+    size_t* b = L->bytes;
+    b[R_ERR] = 16;
+    b[R_CHIST] = (size_t)L->nchunk * E * 4;
+    b[R_COUNTS] = (size_t)E * 4;
+    b[R_OFFS] = (size_t)(E + 1) * 4;
+    b[R_POFFS] = (size_t)(E + 1) * 4;
+    b[R_MTSTART] = (size_t)(E + 1) * 4;
+    b[R_PERM] = (size_t)L->nslots * 4;
+    b[R_INV] = (size_t)L->nslots * 4;
+    b[R_ROWSRC] = R * 4;
+    b[R_ACT1] = (size_t)L->G1 * R * 128;
+    b[R_S1] = R * 4;
+    b[R_AMAX] = R * 4;
+    b[R_H] = R * (size_t)L->Fp * 4;
+    b[R_ACT2] = (size_t)L->G2 * R * 128;
+    b[R_S2] = R * 4;
+    b[R_Y2] = R * (size_t)H * 4;
+    b[R_XIN] = host_io ? (size_t)T * H * 2 : 0;
+    b[R_IDSIN] = host_io ? (size_t)L->nslots * 4 : 0;
+    b[R_WIN] = host_io ? (size_t)L->nslots * 4 : 0;
+    b[R_OUT] = host_io ? (size_t)T * H * 2 : 0;
+    size_t o = 0;
+    for (int r = 0; r < R_COUNT; ++r) {
+        L->off[r] = o;
+        o += align_up(b[r]);
+    }
+    L->off[R_COUNT] = o;
+    return true;
+}
+
+int to_status(cudaError_t e) { return e == cudaSuccess ? W4A8_OK : W4A8_ECUDA; }
+
+#define W4A8_TRY(expr)                                  \
+    do {                                                \
+        cudaError_t _e = (expr);                        \
+        if (_e != cudaSuccess) return W4A8_ECUDA;       \
+    } while (0)
+
+int packed_tiles(int N, int layout) {
+    return layout == W4A8_LAYOUT_GATEUP ? ceil_div(N / 2, kTileRows / 2) : ceil_div(N, kTileRows);
+}
+
+template <typename T>
+T* at(void* base, const MoeLayout& L, Region r) {
+    return reinterpret_cast<T*>(static_cast<uint8_t*>(base) + L.off[r]);
+}
+
+// the forward on device buffers, workspace already validated
+int moe_forward_impl(const void* packed_up, const void* packed_down, int E, int H, int F, const uint16_t* x, int T,
+                     const int32_t* ids, const float* w, int k, uint16_t* out, void* ws, const MoeLayout& L,
+                     cudaStream_t st) {
+    uint32_t* err = at<uint32_t>(ws, L, R_ERR);
+    W4A8_TRY(cudaMemsetAsync(err, 0, 16, st));
+    if (T == 0) return W4A8_OK;
+    int* counts = at<int>(ws, L, R_COUNTS);
+    int* offs = at<int>(ws, L, R_OFFS);
+    int* poffs = at<int>(ws, L, R_POFFS);
+    int* mtstart = at<int>(ws, L, R_MTSTART);
+    int* row_src = at<int>(ws, L, R_ROWSRC);
+    int* inv = at<int>(ws, L, R_INV);
+    float* s1 = at<float>(ws, L, R_S1);
+    float* s2 = at<float>(ws, L, R_S2);
+    uint32_t* amax = at<uint32_t>(ws, L, R_AMAX);
+    float* h = at<float>(ws, L, R_H);
+    float* y2 = at<float>(ws, L, R_Y2);
+    int8_t* act1 = at<int8_t>(ws, L, R_ACT1);
+    int8_t* act2 = at<int8_t>(ws, L, R_ACT2);
+    const size_t plane = (size_t)L.R * 128;
+
+    W4A8_TRY(launch_perm(ids, L.nslots, E, at<int>(ws, L, R_CHIST), L.nchunk, counts, offs, poffs, mtstart,
+                         at<int>(ws, L, R_PERM), inv, row_src, err, st));
+    W4A8_TRY(launch_act_scatter(x, H, k, row_src, poffs, E, L.R, act1, plane, s1, amax, st));
+
+    GemmArgs up{};
+    up.wblocks = static_cast<const uint8_t*>(packed_up) + kHeaderBytes;
+    up.NT = packed_tiles(2 * F, W4A8_LAYOUT_GATEUP);
+    up.G = L.G1;
+    up.act = act1;
+    up.act_plane = plane;
+    up.act_scale = s1;
+    up.counts = counts;
+    up.poffs = poffs;
+    up.mtstart = mtstart;
+    up.E = E;
+    up.mode = 1;
+    up.out = h;
+    up.ldo = L.Fp;
+    up.nvalid = F;
+    up.amax = amax;
+    up.partials = nullptr;
+    up.err = err;
+    W4A8_TRY(launch_gemm(up, sm_count(), st));
+
+    W4A8_TRY(launch_requant(h, L.Fp, F, row_src, poffs, E, L.R, amax, act2, plane, s2, st));
+
+    GemmArgs dn = up;
+    dn.wblocks = static_cast<const uint8_t*>(packed_down) + kHeaderBytes;
+    dn.NT = packed_tiles(H, W4A8_LAYOUT_PLAIN);
+    dn.G = L.G2;
+    dn.act = act2;
+    dn.act_scale = s2;
+    dn.mode = 2;
+    dn.out = y2;
+    dn.ldo = H;
+    dn.nvalid = H;
+    dn.amax = nullptr;
+    W4A8_TRY(launch_gemm(dn, sm_count(), st));
+
+    W4A8_TRY(launch_combine(y2, H, inv, w, T, k, out, st));
+    return W4A8_OK;
+}
+
+int check_moe_args(const void* packed_up, const void* packed_down, int E, int H, int F, int T, int k, void* ws,
+                   size_t ws_bytes, bool host_io, MoeLayout* L) {
+    if (!moe_layout(T, E, k, H, F, host_io, L)) {
+        if (E > kMaxExperts || k > 32) return W4A8_EUNSUPPORTED;
+        return W4A8_EINVAL;
+    }
+    if (packed_up == nullptr || packed_down == nullptr || ws == nullptr) return W4A8_EINVAL;
+    if (!aligned(packed_up, kAlign) || !aligned(packed_down, kAlign) || !aligned(ws, kAlign)) return W4A8_EALIGN;
+    if (ws_bytes < L->off[R_COUNT]) return W4A8_ENOSPACE;
+    return W4A8_OK;
+}
+
+}  // namespace
+}  // namespace w4a8
+
+using namespace w4a8;
+
+W4A8_EXPORT int w4a8_version(void) { return 100; }
+
+W4A8_EXPORT const char* w4a8_status_string(int status) {
+    switch (status) {
+        case W4A8_OK: return "ok";
+        case W4A8_EINVAL: return "invalid argument";
+        case W4A8_EALIGN: return "misaligned pointer";
+        case W4A8_ENOSPACE: return "buffer or workspace too small";
+        case W4A8_ECUDA: return "CUDA error";
+        case W4A8_EUNSUPPORTED: return "unsupported shape";
+        case W4A8_ETIMEOUT: return "device wait timed out";
+        case W4A8_EDEVICE: return "bad data on device";
+        default: return "unknown status";
+    }
+}
+
+W4A8_EXPORT size_t w4a8_packed_bytes(int E, int N, int K, int layout) {
+    if (E < 1 || N < 1 || K < 1) return 0;
+    if (layout != W4A8_LAYOUT_PLAIN && layout != W4A8_LAYOUT_GATEUP) return 0;
+    if (layout == W4A8_LAYOUT_GATEUP && (N & 1)) return 0;
+    const size_t G = (size_t)ceil_div(K, kGroup);
+    return (size_t)kHeaderBytes + (size_t)E * packed_tiles(N, layout) * G * kBlockBytes;
+}
+
+W4A8_EXPORT int w4a8_pack_weights(const void* w_bf16, int E, int N, int K, int layout, void* packed,
+                                  size_t packed_bytes, uint8_t* codes_opt, uint16_t* scale_f16_opt,
+                                  uint16_t* zp_f16_opt, void* stream) {
+    const size_t need = w4a8_packed_bytes(E, N, K, layout);
+    if (need == 0 || w_bf16 == nullptr || packed == nullptr) return W4A8_EINVAL;
+    if (E > 65535) return W4A8_EUNSUPPORTED;
+    if (!aligned(w_bf16, 16) || !aligned(packed, kAlign)) return W4A8_EALIGN;
+    if ((codes_opt && !aligned(codes_opt, 16)) || (scale_f16_opt && !aligned(scale_f16_opt, 2)) ||
+        (zp_f16_opt && !aligned(zp_f16_opt, 2)))
+        return W4A8_EALIGN;
+    if (packed_bytes < need) return W4A8_ENOSPACE;
+    return to_status(launch_pack(static_cast<const uint16_t*>(w_bf16), E, N, K, layout,
+                                 static_cast<uint8_t*>(packed), codes_opt, scale_f16_opt, zp_f16_opt,
+                                 static_cast<cudaStream_t>(stream)));
+}
+
+W4A8_EXPORT int w4a8_quant_act(const void* x_bf16, int T, int K, int8_t* q, float* s, void* stream) {
+    if (T < 0 || K < 1) return W4A8_EINVAL;
+    if (T == 0) return W4A8_OK;
+    if (x_bf16 == nullptr || q == nullptr || s == nullptr) return W4A8_EINVAL;
+    if (!aligned(x_bf16, 16) || !aligned(q, 16) || !aligned(s, 16)) return W4A8_EALIGN;
+    return to_status(launch_quant_act(static_cast<const uint16_t*>(x_bf16), T, K, q, s,
+                                      static_cast<cudaStream_t>(stream)));
+}
+
+W4A8_EXPORT int w4a8_route_topk(const void* logits_bf16, int T, int E, int k, int32_t* ids, float* w,
+                                void* stream) {
+    if (T < 0 || E < 1 || k < 1 || k > E) return W4A8_EINVAL;
+    if (E > kMaxExperts || k > 32) return W4A8_EUNSUPPORTED;
+    if (T == 0) return W4A8_OK;
+    if (logits_bf16 == nullptr || ids == nullptr || w == nullptr) return W4A8_EINVAL;
+    if (!aligned(logits_bf16, 16) || !aligned(ids, 16) || !aligned(w, 16)) return W4A8_EALIGN;
+    return to_status(launch_route_topk(static_cast<const uint16_t*>(logits_bf16), T, E, k, ids, w,
+                                       static_cast<cudaStream_t>(stream)));
+}
+
+W4A8_EXPORT int w4a8_moe_rows_capacity(int T, int E, int k) { return rows_capacity(T, E, k); }
+
+W4A8_EXPORT size_t w4a8_moe_workspace_bytes(int T, int E, int k, int H, int F) {
+    MoeLayout L;
+    if (!moe_layout(T, E, k, H, F, false, &L)) return 0;
+    return L.off[R_COUNT];
+}
+
+W4A8_EXPORT size_t w4a8_moe_host_workspace_bytes(int T, int E, int k, int H, int F) {
+    MoeLayout L;
+    if (!moe_layout(T, E, k, H, F, true, &L)) return 0;
+    return L.off[R_COUNT];
+}
+
+W4A8_EXPORT int w4a8_moe_forward(const void* packed_up, const void* packed_down, int E, int H, int F,
+                                 const void* x_bf16, int T, const int32_t* ids, const float* w, int k,
+                                 void* out_bf16, void* ws, size_t ws_bytes, void* stream) {
+    MoeLayout L;
+    const int st = check_moe_args(packed_up, packed_down, E, H, F, T, k, ws, ws_bytes, false, &L);
+    if (st != W4A8_OK) return st;
+    if (T > 0) {
+        if (x_bf16 == nullptr || ids == nullptr || w == nullptr || out_bf16 == nullptr) return W4A8_EINVAL;
+        if (!aligned(x_bf16, 16) || !aligned(ids, 16) || !aligned(w, 16) || !aligned(out_bf16, 16))
+            return W4A8_EALIGN;
+    }
+    return moe_forward_impl(packed_up, packed_down, E, H, F, static_cast<const uint16_t*>(x_bf16), T, ids, w, k,
+                            static_cast<uint16_t*>(out_bf16), ws, L, static_cast<cudaStream_t>(stream));
+}
+
+W4A8_EXPORT int w4a8_moe_forward_host(const void* packed_up, const void* packed_down, int E, int H, int F,
+                                      const void* x_bf16_host, int T, const int32_t* ids_host, const float* w_host,
+                                      int k, void* out_bf16_host, void* ws, size_t ws_bytes, void* stream) {
+    MoeLayout L;
+    const int st = check_moe_args(packed_up, packed_down, E, H, F, T, k, ws, ws_bytes, true, &L);
+    if (st != W4A8_OK) return st;
+    if (T == 0) return W4A8_OK;
+    if (x_bf16_host == nullptr || ids_host == nullptr || w_host == nullptr || out_bf16_host == nullptr)
+        return W4A8_EINVAL;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint16_t* x = at<uint16_t>(ws, L, R_XIN);
+    int32_t* ids = at<int32_t>(ws, L, R_IDSIN);
+    float* w = at<float>(ws, L, R_WIN);
+    uint16_t* out = at<uint16_t>(ws, L, R_OUT);
+    W4A8_TRY(cudaMemcpyAsync(x, x_bf16_host, L.bytes[R_XIN], cudaMemcpyHostToDevice, s));
+    W4A8_TRY(cudaMemcpyAsync(ids, ids_host, L.bytes[R_IDSIN], cudaMemcpyHostToDevice, s));
+    W4A8_TRY(cudaMemcpyAsync(w, w_host, L.bytes[R_WIN], cudaMemcpyHostToDevice, s));
+    const int r = moe_forward_impl(packed_up, packed_down, E, H, F, x, T, ids, w, k, out, ws, L, s);
+    if (r != W4A8_OK) return r;
+    W4A8_TRY(cudaMemcpyAsync(out_bf16_host, out, L.bytes[R_OUT], cudaMemcpyDeviceToHost, s));
+    return W4A8_OK;
+}
+
+namespace w4a8 {
+namespace {
+struct GemmLayout {
+    size_t err, counts, poffs, mtstart, act, total;
+    int Mp, G;
+};
+bool gemm_layout(int M, int N, int K, GemmLayout* L) {
+    if (M < 0 || N < 1 || K < 1) return false;
+    L->Mp = round_up(M, kRowPad);
+    L->G = ceil_div(K, kGroup);
+    size_t o = 0;
+    L->err = o; o += align_up(16);
+    L->counts = o; o += align_up(4);
+    L->poffs = o; o += align_up(8);
+    L->mtstart = o; o += align_up(8);
+    L->act = o; o += align_up((size_t)L->G * L->Mp * 128);
+    L->total = o;
+    return true;
+}
+}  // namespace
+}  // namespace w4a8
+
+W4A8_EXPORT size_t w4a8_gemm_workspace_bytes(int M, int N, int K) {
+    GemmLayout L;
+    if (!gemm_layout(M, N, K, &L)) return 0;
+    return L.total;
+}
+
+W4A8_EXPORT int w4a8_gemm(const int8_t* qa, const float* sa, int M, const void* packed, int N, int K, float* y,
+                          int32_t* partials_opt, void* ws, size_t ws_bytes, void* stream) {
+    GemmLayout L;
+    if (!gemm_layout(M, N, K, &L)) return W4A8_EINVAL;
+    if (packed == nullptr || ws == nullptr) return W4A8_EINVAL;
+    if (!aligned(packed, kAlign) || !aligned(ws, kAlign)) return W4A8_EALIGN;
+    if (ws_bytes < L.total) return W4A8_ENOSPACE;
+    uint8_t* base = static_cast<uint8_t*>(ws);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint32_t* err = reinterpret_cast<uint32_t*>(base + L.err);
+    W4A8_TRY(cudaMemsetAsync(err, 0, 16, s));
+    if (M == 0) return W4A8_OK;
+    if (qa == nullptr || sa == nullptr || y == nullptr) return W4A8_EINVAL;
+    if (!aligned(qa, 16) || !aligned(sa, 4) || !aligned(y, 4) || (partials_opt && !aligned(partials_opt, 4)))
+        return W4A8_EALIGN;
+    int* counts = reinterpret_cast<int*>(base + L.counts);
+    int* poffs = reinterpret_cast<int*>(base + L.poffs);
+    int* mtstart = reinterpret_cast<int*>(base + L.mtstart);
+    int8_t* act = reinterpret_cast<int8_t*>(base + L.act);
+    const size_t plane = (size_t)L.Mp * 128;
+    W4A8_TRY(launch_dense_prep(qa, M, L.G * kGroup, act, plane, counts, poffs, mtstart, s));
+    GemmArgs a{};
+    a.wblocks = static_cast<const uint8_t*>(packed) + kHeaderBytes;
+    a.NT = packed_tiles(N, W4A8_LAYOUT_PLAIN);
+    a.G = L.G;
+    a.act = act;
+    a.act_plane = plane;
+    a.act_scale = sa;
+    a.counts = counts;
+    a.poffs = poffs;
+    a.mtstart = mtstart;
+    a.E = 1;
+    a.mode = 0;
+    a.out = y;
+    a.ldo = N;
+    a.nvalid = N;
+    a.amax = nullptr;
+    a.partials = partials_opt;
+    a.err = err;
+    W4A8_TRY(launch_gemm(a, sm_count(), s));
+    return W4A8_OK;
+}
+
+W4A8_EXPORT int w4a8_debug_region(int T, int E, int k, int H, int F, int what, size_t* offset, size_t* bytes) {
+    MoeLayout L;
+    if (!moe_layout(T, E, k, H, F, false, &L) || offset == nullptr || bytes == nullptr) return W4A8_EINVAL;
+    static const Region map[] = {R_COUNTS, R_OFFS, R_PERM, R_INV, R_POFFS, R_ACT1,
+                                 R_S1,     R_H,    R_ACT2, R_S2,  R_Y2,    R_ERR};
+    if (what < 0 || what >= (int)(sizeof(map) / sizeof(map[0]))) return W4A8_EINVAL;
+    *offset = L.off[map[what]];
+    *bytes = what == W4A8_DUMP_ERR ? 4 : L.bytes[map[what]];
+    return W4A8_OK;
+}
+
+W4A8_EXPORT int w4a8_debug_dump(const void* ws, int T, int E, int k, int H, int F, int what, void* dst,
+                                size_t bytes, void* stream) {
+    size_t off = 0, n = 0;
+    const int r = w4a8_debug_region(T, E, k, H, F, what, &off, &n);
+    if (r != W4A8_OK) return r;
+    if (ws == nullptr || dst == nullptr) return W4A8_EINVAL;
+    if (bytes < n) n = bytes;
+    if (n == 0) return W4A8_OK;
+    return to_status(cudaMemcpyAsync(dst, static_cast<const uint8_t*>(ws) + off, n, cudaMemcpyDefault,
+                                     static_cast<cudaStream_t>(stream)));
+}
+
+W4A8_EXPORT int w4a8_last_device_error(const void* ws, void* stream) {
+    if (ws == nullptr) return W4A8_EINVAL;
+    uint32_t v = 0;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaMemcpyAsync(&v, ws, 4, cudaMemcpyDeviceToHost, s) != cudaSuccess) return W4A8_ECUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return W4A8_ECUDA;
+    return (int)v;
+}
