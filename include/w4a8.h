@@ -173,6 +173,27 @@ int w4a8_debug_dump(const void* ws, int T, int E, int k, int H, int F, int what,
  * Any workspace from w4a8_moe_forward / w4a8_gemm may be passed. */
 int w4a8_last_device_error(const void* ws, void* stream);
 
+/* Per-kernel device timing, for benchmarks.  After w4a8_profile_start(), every
+ * w4a8_moe_forward / w4a8_moe_forward_host / w4a8_gemm call made from the same
+ * host thread records a pair of CUDA events around each kernel kind it launches
+ * (on the call's stream).  w4a8_profile_stop() waits for those events, writes
+ * per kind the number of kernel launches and their summed device milliseconds
+ * (arrays of n entries, indexed by the W4A8_KERNEL_* values; a "perm" entry covers
+ * the three permutation kernels), stops recording and returns W4A8_OK.  Timing
+ * adds one event record per kernel; it changes no result. */
+enum {
+    W4A8_KERNEL_PERM = 0,      /* histogram + scan + scatter (3 launches)      */
+    W4A8_KERNEL_ACT_QUANT = 1, /* per-token INT8 into the grouped tiled rows    */
+    W4A8_KERNEL_GEMM_UP = 2,   /* grouped W4A8 GEMM, gate|up, SwiGLU epilogue   */
+    W4A8_KERNEL_REQUANT = 3,   /* per-row INT8 of h                             */
+    W4A8_KERNEL_GEMM_DOWN = 4, /* grouped W4A8 GEMM, down projection            */
+    W4A8_KERNEL_COMBINE = 5,   /* weighted sum of the k expert outputs          */
+    W4A8_KERNEL_GEMM_DENSE = 6,/* w4a8_gemm (re-layout + GEMM, 2 launches)      */
+    W4A8_KERNEL_KINDS = 7
+};
+int w4a8_profile_start(void);
+int w4a8_profile_stop(int* launches, float* total_ms, int n);
+
 /* Human-readable name of a w4a8_status value. */
 const char* w4a8_status_string(int status);
 

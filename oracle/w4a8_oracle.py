@@ -99,7 +99,8 @@ def quantize_weights(w: np.ndarray):
         s16 = s32.astype(np.float16)  # round to nearest even fp16 (R5)
         s16[s16 == 0] = np.float16(1.0)  # R3: degenerate (all-zero) group
         sf = s16.astype(np.float32)
-        z = np.clip(np.rint(-mn / sf), 0, INT4_MAX)  # R4, R6
+        # R4, R6; the zero point is an integer index offset, so -0.0 is stored as 0
+        z = np.clip(np.rint(-mn / sf), 0, INT4_MAX) + np.float32(0)
         q = np.rint(v / sf[:, None]) + z[:, None]
         codes[:, g * GROUP:(g + 1) * GROUP] = np.clip(q, 0, INT4_MAX).astype(np.uint8)
         scale[:, g] = s16

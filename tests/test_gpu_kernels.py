@@ -15,6 +15,8 @@ pytestmark = pytest.mark.gpu
 
 
 def dev_bf16(a):
+    a = np.ascontiguousarray(a, dtype=np.float32)
+    assert np.array_equal(synth.bf16_round(a), a), "inputs must be bf16-exact"
     return torch.from_numpy(synth.bf16_bits(a).view(np.int16)).view(torch.bfloat16).cuda()
 
 
@@ -68,6 +70,7 @@ def test_pack_bit_exact(E, N, K, layout):
     w = synth.bf16_round((rng.standard_normal((E, N, K)) * 0.02).astype(np.float32))
     w[0, 0, :] = 0.0  # degenerate group
     w[0, 1, :128] += 0.3  # skewed group
+    w = synth.bf16_round(w)
     packed, codes, scale, zp = pack_on_gpu(w, layout)
     codes_h, scale_h, zp_h = codes.cpu().numpy(), scale.cpu().numpy(), zp.cpu().numpy()
     dc, ds, dz = decode_packed(packed.cpu().numpy(), E, N, K, layout)

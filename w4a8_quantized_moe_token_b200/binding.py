@@ -44,7 +44,11 @@ _SIGS = {
     "w4a8_debug_region": ([_c_int] * 6 + [ctypes.POINTER(_c_size), ctypes.POINTER(_c_size)], _c_int),
     "w4a8_debug_dump": ([_vp] + [_c_int] * 6 + [_vp, _c_size, _vp], _c_int),
     "w4a8_last_device_error": ([_vp, _vp], _c_int),
+    "w4a8_profile_start": ([], _c_int),
+    "w4a8_profile_stop": ([ctypes.POINTER(_c_int), ctypes.POINTER(ctypes.c_float), _c_int], _c_int),
 }
+
+KERNEL_KINDS = ["perm", "act_quant", "gemm_up", "requant", "gemm_down", "combine", "gemm_dense"]
 
 _lib = None
 
@@ -214,3 +218,16 @@ def empty_aligned(nbytes: int, device="cuda") -> torch.Tensor:
     if t.data_ptr() % 256:
         raise W4A8Error("allocator returned a buffer that is not 256-byte aligned")
     return t
+
+
+def w4a8_profile_start():
+    _check(lib().w4a8_profile_start(), "w4a8_profile_start")
+
+
+def w4a8_profile_stop() -> dict:
+    """{kernel kind: (launches, total device ms)} since w4a8_profile_start()."""
+    n = len(KERNEL_KINDS)
+    launches = (ctypes.c_int * n)()
+    ms = (ctypes.c_float * n)()
+    _check(lib().w4a8_profile_stop(launches, ms, n), "w4a8_profile_stop")
+    return {k: (launches[i], ms[i]) for i, k in enumerate(KERNEL_KINDS)}

@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 
 #include <mutex>
+#include <vector>
 
 #include "../../include/w4a8.h"
 #include "w4a8_common.cuh"
@@ -99,6 +100,49 @@ bool moe_layout(int T, int E, int k, int H, int F, bool host_io, MoeLayout* L) {
 
 int to_status(cudaError_t e) { return e == cudaSuccess ? W4A8_OK : W4A8_ECUDA; }
 
+// Optional per-kernel event timing (w4a8_profile_start / w4a8_profile_stop),
+// kept per host thread.
+struct Profiler {
+    bool on = false;
+    struct Rec {
+        int kind;
+        cudaEvent_t a, b;
+    };
+    std::vector<cudaEvent_t> pool;
+    std::vector<Rec> recs;
+    int launches[W4A8_KERNEL_KINDS] = {0};
+};
+thread_local Profiler g_prof;
+
+cudaEvent_t prof_event() {
+    if (!g_prof.pool.empty()) {
+        cudaEvent_t e = g_prof.pool.back();
+        g_prof.pool.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    return e;
+}
+
+// RAII: records an event pair around the kernels launched in its scope
+struct ProfScope {
+    int kind, nlaunch;
+    cudaStream_t st;
+    cudaEvent_t a = nullptr;
+    ProfScope(int k, int n, cudaStream_t s) : kind(k), nlaunch(n), st(s) {
+        if (g_prof.on && (a = prof_event()) != nullptr) cudaEventRecord(a, st);
+    }
+    ~ProfScope() {
+        if (a == nullptr) return;
+        cudaEvent_t b = prof_event();
+        if (b == nullptr) return;
+        cudaEventRecord(b, st);
+        g_prof.recs.push_back({kind, a, b});
+        g_prof.launches[kind] += nlaunch;
+    }
+};
+
 #define W4A8_TRY(expr)                                  \
     do {                                                \
         cudaError_t _e = (expr);                        \
@@ -136,9 +180,15 @@ int moe_forward_impl(const void* packed_up, const void* packed_down, int E, int 
     int8_t* act2 = at<int8_t>(ws, L, R_ACT2);
     const size_t plane = (size_t)L.R * 128;
 
-    W4A8_TRY(launch_perm(ids, L.nslots, E, at<int>(ws, L, R_CHIST), L.nchunk, counts, offs, poffs, mtstart,
-                         at<int>(ws, L, R_PERM), inv, row_src, err, st));
-    W4A8_TRY(launch_act_scatter(x, H, k, row_src, poffs, E, L.R, act1, plane, s1, amax, st));
+    {
+        ProfScope p(W4A8_KERNEL_PERM, 3, st);
+        W4A8_TRY(launch_perm(ids, L.nslots, E, at<int>(ws, L, R_CHIST), L.nchunk, counts, offs, poffs, mtstart,
+                             at<int>(ws, L, R_PERM), inv, row_src, err, st));
+    }
+    {
+        ProfScope p(W4A8_KERNEL_ACT_QUANT, 1, st);
+        W4A8_TRY(launch_act_scatter(x, H, k, row_src, poffs, E, L.R, act1, plane, s1, amax, st));
+    }
 
     GemmArgs up{};
     up.wblocks = static_cast<const uint8_t*>(packed_up) + kHeaderBytes;
@@ -158,9 +208,14 @@ int moe_forward_impl(const void* packed_up, const void* packed_down, int E, int 
     up.amax = amax;
     up.partials = nullptr;
     up.err = err;
-    W4A8_TRY(launch_gemm(up, sm_count(), st));
-
-    W4A8_TRY(launch_requant(h, L.Fp, F, row_src, poffs, E, L.R, amax, act2, plane, s2, st));
+    {
+        ProfScope p(W4A8_KERNEL_GEMM_UP, 1, st);
+        W4A8_TRY(launch_gemm(up, sm_count(), st));
+    }
+    {
+        ProfScope p(W4A8_KERNEL_REQUANT, 1, st);
+        W4A8_TRY(launch_requant(h, L.Fp, F, row_src, poffs, E, L.R, amax, act2, plane, s2, st));
+    }
 
     GemmArgs dn = up;
     dn.wblocks = static_cast<const uint8_t*>(packed_down) + kHeaderBytes;
@@ -173,9 +228,14 @@ int moe_forward_impl(const void* packed_up, const void* packed_down, int E, int 
     dn.ldo = H;
     dn.nvalid = H;
     dn.amax = nullptr;
-    W4A8_TRY(launch_gemm(dn, sm_count(), st));
-
-    W4A8_TRY(launch_combine(y2, H, inv, w, T, k, out, st));
+    {
+        ProfScope p(W4A8_KERNEL_GEMM_DOWN, 1, st);
+        W4A8_TRY(launch_gemm(dn, sm_count(), st));
+    }
+    {
+        ProfScope p(W4A8_KERNEL_COMBINE, 1, st);
+        W4A8_TRY(launch_combine(y2, H, inv, w, T, k, out, st));
+    }
     return W4A8_OK;
 }
 
@@ -356,6 +416,7 @@ W4A8_EXPORT int w4a8_gemm(const int8_t* qa, const float* sa, int M, const void* 
     int* mtstart = reinterpret_cast<int*>(base + L.mtstart);
     int8_t* act = reinterpret_cast<int8_t*>(base + L.act);
     const size_t plane = (size_t)L.Mp * 128;
+    ProfScope prof(W4A8_KERNEL_GEMM_DENSE, 2, s);
     W4A8_TRY(launch_dense_prep(qa, M, L.G * kGroup, act, plane, counts, poffs, mtstart, s));
     GemmArgs a{};
     a.wblocks = static_cast<const uint8_t*>(packed) + kHeaderBytes;
@@ -409,4 +470,30 @@ W4A8_EXPORT int w4a8_last_device_error(const void* ws, void* stream) {
     if (cudaMemcpyAsync(&v, ws, 4, cudaMemcpyDeviceToHost, s) != cudaSuccess) return W4A8_ECUDA;
     if (cudaStreamSynchronize(s) != cudaSuccess) return W4A8_ECUDA;
     return (int)v;
+}
+
+W4A8_EXPORT int w4a8_profile_start(void) {
+    g_prof.on = true;
+    return W4A8_OK;
+}
+
+W4A8_EXPORT int w4a8_profile_stop(int* launches, float* total_ms, int n) {
+    float ms[W4A8_KERNEL_KINDS] = {0.f};
+    int rc = W4A8_OK;
+    for (auto& r : g_prof.recs) {
+        float t = 0.f;
+        if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&t, r.a, r.b) != cudaSuccess)
+            rc = W4A8_ECUDA;
+        ms[r.kind] += t;
+        g_prof.pool.push_back(r.a);
+        g_prof.pool.push_back(r.b);
+    }
+    for (int i = 0; i < n && i < W4A8_KERNEL_KINDS; ++i) {
+        if (launches) launches[i] = g_prof.launches[i];
+        if (total_ms) total_ms[i] = ms[i];
+    }
+    g_prof.recs.clear();
+    for (int i = 0; i < W4A8_KERNEL_KINDS; ++i) g_prof.launches[i] = 0;
+    g_prof.on = false;
+    return rc;
 }
