@@ -1,0 +1,589 @@
+#!/usr/bin/env python
+"""Benchmark of the W4A8 MoE expert FFN on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload toy_moe] [--impl ours|reference]
+
+One step = one forward of the whole hot path (routing when the workload routes
+from logits, permutation, INT8 activation quant, up GEMM + SwiGLU, requant, down
+GEMM, combine) over one batch of seeded synthetic input already resident in HBM.
+L2 is flushed (a 256 MiB write) before every timed step, outside the timed span.
+Steps are timed with CUDA events on the launching stream; per-kernel times come
+from the library's event profiler over the same timed region.  With N > 1 (one
+process per GPU under torchrun) every rank runs an independent replica of the
+layer -- the layer has no cross-GPU exchange -- and the slowest rank's time is
+reported ("scaling": "weak").  Rank 0 prints one JSON line.
+
+--impl reference times the CPU oracle (numpy, fp64 GEMMs through BLAS) on a
+bounded token sample of the same workload, on the host cores.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from w4a8_quantized_moe_token_b200 import synth  # noqa: E402
+
+METRIC = "W4A8 MoE FFN tokens/s, TOPS and weight GB/s on 1 B200; % of HBM / INT8 roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+INT8_OVER_BF16 = 4.5 / 2.25  # nominal dense INT8 / BF16 tensor peak ratio on B200
+
+
+# --------------------------------------------------------------------------- #
+# accounting (algorithmic work; pages' storage format: 0.5 B/weight + 4 B per 128-group)
+# --------------------------------------------------------------------------- #
+def padded(k):
+    return (k + 127) // 128 * 128
+
+
+def packed_matrix_bytes(N, K):
+    """4-bit codes + one fp16 scale and one fp16 zero point per 128-group."""
+    Kp = padded(K)
+    return N * Kp // 2 + N * (Kp // 128) * 4
+
+
+def moe_accounting(W, ids):
+    T, k, H, F = W.T, W.topk, W.H, W.F
+    touched = int(np.unique(ids).size)
+    slots = T * k
+    Hp, Fp = padded(H), padded(F)
+    up_w = touched * packed_matrix_bytes(2 * F, H)
+    dn_w = touched * packed_matrix_bytes(H, F)
+    k_ops = {
+        "gemm_up": 2.0 * slots * 2 * F * H,
+        "gemm_down": 2.0 * slots * H * F,
+    }
+    k_bytes = {
+        "perm": slots * 4 * 3.0,
+        "act_quant": T * H * 2.0 + slots * Hp + slots * 4,
+        "gemm_up": up_w + slots * Hp + slots * F * 4.0,
+        "requant": slots * F * 4.0 + slots * Fp,
+        "gemm_down": dn_w + slots * Fp + slots * H * 4.0,
+        "combine": slots * H * 4.0 + T * H * 2.0 + slots * 8,
+        "route": T * W.E * 2.0 + slots * 8,
+    }
+    return {"touched_experts": touched, "weight_bytes": up_w + dn_w, "ops": k_ops["gemm_up"] + k_ops["gemm_down"],
+            "kernel_ops": k_ops, "kernel_bytes": k_bytes}
+
+
+def gemm_accounting(W):
+    M, N, K = W.M, W.N, W.K
+    wb = packed_matrix_bytes(N, K)
+    return {"touched_experts": 1, "weight_bytes": wb, "ops": 2.0 * M * N * K,
+            "kernel_ops": {"gemm_dense": 2.0 * M * N * K},
+            "kernel_bytes": {"gemm_dense": wb + M * padded(K) * 2 + M * N * 4.0, "act_quant": M * K * 2.0 + M * K}}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        d["source"] = "measured"
+        return d
+    return dict(FALLBACK_PEAKS)
+
+
+# --------------------------------------------------------------------------- #
+# clocks during the timed region (NVML reads only)
+# --------------------------------------------------------------------------- #
+class ClockSampler:
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting", 0x1: "gpu_idle"}
+
+    def __init__(self, index, period=0.005):
+        self.index, self.period = index, period
+        self.samples, self.reasons, self.max_mhz = [], 0, None
+        self._stop = threading.Event()
+        self._t = None
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+
+    def _run(self):
+        nv = self._nv
+        get_r = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            getattr(nv, "nvmlDeviceGetCurrentClocksThrottleReasons")
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                self.reasons |= int(get_r(self._h))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+
+    def stop(self):
+        if self._t:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        rs = [n for b, n in self.REASONS.items() if self.reasons & b and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None, "sm_max_mhz": self.max_mhz,
+                "reasons": rs, "samples": len(self.samples)}
+
+
+# --------------------------------------------------------------------------- #
+# setup on the device
+# --------------------------------------------------------------------------- #
+def dev_bf16(a, device):
+    import torch
+    return torch.from_numpy(synth.bf16_bits(a).view(np.int16)).view(torch.bfloat16).to(device)
+
+
+def pack_experts(B, torch, W, seed, device):
+    """Pack every expert's up (gate|up) and down weights on the device, one expert at a time."""
+    E, H, F = W.E, W.H, W.F
+    up = B.empty_aligned(B.w4a8_packed_bytes(E, 2 * F, H, B.W4A8_LAYOUT_GATEUP), device)
+    dn = B.empty_aligned(B.w4a8_packed_bytes(E, H, F, B.W4A8_LAYOUT_PLAIN), device)
+    su = (up.numel() - 256) // E
+    sd = (dn.numel() - 256) // E
+    tu = B.empty_aligned(B.w4a8_packed_bytes(1, 2 * F, H, 1), device)
+    td = B.empty_aligned(B.w4a8_packed_bytes(1, H, F, 0), device)
+    for which, (buf, tmp, stride, rows, cols, layout) in (("up", (up, tu, su, 2 * F, H, 1)),
+                                                           ("down", (dn, td, sd, H, F, 0))):
+        for e, w in synth.expert_weights_parallel(seed, E, which, rows, cols):
+            B.w4a8_pack_weights(dev_bf16(w, device), layout, tmp)
+            buf[256 + e * stride:256 + (e + 1) * stride].copy_(tmp[256:])
+    torch.cuda.synchronize(device)
+    return up, dn
+
+
+class MoeStep:
+    def __init__(self, B, torch, W, seed, device):
+        self.B, self.torch, self.W, self.device = B, torch, W, device
+        inp = synth.moe_inputs(W, seed)
+        self.x_host = inp["x"]
+        T, E, k, H, F = W.T, W.E, W.topk, W.H, W.F
+        self.x = dev_bf16(inp["x"], device)
+        self.ids = torch.empty((T, k), dtype=torch.int32, device=device)
+        self.w = torch.empty((T, k), dtype=torch.float32, device=device)
+        self.logits = None
+        if "logits" in inp:
+            self.logits = dev_bf16(inp["logits"], device)
+            B.w4a8_route_topk(self.logits, k, self.ids, self.w)
+            torch.cuda.synchronize(device)
+            self.ids_host = self.ids.cpu().numpy()
+            self.w_host = self.w.cpu().numpy()
+        else:
+            self.ids_host, self.w_host = inp["ids"], inp["wts"]
+            self.ids.copy_(torch.from_numpy(inp["ids"]))
+            self.w.copy_(torch.from_numpy(inp["wts"]))
+        self.logits_host = inp.get("logits")
+        self.packed_up, self.packed_down = pack_experts(B, torch, W, seed, device)
+        self.out = torch.empty((T, H), dtype=torch.bfloat16, device=device)
+        self.ws = B.empty_aligned(B.w4a8_moe_workspace_bytes(T, E, k, H, F), device)
+        self.acct = moe_accounting(W, self.ids_host)
+        self.route_ms = 0.0
+        self.route_launches = 0
+        self.timing_route = False
+
+    def __call__(self):
+        B, W = self.B, self.W
+        if self.logits is not None:
+            if self.timing_route:
+                a = self.torch.cuda.Event(enable_timing=True)
+                b = self.torch.cuda.Event(enable_timing=True)
+                a.record()
+            B.w4a8_route_topk(self.logits, W.topk, self.ids, self.w)
+            if self.timing_route:
+                b.record()
+                self._route_events.append((a, b))
+                self.route_launches += 1
+        B.w4a8_moe_forward(self.packed_up, self.packed_down, W.E, W.H, W.F, self.x, self.ids, self.w, self.out,
+                           self.ws)
+
+    def start_route_timing(self):
+        self._route_events = []
+        self.route_launches = 0
+        self.timing_route = True
+
+    def stop_route_timing(self):
+        self.timing_route = False
+        self.route_ms = sum(a.elapsed_time(b) for a, b in self._route_events)
+
+    def e2e(self, steps, warmup):
+        """Same metric through the public API with HOST inputs/outputs: per step the
+        pinned-host inputs are copied in and the bf16 output copied back."""
+        torch, B, W = self.torch, self.B, self.W
+        T, E, k, H, F = W.T, W.E, W.topk, W.H, W.F
+        pin = lambda a: torch.from_numpy(a).pin_memory()
+        x_h = torch.from_numpy(synth.bf16_bits(self.x_host).view(np.int16)).view(torch.bfloat16).pin_memory()
+        out_h = torch.empty((T, H), dtype=torch.bfloat16).pin_memory()
+        if self.logits is None:
+            ids_h, w_h = pin(np.ascontiguousarray(self.ids_host)), pin(np.ascontiguousarray(self.w_host))
+            ws = B.empty_aligned(B.w4a8_moe_host_workspace_bytes(T, E, k, H, F), self.device)
+            h2d = x_h.numel() * 2 + ids_h.numel() * 4 + w_h.numel() * 4
+
+            def step():
+                B.w4a8_moe_forward_host(self.packed_up, self.packed_down, E, H, F, x_h, ids_h, w_h, out_h, ws)
+        else:
+            lg_h = torch.from_numpy(synth.bf16_bits(self.logits_host).view(np.int16)).view(torch.bfloat16).pin_memory()
+            x_d = torch.empty_like(self.x)
+            lg_d = torch.empty_like(self.logits)
+            h2d = x_h.numel() * 2 + lg_h.numel() * 2
+
+            def step():
+                x_d.copy_(x_h, non_blocking=True)
+                lg_d.copy_(lg_h, non_blocking=True)
+                B.w4a8_route_topk(lg_d, k, self.ids, self.w)
+                B.w4a8_moe_forward(self.packed_up, self.packed_down, E, H, F, x_d, self.ids, self.w, self.out,
+                                   self.ws)
+                out_h.copy_(self.out, non_blocking=True)
+        for _ in range(warmup):
+            step()
+        torch.cuda.synchronize()
+        total = 0.0
+        for _ in range(steps):
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            step()
+            b.record()
+            b.synchronize()
+            total += a.elapsed_time(b)
+        return total / steps, h2d, T * H * 2
+
+
+class GemmStep:
+    """Dense W4A8 linear: per-token INT8 of x, then the W4A8 GEMM."""
+
+    def __init__(self, B, torch, W, seed, device):
+        self.B, self.torch, self.W, self.device = B, torch, W, device
+        x, w = synth.dense_gemm_inputs(seed, W.M, W.K, W.N)
+        self.x = dev_bf16(x, device)
+        self.packed = B.empty_aligned(B.w4a8_packed_bytes(1, W.N, W.K, 0), device)
+        B.w4a8_pack_weights(dev_bf16(w, device), 0, self.packed)
+        Kp = padded(W.K)
+        self.q = torch.empty((W.M, Kp), dtype=torch.int8, device=device)
+        self.s = torch.empty(W.M, dtype=torch.float32, device=device)
+        self.y = torch.empty((W.M, W.N), dtype=torch.float32, device=device)
+        self.ws = B.empty_aligned(B.w4a8_gemm_workspace_bytes(W.M, W.N, W.K), device)
+        self.acct = gemm_accounting(W)
+        self.route_ms, self.route_launches = 0.0, 0
+
+    def __call__(self):
+        self.B.w4a8_quant_act(self.x, self.q, self.s)
+        self.B.w4a8_gemm(self.q, self.s, self.packed, self.W.N, self.W.K, self.y, self.ws)
+
+    def start_route_timing(self):
+        pass
+
+    def stop_route_timing(self):
+        pass
+
+    def e2e(self, steps, warmup):
+        torch = self.torch
+        x_h = self.x.cpu().pin_memory()
+        y_h = torch.empty_like(self.y, device="cpu").pin_memory()
+
+        def step():
+            self.x.copy_(x_h, non_blocking=True)
+            self()
+            y_h.copy_(self.y, non_blocking=True)
+        for _ in range(warmup):
+            step()
+        torch.cuda.synchronize()
+        total = 0.0
+        for _ in range(steps):
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            step()
+            b.record()
+            b.synchronize()
+            total += a.elapsed_time(b)
+        return total / steps, x_h.numel() * 2, y_h.numel() * 4
+
+
+# --------------------------------------------------------------------------- #
+# CPU oracle timing (the reported CPU baseline and the reference arm)
+# --------------------------------------------------------------------------- #
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+class OracleSample:
+    """The oracle forward on a bounded token sample of the workload (weights
+    quantised once beforehand, untimed -- the GPU step excludes packing too)."""
+
+    def __init__(self, W, seed, target_s):
+        from oracle import w4a8_oracle as O
+        self.O, self.W, self.seed = O, W, seed
+        if W.kind == "gemm":
+            x, w = synth.dense_gemm_inputs(seed, W.M, W.K, W.N)
+            self.x, self.qw = x, O.quantize_weights(w)
+            self.tokens = W.M
+            self.sample_desc = f"all {W.M} rows"
+            return
+        inp = synth.moe_inputs(W, seed)
+        self.x = inp["x"]
+        if "logits" in inp:
+            self.logits = inp["logits"]
+            self.ids, self.w = O.route_topk(self.logits, W.topk)
+        else:
+            self.logits = None
+            self.ids, self.w = inp["ids"], inp["wts"].astype(np.float64)
+        # size the token sample: time a few tokens, scale to the target
+        self.experts = {}
+        n = min(W.T, 8)
+        t = self._time(n)
+        per_tok = t / n
+        self.tokens = int(max(1, min(W.T, target_s / max(per_tok, 1e-6))))
+        self.sample_desc = f"{self.tokens} of {W.T} tokens ({self._touched(self.tokens)} experts)"
+
+    def _touched(self, n):
+        return int(np.unique(self.ids[:n]).size)
+
+    def _ensure_experts(self, n):
+        for e in np.unique(self.ids[:n]):
+            e = int(e)
+            if e not in self.experts:
+                W = self.W
+                self.experts[e] = self.O.QuantExpert(synth.expert_weight(self.seed, e, "up", 2 * W.F, W.H),
+                                                     synth.expert_weight(self.seed, e, "down", W.H, W.F))
+
+    def _time(self, n):
+        self._ensure_experts(n)
+        t0 = time.perf_counter()
+        self.run(n)
+        return time.perf_counter() - t0
+
+    def run(self, n=None):
+        O, W = self.O, self.W
+        if W.kind == "gemm":
+            qa, sa = O.quantize_act(self.x)
+            return O.w4a8_linear(qa, sa, *self.qw)
+        n = self.tokens if n is None else n
+        if self.logits is not None:
+            O.route_topk(self.logits[:n], W.topk)
+        return O.moe_forward(self.x[:n], self.ids[:n], self.w[:n], self.experts, W.E, W.F)
+
+    def timed(self, reps=1):
+        if self.W.kind != "gemm":
+            self._ensure_experts(self.tokens)
+        t0 = time.perf_counter()
+        for _ in range(reps):
+            self.run()
+        return (time.perf_counter() - t0) / reps
+
+
+# --------------------------------------------------------------------------- #
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def run_reference(args, W):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    target = max(0.5, min(10.0, 150.0 / max(1, args.steps + args.warmup)))
+    S = OracleSample(W, args.seed, target)
+    for _ in range(args.warmup):
+        S.run()
+    t = sum(S.timed() for _ in range(args.steps)) / args.steps
+    tokens = S.tokens
+    value = tokens / t
+    cores = blas_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_of(W, "none"),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": S.sample_desc},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_of(W, l2):
+    if W.kind == "gemm":
+        c = {"workload": W.name, "M": W.M, "K": W.K, "N": W.N}
+    else:
+        c = {"workload": W.name, "T": W.T, "E": W.E, "topk": W.topk, "H": W.H, "F": W.F, "routing": W.routing}
+    c.update({"weights": "int4 g128 asym (fp16 scale+zp)", "acts": "int8 per-token", "l2": l2,
+              "parallelism": "replicas (no cross-GPU exchange)"})
+    return c
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(synth.WORKLOADS), default="toy_moe")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--cpu-baseline-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    W = synth.WORKLOADS[args.workload]
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    if args.impl == "reference":
+        return run_reference(args, W)
+
+    import torch
+    from w4a8_quantized_moe_token_b200 import binding as B
+
+    world, rank, local = dist_env()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+
+    step = (GemmStep if W.kind == "gemm" else MoeStep)(B, torch, W, args.seed + rank * 0, device)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    sampler = ClockSampler(torch.cuda.current_device())
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    B.w4a8_profile_start()
+    step.start_route_timing()
+    sampler.start()
+    barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.zero_()
+        starts[i].record()
+        step()
+        ends[i].record()
+    torch.cuda.synchronize()
+    barrier()
+    sampler.stop()
+    step.stop_route_timing()
+    prof = B.w4a8_profile_stop()
+    assert B.w4a8_last_device_error(step.ws) == 0, "device error during the timed steps"
+    ms = sum(a.elapsed_time(b) for a, b in zip(starts, ends)) / args.steps
+    ms_t = torch.tensor([ms], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(ms_t, op=torch.distributed.ReduceOp.MAX)
+    ms_max = float(ms_t.item())
+
+    e2e_ms, h2d, d2h = step.e2e(args.steps, args.warmup)
+    e2e_t = torch.tensor([e2e_ms], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(e2e_t, op=torch.distributed.ReduceOp.MAX)
+    e2e_ms = float(e2e_t.item())
+
+    acct = step.acct
+    tokens = (W.T if W.kind == "moe" else W.M) * world
+    sec = ms_max / 1e3
+    peaks = load_peaks()
+    hbm = float(peaks["hbm_gbs"])
+    i8 = float(peaks["bf16_tflops"]) * INT8_OVER_BF16
+
+    # per-kernel table and the dominant kernel's roofline
+    kernels = {}
+    for kind, (n, tot) in prof.items():
+        if n:
+            kernels[kind] = {"launches": n, "ms_per_step": tot / args.steps}
+    if step.route_launches:
+        kernels["route"] = {"launches": step.route_launches, "ms_per_step": step.route_ms / args.steps}
+    dom = max(kernels, key=lambda k: kernels[k]["ms_per_step"])
+    per_launch_ms = kernels[dom]["ms_per_step"] * args.steps / kernels[dom]["launches"]
+    ops = acct["kernel_ops"].get(dom, 0.0)
+    byt = acct["kernel_bytes"].get(dom, 0.0)
+    ridge = i8 * 1e12 / (hbm * 1e9)
+    if ops and ops / max(byt, 1) > ridge:
+        roof = {"bound": "tensor", "achieved": ops / (per_launch_ms / 1e3) / 1e12, "peak": i8, "unit": "TFLOP/s"}
+    else:
+        roof = {"bound": "hbm", "achieved": byt / (per_launch_ms / 1e3) / 1e9, "peak": hbm, "unit": "GB/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = None
+    roof["kernel"] = dom
+    roof["peak_source"] = (f"{peaks['source']}: " + ("MEASURED_PEAKS hbm_gbs" if roof["bound"] == "hbm" else
+                           "bf16_tflops x 2 (nominal int8/bf16 ratio)"))
+    for kind, v in kernels.items():
+        kb = acct["kernel_bytes"].get(kind, 0.0)
+        ko = acct["kernel_ops"].get(kind, 0.0)
+        t = v["ms_per_step"] * args.steps / v["launches"] / 1e3
+        v["gbs"] = kb / t / 1e9 if t > 0 else None
+        if ko:
+            v["tops"] = ko / t / 1e12 if t > 0 else None
+
+    line = {
+        "metric": METRIC,
+        "value": tokens / sec,
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_max,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "int8",
+        "data": "synthetic",
+        "config": config_of(W, "flushed before every timed step (256 MiB write, outside the timed span)"),
+        "tops": acct["ops"] * world / sec / 1e12,
+        "weight_gbs": acct["weight_bytes"] * world / sec / 1e9,
+        "touched_experts": acct["touched_experts"],
+        "roofline": roof,
+        "kernels": kernels,
+        "gpu_launches": sum(v["launches"] for v in kernels.values()),
+        "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "clocks": sampler.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        S = OracleSample(W, args.seed, args.cpu_baseline_seconds)
+        t = S.timed()
+        line["cpu_baseline"] = {"value": S.tokens / t, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                                "sample": S.sample_desc}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

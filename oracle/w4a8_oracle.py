@@ -276,6 +276,23 @@ def combine(y2: np.ndarray, w: np.ndarray, inv: np.ndarray, T: int, k: int) -> n
     return out
 
 
+def round_to_bf16(x: np.ndarray) -> np.ndarray:
+    """Round fp64 values to the nearest bf16 (ties to even), returned as fp64.
+
+    [P1] §4.3 step 4: the result is converted back to 16-bit float (BF16) for the
+    layers that follow.  bf16 keeps 8 significant bits; the fp64 mantissa is cut to
+    its top 7 stored bits with round-half-to-even on the integer bit pattern, a
+    single correctly rounded step for every normal value (the layer's outputs are
+    far from the bf16 subnormal and overflow ranges).
+    """
+    b = np.ascontiguousarray(x, dtype=np.float64).view(np.uint64)
+    drop = np.uint64(52 - 7)
+    half = np.uint64(1) << (drop - np.uint64(1))
+    lsb = (b >> drop) & np.uint64(1)
+    r = (b + (half - np.uint64(1)) + lsb) & ~((np.uint64(1) << drop) - np.uint64(1))
+    return r.view(np.float64)
+
+
 # --------------------------------------------------------------------------- #
 # the whole layer
 # --------------------------------------------------------------------------- #
@@ -306,7 +323,8 @@ def expert_forward(xq, xs, qe: QuantExpert, F: int, stages: dict | None = None):
 
 
 def moe_forward(x, ids, w, experts: dict, E: int, F: int, stages: dict | None = None):
-    """Full W4A8 MoE expert FFN (fp64 result, [T][H]).
+    """Full W4A8 MoE expert FFN, [T][H]: the fp64 sum of a8 rounded to bf16
+    ([P1] §4.3 step 4), returned as fp64 values.
 
     x [T][H] float32 (bf16 values); ids [T][k]; w [T][k]; experts[e] = QuantExpert
     (only experts that receive tokens are needed).
@@ -325,14 +343,14 @@ def moe_forward(x, ids, w, experts: dict, E: int, F: int, stages: dict | None = 
         y2[offs[e]:offs[e + 1]] = expert_forward(xq[tok], xs[tok], experts[e], F, stages)[:, :H]
     if stages is not None:
         stages.update(counts=counts, offs=offs, perm=perm, inv=inv, xq=xq, xs=xs, y2=y2)
-    return combine(y2, w, inv, T, k)
+    return round_to_bf16(combine(y2, w, inv, T, k))
 
 
 def token_forward(t: int, x, ids, w, experts: dict, F: int) -> np.ndarray:
-    """The layer's output for one token only (used to sample large layers)."""
+    """The layer's output (bf16-rounded) for one token only (used to sample large layers)."""
     xq, xs = quantize_act(np.asarray(x, dtype=np.float32)[t:t + 1])
     out = 0.0
     for j in range(ids.shape[1]):
         y2 = expert_forward(xq, xs, experts[int(ids[t, j])], F)[0]
         out = out + float(w[t, j]) * y2
-    return out
+    return round_to_bf16(out)

@@ -141,7 +141,7 @@ def check_stages(L: Layer, out):
             y2_ref[sl] = O.w4a8_linear(qh[sl], sh[sl], *qe.down)
     assert_close(y2[rows], y2_ref, max_rel=1e-4, mae_rel=1e-5, what="y2")
     # a8: combine of the dumped y2
-    comb = O.combine(y2[rows].astype(np.float64), L.w, np.arange(T * k), T, k)
+    comb = O.round_to_bf16(O.combine(y2[rows].astype(np.float64), L.w, np.arange(T * k), T, k))
     assert_close(out, comb, max_rel=1e-2, mae_rel=1e-3, what="combine")
 
 

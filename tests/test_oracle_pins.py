@@ -347,7 +347,8 @@ def test_moe_forward_equals_per_token_dequantized_formulation():
             hh = (yu[:F] / (1 + np.exp(-yu[:F])) * yu[F:]).astype(np.float32)
             qh, sh = O.quantize_act(hh[None, :])
             acc += float(w[t, j]) * (wd @ (qh[0].astype(np.float64) * float(sh[0])))
-        np.testing.assert_allclose(out[t], acc, rtol=1e-9, atol=1e-12)
+        # the layer's output is rounded to bf16: within half a bf16 ulp of the fp64 value
+        assert np.all(np.abs(out[t] - acc) <= np.abs(acc) * 2.0 ** -8 + 1e-30)
         np.testing.assert_allclose(O.token_forward(t, x, ids, w, experts, F), out[t], rtol=1e-12, atol=1e-15)
 
 
@@ -369,3 +370,17 @@ def test_planted_mistakes_are_caught():
     good = O.w4a8_linear(qa, sa, codes, scale, zp, acc)
     bad = sa[:, None] * np.einsum("mng,mg->mn", acc.astype(np.float64), scale.astype(np.float64))
     assert np.abs(good - bad).max() > 1e-6
+
+
+def test_round_to_bf16_against_library_rounding():
+    # independent: torch's float32 -> bfloat16 conversion is round-half-to-even; on
+    # fp64 values that are exactly float32 the two single roundings must agree
+    import torch
+    rng = np.random.default_rng(8)
+    v = (rng.standard_normal(20000) * 10.0 ** rng.integers(-6, 6, 20000)).astype(np.float32).astype(np.float64)
+    ties = np.array([1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8, -(1.0 + 2.0 ** -8), 0.0, 3.0])  # exact midpoints
+    v = np.concatenate([v, ties])
+    ref = torch.from_numpy(v.astype(np.float32)).to(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(O.round_to_bf16(v), ref)
+    assert O.round_to_bf16(np.array([1.0 + 2.0 ** -8]))[0] == 1.0  # tie to even
+    assert O.round_to_bf16(np.array([1.0 + 3 * 2.0 ** -8]))[0] == 1.0 + 2.0 ** -6
