@@ -141,6 +141,29 @@ size_t w4a8_gemm_workspace_bytes(int M, int N, int K);
 int w4a8_gemm(const int8_t* qa, const float* sa, int M, const void* packed, int N, int K,
               float* y, int32_t* partials_opt, void* ws, size_t ws_bytes, void* stream);
 
+/* w4a8_gemm for callers that cannot allocate device memory.  (The pages describe
+ * no such variant: it exists for integration, not for the method.)
+ * Some callers cannot hand this library a workspace: a plugin inside a host
+ * framework that owns every device allocation and forbids new ones on its
+ * execution path, code running where a cudaMalloc would synchronise the device
+ * or is not allowed, a binding with no allocator at hand.  This entry point takes
+ * the same inputs and outputs as w4a8_gemm and uses instead a fixed 8 MiB device
+ * array inside the library (reserved on every GPU that loads the library, until
+ * the process exits).  It calls no cudaMalloc, cudaFree or other allocating
+ * routine.
+ *   - Limit: w4a8_gemm_workspace_bytes(M, N, K) must not exceed 8 MiB (about
+ *     8.3 million INT8 values of M x Kp, e.g. M = 1024 at K = 7168); larger
+ *     sizes return W4A8_ENOSPACE before anything is launched.
+ *   - The first call on a device looks up the array's device address (once per
+ *     device, with that device current); make that first call before any stream
+ *     capture.
+ *   - Every call, on every stream, shares the one array: calls whose work
+ *     overlaps on the GPU race with each other and give wrong results.  Each call
+ *     rewrites all of the scratch it reads, so nothing carries over between calls.
+ *   - The device error word lives in that array and is not readable by the caller. */
+int w4a8_gemm_noalloc(const int8_t* qa, const float* sa, int M, const void* packed, int N, int K,
+                      float* y, int32_t* partials_opt, void* stream);
+
 /* Intermediate results kept in a w4a8_moe_forward workspace, for stage tests. */
 enum {
     W4A8_DUMP_COUNTS = 0, /* int32 [E]      tokens routed to each expert             */

@@ -41,6 +41,7 @@ _SIGS = {
                                _vp], _c_int),
     "w4a8_gemm_workspace_bytes": ([_c_int] * 3, _c_size),
     "w4a8_gemm": ([_vp, _vp, _c_int, _vp, _c_int, _c_int, _vp, _vp, _vp, _c_size, _vp], _c_int),
+    "w4a8_gemm_noalloc": ([_vp, _vp, _c_int, _vp, _c_int, _c_int, _vp, _vp, _vp], _c_int),
     "w4a8_debug_region": ([_c_int] * 6 + [ctypes.POINTER(_c_size), ctypes.POINTER(_c_size)], _c_int),
     "w4a8_debug_dump": ([_vp] + [_c_int] * 6 + [_vp, _c_size, _vp], _c_int),
     "w4a8_last_device_error": ([_vp, _vp], _c_int),
@@ -186,6 +187,17 @@ def w4a8_gemm(qa, sa, packed, N, K, y, ws, partials=None):
     M = qa.shape[0]
     _check(lib().w4a8_gemm(_ptr(qa), _ptr(sa), M, _ptr(packed), N, K, _ptr(y), _ptr(partials), _ptr(ws), ws.numel(),
                            _stream()), "w4a8_gemm")
+
+
+def w4a8_gemm_noalloc(qa, sa, packed, N, K, y, partials=None):
+    """w4a8_gemm without a caller workspace: the library's own fixed scratch array
+    is used (for callers that cannot allocate; concurrent calls race)."""
+    _dev(qa, torch.int8, "qa")
+    _dev(sa, torch.float32, "sa")
+    _dev(y, torch.float32, "y")
+    M = qa.shape[0]
+    _check(lib().w4a8_gemm_noalloc(_ptr(qa), _ptr(sa), M, _ptr(packed), N, K, _ptr(y), _ptr(partials), _stream()),
+           "w4a8_gemm_noalloc")
 
 
 def w4a8_debug_region(T, E, k, H, F, what) -> tuple[int, int]:
