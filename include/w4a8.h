@@ -171,17 +171,22 @@ enum {
     W4A8_DUMP_PERM = 2,   /* int32 [T*k]    slot (t*k+j) at each grouped position     */
     W4A8_DUMP_INV = 3,    /* int32 [T*k]    padded row of each slot                   */
     W4A8_DUMP_POFFS = 4,  /* int32 [E+1]    row offsets with every expert padded to 16 */
-    W4A8_DUMP_ACT1 = 5,   /* int8 [Hp/128][R][128] INT8 x rows (tiled, see below)     */
+    W4A8_DUMP_ACT1 = 5,   /* int8, R x Hp: INT8 x rows (tiled, see below)             */
     W4A8_DUMP_S1 = 6,     /* float [R]      token scale of each padded row            */
     W4A8_DUMP_H = 7,      /* float [R][Fp]  SwiGLU output h (fp32) per padded row      */
-    W4A8_DUMP_ACT2 = 8,   /* int8 [Fp/128][R][128] requantised h (tiled)              */
+    W4A8_DUMP_ACT2 = 8,   /* int8, R x Fp: requantised h (tiled, see below)           */
     W4A8_DUMP_S2 = 9,     /* float [R]      scale of the requantised h rows           */
     W4A8_DUMP_Y2 = 10,    /* float [R][H]   down-projection output per padded row     */
     W4A8_DUMP_ERR = 11    /* uint32 [1]     device error word                         */
 };
-/* R = w4a8_moe_rows_capacity(T,E,k).  Tiled INT8 planes: plane g holds K columns
- * [128g, 128g+128); row r's 16-byte chunk c sits at r*128 + ((c ^ (r & 7)) * 16). */
+/* R = w4a8_moe_rows_capacity(T,E,k).  Tiled INT8 rows: rows are grouped in blocks of
+ * RB = w4a8_moe_act_block_rows(T,E,k) rows (16 for decode-shaped layers, whose mean
+ * tokens per expert is at most 16; otherwise RB = R); the buffer is
+ * [R/RB][Kp/128][RB][128 bytes]: block b, K group g, row i (= r % RB) starts at byte
+ * ((b * Kp/128 + g) * RB + i) * 128, and the row's 16-byte chunk c (K columns
+ * 128g + 16c .. +15) sits at chunk position c ^ (i & 7). */
 int w4a8_moe_rows_capacity(int T, int E, int k);
+int w4a8_moe_act_block_rows(int T, int E, int k);
 
 /* Byte offset and size of dump region `what` inside the workspace. */
 int w4a8_debug_region(int T, int E, int k, int H, int F, int what, size_t* offset, size_t* bytes);

@@ -87,14 +87,16 @@ def decode_packed(buf: np.ndarray, E: int, N: int, K: int, layout: int):
     return codes, scale, zp
 
 
-def untile_act(planes: np.ndarray, R: int, Kp: int) -> np.ndarray:
-    """Tiled INT8 planes [Kp/128][R][128] (16-byte chunk c of row r at c ^ (r & 7)) -> [R][Kp]."""
+def untile_act(buf: np.ndarray, R: int, Kp: int, RB: int | None = None) -> np.ndarray:
+    """Tiled INT8 rows [R/RB][Kp/128][RB][128] (16-byte chunk c of row i of a block at
+    chunk position c ^ (i & 7)) -> [R][Kp].  RB defaults to R (plain planes)."""
+    RB = R if RB is None else RB
     G = Kp // 128
-    p = np.asarray(planes).reshape(G, R, 8, 16)
-    r = np.arange(R)
+    p = np.asarray(buf).reshape(R // RB, G, RB, 8, 16)
     out = np.zeros((R, Kp), dtype=p.dtype)
+    i = np.arange(RB)
     for c in range(8):
-        phys = (c ^ (r & 7))
+        phys = c ^ (i & 7)
         for g in range(G):
-            out[:, g * 128 + c * 16:g * 128 + (c + 1) * 16] = p[g, r, phys]
+            out.reshape(R // RB, RB, Kp)[:, :, g * 128 + c * 16:g * 128 + (c + 1) * 16] = p[:, g, i, phys]
     return out

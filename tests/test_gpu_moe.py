@@ -110,7 +110,9 @@ def check_stages(L: Layer, out):
     assert np.array_equal(inv_d - poffs[flat] + offs[flat], inv)
     # a2: INT8 activations of the grouped rows, bit-exact
     xq, xs = O.quantize_act(L.x)
-    act1 = untile_act(L.dump("act1", np.int8), R, Hp)
+    RB = B.w4a8_moe_act_block_rows(T, E, k)
+    assert RB in (16, R)
+    act1 = untile_act(L.dump("act1", np.int8), R, Hp, RB)
     s1 = L.dump("s1", np.float32)
     rows = inv_d  # padded row of each slot
     tok = np.arange(T * k) // k
@@ -127,7 +129,7 @@ def check_stages(L: Layer, out):
             h_ref[sl] = O.swiglu(O.w4a8_linear(xq[t_e], xs[t_e], *qe.up), F)
     assert_close(h[rows, :F], h_ref, max_rel=1e-4, mae_rel=1e-5, what="h")
     # a6: requantisation of the dumped h, bit-exact
-    act2 = untile_act(L.dump("act2", np.int8), R, Fp)
+    act2 = untile_act(L.dump("act2", np.int8), R, Fp, RB)
     s2 = L.dump("s2", np.float32)
     qh, sh = O.quantize_act(h[rows, :F].astype(np.float32))
     assert np.array_equal(act2[rows], qh)

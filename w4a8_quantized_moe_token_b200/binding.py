@@ -35,6 +35,7 @@ _SIGS = {
     "w4a8_moe_workspace_bytes": ([_c_int] * 5, _c_size),
     "w4a8_moe_host_workspace_bytes": ([_c_int] * 5, _c_size),
     "w4a8_moe_rows_capacity": ([_c_int] * 3, _c_int),
+    "w4a8_moe_act_block_rows": ([_c_int] * 3, _c_int),
     "w4a8_moe_forward": ([_vp, _vp, _c_int, _c_int, _c_int, _vp, _c_int, _vp, _vp, _c_int, _vp, _vp, _c_size, _vp],
                          _c_int),
     "w4a8_moe_forward_host": ([_vp, _vp, _c_int, _c_int, _c_int, _vp, _c_int, _vp, _vp, _c_int, _vp, _vp, _c_size,
@@ -152,6 +153,10 @@ def w4a8_moe_host_workspace_bytes(T, E, k, H, F) -> int:
 
 def w4a8_moe_rows_capacity(T, E, k) -> int:
     return lib().w4a8_moe_rows_capacity(T, E, k)
+
+
+def w4a8_moe_act_block_rows(T, E, k) -> int:
+    return lib().w4a8_moe_act_block_rows(T, E, k)
 
 
 def w4a8_moe_forward(packed_up, packed_down, E, H, F, x, ids, w, out, ws):

@@ -45,8 +45,8 @@ int rows_capacity(int T, int E, int k) {
 
 // Workspace of w4a8_moe_forward: regions in the order of the enum below.
 enum Region {
-    R_ERR, R_CHIST, R_COUNTS, R_OFFS, R_POFFS, R_MTSTART, R_PERM, R_INV, R_ROWSRC,
-    R_ACT1, R_S1, R_AMAX, R_H, R_ACT2, R_S2, R_Y2,
+    R_ERR, R_CHIST, R_COUNTS, R_OFFS, R_POFFS, R_MTSTART, R_MTTAB, R_PERM, R_INV, R_ROWSRC,
+    R_ACT1, R_S1, R_H, R_ACT2, R_S2, R_Y2,
     R_XIN, R_IDSIN, R_WIN, R_OUT,  // host-buffer variant only
     R_COUNT
 };
@@ -75,12 +75,12 @@ bool moe_layout(int T, int E, int k, int H, int F, bool host_io, MoeLayout* L) {
     b[R_OFFS] = (size_t)(E + 1) * 4;
     b[R_POFFS] = (size_t)(E + 1) * 4;
     b[R_MTSTART] = (size_t)(E + 1) * 4;
+    b[R_MTTAB] = (size_t)mt_tab_capacity(L->nslots, E) * 16;
     b[R_PERM] = (size_t)L->nslots * 4;
     b[R_INV] = (size_t)L->nslots * 4;
     b[R_ROWSRC] = R * 4;
     b[R_ACT1] = (size_t)L->G1 * R * 128;
     b[R_S1] = R * 4;
-    b[R_AMAX] = R * 4;
     b[R_H] = R * (size_t)L->Fp * 4;
     b[R_ACT2] = (size_t)L->G2 * R * 128;
     b[R_S2] = R * 4;
@@ -169,25 +169,28 @@ int moe_forward_impl(const void* packed_up, const void* packed_down, int E, int 
     int* offs = at<int>(ws, L, R_OFFS);
     int* poffs = at<int>(ws, L, R_POFFS);
     int* mtstart = at<int>(ws, L, R_MTSTART);
+    int4* mt_tab = at<int4>(ws, L, R_MTTAB);
     int* row_src = at<int>(ws, L, R_ROWSRC);
     int* inv = at<int>(ws, L, R_INV);
     float* s1 = at<float>(ws, L, R_S1);
     float* s2 = at<float>(ws, L, R_S2);
-    uint32_t* amax = at<uint32_t>(ws, L, R_AMAX);
     float* h = at<float>(ws, L, R_H);
     float* y2 = at<float>(ws, L, R_Y2);
     int8_t* act1 = at<int8_t>(ws, L, R_ACT1);
     int8_t* act2 = at<int8_t>(ws, L, R_ACT2);
-    const size_t plane = (size_t)L.R * 128;
+    // tokens per GEMM tile from the mean tokens per expert (decode-like layers use the
+    // decode kernel with 16-token tiles and 16-row blocks of token rows)
+    const int tile = gemm_tile_tokens(L.nslots / E);
+    const int rb = act_block_rows(tile, L.R);
 
     {
         ProfScope p(W4A8_KERNEL_PERM, 3, st);
-        W4A8_TRY(launch_perm(ids, L.nslots, E, at<int>(ws, L, R_CHIST), L.nchunk, counts, offs, poffs, mtstart,
-                             at<int>(ws, L, R_PERM), inv, row_src, err, st));
+        W4A8_TRY(launch_perm(ids, L.nslots, E, tile, at<int>(ws, L, R_CHIST), L.nchunk, counts, offs, poffs, mtstart,
+                             mt_tab, at<int>(ws, L, R_PERM), inv, row_src, err, st));
     }
     {
         ProfScope p(W4A8_KERNEL_ACT_QUANT, 1, st);
-        W4A8_TRY(launch_act_scatter(x, H, k, row_src, poffs, E, L.R, act1, plane, s1, amax, st));
+        W4A8_TRY(launch_act_scatter(x, H, k, row_src, poffs, E, L.R, rb, act1, s1, st));
     }
 
     GemmArgs up{};
@@ -195,26 +198,24 @@ int moe_forward_impl(const void* packed_up, const void* packed_down, int E, int 
     up.NT = packed_tiles(2 * F, W4A8_LAYOUT_GATEUP);
     up.G = L.G1;
     up.act = act1;
-    up.act_plane = plane;
+    up.act_plane = (size_t)rb * 128;
+    up.act_rb_stride = (size_t)L.G1 * rb * 128;
     up.act_scale = s1;
-    up.counts = counts;
-    up.poffs = poffs;
-    up.mtstart = mtstart;
-    up.E = E;
+    up.mt_tab = mt_tab;
+    up.n_mtiles = mtstart + E;
     up.mode = 1;
     up.out = h;
     up.ldo = L.Fp;
     up.nvalid = F;
-    up.amax = amax;
     up.partials = nullptr;
     up.err = err;
     {
         ProfScope p(W4A8_KERNEL_GEMM_UP, 1, st);
-        W4A8_TRY(launch_gemm(up, sm_count(), st));
+        W4A8_TRY(launch_gemm(up, tile, sm_count(), st));
     }
     {
         ProfScope p(W4A8_KERNEL_REQUANT, 1, st);
-        W4A8_TRY(launch_requant(h, L.Fp, F, row_src, poffs, E, L.R, amax, act2, plane, s2, st));
+        W4A8_TRY(launch_requant(h, L.Fp, F, row_src, poffs, E, L.R, rb, act2, s2, st));
     }
 
     GemmArgs dn = up;
@@ -222,15 +223,15 @@ int moe_forward_impl(const void* packed_up, const void* packed_down, int E, int 
     dn.NT = packed_tiles(H, W4A8_LAYOUT_PLAIN);
     dn.G = L.G2;
     dn.act = act2;
+    dn.act_rb_stride = (size_t)L.G2 * rb * 128;
     dn.act_scale = s2;
     dn.mode = 2;
     dn.out = y2;
     dn.ldo = H;
     dn.nvalid = H;
-    dn.amax = nullptr;
     {
         ProfScope p(W4A8_KERNEL_GEMM_DOWN, 1, st);
-        W4A8_TRY(launch_gemm(dn, sm_count(), st));
+        W4A8_TRY(launch_gemm(dn, tile, sm_count(), st));
     }
     {
         ProfScope p(W4A8_KERNEL_COMBINE, 1, st);
@@ -318,6 +319,11 @@ W4A8_EXPORT int w4a8_route_topk(const void* logits_bf16, int T, int E, int k, in
 
 W4A8_EXPORT int w4a8_moe_rows_capacity(int T, int E, int k) { return rows_capacity(T, E, k); }
 
+W4A8_EXPORT int w4a8_moe_act_block_rows(int T, int E, int k) {
+    if (T < 0 || E < 1 || k < 1) return 0;
+    return act_block_rows(gemm_tile_tokens((int)((long long)T * k / E)), rows_capacity(T, E, k));
+}
+
 W4A8_EXPORT size_t w4a8_moe_workspace_bytes(int T, int E, int k, int H, int F) {
     MoeLayout L;
     if (!moe_layout(T, E, k, H, F, false, &L)) return 0;
@@ -371,7 +377,7 @@ W4A8_EXPORT int w4a8_moe_forward_host(const void* packed_up, const void* packed_
 namespace w4a8 {
 namespace {
 struct GemmLayout {
-    size_t err, counts, poffs, mtstart, act, total;
+    size_t err, nmt, mttab, act, total;
     int Mp, G;
 };
 bool gemm_layout(int M, int N, int K, GemmLayout* L) {
@@ -380,9 +386,8 @@ bool gemm_layout(int M, int N, int K, GemmLayout* L) {
     L->G = ceil_div(K, kGroup);
     size_t o = 0;
     L->err = o; o += align_up(16);
-    L->counts = o; o += align_up(4);
-    L->poffs = o; o += align_up(8);
-    L->mtstart = o; o += align_up(8);
+    L->nmt = o; o += align_up(4);
+    L->mttab = o; o += align_up((size_t)(M / 32 + 2) * 16);
     L->act = o; o += align_up((size_t)L->G * L->Mp * 128);
     L->total = o;
     return true;
@@ -411,32 +416,30 @@ W4A8_EXPORT int w4a8_gemm(const int8_t* qa, const float* sa, int M, const void* 
     if (qa == nullptr || sa == nullptr || y == nullptr) return W4A8_EINVAL;
     if (!aligned(qa, 16) || !aligned(sa, 4) || !aligned(y, 4) || (partials_opt && !aligned(partials_opt, 4)))
         return W4A8_EALIGN;
-    int* counts = reinterpret_cast<int*>(base + L.counts);
-    int* poffs = reinterpret_cast<int*>(base + L.poffs);
-    int* mtstart = reinterpret_cast<int*>(base + L.mtstart);
+    int* n_mtiles = reinterpret_cast<int*>(base + L.nmt);
+    int4* mt_tab = reinterpret_cast<int4*>(base + L.mttab);
     int8_t* act = reinterpret_cast<int8_t*>(base + L.act);
-    const size_t plane = (size_t)L.Mp * 128;
     ProfScope prof(W4A8_KERNEL_GEMM_DENSE, 2, s);
-    W4A8_TRY(launch_dense_prep(qa, M, L.G * kGroup, act, plane, counts, poffs, mtstart, s));
+    const int tile = gemm_tile_tokens(M);
+    const int rb = act_block_rows(tile, L.Mp);
+    W4A8_TRY(launch_dense_prep(qa, M, L.G * kGroup, tile, rb, act, mt_tab, n_mtiles, s));
     GemmArgs a{};
     a.wblocks = static_cast<const uint8_t*>(packed) + kHeaderBytes;
     a.NT = packed_tiles(N, W4A8_LAYOUT_PLAIN);
     a.G = L.G;
     a.act = act;
-    a.act_plane = plane;
+    a.act_plane = (size_t)rb * 128;
+    a.act_rb_stride = (size_t)L.G * rb * 128;
     a.act_scale = sa;
-    a.counts = counts;
-    a.poffs = poffs;
-    a.mtstart = mtstart;
-    a.E = 1;
+    a.mt_tab = mt_tab;
+    a.n_mtiles = n_mtiles;
     a.mode = 0;
     a.out = y;
     a.ldo = N;
     a.nvalid = N;
-    a.amax = nullptr;
     a.partials = partials_opt;
     a.err = err;
-    W4A8_TRY(launch_gemm(a, sm_count(), s));
+    W4A8_TRY(launch_gemm(a, tile, sm_count(), s));
     return W4A8_OK;
 }
 

@@ -1,0 +1,458 @@
+// Grouped W4A8 GEMM for decode-shaped layers (at most 16 tokens per tile), sm_100a.
+//
+// Same method as gemm_w4a8.cu (INT4 group-128 weights x per-token INT8 tokens on
+// tcgen05 kind::i8 MMAs, one exact INT32 partial per 128-wide K group, scales folded
+// in fp32): «Kimi 2.7 Moe 从 4 bit 存储到 INT8 拆解» (pptc.cn) sections 2.1 and 3.2,
+// the Kimi 2.7T MoE W4A8 article (hotelren.com 5173946) section 4.3.
+//
+// Decode streams every touched expert's weights once for a handful of tokens, so the
+// kernel must run at HBM speed.  Every synchronisation between the roles (mbarrier
+// wait / arrive, tcgen05 commit, tensor-memory store + wait) costs a few hundred
+// cycles, which is as long as one 8.7 KB weight block takes to arrive at full
+// bandwidth; so one pipeline step here carries GPS = 4 consecutive K groups of a tile
+// (35 KB of weights, 16 MMAs), paying the synchronisation once per 4 groups.
+//
+// Roles (one persistent CTA per SM, 16 warps):
+//   2 producer warps   : (alternate steps) one 1-D bulk copy of the step's weight blocks
+//                        (contiguous in the packed layout) and one of its token rows
+//                        (contiguous in the 16-row-block activation layout);
+//   2 converter groups : (alternate steps) each thread expands one weight row's codes
+//                        to unsigned INT8 (raw 4-bit codes 0..15: a mask and a
+//                        multiply-high per 8 codes), stores them to a tensor-memory A
+//                        slot, publishes the row's scale and zero point, and sums each
+//                        token's 128 INT8 codes per group (S, with dp4a);
+//   2 MMA warps        : (alternate steps) per group 4 x tcgen05.mma.kind::i8 u8 x s8,
+//                        M=128 weight rows, N=16 tokens, K=32, into the group's own
+//                        INT32 accumulator (preloaded with 1.5 * 2^23, see below);
+//   1 epilogue group   : reads the partials, removes the zero point exactly
+//                        (P = sum a*c - zp * S), acc += scale * P in fp32 (packed
+//                        fp32x2), then applies the token scale and stores.
+// The accumulators start at the bit pattern 0x4B400000 (1.5 * 2^23): the MMAs add
+// the partial (|P| < 2^22), so the bits read back as fp32 are exactly 1.5 * 2^23 + P,
+// and one packed fp32 subtraction yields P without an int -> float conversion.
+#include "w4a8_common.cuh"
+#include "w4a8_internal.h"
+
+namespace w4a8 {
+
+namespace {
+
+constexpr uint32_t kMagicBits = 0x4B400000u;  // 1.5 * 2^23
+constexpr float kMagicF = 12582912.0f;
+constexpr long long kWaitLimitCycles = 4000000000ll;  // ~2 s: a bounded wait
+
+constexpr int GPS = 4;    // K groups per pipeline step
+constexpr int BN = 16;    // tokens per tile (one 16-row block)
+constexpr int NS = 4;     // shared-memory stages
+constexpr int NA = 2;     // tensor-memory A slots (GPS x 32 columns each)
+constexpr int ND = 4;     // tensor-memory accumulators (GPS x BN columns each)
+constexpr int NSC = 8;    // side-information ring slots (>= NA + ND)
+constexpr int kAStage = GPS * kBlockBytes;  // weight blocks of one step
+constexpr int kBStage = GPS * BN * 128;     // token rows of one step
+constexpr int kACols = GPS * 32;
+constexpr int kDCols = GPS * BN;
+constexpr uint32_t kACol0 = 0;
+constexpr uint32_t kDCol0 = NA * kACols;
+constexpr uint32_t kTmemCols = 512;
+static_assert(kDCol0 + ND * kDCols <= kTmemCols, "tensor memory over-subscribed");
+static_assert(NSC >= NA + ND, "side-information ring too small");
+static_assert(NS % 2 == 0, "the two producers own the stages of one parity each");
+
+// warps: 0-7 converters (2 groups), 8-11 epilogue, 12 producer 0, 13-14 MMA, 15 producer 1
+constexpr int kThreads = 512;
+constexpr int kEpiWarp0 = 8, kCtrlWarp0 = 12;
+constexpr int kRegLaunch = 128;  // 65536 / 512
+constexpr int kRegConv = 96, kRegCtrl = 48, kRegEpi = 200;
+static_assert(128 * (2 * kRegConv + kRegCtrl + kRegEpi) <= kRegLaunch * kThreads, "register split");
+
+// shared memory carve-up (offsets from a 1024-aligned base)
+constexpr int kOffB = 0;
+constexpr int kOffA = kOffB + NS * kBStage;
+constexpr int kOffSc = kOffA + NS * kAStage;      // ring: fp32 scale   [NSC][GPS][128]
+constexpr int kOffZp = kOffSc + NSC * GPS * 128 * 4;  // ring: zero point  [NSC][GPS][128]
+constexpr int kOffS = kOffZp + NSC * GPS * 128 * 4;   // ring: group sums  [NSC][GPS][BN]
+constexpr int kOffBar = kOffS + NSC * GPS * BN * 4;
+// full[NS] empty[NS] conv[NA] aempty[NA] dfull[ND] dempty[ND] side[NSC] final[2]
+constexpr int kNumBars = 2 * NS + 2 * NA + 2 * ND + NSC + 2;
+constexpr int kOffMisc = kOffBar + kNumBars * 8;
+constexpr int kSmemBytes = kOffMisc + 16 + 1024;
+static_assert(kSmemBytes <= 227 * 1024, "shared memory over-subscribed");
+
+#define FULL_BAR(s) (bar0 + 8u * (uint32_t)(s))
+#define EMPTY_BAR(s) (bar0 + 8u * (uint32_t)(NS + (s)))
+#define CONV_BAR(x) (bar0 + 8u * (uint32_t)(2 * NS + (x)))
+#define AEMPTY_BAR(x) (bar0 + 8u * (uint32_t)(2 * NS + NA + (x)))
+#define DFULL_BAR(b) (bar0 + 8u * (uint32_t)(2 * NS + 2 * NA + (b)))
+#define DEMPTY_BAR(b) (bar0 + 8u * (uint32_t)(2 * NS + 2 * NA + ND + (b)))
+#define SIDE_BAR(i) (bar0 + 8u * (uint32_t)(2 * NS + 2 * NA + 2 * ND + (i)))
+#define FINAL_BAR(m) (bar0 + 8u * (uint32_t)(2 * NS + 2 * NA + 2 * ND + NSC + (m)))
+
+struct Item {
+    int e, nt, row0, nrows;
+};
+
+__device__ __forceinline__ Item decode_item(int u, const GemmArgs& a) {
+    const int mt = u / a.NT;
+    const int4 t = __ldg(a.mt_tab + mt);
+    return Item{t.x, u - mt * a.NT, t.y, t.z};
+}
+
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag, uint32_t* err) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    for (uint32_t n = 1;; ++n) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((n & 15u) == 0) {
+            if (*abort_flag) return false;
+            if (clock64() - t0 > kWaitLimitCycles) {
+                *abort_flag = 1;
+                atomicOr(err, kErrTimeout);
+                return false;
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint32_t* err) {
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity)) {
+        if (clock64() - t0 > kWaitLimitCycles) {
+            atomicOr(err, kErrTimeout);
+            return;
+        }
+    }
+}
+
+__device__ __forceinline__ void tmem_st16_const(uint32_t taddr, uint32_t v) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1};" ::"r"(taddr),
+        "r"(v)
+        : "memory");
+}
+
+// (a0, a1) += s * ((x0, x1) - 1.5*2^23 - zp * (S0, S1)), packed fp32x2.  With x the
+// bits of 1.5*2^23 + P_raw, the subtraction and the zero-point term are exact (all
+// values are integers below 2^24), so the fold sees the exact INT32 partial.
+__device__ __forceinline__ void fold2_zp(float& a0, float& a1, float s, float nzp, uint32_t x0, uint32_t x1, float s0,
+                                         float s1) {
+    asm("{\n\t.reg .b64 a, x, m, sc, z, sg;\n\t"
+        "mov.b64 a, {%0, %1};\n\t"
+        "mov.b64 x, {%2, %3};\n\t"
+        "mov.b64 m, {%4, %4};\n\t"
+        "mov.b64 sc, {%5, %5};\n\t"
+        "mov.b64 z, {%6, %6};\n\t"
+        "mov.b64 sg, {%7, %8};\n\t"
+        "sub.rn.f32x2 x, x, m;\n\t"
+        "fma.rn.f32x2 x, z, sg, x;\n\t"
+        "fma.rn.f32x2 a, sc, x, a;\n\t"
+        "mov.b64 {%0, %1}, a;\n\t}"
+        : "+f"(a0), "+f"(a1)
+        : "r"(x0), "r"(x1), "f"(kMagicF), "f"(s), "f"(nzp), "f"(s0), "f"(s1));
+}
+
+__device__ __forceinline__ float silu_mul(float g, float u) { return __fdividef(g, 1.0f + __expf(-g)) * u; }
+
+__global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_addr = smem_u32(smem_raw);
+    const uint32_t base_addr = (raw_addr + 1023u) & ~1023u;
+    uint8_t* smem = smem_raw + (base_addr - raw_addr);
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    const uint8_t* smA = smem + kOffA;
+    const uint8_t* smB = smem + kOffB;
+    float* sc_ring = reinterpret_cast<float*>(smem + kOffSc);
+    float* zp_ring = reinterpret_cast<float*>(smem + kOffZp);
+    float* s_ring = reinterpret_cast<float*>(smem + kOffS);
+    const uint32_t sA = base_addr + kOffA, sB = base_addr + kOffB;
+    const uint32_t bar0 = base_addr + kOffBar;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(FULL_BAR(s), 1);
+            mbar_init(EMPTY_BAR(s), 1);
+        }
+        for (int x = 0; x < NA; ++x) {
+            mbar_init(CONV_BAR(x), 4);
+            mbar_init(AEMPTY_BAR(x), 1);
+        }
+        for (int b = 0; b < ND; ++b) {
+            mbar_init(DFULL_BAR(b), 1);
+            mbar_init(DEMPTY_BAR(b), 4);
+        }
+        for (int i = 0; i < NSC; ++i) mbar_init(SIDE_BAR(i), 4);
+        mbar_init(FINAL_BAR(0), 1);
+        mbar_init(FINAL_BAR(1), 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == kCtrlWarp0 + 1) {
+        tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const int q = warp & 3;
+    const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+    const bool is_epi = warp >= kEpiWarp0 && warp < kCtrlWarp0;
+    if (is_epi) {
+        for (int c = 0; c < ND * kDCols / 16; ++c) tmem_st16_const(tmem_base + lane_base + kDCol0 + c * 16, kMagicBits);
+        tmem_st_wait();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    const int total = a.NT * __ldg(a.n_mtiles);
+    const int G = a.G;
+    const int steps_per_item = (G + GPS - 1) / GPS;
+
+    if (warp >= kCtrlWarp0) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegCtrl));
+        const int cw = warp - kCtrlWarp0;  // 0: producer 0, 1-2: MMA, 3: producer 1
+        if (cw == 0 || cw == 3) {
+            // ---------------- producers ----------------
+            const int pi = cw == 0 ? 0 : 1;
+            if (lane == 0) {
+                uint32_t j = 0, last = 0;
+                bool ok = true;
+                for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
+                    const Item it = decode_item(u, a);
+                    const uint8_t* wsrc = a.wblocks + (size_t)(it.e * a.NT + it.nt) * G * kBlockBytes;
+                    const int8_t* bsrc = a.act + (size_t)(it.row0 / BN) * a.act_rb_stride;
+                    for (int t = 0; t < steps_per_item; ++t, ++j) {
+                        if ((int)(j & 1u) != pi) continue;
+                        last = j + 1;
+                        const int g0 = t * GPS, ng = min(GPS, G - g0);
+                        const int s = j % NS;
+                        if (!wait_bar(EMPTY_BAR(s), ((j / NS) & 1u) ^ 1u, abort_flag, a.err)) { ok = false; break; }
+                        mbar_arrive_expect_tx(FULL_BAR(s), (uint32_t)ng * (kBlockBytes + BN * 128));
+                        bulk_g2s(sA + s * kAStage, wsrc + (size_t)g0 * kBlockBytes, ng * kBlockBytes, FULL_BAR(s));
+                        bulk_g2s(sB + s * kBStage, bsrc + (size_t)g0 * BN * 128, ng * BN * 128, FULL_BAR(s));
+                    }
+                }
+                for (uint32_t qq = (last > (uint32_t)NS ? last - NS : 0u); qq < last; ++qq)
+                    if ((int)(qq & 1u) == pi) drain_wait(FULL_BAR(qq % NS), (qq / NS) & 1u, a.err);
+            }
+            __syncwarp();
+        } else {
+            // ---------------- MMA issuers ----------------
+            const int mi = cw - 1;
+            if (lane == 0) {
+                uint32_t j = 0;
+                bool ok = true;
+                const uint32_t idesc = idesc_i8(128, BN, false);
+                for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
+                    for (int t = 0; t < steps_per_item; ++t, ++j) {
+                        if ((int)(j & 1u) != mi) continue;
+                        const int ng = min(GPS, G - t * GPS);
+                        const int s = j % NS, x = j % NA, b = j % ND;
+                        if (!wait_bar(CONV_BAR(x), (j / NA) & 1u, abort_flag, a.err)) { ok = false; break; }
+                        if (!wait_bar(DEMPTY_BAR(b), ((j / ND) & 1u) ^ 1u, abort_flag, a.err)) { ok = false; break; }
+                        tc_fence_after();
+                        for (int gq = 0; gq < ng; ++gq) {
+                            const uint32_t dt = tmem_base + kDCol0 + (uint32_t)(b * kDCols + gq * BN);
+                            const uint32_t at = tmem_base + kACol0 + (uint32_t)(x * kACols + gq * 32);
+                            const uint32_t sb = sB + s * kBStage + gq * BN * 128;
+#pragma unroll
+                            for (int kk = 0; kk < 4; ++kk)
+                                mma_i8_ts(dt, at + kk * 8, smem_desc_sw128(sb + kk * 32), idesc, 1u);
+                        }
+                        tc_commit(EMPTY_BAR(s));
+                        tc_commit(AEMPTY_BAR(x));
+                        tc_commit(DFULL_BAR(b));
+                    }
+                }
+                tc_commit(FINAL_BAR(mi));
+                drain_wait(FINAL_BAR(mi), 0, a.err);
+            }
+            __syncwarp();
+        }
+    } else if (warp < kEpiWarp0) {
+        // ---------------- converters ----------------
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegConv));
+        const int cg = warp >> 2;
+        const int r = threadIdx.x & 127;
+        // group sums: this thread adds half (64 bytes) of token m's row in group gs
+        const int gs = r >> 5, m = (r & 31) >> 1, half = r & 1;
+        uint32_t m28;
+        asm volatile("mov.u32 %0, 0x10000000;" : "=r"(m28));  // x * 2^28 >> 32 = x >> 4, on the FMA pipe
+        const int nsteps = ((total - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x) * steps_per_item;
+        for (int j = cg; j < nsteps; j += 2) {
+            const int t = j % steps_per_item;
+            const int ng = min(GPS, G - t * GPS);
+            const int s = j % NS, x = j % NA, slot = j % NSC;
+            if (!wait_bar(FULL_BAR(s), (j / NS) & 1u, abort_flag, a.err)) break;
+            if (!wait_bar(AEMPTY_BAR(x), ((j / NA) & 1u) ^ 1u, abort_flag, a.err)) break;
+            for (int gq = 0; gq < ng; ++gq) {
+                const uint8_t* blk = smA + s * kAStage + gq * kBlockBytes;
+                uint4 w[4];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) w[c] = *reinterpret_cast<const uint4*>(blk + code_chunk_offset(r, c));
+                sc_ring[(slot * GPS + gq) * 128 + r] = __half2float(reinterpret_cast<const __half*>(blk + kScaleOff)[r]);
+                zp_ring[(slot * GPS + gq) * 128 + r] = __half2float(reinterpret_cast<const __half*>(blk + kZpOff)[r]);
+                uint32_t v[32];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const uint32_t xw[4] = {w[c].x, w[c].y, w[c].z, w[c].w};
+#pragma unroll
+                    for (int qq = 0; qq < 4; ++qq) {
+                        const int i = 4 * c + qq;  // word i holds K = 8i .. 8i+7 of the group
+                        v[2 * i] = xw[qq] & 0x0F0F0F0Fu;
+                        v[2 * i + 1] = __umulhi(xw[qq], m28) & 0x0F0F0F0Fu;
+                    }
+                }
+                tmem_st32(tmem_base + lane_base + kACol0 + (uint32_t)(x * kACols + gq * 32), v);
+            }
+            if (gs < ng) {
+                // S[gs][m] = sum of token m's 128 INT8 codes of group gs (the swizzle only
+                // permutes the 16-byte chunks inside the row, so the row sum is unaffected)
+                const uint4* rowp = reinterpret_cast<const uint4*>(smB + s * kBStage + gs * BN * 128 + m * 128 + half * 64);
+                int sum = 0;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const uint4 b4 = rowp[c];
+                    sum = __dp4a((int)b4.x, 0x01010101, sum);
+                    sum = __dp4a((int)b4.y, 0x01010101, sum);
+                    sum = __dp4a((int)b4.z, 0x01010101, sum);
+                    sum = __dp4a((int)b4.w, 0x01010101, sum);
+                }
+                sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+                if (half == 0) s_ring[(slot * GPS + gs) * BN + m] = (float)sum;
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(CONV_BAR(x));
+                mbar_arrive(SIDE_BAR(slot));
+            }
+        }
+    } else {
+        // ---------------- epilogue ----------------
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegEpi));
+        const int r = q * 32 + lane;
+        uint32_t j = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
+            const Item it = decode_item(u, a);
+            float acc[BN];
+#pragma unroll
+            for (int i = 0; i < BN; ++i) acc[i] = 0.f;
+            const int n_out = (a.mode == 1) ? -1 : it.nt * kTileRows + r;
+            for (int t = 0; t < steps_per_item; ++t, ++j) {
+                const int ng = min(GPS, G - t * GPS);
+                const int b = j % ND, slot = j % NSC;
+                if (!wait_bar(DFULL_BAR(b), (j / ND) & 1u, abort_flag, a.err)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t taddr = tmem_base + lane_base + kDCol0 + (uint32_t)(b * kDCols);
+                uint32_t v[GPS][BN];
+#pragma unroll
+                for (int gq = 0; gq < GPS; ++gq)
+                    if (gq < ng) tmem_ld16(taddr + gq * BN, v[gq]);
+                tmem_ld_wait();
+#pragma unroll
+                for (int gq = 0; gq < GPS; ++gq)
+                    if (gq < ng) tmem_st16_const(taddr + gq * BN, kMagicBits);
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(DEMPTY_BAR(b));
+                if (!wait_bar(SIDE_BAR(slot), (j / NSC) & 1u, abort_flag, a.err)) { ok = false; break; }
+#pragma unroll
+                for (int gq = 0; gq < GPS; ++gq) {
+                    if (gq < ng) {
+                        const float sc = sc_ring[(slot * GPS + gq) * 128 + r];
+                        const float zpf = zp_ring[(slot * GPS + gq) * 128 + r];
+                        const float4* sp = reinterpret_cast<const float4*>(s_ring + (slot * GPS + gq) * BN);
+                        float sg[BN];
+#pragma unroll
+                        for (int i = 0; i < BN / 4; ++i) {
+                            const float4 f4 = sp[i];
+                            sg[4 * i] = f4.x; sg[4 * i + 1] = f4.y; sg[4 * i + 2] = f4.z; sg[4 * i + 3] = f4.w;
+                        }
+                        if (a.partials != nullptr && n_out < a.nvalid) {
+                            int32_t* pp = a.partials + ((size_t)it.row0 * a.nvalid + n_out) * G + t * GPS + gq;
+                            const size_t pstride = (size_t)a.nvalid * G;
+#pragma unroll
+                            for (int i = 0; i < BN; ++i)
+                                if (i < it.nrows)
+                                    pp[i * pstride] = (int32_t)(v[gq][i] - kMagicBits) - (int32_t)zpf * (int32_t)sg[i];
+                        }
+#pragma unroll
+                        for (int i = 0; i < BN; i += 2)
+                            fold2_zp(acc[i], acc[i + 1], sc, -zpf, v[gq][i], v[gq][i + 1], sg[i], sg[i + 1]);
+                    }
+                }
+            }
+            if (!ok) break;
+            const float* sap = a.act_scale + it.row0;
+            if (a.mode != 1) {
+                if (n_out < a.nvalid) {
+                    float* op = a.out + (size_t)it.row0 * a.ldo + n_out;
+#pragma unroll
+                    for (int i = 0; i < BN; ++i)
+                        if (i < it.nrows) op[(size_t)i * a.ldo] = acc[i] * __ldg(sap + i);
+                }
+            } else {
+                // SwiGLU: even tile rows hold gate channel f, odd rows the matching up channel
+                const int f = it.nt * (kTileRows / 2) + (r >> 1);
+                const bool valid = ((r & 1) == 0) && f < a.nvalid;
+                float* op = a.out + (size_t)it.row0 * a.ldo + f;
+#pragma unroll
+                for (int i = 0; i < BN; ++i) {
+                    if (i < it.nrows) {
+                        const float y = acc[i] * __ldg(sap + i);
+                        const float yo = __shfl_xor_sync(0xffffffffu, y, 1);
+                        if (valid) op[(size_t)i * a.ldo] = silu_mul(y, yo);
+                    }
+                }
+            }
+        }
+    }
+
+    __syncthreads();
+    if (warp == kCtrlWarp0 + 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, kTmemCols);
+    }
+}
+
+#undef FULL_BAR
+#undef EMPTY_BAR
+#undef CONV_BAR
+#undef AEMPTY_BAR
+#undef DFULL_BAR
+#undef DEMPTY_BAR
+#undef SIDE_BAR
+#undef FINAL_BAR
+
+}  // namespace
+
+int gemm_decode_tile_tokens() { return BN; }
+
+cudaError_t launch_gemm_decode(const GemmArgs& a, int num_ctas, cudaStream_t stream) {
+    static int attr_done[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64 || !attr_done[dev]) {
+        // the register split assumes kRegLaunch registers per thread at launch
+        cudaFuncAttributes fa;
+        cudaError_t e = cudaFuncGetAttributes(&fa, gemm_decode_kernel);
+        if (e != cudaSuccess) return e;
+        if (fa.numRegs != kRegLaunch) return cudaErrorInvalidConfiguration;
+        e = cudaFuncSetAttribute(gemm_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+        if (e != cudaSuccess) return e;
+        if (dev >= 0 && dev < 64) attr_done[dev] = 1;
+    }
+    gemm_decode_kernel<<<num_ctas, kThreads, kSmemBytes, stream>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace w4a8

@@ -5,26 +5,38 @@
 // -- the INT4 weights are expanded to INT8, multiplied with INT8 activations,
 // accumulated in INT32, then scaled back to floating point; section 2.1 -- one scale
 // and zero point per 128 weights; the Kimi 2.7T MoE W4A8 article (hotelren.com
-// 5173946) section 4.3 -- the 4-bit -> INT8 expansion and the requantisation are
-// fused into the kernel instead of going through memory.
+// 5173946) section 4.3 -- the 4-bit -> INT8 expansion is fused into the kernel
+// instead of going through memory.
 //
-// Design (one persistent CTA per SM, warp-specialised, 320 threads):
-//   warp 8   producer : 1-D bulk copies of one packed weight block (8192 B of
-//                       nibbles + fp16 scales + fp16 zero points for 128 output
-//                       channels x 128 K) and of the matching rows of the tiled INT8
-//                       token planes into an 8-stage shared-memory ring;
-//   warps 0-3 converter: each thread owns one weight row, expands its 128 nibbles to
-//                       signed INT8 (code - zp) in registers and writes them to a
-//                       tensor-memory A slot with tcgen05.st (the expanded weights never
-//                       touch shared memory);
-//   warp 9   MMA       : 4 x tcgen05.mma.kind::i8 (M=128 channels, N=tokens, K=32)
-//                       per group into a fresh INT32 accumulator (double-buffered);
-//   warps 4-7 epilogue : tcgen05.ld of the group's INT32 partials, acc += scale[n,g] *
-//                       partial in fp32 registers; after the last group the token
-//                       scale is applied and the tile is written (plain, or with
-//                       SwiGLU + per-row amax for the requantisation that follows).
-// Weights take the MMA's M slot ("swap AB"): tokens per expert are few in decode,
-// output channels are many, so M=128 is always full and N = tokens rounded to 16.
+// One persistent CTA per SM, warp-specialised.  A "step" is one 128-wide K group of
+// one tile (128 output channels x up to BN tokens); steps are numbered j = 0, 1, ...
+// over all the tiles a CTA processes, and every role walks the same sequence.
+//   2 producer warps    : (alternate steps) 1-D bulk copies of the step's packed weight block (8192 B
+//                         of nibbles + fp16 scales + fp16 zero points) and of its run
+//                         of tiled INT8 token rows into an NS-stage shared-memory ring;
+//   converter groups    : (4 warps each, alternate steps) each thread owns one weight
+//                         row, expands its 128 nibbles to signed INT8 (code - zp) in
+//                         registers and stores them to one of NA tensor-memory A slots
+//                         with tcgen05.st; it also publishes the row's fp32 scale in a
+//                         ring for the epilogue;
+//   2 MMA warps         : (alternate steps; the issue rate of tcgen05.mma is a
+//                         per-thread limit, two issuers double it) 4 x
+//                         tcgen05.mma.kind::i8 per step (M=128 channels, N=tokens,
+//                         K=32, A in tensor memory, B in shared memory) into one of ND
+//                         INT32 accumulators;
+//   epilogue warpgroups : tcgen05.ld of a step's partials and acc += scale[n,g] *
+//                         partial in fp32 registers; after the tile's last step the
+//                         token scale is applied and the tile stored (plain, or
+//                         SwiGLU on gate/up lane pairs).
+// Weights take the MMA's M slot ("swap AB"): decode has few tokens per expert and
+// many channels, so M=128 is always full and N shrinks to the tokens.
+//
+// This kernel serves layers with many tokens per expert (tiles of up to 128 tokens);
+// decode-shaped layers use gemm_decode.cu.  Every accumulator holds 0x4B400000 (the
+// fp32 bit pattern of 1.5 * 2^23) before its step's MMAs, which add the INT32 partial
+// P (|P| < 2^22) on top, so the result read as fp32 is exactly 1.5 * 2^23 + P and the
+// epilogue recovers P with one packed fp32 subtraction instead of an int -> float
+// conversion, then writes the constant back.
 #include "w4a8_common.cuh"
 #include "w4a8_internal.h"
 
@@ -32,65 +44,148 @@ namespace w4a8 {
 
 namespace {
 
-constexpr int kStages = 8;
-constexpr int kBStageBytes = kBN * 128;  // 16 KB of token rows per stage
-constexpr int kThreads = 320;
-constexpr int kEpiWarp0 = 4, kProdWarp = 8, kMmaWarp = 9;
-constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kDCol0 = 0;          // two INT32 accumulators of kBN columns
-constexpr uint32_t kACol0 = 2 * kBN;    // kStages A slots of 32 columns (128 x 128 int8)
-static_assert(kACol0 + kStages * 32 <= kTmemCols, "tensor memory over-subscribed");
-
-constexpr int kOffB = 0;
-constexpr int kOffA = kOffB + kStages * kBStageBytes;
-constexpr int kOffRed = kOffA + kStages * kBlockBytes;
-constexpr int kOffBar = kOffRed + 4 * kBN * 4;
-constexpr int kNumBars = 3 * kStages + 2 * 2 + 1;
-constexpr int kOffMisc = kOffBar + kNumBars * 8;
-constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
+constexpr uint32_t kMagicBits = 0x4B400000u;  // 1.5 * 2^23
+constexpr float kMagicF = 12582912.0f;
 
 constexpr long long kWaitLimitCycles = 4000000000ll;  // ~2 s: a bounded wait
+#ifndef W4A8_BACKOFF
+#define W4A8_BACKOFF() ((void)0)
+#endif
+
+// Compile-time shape of one kernel instance.
+//   BN    : tokens per tile at most (MMA N <= BN)
+//   NS    : shared-memory stages        NA : tensor-memory A slots
+//   ND    : INT32 accumulators          NEPI: epilogue warpgroups (split the columns)
+//   MAGIC : accumulator pre-load (see above)
+//   NCG   : converter warpgroups (they take alternate steps)
+template <int BN_, int NS_, int NA_, int ND_, int NEPI_, bool MAGIC_, int NCG_>
+struct Cfg {
+    static constexpr int BN = BN_, NS = NS_, NA = NA_, ND = ND_, NEPI = NEPI_, NCG = NCG_;
+    static constexpr bool kMagic = MAGIC_;
+    static constexpr int kNSC = 32;       // scale ring slots (>= NA + ND)
+    static constexpr int kCW = BN / NEPI;  // accumulator columns per epilogue thread
+    // warpgroups: NCG converter groups, NEPI epilogue groups, 1 control group
+    // (producer warp, two MMA warps, second producer warp)
+    static constexpr int kConvWarps = 4 * NCG;
+    static constexpr int kEpiWarp0 = kConvWarps;
+    static constexpr int kProdWarp = kEpiWarp0 + 4 * NEPI;
+    static constexpr int kMmaWarp0 = kProdWarp + 1;
+    static constexpr int kThreads = 32 * (kProdWarp + 4);
+    // register split (setmaxnreg): the launch gives every thread kRegLaunch; the
+    // converter and control groups shrink, the epilogue groups grow
+    static constexpr int kRegLaunch = (65536 / kThreads) / 8 * 8;
+    static constexpr int kRegConv = 80;
+    static constexpr int kRegCtrl = 48;
+    static constexpr int kRegEpiFit = ((kRegLaunch * kThreads / 128 - NCG * kRegConv - kRegCtrl) / NEPI) / 8 * 8;
+    static constexpr int kRegEpi = kRegEpiFit > 232 ? 232 : kRegEpiFit;
+    static_assert(128 * (NCG * kRegConv + kRegCtrl + NEPI * kRegEpi) <= kRegLaunch * kThreads, "register split");
+    static constexpr int kBStageBytes = BN * 128;
+    static constexpr uint32_t kTmemCols = 512;
+    static constexpr uint32_t kACol0 = 0;
+    static constexpr uint32_t kDCol0 = NA * 32;
+    static_assert(kDCol0 + ND * BN <= kTmemCols, "tensor memory over-subscribed");
+    static_assert(kNSC >= NA + ND, "scale ring too small");
+    static_assert(NS % 2 == 0, "the two producers own the stages of one parity each");
+    static_assert(kCW % 16 == 0, "epilogue column split");
+    static_assert(MAGIC_, "accumulators are preloaded with 1.5 * 2^23");
+    // shared memory carve-up
+    static constexpr int kOffB = 0;  // 1024-aligned (128-byte swizzle atoms)
+    static constexpr int kOffA = kOffB + NS * kBStageBytes;
+    static constexpr int kOffSc = kOffA + NS * kBlockBytes;  // ring: fp32 scale per row
+    static constexpr int kOffBar = kOffSc + kNSC * kTileRows * 4;
+    // full[NS] empty[NS] conv[NA] aempty[NA] dfull[ND] dempty[ND] scfull[NSC] final[2]
+    static constexpr int kNumBars = 2 * NS + 2 * NA + 2 * ND + kNSC + 2;
+    static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+    static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
+    static_assert(kSmemBytes <= 227 * 1024, "shared memory over-subscribed");
+};
 
 struct Item {
     int e, nt, row0, nrows;
 };
 
+// Tiles are ordered row-tile-major, weight tile fastest: the CTAs working at the
+// same time share the row tile's tokens (and, for experts with several row tiles,
+// the weights of nearby tiles) in L2.
+template <int BN>
 __device__ __forceinline__ Item decode_item(int u, const GemmArgs& a) {
-    int lo = 0, hi = a.E;  // largest e in [0, E) with NT * mtstart[e] <= u
-    while (hi - lo > 1) {
-        int mid = (lo + hi) >> 1;
-        if (a.NT * __ldg(a.mtstart + mid) <= u) lo = mid; else hi = mid;
-    }
+    const int mt = u / a.NT;
+    const int4 t = __ldg(a.mt_tab + mt);
     Item it;
-    it.e = lo;
-    const int m0 = __ldg(a.mtstart + lo);
-    const int nmt = __ldg(a.mtstart + lo + 1) - m0;
-    const int local = u - a.NT * m0;
-    it.nt = local / nmt;
-    const int j = local - it.nt * nmt;
-    it.row0 = __ldg(a.poffs + lo) + j * kBN;
-    it.nrows = min(kBN, __ldg(a.counts + lo) - j * kBN);
+    it.e = t.x;
+    it.nt = u - mt * a.NT;
+    it.row0 = t.y;
+    it.nrows = t.z;
     return it;
 }
 
 // Bounded wait on an mbarrier phase.  Returns false (and flags the CTA and the
 // device error word) when the wait runs out or another role already gave up.
-__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                         uint32_t* err) {
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag, uint32_t* err) {
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
-    while (true) {
+    for (uint32_t n = 1;; ++n) {
+        W4A8_BACKOFF();
         if (mbar_try_wait(bar, parity)) return true;
-        if (*abort_flag) return false;
-        if (clock64() - t0 > kWaitLimitCycles) {
-            *abort_flag = 1;
-            atomicOr(err, kErrTimeout);
-            return false;
+        if ((n & 15u) == 0) {
+            if (*abort_flag) return false;
+            if (clock64() - t0 > kWaitLimitCycles) {
+                *abort_flag = 1;
+                atomicOr(err, kErrTimeout);
+                return false;
+            }
         }
     }
 }
 
-__global__ void __launch_bounds__(kThreads, 1) gemm_w4a8_kernel(const GemmArgs a) {
+// wait without the abort bookkeeping, for draining at exit
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint32_t* err) {
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity)) {
+        if (clock64() - t0 > kWaitLimitCycles) {
+            atomicOr(err, kErrTimeout);
+            return;
+        }
+    }
+}
+
+__device__ __forceinline__ void tmem_st16_const(uint32_t taddr, uint32_t v) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1};" ::"r"(taddr),
+        "r"(v)
+        : "memory");
+}
+
+// acc0/acc1 += s * (x0 - 1.5*2^23, x1 - 1.5*2^23) with packed fp32x2 arithmetic
+__device__ __forceinline__ void fold2_magic(float& acc0, float& acc1, float s, uint32_t x0, uint32_t x1) {
+    asm("{\n\t.reg .b64 a, x, m, sc;\n\t"
+        "mov.b64 a, {%0, %1};\n\t"
+        "mov.b64 x, {%2, %3};\n\t"
+        "mov.b64 m, {%4, %4};\n\t"
+        "mov.b64 sc, {%5, %5};\n\t"
+        "sub.rn.f32x2 x, x, m;\n\t"
+        "fma.rn.f32x2 a, sc, x, a;\n\t"
+        "mov.b64 {%0, %1}, a;\n\t}"
+        : "+f"(acc0), "+f"(acc1)
+        : "r"(x0), "r"(x1), "f"(kMagicF), "f"(s));
+}
+
+__device__ __forceinline__ float silu_mul(float g, float u) { return __fdividef(g, 1.0f + __expf(-g)) * u; }
+
+// mbarrier addresses (used with bar0, NS, NA, ND, kNSC of the kernel's configuration in scope)
+#define FULL_BAR(s) (bar0 + 8u * (uint32_t)(s))
+#define EMPTY_BAR(s) (bar0 + 8u * (uint32_t)(NS + (s)))
+#define CONV_BAR(x) (bar0 + 8u * (uint32_t)(2 * NS + (x)))
+#define AEMPTY_BAR(x) (bar0 + 8u * (uint32_t)(2 * NS + NA + (x)))
+#define DFULL_BAR(b) (bar0 + 8u * (uint32_t)(2 * NS + 2 * NA + (b)))
+#define DEMPTY_BAR(b) (bar0 + 8u * (uint32_t)(2 * NS + 2 * NA + ND + (b)))
+#define SCFULL_BAR(i) (bar0 + 8u * (uint32_t)(2 * NS + 2 * NA + 2 * ND + (i)))
+#define FINAL_BAR(m) (bar0 + 8u * (uint32_t)(2 * NS + 2 * NA + 2 * ND + kNSC + (m)))
+
+template <class C>
+__global__ void __launch_bounds__(C::kThreads, 1) gemm_w4a8_kernel(const GemmArgs a) {
+    constexpr int BN = C::BN, NS = C::NS, NA = C::NA, ND = C::ND, kNSC = C::kNSC, kCW = C::kCW;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
     const uint32_t base_addr = (raw_addr + 1023u) & ~1023u;
@@ -99,36 +194,35 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_w4a8_kernel(const GemmArgs a
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    uint8_t* smA = smem + kOffA;
-    float* red = reinterpret_cast<float*>(smem + kOffRed);
-    const uint32_t sA = base_addr + kOffA;
-    const uint32_t sB = base_addr + kOffB;
-    const uint32_t bar0 = base_addr + kOffBar;
-    auto full_bar = [&](int s) { return bar0 + 8u * s; };
-    auto empty_bar = [&](int s) { return bar0 + 8u * (kStages + s); };
-    auto conv_bar = [&](int s) { return bar0 + 8u * (2 * kStages + s); };
-    auto dfull_bar = [&](int b) { return bar0 + 8u * (3 * kStages + b); };
-    auto dempty_bar = [&](int b) { return bar0 + 8u * (3 * kStages + 2 + b); };
-    const uint32_t final_bar = bar0 + 8u * (3 * kStages + 4);
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
+    uint8_t* smA = smem + C::kOffA;
+    float* sc_ring = reinterpret_cast<float*>(smem + C::kOffSc);
+    const uint32_t sA = base_addr + C::kOffA;
+    const uint32_t sB = base_addr + C::kOffB;
+    const uint32_t bar0 = base_addr + C::kOffBar;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
-            mbar_init(full_bar(s), 1);
-            mbar_init(empty_bar(s), 1 + 4);  // MMA commit + 4 epilogue warps (scale read)
-            mbar_init(conv_bar(s), 4);       // 4 converter warps
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(FULL_BAR(s), 1);
+            mbar_init(EMPTY_BAR(s), 1);  // commit of the MMAs that read the stage
         }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(dfull_bar(b), 1);
-            mbar_init(dempty_bar(b), 4);
+        for (int x = 0; x < NA; ++x) {
+            mbar_init(CONV_BAR(x), 4);    // the 4 warps of one converter group
+            mbar_init(AEMPTY_BAR(x), 1);  // commit of the MMAs that read the A slot
         }
-        mbar_init(final_bar, 1);
+        for (int b = 0; b < ND; ++b) {
+            mbar_init(DFULL_BAR(b), 1);
+            mbar_init(DEMPTY_BAR(b), 4 * C::NEPI);
+        }
+        for (int i = 0; i < kNSC; ++i) mbar_init(SCFULL_BAR(i), 4);
+        mbar_init(FINAL_BAR(0), 1);
+        mbar_init(FINAL_BAR(1), 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == kMmaWarp) {
-        tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    if (warp == C::kMmaWarp0) {
+        tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -136,215 +230,259 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_w4a8_kernel(const GemmArgs a
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
-    const int total = a.NT * __ldg(a.mtstart + a.E);
+    const bool is_epi = warp >= C::kEpiWarp0 && warp < C::kProdWarp;
+    const int q = warp & 3;  // TMEM lane quarter of this warp
+
+    const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+    if (is_epi) {
+        const int eh = (warp - C::kEpiWarp0) >> 2;
+#pragma unroll
+        for (int b = 0; b < ND; ++b)
+#pragma unroll
+            for (int c = 0; c < kCW / 16; ++c)
+                tmem_st16_const(tmem_base + lane_base + C::kDCol0 + b * BN + eh * kCW + c * 16, kMagicBits);
+        tmem_st_wait();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    const int total = a.NT * __ldg(a.n_mtiles);
     const int G = a.G;
 
-    if (warp == kProdWarp) {
+    // each role first moves its warpgroup's register budget (converter and control
+    // groups give registers to the epilogue groups), then runs
+    if (warp >= C::kProdWarp) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::kRegCtrl));
+    }
+    if (warp == C::kProdWarp || warp == C::kProdWarp + 3) {
+        // ---------------- producers: warp pi takes the steps with j % 2 == pi ----------------
+        // (the time a thread needs per ring step is fixed, whatever the copy size, so two
+        // issuing threads are needed to keep HBM busy with 8.7 KB weight blocks)
+        const int pi = warp == C::kProdWarp ? 0 : 1;
         if (lane == 0) {
-            uint32_t j = 0;
+            uint32_t j = 0, last = 0;
             bool ok = true;
             for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
-                const Item it = decode_item(u, a);
+                const Item it = decode_item<BN>(u, a);
                 const uint32_t bbytes = (uint32_t)round_up(it.nrows, 16) * 128u;
                 const uint8_t* wsrc = a.wblocks + (size_t)(it.e * a.NT + it.nt) * G * kBlockBytes;
                 const int8_t* asrc = a.act + (size_t)it.row0 * 128;
                 for (int g = 0; g < G; ++g, ++j) {
-                    const int s = j % kStages;
-                    const uint32_t ph = (j / kStages) & 1u;
-                    if (!wait_bar(empty_bar(s), ph ^ 1u, abort_flag, a.err)) { ok = false; break; }
-                    mbar_arrive_expect_tx(full_bar(s), kBlockBytes + bbytes);
-                    bulk_g2s(sA + s * kBlockBytes, wsrc + (size_t)g * kBlockBytes, kBlockBytes, full_bar(s));
-                    bulk_g2s(sB + s * kBStageBytes, asrc + (size_t)g * a.act_plane, bbytes, full_bar(s));
+                    if ((int)(j & 1u) != pi) continue;
+                    last = j + 1;
+                    const int s = j % NS;
+                    if (!wait_bar(EMPTY_BAR(s), ((j / NS) & 1u) ^ 1u, abort_flag, a.err)) { ok = false; break; }
+                    mbar_arrive_expect_tx(FULL_BAR(s), kBlockBytes + bbytes);
+                    bulk_g2s(sA + s * kBlockBytes, wsrc + (size_t)g * kBlockBytes, kBlockBytes, FULL_BAR(s));
+                    bulk_g2s(sB + s * C::kBStageBytes, asrc + (size_t)g * a.act_plane, bbytes, FULL_BAR(s));
                 }
             }
             // never leave the CTA with copies still landing in its shared memory
-            const uint32_t first = j > (uint32_t)kStages ? j - kStages : 0u;
-            for (uint32_t q = first; q < j; ++q) {
-                const long long t0 = clock64();
-                while (!mbar_try_wait(full_bar(q % kStages), (q / kStages) & 1u)) {
-                    if (clock64() - t0 > kWaitLimitCycles) { atomicOr(a.err, kErrTimeout); break; }
-                }
-            }
+            for (uint32_t qq = (last > (uint32_t)NS ? last - NS : 0u); qq < last; ++qq)
+                if ((int)(qq & 1u) == pi) drain_wait(FULL_BAR(qq % NS), (qq / NS) & 1u, a.err);
         }
         __syncwarp();
-    } else if (warp < 4) {
-        // ---------------- converter: nibbles -> signed INT8 (code - zp) in TMEM ----------------
-        const int r = threadIdx.x;  // tile row = TMEM lane
-        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-        uint32_t j = 0;
-        bool ok = true;
-        for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
-            for (int g = 0; g < G; ++g, ++j) {
-                const int s = j % kStages;
-                const uint32_t ph = (j / kStages) & 1u;
-                if (!wait_bar(full_bar(s), ph, abort_flag, a.err)) { ok = false; break; }
-                const uint8_t* blk = smA + s * kBlockBytes;
-                uint4 w[4];
+    } else if (warp < C::kConvWarps) {
+        // ---------------- converters: nibbles -> signed INT8 (code - zp) in TMEM ----------------
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::kRegConv));
+        const int cg = warp >> 2;         // converter group: takes the steps with j % NCG == cg
+        const int r = threadIdx.x & 127;  // tile row = TMEM lane
+        const int nsteps = ((total - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x) * G;
+        for (int j = cg; j < nsteps; j += C::NCG) {
+            const int s = j % NS;
+            const int x = j % NA;
+            if (!wait_bar(FULL_BAR(s), (j / NS) & 1u, abort_flag, a.err)) break;
+            if (!wait_bar(AEMPTY_BAR(x), ((j / NA) & 1u) ^ 1u, abort_flag, a.err)) break;
+            const uint8_t* blk = smA + s * kBlockBytes;
+            uint4 w[4];
 #pragma unroll
-                for (int c = 0; c < 4; ++c) w[c] = *reinterpret_cast<const uint4*>(blk + code_chunk_offset(r, c));
-                const int zp = (int)__half2float(reinterpret_cast<const __half*>(blk + kZpOff)[r]);
+            for (int c = 0; c < 4; ++c) w[c] = *reinterpret_cast<const uint4*>(blk + code_chunk_offset(r, c));
+            const int zp = (int)__half2float(reinterpret_cast<const __half*>(blk + kZpOff)[r]);
+            const int slot = j % kNSC;
+            sc_ring[slot * kTileRows + r] = __half2float(reinterpret_cast<const __half*>(blk + kScaleOff)[r]);
+            uint32_t v[32];
+            {
+                // signed INT8 (code - zp): byte-wise (code + 128 - zp) ^ 128, no carries
                 const uint32_t nz = (uint32_t)(0x80 - zp) * 0x01010101u;
-                uint32_t v[32];
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
-                    const uint32_t x[4] = {w[c].x, w[c].y, w[c].z, w[c].w};
+                    const uint32_t xw[4] = {w[c].x, w[c].y, w[c].z, w[c].w};
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const int i = 4 * c + q;  // word i holds K = 8i .. 8i+7 of the group
-                        v[2 * i] = ((x[q] & 0x0F0F0F0Fu) + nz) ^ 0x80808080u;
-                        v[2 * i + 1] = (((x[q] >> 4) & 0x0F0F0F0Fu) + nz) ^ 0x80808080u;
+                    for (int qq = 0; qq < 4; ++qq) {
+                        const int i = 4 * c + qq;  // word i holds K = 8i .. 8i+7 of the group
+                        v[2 * i] = ((xw[qq] & 0x0F0F0F0Fu) + nz) ^ 0x80808080u;
+                        v[2 * i + 1] = (((xw[qq] >> 4) & 0x0F0F0F0Fu) + nz) ^ 0x80808080u;
                     }
                 }
-                tmem_st32(tmem_base + lane_base + kACol0 + (uint32_t)s * 32u, v);
-                tmem_st_wait();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(conv_bar(s));
+            }
+            tmem_st32(tmem_base + lane_base + C::kACol0 + (uint32_t)x * 32u, v);
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(CONV_BAR(x));
+                mbar_arrive(SCFULL_BAR(slot));
             }
         }
-    } else if (warp == kMmaWarp) {
-        // ---------------- MMA issue (one thread) ----------------
+    } else if (warp >= C::kMmaWarp0) {
+        // ---------------- MMA issue: warp mi takes the steps with j % 2 == mi ----------------
+        const int mi = warp - C::kMmaWarp0;
         if (lane == 0) {
-            uint32_t j = 0, d = 0;
+            uint32_t j = 0;
             bool ok = true;
             for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
-                const Item it = decode_item(u, a);
+                const Item it = decode_item<BN>(u, a);
                 const uint32_t idesc = idesc_i8(128, round_up(it.nrows, 16));
-                for (int g = 0; g < G; ++g, ++j, ++d) {
-                    const int s = j % kStages;
-                    const uint32_t ph = (j / kStages) & 1u;
-                    const int b = d & 1;
-                    const uint32_t dph = (d >> 1) & 1u;
-                    if (!wait_bar(conv_bar(s), ph, abort_flag, a.err)) { ok = false; break; }
-                    if (!wait_bar(dempty_bar(b), dph ^ 1u, abort_flag, a.err)) { ok = false; break; }
+                for (int g = 0; g < G; ++g, ++j) {
+                    if ((int)(j & 1u) != mi) continue;
+                    const int s = j % NS, x = j % NA, b = j % ND;
+                    if (!wait_bar(CONV_BAR(x), (j / NA) & 1u, abort_flag, a.err)) { ok = false; break; }
+                    if (!wait_bar(DEMPTY_BAR(b), ((j / ND) & 1u) ^ 1u, abort_flag, a.err)) { ok = false; break; }
                     tc_fence_after();
-                    const uint32_t dt = tmem_base + kDCol0 + (uint32_t)b * kBN;
-                    const uint32_t at = tmem_base + kACol0 + (uint32_t)s * 32u;
-                    const uint32_t sb = sB + s * kBStageBytes;
+                    const uint32_t dt = tmem_base + C::kDCol0 + (uint32_t)b * BN;
+                    const uint32_t at = tmem_base + C::kACol0 + (uint32_t)x * 32u;
+                    const uint32_t sb = sB + s * C::kBStageBytes;
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        mma_i8_ts(dt, at + kk * 8, smem_desc_sw128(sb + kk * 32), idesc, kk > 0 ? 1u : 0u);
-                    tc_commit(empty_bar(s));
-                    tc_commit(dfull_bar(b));
+                        mma_i8_ts(dt, at + kk * 8, smem_desc_sw128(sb + kk * 32), idesc, 1u);
+                    tc_commit(EMPTY_BAR(s));
+                    tc_commit(AEMPTY_BAR(x));
+                    tc_commit(DFULL_BAR(b));
                 }
             }
-            // every MMA issued above must be complete before tensor memory is freed
-            tc_commit(final_bar);
-            const long long t0 = clock64();
-            while (!mbar_try_wait(final_bar, 0)) {
-                if (clock64() - t0 > kWaitLimitCycles) { atomicOr(a.err, kErrTimeout); break; }
-            }
+            // every MMA this warp issued must be complete before tensor memory is freed
+            tc_commit(FINAL_BAR(mi));
+            drain_wait(FINAL_BAR(mi), 0, a.err);
         }
         __syncwarp();
     } else {
-        // ---------------- epilogue: fold partials, apply scales, write ----------------
-        const int q = warp - kEpiWarp0;  // TMEM lane quarter
-        const int r = q * 32 + lane;     // tile row
-        const int et = threadIdx.x - kEpiWarp0 * 32;
-        const uint32_t lane_base = (uint32_t)(q * 32) << 16;
-        uint32_t j = 0, d = 0;
+        // ---------------- epilogue ----------------
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::kRegEpi));
+        const int eh = (warp - C::kEpiWarp0) >> 2;  // epilogue warpgroup: columns [eh*kCW, eh*kCW + kCW)
+        const int r = q * 32 + lane;                 // tile row = TMEM lane
+        const int col0 = eh * kCW;
+        uint32_t j = 0;
         bool ok = true;
         for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
-            const Item it = decode_item(u, a);
-            const int nch = round_up(it.nrows, 16) >> 4;
-            float acc[kBN];
+            const Item it = decode_item<BN>(u, a);
+            const int nb = round_up(it.nrows, 16);
+            float acc[kCW];
 #pragma unroll
-            for (int i = 0; i < kBN; ++i) acc[i] = 0.f;
+            for (int i = 0; i < kCW; ++i) acc[i] = 0.f;
             const int n_out = (a.mode == 1) ? -1 : it.nt * kTileRows + r;
-            for (int g = 0; g < G; ++g, ++j, ++d) {
-                const int s = j % kStages;
-                const int b = d & 1;
-                const uint32_t dph = (d >> 1) & 1u;
-                if (!wait_bar(dfull_bar(b), dph, abort_flag, a.err)) { ok = false; break; }
-                tc_fence_after();
-                const float sc = __half2float(reinterpret_cast<const __half*>(smA + s * kBlockBytes + kScaleOff)[r]);
-                const uint32_t taddr = tmem_base + lane_base + kDCol0 + (uint32_t)b * kBN;
+            int g = 0;
+            while (g < G) {
+                {
+                    // wide tiles: one step per pass, magic-constant accumulators
+                    const int b = j % ND;
+                    if (!wait_bar(DFULL_BAR(b), (j / ND) & 1u, abort_flag, a.err)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t taddr = tmem_base + lane_base + C::kDCol0 + (uint32_t)b * BN + col0;
+                    if (!wait_bar(SCFULL_BAR(j % kNSC), (j / kNSC) & 1u, abort_flag, a.err)) { ok = false; break; }
+                    const float sc = sc_ring[(j % kNSC) * kTileRows + r];
 #pragma unroll
-                for (int c = 0; c < kBN / 16; ++c) {
-                    if (c < nch) {
-                        uint32_t v[16];
-                        tmem_ld16(taddr + c * 16, v);
-                        tmem_ld_wait();
-                        if (a.partials != nullptr && n_out < a.nvalid) {
+                    for (int rd = 0; rd < kCW / 16; ++rd) {
+                        if (col0 + rd * 16 < nb) {
+                            uint32_t v[16];
+                            tmem_ld16(taddr + rd * 16, v);
+                            tmem_ld_wait();
+                            if (a.partials != nullptr && n_out < a.nvalid) {
+                                const int m0 = col0 + rd * 16;
+                                int32_t* pp = a.partials + ((size_t)(it.row0 + m0) * a.nvalid + n_out) * G + g;
+                                const size_t pstride = (size_t)a.nvalid * G;
 #pragma unroll
-                            for (int i = 0; i < 16; ++i) {
-                                const int m = c * 16 + i;
-                                if (m < it.nrows)
-                                    a.partials[((size_t)(it.row0 + m) * a.nvalid + n_out) * G + g] = (int32_t)v[i];
+                                for (int i = 0; i < 16; ++i)
+                                    if (m0 + i < it.nrows) pp[i * pstride] = (int32_t)(v[i] - kMagicBits);
                             }
-                        }
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) acc[c * 16 + i] = fmaf(sc, (float)(int32_t)v[i], acc[c * 16 + i]);
+                            for (int i = 0; i < 16; i += 2)
+                                fold2_magic(acc[rd * 16 + i], acc[rd * 16 + i + 1], sc, v[i], v[i + 1]);
+                        }
                     }
-                }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(dempty_bar(b));
-                    mbar_arrive(empty_bar(s));
+#pragma unroll
+                    for (int c = 0; c < kCW / 16; ++c)
+                        if (col0 + c * 16 < nb) tmem_st16_const(taddr + c * 16, kMagicBits);
+                    tmem_st_wait();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(DEMPTY_BAR(b));
+                    ++j;
+                    ++g;
                 }
             }
             if (!ok) break;
+            const float* sap = a.act_scale + it.row0 + col0;
             if (a.mode != 1) {
                 if (n_out < a.nvalid) {
+                    float* op = a.out + (size_t)(it.row0 + col0) * a.ldo + n_out;
 #pragma unroll
-                    for (int m = 0; m < kBN; ++m) {
-                        if (m < it.nrows) {
-                            const float sa = __ldg(a.act_scale + it.row0 + m);
-                            a.out[(size_t)(it.row0 + m) * a.ldo + n_out] = acc[m] * sa;
-                        }
-                    }
+                    for (int i = 0; i < kCW; ++i)
+                        if (col0 + i < it.nrows) op[(size_t)i * a.ldo] = acc[i] * __ldg(sap + i);
                 }
             } else {
                 // SwiGLU: even tile rows hold gate channel f, odd rows the matching up channel
                 const int f = it.nt * (kTileRows / 2) + (r >> 1);
-                const bool is_gate = (r & 1) == 0;
-                const bool valid = is_gate && f < a.nvalid;
+                const bool valid = ((r & 1) == 0) && f < a.nvalid;
+                float* op = a.out + (size_t)(it.row0 + col0) * a.ldo + f;
 #pragma unroll
-                for (int m = 0; m < kBN; ++m) {
-                    if (m < it.nrows) {
-                        const float sa = __ldg(a.act_scale + it.row0 + m);
-                        const float y = acc[m] * sa;
+                for (int i = 0; i < kCW; ++i) {
+                    if (col0 + i < it.nrows) {
+                        const float y = acc[i] * __ldg(sap + i);
                         const float yo = __shfl_xor_sync(0xffffffffu, y, 1);
-                        float hv = 0.f;
-                        if (valid) {
-                            hv = (y / (1.0f + expf(-y))) * yo;
-                            a.out[(size_t)(it.row0 + m) * a.ldo + f] = hv;
-                        }
-                        const uint32_t am = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(hv)));
-                        if (lane == 0) red[q * kBN + m] = __uint_as_float(am);
+                        if (valid) op[(size_t)i * a.ldo] = silu_mul(y, yo);
                     }
                 }
-                named_bar_sync(1, 128);
-                for (int m = et; m < it.nrows; m += 128) {
-                    const float mx = fmaxf(fmaxf(red[m], red[kBN + m]), fmaxf(red[2 * kBN + m], red[3 * kBN + m]));
-                    atomicMax(a.amax + it.row0 + m, __float_as_uint(mx));
-                }
-                named_bar_sync(1, 128);
             }
         }
     }
 
     __syncthreads();
-    if (warp == kMmaWarp) {
+    if (warp == C::kMmaWarp0) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, kTmemCols);
+        tmem_dealloc(tmem_base, C::kTmemCols);
     }
+}
+
+#undef FULL_BAR
+#undef EMPTY_BAR
+#undef CONV_BAR
+#undef AEMPTY_BAR
+#undef DFULL_BAR
+#undef DEMPTY_BAR
+#undef SCFULL_BAR
+#undef FINAL_BAR
+
+using CfgLarge = Cfg<128, 8, 4, 3, 2, true, 1>;  // many tokens per expert
+
+template <class C>
+cudaError_t launch_cfg(const GemmArgs& a, int num_ctas, cudaStream_t stream) {
+    static int attr_done[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64 || !attr_done[dev]) {
+        // the register split only holds if the kernel really launches with
+        // kRegLaunch registers per thread; otherwise setmaxnreg.inc could not be
+        // satisfied, so refuse to launch
+        cudaFuncAttributes fa;
+        cudaError_t e = cudaFuncGetAttributes(&fa, gemm_w4a8_kernel<C>);
+        if (e != cudaSuccess) return e;
+        if (fa.numRegs != C::kRegLaunch) return cudaErrorInvalidConfiguration;
+        e = cudaFuncSetAttribute(gemm_w4a8_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+        if (e != cudaSuccess) return e;
+        if (dev >= 0 && dev < 64) attr_done[dev] = 1;
+    }
+    gemm_w4a8_kernel<C><<<num_ctas, C::kThreads, C::kSmemBytes, stream>>>(a);
+    return cudaGetLastError();
 }
 
 }  // namespace
 
-size_t gemm_smem_bytes() { return (size_t)kSmemBytes; }
+int gemm_tile_tokens(int avg_tokens_per_expert) { return avg_tokens_per_expert <= 16 ? 16 : CfgLarge::BN; }
 
-cudaError_t launch_gemm(const GemmArgs& a, int num_ctas, cudaStream_t stream) {
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(gemm_w4a8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
-    gemm_w4a8_kernel<<<num_ctas, kThreads, kSmemBytes, stream>>>(a);
-    return cudaGetLastError();
+cudaError_t launch_gemm(const GemmArgs& a, int tile_tokens, int num_ctas, cudaStream_t stream) {
+    if (tile_tokens == 16) return launch_gemm_decode(a, num_ctas, stream);
+    return launch_cfg<CfgLarge>(a, num_ctas, stream);
 }
 
 }  // namespace w4a8

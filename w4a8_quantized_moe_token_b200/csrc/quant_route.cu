@@ -271,10 +271,10 @@ __device__ int block_exclusive_scan(int v, int* sh, int* total) {
     return before;
 }
 
-__global__ void __launch_bounds__(1024) perm_scan_kernel(int* __restrict__ chist, int nchunk, int E,
+__global__ void __launch_bounds__(1024) perm_scan_kernel(int* __restrict__ chist, int nchunk, int E, int tile_tokens,
                                                         int* __restrict__ counts, int* __restrict__ offs,
                                                         int* __restrict__ poffs, int* __restrict__ mtstart,
-                                                        int* __restrict__ row_src) {
+                                                        int4* __restrict__ mt_tab, int* __restrict__ row_src) {
     __shared__ int sh[32];
     const int e = threadIdx.x;
     int c_e = 0;
@@ -289,13 +289,16 @@ __global__ void __launch_bounds__(1024) perm_scan_kernel(int* __restrict__ chist
     int t0, t1, t2;
     const int o0 = block_exclusive_scan(c_e, sh, &t0);
     const int o1 = block_exclusive_scan(round_up(c_e, kRowPad), sh, &t1);
-    const int o2 = block_exclusive_scan(ceil_div(c_e, kBN), sh, &t2);
+    const int o2 = block_exclusive_scan(ceil_div(c_e, tile_tokens), sh, &t2);
     if (e < E) {
         counts[e] = c_e;
         offs[e] = o0;
         poffs[e] = o1;
         mtstart[e] = o2;
         for (int rr = o1 + c_e; rr < o1 + round_up(c_e, kRowPad); ++rr) row_src[rr] = -1;
+        // one entry per row tile of this expert: (expert, first row, rows)
+        for (int t = 0; t < ceil_div(c_e, tile_tokens); ++t)
+            mt_tab[o2 + t] = make_int4(e, o1 + t * tile_tokens, min(tile_tokens, c_e - t * tile_tokens), 0);
     }
     if (e == 0) {
         offs[E] = t0;
@@ -342,19 +345,17 @@ __global__ void __launch_bounds__(kPermChunk) perm_scatter_kernel(const int32_t*
 __global__ void __launch_bounds__(256) act_scatter_kernel(const uint16_t* __restrict__ x, int H, int k,
                                                           const int* __restrict__ row_src,
                                                           const int* __restrict__ poffs, int E,
-                                                          int8_t* __restrict__ act, size_t plane,
-                                                          float* __restrict__ s, uint32_t* __restrict__ amax_h) {
+                                                          int RB, int8_t* __restrict__ act,
+                                                          float* __restrict__ s) {
     const int r = blockIdx.x * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (r >= __ldg(poffs + E)) return;
     const int Hp = round_up(H, kGroup);
     const int nchunks = Hp / 16;  // 16-byte chunks of the row
     const int src = row_src[r];
-    if (lane == 0) amax_h[r] = 0u;
     if (src < 0) {
         for (int ci = lane; ci < nchunks; ci += 32)
-            *reinterpret_cast<uint4*>(act + (size_t)(ci >> 3) * plane + act_tiled_offset(r, (ci & 7) * 16)) =
-                make_uint4(0, 0, 0, 0);
+            *reinterpret_cast<uint4*>(act + act_offset(r, ci * 16, Hp / kGroup, RB)) = make_uint4(0, 0, 0, 0);
         if (lane == 0) s[r] = 0.f;
         return;
     }
@@ -375,10 +376,11 @@ __global__ void __launch_bounds__(256) act_scatter_kernel(const uint16_t* __rest
     }
     amax = warp_max(amax);
     const float sc = __fdiv_rn(amax, 127.0f);
-    for (int ci = lane; ci < nchunks; ci += 32) {
+    for (int base = 0; base < nchunks; base += 32) {
+        const int ci = base + lane;
         const int k0 = ci * 16;
         uint32_t out[4] = {0u, 0u, 0u, 0u};
-        if (amax > 0.f) {
+        if (ci < nchunks && amax > 0.f) {
             float vals[16];
             if (vec && k0 < H) {
                 const uint4 p0 = *reinterpret_cast<const uint4*>(xr + k0);
@@ -399,33 +401,45 @@ __global__ void __launch_bounds__(256) act_scatter_kernel(const uint16_t* __rest
                 out[i >> 2] |= c << (8 * (i & 3));
             }
         }
-        *reinterpret_cast<uint4*>(act + (size_t)(ci >> 3) * plane + act_tiled_offset(r, (ci & 7) * 16)) =
-            make_uint4(out[0], out[1], out[2], out[3]);
+        if (ci < nchunks)
+            *reinterpret_cast<uint4*>(act + act_offset(r, k0, Hp / kGroup, RB)) = make_uint4(out[0], out[1], out[2], out[3]);
     }
     if (lane == 0) s[r] = sc;
 }
 
 // ---------------------------------------------------------------------------
-// a6 (second half): requantise h per row with the row max gathered by the up GEMM.
+// a6 (second half): requantise h per row (max |h| over the row, then INT8 codes).
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) requant_kernel(const float* __restrict__ h, int ldh, int F,
                                                       const int* __restrict__ row_src, const int* __restrict__ poffs,
-                                                      int E, const uint32_t* __restrict__ amax_h,
-                                                      int8_t* __restrict__ act, size_t plane, float* __restrict__ s) {
+                                                      int E, int RB, int8_t* __restrict__ act,
+                                                      float* __restrict__ s) {
     const int r = blockIdx.x * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (r >= __ldg(poffs + E)) return;
     const int Fp = round_up(F, kGroup);
     const int nchunks = Fp / 16;
     const bool live = row_src[r] >= 0;
-    const float amax = live ? __uint_as_float(amax_h[r]) : 0.f;
-    const float sc = __fdiv_rn(amax, 127.0f);
     const float* hr = h + (size_t)r * ldh;
     const bool vec = (F & 15) == 0;
-    for (int ci = lane; ci < nchunks; ci += 32) {
+    float amax = 0.f;
+    if (live) {
+        if (vec) {
+            for (int i = lane; i < F / 4; i += 32) {
+                const float4 p = *reinterpret_cast<const float4*>(hr + 4 * i);
+                amax = fmaxf(amax, fmaxf(fmaxf(fabsf(p.x), fabsf(p.y)), fmaxf(fabsf(p.z), fabsf(p.w))));
+            }
+        } else {
+            for (int i = lane; i < F; i += 32) amax = fmaxf(amax, fabsf(hr[i]));
+        }
+        amax = warp_max(amax);
+    }
+    const float sc = __fdiv_rn(amax, 127.0f);
+    for (int base = 0; base < nchunks; base += 32) {
+        const int ci = base + lane;
         const int k0 = ci * 16;
         uint32_t out[4] = {0u, 0u, 0u, 0u};
-        if (amax > 0.f) {
+        if (ci < nchunks && amax > 0.f) {
             float vals[16];
             if (vec && k0 < F) {
 #pragma unroll
@@ -443,8 +457,8 @@ __global__ void __launch_bounds__(256) requant_kernel(const float* __restrict__ 
                 out[i >> 2] |= c << (8 * (i & 3));
             }
         }
-        *reinterpret_cast<uint4*>(act + (size_t)(ci >> 3) * plane + act_tiled_offset(r, (ci & 7) * 16)) =
-            make_uint4(out[0], out[1], out[2], out[3]);
+        if (ci < nchunks)
+            *reinterpret_cast<uint4*>(act + act_offset(r, k0, Fp / kGroup, RB)) = make_uint4(out[0], out[1], out[2], out[3]);
     }
     if (lane == 0) s[r] = sc;
 }
@@ -499,25 +513,20 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
 
 // dense GEMM: copy INT8 rows into the tiled planes (pad rows zero) and describe
 // them as one "expert" with M rows.
-__global__ void __launch_bounds__(256) dense_prep_kernel(const int8_t* __restrict__ qa, int M, int Kp,
-                                                         int8_t* __restrict__ act, size_t plane, int* counts, int* poffs,
-                                                         int* mtstart) {
+__global__ void __launch_bounds__(256) dense_prep_kernel(const int8_t* __restrict__ qa, int M, int Kp, int tile_tokens,
+                                                         int RB, int8_t* __restrict__ act, int4* mt_tab, int* n_mtiles) {
     const int Mp = round_up(M, kRowPad);
     const int nch = Kp / 16;
     const size_t idx = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (idx == 0) {
-        counts[0] = M;
-        poffs[0] = 0;
-        poffs[1] = Mp;
-        mtstart[0] = 0;
-        mtstart[1] = ceil_div(M, kBN);
-    }
+    const int nmt = ceil_div(M, tile_tokens);
+    if (idx == 0) *n_mtiles = nmt;
+    if (idx < (size_t)nmt) mt_tab[idx] = make_int4(0, (int)idx * tile_tokens, min(tile_tokens, M - (int)idx * tile_tokens), 0);
     if (idx >= (size_t)Mp * nch) return;
     const int r = (int)(idx / nch);
     const int ci = (int)(idx % nch);
     uint4 v = make_uint4(0, 0, 0, 0);
     if (r < M) v = *reinterpret_cast<const uint4*>(qa + (size_t)r * Kp + ci * 16);
-    *reinterpret_cast<uint4*>(act + (size_t)(ci >> 3) * plane + act_tiled_offset(r, (ci & 7) * 16)) = v;
+    *reinterpret_cast<uint4*>(act + act_offset(r, ci * 16, Kp / kGroup, RB)) = v;
 }
 
 }  // namespace
@@ -543,26 +552,25 @@ cudaError_t launch_route_topk(const uint16_t* logits, int T, int E, int k, int32
     return cudaGetLastError();
 }
 
-cudaError_t launch_perm(const int32_t* ids, int nslots, int E, int* chist, int nchunk, int* counts, int* offs,
-                        int* poffs, int* mtstart, int* perm, int* inv, int* row_src, uint32_t* err,
-                        cudaStream_t stream) {
+cudaError_t launch_perm(const int32_t* ids, int nslots, int E, int tile_tokens, int* chist, int nchunk, int* counts,
+                        int* offs, int* poffs, int* mtstart, int4* mt_tab, int* perm, int* inv, int* row_src,
+                        uint32_t* err, cudaStream_t stream) {
     perm_hist_kernel<<<nchunk, kPermChunk, 0, stream>>>(ids, nslots, E, chist, err);
-    perm_scan_kernel<<<1, 1024, 0, stream>>>(chist, nchunk, E, counts, offs, poffs, mtstart, row_src);
+    perm_scan_kernel<<<1, 1024, 0, stream>>>(chist, nchunk, E, tile_tokens, counts, offs, poffs, mtstart, mt_tab,
+                                             row_src);
     perm_scatter_kernel<<<nchunk, kPermChunk, 0, stream>>>(ids, nslots, E, chist, offs, poffs, perm, inv, row_src);
     return cudaGetLastError();
 }
 
 cudaError_t launch_act_scatter(const uint16_t* x, int H, int k, const int* row_src, const int* poffs, int E,
-                               int rows_cap, int8_t* act, size_t plane, float* s, uint32_t* amax,
-                               cudaStream_t stream) {
-    act_scatter_kernel<<<ceil_div(rows_cap, 8), 256, 0, stream>>>(x, H, k, row_src, poffs, E, act, plane, s, amax);
+                               int rows_cap, int rb, int8_t* act, float* s, cudaStream_t stream) {
+    act_scatter_kernel<<<ceil_div(rows_cap, 8), 256, 0, stream>>>(x, H, k, row_src, poffs, E, rb, act, s);
     return cudaGetLastError();
 }
 
 cudaError_t launch_requant(const float* h, int ldh, int F, const int* row_src, const int* poffs, int E,
-                           int rows_cap, const uint32_t* amax, int8_t* act, size_t plane, float* s,
-                           cudaStream_t stream) {
-    requant_kernel<<<ceil_div(rows_cap, 8), 256, 0, stream>>>(h, ldh, F, row_src, poffs, E, amax, act, plane, s);
+                           int rows_cap, int rb, int8_t* act, float* s, cudaStream_t stream) {
+    requant_kernel<<<ceil_div(rows_cap, 8), 256, 0, stream>>>(h, ldh, F, row_src, poffs, E, rb, act, s);
     return cudaGetLastError();
 }
 
@@ -574,11 +582,11 @@ cudaError_t launch_combine(const float* y2, int H, const int* inv, const float* 
     return cudaGetLastError();
 }
 
-cudaError_t launch_dense_prep(const int8_t* qa, int M, int Kp, int8_t* act, size_t plane, int* counts, int* poffs,
-                              int* mtstart, cudaStream_t stream) {
+cudaError_t launch_dense_prep(const int8_t* qa, int M, int Kp, int tile_tokens, int rb, int8_t* act, int4* mt_tab,
+                              int* n_mtiles, cudaStream_t stream) {
     const size_t n = (size_t)round_up(M, kRowPad) * (Kp / 16);
-    dense_prep_kernel<<<(unsigned)((n + 255) / 256 + 1), 256, 0, stream>>>(qa, M, Kp, act, plane, counts, poffs,
-                                                                          mtstart);
+    dense_prep_kernel<<<(unsigned)((n + 255) / 256 + 1), 256, 0, stream>>>(qa, M, Kp, tile_tokens, rb, act, mt_tab,
+                                                                          n_mtiles);
     return cudaGetLastError();
 }
 

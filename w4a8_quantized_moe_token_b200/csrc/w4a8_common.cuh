@@ -22,7 +22,6 @@ constexpr int kBlockBytes = kZpOff + kTileRows * 2;  // 8704 bytes per (tile, gr
 constexpr int kHeaderBytes = 256;
 constexpr uint32_t kPackMagic = 0x38413457u;         // "W4A8"
 constexpr int kRowPad = 16;           // each expert's row segment is padded to 16 rows
-constexpr int kBN = 128;              // tokens per GEMM tile (MMA N, at most)
 constexpr int kMaxExperts = 1024;
 
 // device error word bits
@@ -39,6 +38,14 @@ __host__ __device__ inline int round_up(int a, int b) { return ceil_div(a, b) * 
 // be moved into shared memory with one plain bulk copy.
 __host__ __device__ inline uint32_t act_tiled_offset(int r, int k) {
     return (uint32_t)r * 128u + ((uint32_t)(((k >> 4) ^ (r & 7)) & 7) << 4) + (uint32_t)(k & 15);
+}
+
+// Byte offset of (row r, column k) in the whole tiled activation buffer of G planes:
+// rows are grouped in blocks of RB rows, each block stores its G planes one after the
+// other ([rows/RB][G][RB][128]).  RB = 16 lets one copy fetch several K groups of a
+// 16-row tile; RB = all rows gives plain planes [G][rows][128].
+__host__ __device__ inline size_t act_offset(int r, int k, int G, int RB) {
+    return ((size_t)(r / RB) * G + (size_t)(k >> 7)) * (size_t)RB * 128u + act_tiled_offset(r % RB, k & 127);
 }
 
 // Byte offset of 16-byte chunk c (K columns 32c..32c+31 of the group) of tiled row r
@@ -72,14 +79,17 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
                  : "memory");
 }
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+// Test an mbarrier phase.  A thread whose phase is not complete yet is suspended
+// by the hardware until it completes or about `suspend_ns` pass, so waiting warps
+// do not spin on the issue slots that working warps on the same SM need.
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity, uint32_t suspend_ns = 20000u) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.b32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(bar), "r"(parity)
+        : "r"(bar), "r"(parity), "r"(suspend_ns)
         : "memory");
     return ok != 0;
 }
@@ -126,10 +136,12 @@ __device__ __forceinline__ void mma_i8_ts(uint32_t d_tmem, uint32_t a_tmem, uint
         : "memory");
 }
 
-// Instruction descriptor for kind::i8: D = s32 (bits 4-5 = 2), A = s8 (bits 7-9 = 1),
+// Instruction descriptor for kind::i8: D = s32 (bits 4-5 = 2), A = s8 or u8 (bits 7-9),
 // B = s8 (bits 10-12 = 1), both K-major, N >> 3 at bits 17-22, M >> 4 at bits 24-28.
-__host__ __device__ constexpr uint32_t idesc_i8(int M, int N) {
-    return (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+// a_signed = false selects unsigned 8-bit A (bits 7-9 = 0).
+__host__ __device__ constexpr uint32_t idesc_i8(int M, int N, bool a_signed = true) {
+    return (2u << 4) | ((a_signed ? 1u : 0u) << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |
+           ((uint32_t)(M >> 4) << 24);
 }
 
 // Shared-memory matrix descriptor: K-major, 128-byte swizzle, rows of 128 bytes,
