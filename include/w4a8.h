@@ -207,10 +207,10 @@ int w4a8_last_device_error(const void* ws, void* stream);
  * (on the call's stream).  w4a8_profile_stop() waits for those events, writes
  * per kind the number of kernel launches and their summed device milliseconds
  * (arrays of n entries, indexed by the W4A8_KERNEL_* values; a "perm" entry covers
- * the three permutation kernels), stops recording and returns W4A8_OK.  Timing
+ * the permutation kernels), stops recording and returns W4A8_OK.  Timing
  * adds one event record per kernel; it changes no result. */
 enum {
-    W4A8_KERNEL_PERM = 0,      /* histogram + scan + scatter (3 launches)      */
+    W4A8_KERNEL_PERM = 0,      /* histogram, scan, scatter (1 or 3 launches)  */
     W4A8_KERNEL_ACT_QUANT = 1, /* per-token INT8 into the grouped tiled rows    */
     W4A8_KERNEL_GEMM_UP = 2,   /* grouped W4A8 GEMM, gate|up, SwiGLU epilogue   */
     W4A8_KERNEL_REQUANT = 3,   /* per-row INT8 of h                             */

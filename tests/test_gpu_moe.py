@@ -154,6 +154,8 @@ SMALL = [
     (3, 16, 1, 256, 128, "uniform"),   # most experts empty
     (300, 4, 2, 512, 256, "uniform"),  # several row tiles per expert
     (64, 12, 4, 384, 192, "zipf"),
+    (64, 32, 4, 256, 256, "zipf"),     # decode kernel, hot experts span several 16-token tiles
+    (4500, 16, 4, 256, 128, "uniform"),  # > 16384 slots: multi-CTA permutation
 ]
 
 

@@ -184,7 +184,7 @@ int moe_forward_impl(const void* packed_up, const void* packed_down, int E, int 
     const int rb = act_block_rows(tile, L.R);
 
     {
-        ProfScope p(W4A8_KERNEL_PERM, 3, st);
+        ProfScope p(W4A8_KERNEL_PERM, perm_launch_count(L.nslots), st);
         W4A8_TRY(launch_perm(ids, L.nslots, E, tile, at<int>(ws, L, R_CHIST), L.nchunk, counts, offs, poffs, mtstart,
                              mt_tab, at<int>(ws, L, R_PERM), inv, row_src, err, st));
     }
@@ -387,7 +387,7 @@ bool gemm_layout(int M, int N, int K, GemmLayout* L) {
     size_t o = 0;
     L->err = o; o += align_up(16);
     L->nmt = o; o += align_up(4);
-    L->mttab = o; o += align_up((size_t)(M / 32 + 2) * 16);
+    L->mttab = o; o += align_up((size_t)(M / 16 + 2) * 16);
     L->act = o; o += align_up((size_t)L->G * L->Mp * 128);
     L->total = o;
     return true;

@@ -86,7 +86,7 @@ struct Cfg {
     static_assert(kDCol0 + ND * BN <= kTmemCols, "tensor memory over-subscribed");
     static_assert(kNSC >= NA + ND, "scale ring too small");
     static_assert(NS % 2 == 0, "the two producers own the stages of one parity each");
-    static_assert(kCW % 16 == 0, "epilogue column split");
+    static_assert(kCW % 64 == 0, "epilogue column split (batches of 64)");
     static_assert(MAGIC_, "accumulators are preloaded with 1.5 * 2^23");
     // shared memory carve-up
     static constexpr int kOffB = 0;  // 1024-aligned (128-byte swizzle atoms)
@@ -183,7 +183,7 @@ __device__ __forceinline__ float silu_mul(float g, float u) { return __fdividef(
 #define SCFULL_BAR(i) (bar0 + 8u * (uint32_t)(2 * NS + 2 * NA + 2 * ND + (i)))
 #define FINAL_BAR(m) (bar0 + 8u * (uint32_t)(2 * NS + 2 * NA + 2 * ND + kNSC + (m)))
 
-template <class C>
+template <class C, bool kPartials>
 __global__ void __launch_bounds__(C::kThreads, 1) gemm_w4a8_kernel(const GemmArgs a) {
     constexpr int BN = C::BN, NS = C::NS, NA = C::NA, ND = C::ND, kNSC = C::kNSC, kCW = C::kCW;
     extern __shared__ uint8_t smem_raw[];
@@ -381,23 +381,34 @@ __global__ void __launch_bounds__(C::kThreads, 1) gemm_w4a8_kernel(const GemmArg
                     const uint32_t taddr = tmem_base + lane_base + C::kDCol0 + (uint32_t)b * BN + col0;
                     if (!wait_bar(SCFULL_BAR(j % kNSC), (j / kNSC) & 1u, abort_flag, a.err)) { ok = false; break; }
                     const float sc = sc_ring[(j % kNSC) * kTileRows + r];
+                    // batches of kLdB columns: kLdB/16 loads, one wait, fold (the partials
+                    // instance keeps its batches small so that it needs no spill)
+                    constexpr int kLdB = kPartials ? 16 : 64;
 #pragma unroll
-                    for (int rd = 0; rd < kCW / 16; ++rd) {
-                        if (col0 + rd * 16 < nb) {
-                            uint32_t v[16];
-                            tmem_ld16(taddr + rd * 16, v);
+                    for (int rd = 0; rd < kCW / kLdB; ++rd) {
+                        const int m0 = col0 + rd * kLdB;
+                        if (m0 < nb) {
+                            uint32_t v[kLdB];
+#pragma unroll
+                            for (int c = 0; c < kLdB / 16; ++c)
+                                if (m0 + c * 16 < nb)
+                                    tmem_ld16(taddr + rd * kLdB + c * 16, *reinterpret_cast<uint32_t(*)[16]>(&v[c * 16]));
                             tmem_ld_wait();
-                            if (a.partials != nullptr && n_out < a.nvalid) {
-                                const int m0 = col0 + rd * 16;
+                            if (kPartials && n_out < a.nvalid) {
                                 int32_t* pp = a.partials + ((size_t)(it.row0 + m0) * a.nvalid + n_out) * G + g;
                                 const size_t pstride = (size_t)a.nvalid * G;
 #pragma unroll
-                                for (int i = 0; i < 16; ++i)
+                                for (int i = 0; i < kLdB; ++i)
                                     if (m0 + i < it.nrows) pp[i * pstride] = (int32_t)(v[i] - kMagicBits);
                             }
 #pragma unroll
-                            for (int i = 0; i < 16; i += 2)
-                                fold2_magic(acc[rd * 16 + i], acc[rd * 16 + i + 1], sc, v[i], v[i + 1]);
+                            for (int c = 0; c < kLdB / 16; ++c)
+                                if (m0 + c * 16 < nb) {
+#pragma unroll
+                                    for (int i = 0; i < 16; i += 2)
+                                        fold2_magic(acc[rd * kLdB + c * 16 + i], acc[rd * kLdB + c * 16 + i + 1], sc,
+                                                    v[c * 16 + i], v[c * 16 + i + 1]);
+                                }
                         }
                     }
 #pragma unroll
@@ -417,8 +428,10 @@ __global__ void __launch_bounds__(C::kThreads, 1) gemm_w4a8_kernel(const GemmArg
                 if (n_out < a.nvalid) {
                     float* op = a.out + (size_t)(it.row0 + col0) * a.ldo + n_out;
 #pragma unroll
-                    for (int i = 0; i < kCW; ++i)
-                        if (col0 + i < it.nrows) op[(size_t)i * a.ldo] = acc[i] * __ldg(sap + i);
+                    for (int i = 0; i < kCW; ++i) {
+                        if (col0 + i < it.nrows) *op = acc[i] * __ldg(sap + i);
+                        op += a.ldo;
+                    }
                 }
             } else {
                 // SwiGLU: even tile rows hold gate channel f, odd rows the matching up channel
@@ -430,8 +443,9 @@ __global__ void __launch_bounds__(C::kThreads, 1) gemm_w4a8_kernel(const GemmArg
                     if (col0 + i < it.nrows) {
                         const float y = acc[i] * __ldg(sap + i);
                         const float yo = __shfl_xor_sync(0xffffffffu, y, 1);
-                        if (valid) op[(size_t)i * a.ldo] = silu_mul(y, yo);
+                        if (valid) *op = silu_mul(y, yo);
                     }
+                    op += a.ldo;
                 }
             }
         }
@@ -455,7 +469,7 @@ __global__ void __launch_bounds__(C::kThreads, 1) gemm_w4a8_kernel(const GemmArg
 
 using CfgLarge = Cfg<128, 8, 4, 3, 2, true, 1>;  // many tokens per expert
 
-template <class C>
+template <class C, bool kPartials>
 cudaError_t launch_cfg(const GemmArgs& a, int num_ctas, cudaStream_t stream) {
     static int attr_done[64] = {0};
     int dev = 0;
@@ -465,14 +479,15 @@ cudaError_t launch_cfg(const GemmArgs& a, int num_ctas, cudaStream_t stream) {
         // kRegLaunch registers per thread; otherwise setmaxnreg.inc could not be
         // satisfied, so refuse to launch
         cudaFuncAttributes fa;
-        cudaError_t e = cudaFuncGetAttributes(&fa, gemm_w4a8_kernel<C>);
+        cudaError_t e = cudaFuncGetAttributes(&fa, gemm_w4a8_kernel<C, kPartials>);
         if (e != cudaSuccess) return e;
         if (fa.numRegs != C::kRegLaunch) return cudaErrorInvalidConfiguration;
-        e = cudaFuncSetAttribute(gemm_w4a8_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+        e = cudaFuncSetAttribute(gemm_w4a8_kernel<C, kPartials>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 C::kSmemBytes);
         if (e != cudaSuccess) return e;
         if (dev >= 0 && dev < 64) attr_done[dev] = 1;
     }
-    gemm_w4a8_kernel<C><<<num_ctas, C::kThreads, C::kSmemBytes, stream>>>(a);
+    gemm_w4a8_kernel<C, kPartials><<<num_ctas, C::kThreads, C::kSmemBytes, stream>>>(a);
     return cudaGetLastError();
 }
 
@@ -482,7 +497,9 @@ int gemm_tile_tokens(int avg_tokens_per_expert) { return avg_tokens_per_expert <
 
 cudaError_t launch_gemm(const GemmArgs& a, int tile_tokens, int num_ctas, cudaStream_t stream) {
     if (tile_tokens == 16) return launch_gemm_decode(a, num_ctas, stream);
-    return launch_cfg<CfgLarge>(a, num_ctas, stream);
+    // the INT32-partials output (a parity check of the dense entry point) has its own instance
+    if (a.partials != nullptr) return launch_cfg<CfgLarge, true>(a, num_ctas, stream);
+    return launch_cfg<CfgLarge, false>(a, num_ctas, stream);
 }
 
 }  // namespace w4a8

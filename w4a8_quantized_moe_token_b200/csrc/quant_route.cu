@@ -338,129 +338,207 @@ __global__ void __launch_bounds__(kPermChunk) perm_scatter_kernel(const int32_t*
     }
 }
 
-// ---------------------------------------------------------------------------
-// a2 in the layer: per-token INT8 of x, written straight into the tiled planes in
-// expert-grouped row order (one warp per grouped row; pad rows get zeros).
-// ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) act_scatter_kernel(const uint16_t* __restrict__ x, int H, int k,
-                                                          const int* __restrict__ row_src,
-                                                          const int* __restrict__ poffs, int E,
-                                                          int RB, int8_t* __restrict__ act,
-                                                          float* __restrict__ s) {
-    const int r = blockIdx.x * 8 + (threadIdx.x >> 5);
-    const int lane = threadIdx.x & 31;
-    if (r >= __ldg(poffs + E)) return;
-    const int Hp = round_up(H, kGroup);
-    const int nchunks = Hp / 16;  // 16-byte chunks of the row
-    const int src = row_src[r];
-    if (src < 0) {
-        for (int ci = lane; ci < nchunks; ci += 32)
-            *reinterpret_cast<uint4*>(act + act_offset(r, ci * 16, Hp / kGroup, RB)) = make_uint4(0, 0, 0, 0);
-        if (lane == 0) s[r] = 0.f;
-        return;
+// a4 for small batches (up to kPermSmallSlots slots): histogram, scans and the
+// stable scatter in one CTA, in slot order, 1024 slots at a time.
+__global__ void __launch_bounds__(1024) perm_small_kernel(const int32_t* __restrict__ ids, int nslots, int E,
+                                                         int tile_tokens, int* __restrict__ counts,
+                                                         int* __restrict__ offs, int* __restrict__ poffs,
+                                                         int* __restrict__ mtstart, int4* __restrict__ mt_tab,
+                                                         int* __restrict__ perm, int* __restrict__ inv,
+                                                         int* __restrict__ row_src, uint32_t* err) {
+    extern __shared__ int psm[];
+    int* s_off = psm;          // [E] counts, then the exclusive offsets
+    int* s_poff = psm + E;     // [E] padded offsets
+    int* s_run = psm + 2 * E;  // [E] slots of e placed so far
+    int* s_wcnt = psm + 3 * E; // [32][E] slots of e in each warp of the current chunk
+    __shared__ int sh[32];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    for (int e = tid; e < E; e += blockDim.x) {
+        s_off[e] = 0;
+        s_run[e] = 0;
     }
-    const uint16_t* xr = x + (size_t)(src / k) * H;
-    float amax = 0.f;
-    const bool vec = (H & 15) == 0;
-    if (vec) {
-        for (int ci = lane; ci < H / 8; ci += 32) {
-            const uint4 p = *reinterpret_cast<const uint4*>(xr + 8 * ci);
-            const uint32_t pw[4] = {p.x, p.y, p.z, p.w};
-#pragma unroll
-            for (int h = 0; h < 4; ++h)
-                amax = fmaxf(amax, fmaxf(fabsf(bf16_to_f32((uint16_t)(pw[h] & 0xFFFFu))),
-                                         fabsf(bf16_to_f32((uint16_t)(pw[h] >> 16)))));
+    __syncthreads();
+    for (int i = tid; i < nslots; i += blockDim.x) {
+        const int e = ids[i];
+        if (e >= 0 && e < E) atomicAdd(&s_off[e], 1);
+        else atomicOr(err, kErrBadExpert);
+    }
+    __syncthreads();
+    const int c_e = tid < E ? s_off[tid] : 0;
+    int t0, t1, t2;
+    const int o0 = block_exclusive_scan(c_e, sh, &t0);
+    const int o1 = block_exclusive_scan(round_up(c_e, kRowPad), sh, &t1);
+    const int o2 = block_exclusive_scan(ceil_div(c_e, tile_tokens), sh, &t2);
+    if (tid < E) {
+        counts[tid] = c_e;
+        offs[tid] = o0;
+        poffs[tid] = o1;
+        mtstart[tid] = o2;
+        s_off[tid] = o0;
+        s_poff[tid] = o1;
+        for (int rr = o1 + c_e; rr < o1 + round_up(c_e, kRowPad); ++rr) row_src[rr] = -1;
+        for (int t = 0; t < ceil_div(c_e, tile_tokens); ++t)
+            mt_tab[o2 + t] = make_int4(tid, o1 + t * tile_tokens, min(tile_tokens, c_e - t * tile_tokens), 0);
+    }
+    if (tid == 0) {
+        offs[E] = t0;
+        poffs[E] = t1;
+        mtstart[E] = t2;
+    }
+    for (int c0 = 0; c0 < nslots; c0 += blockDim.x) {
+        for (int idx = tid; idx < 32 * E; idx += blockDim.x) s_wcnt[idx] = 0;
+        __syncthreads();
+        const int i = c0 + tid;
+        const bool valid = i < nslots;
+        const int e = valid ? ids[i] : -1;
+        const bool good = valid && e >= 0 && e < E;
+        const uint32_t mask = __match_any_sync(0xffffffffu, good ? e : E + lane);
+        const int rank_w = __popc(mask & ((1u << lane) - 1u));
+        if (good && lane == __ffs(mask) - 1) s_wcnt[warp * E + e] = __popc(mask);
+        __syncthreads();
+        if (good) {
+            int p = s_run[e] + rank_w;
+            for (int w2 = 0; w2 < warp; ++w2) p += s_wcnt[w2 * E + e];
+            perm[s_off[e] + p] = i;
+            inv[i] = s_poff[e] + p;
+            row_src[s_poff[e] + p] = i;
+        } else if (valid) {
+            inv[i] = -1;
         }
-    } else {
-        for (int kk = lane; kk < H; kk += 32) amax = fmaxf(amax, fabsf(bf16_to_f32(xr[kk])));
-    }
-    amax = warp_max(amax);
-    const float sc = __fdiv_rn(amax, 127.0f);
-    for (int base = 0; base < nchunks; base += 32) {
-        const int ci = base + lane;
-        const int k0 = ci * 16;
-        uint32_t out[4] = {0u, 0u, 0u, 0u};
-        if (ci < nchunks && amax > 0.f) {
-            float vals[16];
-            if (vec && k0 < H) {
-                const uint4 p0 = *reinterpret_cast<const uint4*>(xr + k0);
-                const uint4 p1 = *reinterpret_cast<const uint4*>(xr + k0 + 8);
-                const uint32_t pw[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
-#pragma unroll
-                for (int h = 0; h < 8; ++h) {
-                    vals[2 * h] = bf16_to_f32((uint16_t)(pw[h] & 0xFFFFu));
-                    vals[2 * h + 1] = bf16_to_f32((uint16_t)(pw[h] >> 16));
-                }
-            } else {
-#pragma unroll
-                for (int i = 0; i < 16; ++i) vals[i] = (k0 + i < H) ? bf16_to_f32(xr[k0 + i]) : 0.f;
-            }
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const uint32_t c = (uint32_t)(quant_i8(vals[i], sc) & 0xFF);
-                out[i >> 2] |= c << (8 * (i & 3));
-            }
+        __syncthreads();
+        for (int ee = tid; ee < E; ee += blockDim.x) {
+            int add = 0;
+            for (int w2 = 0; w2 < 32; ++w2) add += s_wcnt[w2 * E + ee];
+            s_run[ee] += add;
         }
-        if (ci < nchunks)
-            *reinterpret_cast<uint4*>(act + act_offset(r, k0, Hp / kGroup, RB)) = make_uint4(out[0], out[1], out[2], out[3]);
+        __syncthreads();
     }
-    if (lane == 0) s[r] = sc;
 }
 
 // ---------------------------------------------------------------------------
-// a6 (second half): requantise h per row (max |h| over the row, then INT8 codes).
+// a2 / a6 in the layer: per-row symmetric INT8 into the tiled token rows.  One CTA
+// of 128 threads per grouped row; thread t owns the 16-value chunks t, t+128, ...
+// of the row and keeps up to kRowCache of them in registers between the max pass
+// and the quantisation pass.  Pad rows (row_src < 0) get zero codes and scale 0.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) requant_kernel(const float* __restrict__ h, int ldh, int F,
-                                                      const int* __restrict__ row_src, const int* __restrict__ poffs,
-                                                      int E, int RB, int8_t* __restrict__ act,
-                                                      float* __restrict__ s) {
-    const int r = blockIdx.x * 8 + (threadIdx.x >> 5);
-    const int lane = threadIdx.x & 31;
-    if (r >= __ldg(poffs + E)) return;
-    const int Fp = round_up(F, kGroup);
-    const int nchunks = Fp / 16;
-    const bool live = row_src[r] >= 0;
-    const float* hr = h + (size_t)r * ldh;
-    const bool vec = (F & 15) == 0;
-    float amax = 0.f;
-    if (live) {
-        if (vec) {
-            for (int i = lane; i < F / 4; i += 32) {
-                const float4 p = *reinterpret_cast<const float4*>(hr + 4 * i);
-                amax = fmaxf(amax, fmaxf(fmaxf(fabsf(p.x), fabsf(p.y)), fmaxf(fabsf(p.z), fabsf(p.w))));
-            }
-        } else {
-            for (int i = lane; i < F; i += 32) amax = fmaxf(amax, fabsf(hr[i]));
+constexpr int kRowCache = 4;
+
+struct Chunk16 {
+    float v[16];
+};
+
+__device__ __forceinline__ void load_chunk(const uint16_t* row, int len, int k0, Chunk16& c) {
+    if ((len & 15) == 0 && k0 + 16 <= len) {
+        const uint4 p0 = *reinterpret_cast<const uint4*>(row + k0);
+        const uint4 p1 = *reinterpret_cast<const uint4*>(row + k0 + 8);
+        const uint32_t pw[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+#pragma unroll
+        for (int h = 0; h < 8; ++h) {
+            c.v[2 * h] = bf16_to_f32((uint16_t)(pw[h] & 0xFFFFu));
+            c.v[2 * h + 1] = bf16_to_f32((uint16_t)(pw[h] >> 16));
         }
-        amax = warp_max(amax);
+    } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) c.v[i] = (k0 + i < len) ? bf16_to_f32(row[k0 + i]) : 0.f;
     }
-    const float sc = __fdiv_rn(amax, 127.0f);
-    for (int base = 0; base < nchunks; base += 32) {
-        const int ci = base + lane;
-        const int k0 = ci * 16;
-        uint32_t out[4] = {0u, 0u, 0u, 0u};
-        if (ci < nchunks && amax > 0.f) {
-            float vals[16];
-            if (vec && k0 < F) {
+}
+__device__ __forceinline__ void load_chunk(const float* row, int len, int k0, Chunk16& c) {
+    if ((len & 15) == 0 && k0 + 16 <= len) {
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const float4 p = *reinterpret_cast<const float4*>(hr + k0 + 4 * i);
-                    vals[4 * i] = p.x; vals[4 * i + 1] = p.y; vals[4 * i + 2] = p.z; vals[4 * i + 3] = p.w;
-                }
-            } else {
+        for (int i = 0; i < 4; ++i) {
+            const float4 p = *reinterpret_cast<const float4*>(row + k0 + 4 * i);
+            c.v[4 * i] = p.x; c.v[4 * i + 1] = p.y; c.v[4 * i + 2] = p.z; c.v[4 * i + 3] = p.w;
+        }
+    } else {
 #pragma unroll
-                for (int i = 0; i < 16; ++i) vals[i] = (k0 + i < F) ? hr[k0 + i] : 0.f;
+        for (int i = 0; i < 16; ++i) c.v[i] = (k0 + i < len) ? row[k0 + i] : 0.f;
+    }
+}
+
+template <typename TIn>
+__device__ __forceinline__ void quant_row_cta(const TIn* row, int len, int r, int RB, int8_t* __restrict__ act,
+                                              float* __restrict__ s) {
+    __shared__ float red[4];
+    const int Kp = round_up(len, kGroup);
+    const int nch = Kp / 16;
+    const int G = Kp / kGroup;
+    const int t = threadIdx.x;
+    Chunk16 cache[kRowCache];
+    float amax = 0.f;
+    if (row != nullptr) {
+#pragma unroll
+        for (int c = 0; c < kRowCache; ++c) {
+            const int ci = t + c * 128;
+            if (ci < nch) {
+                load_chunk(row, len, ci * 16, cache[c]);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(cache[c].v[i]));
             }
+        }
+        for (int ci = t + kRowCache * 128; ci < nch; ci += 128) {
+            Chunk16 tmp;
+            load_chunk(row, len, ci * 16, tmp);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(tmp.v[i]));
+        }
+    }
+    amax = warp_max(amax);
+    if ((t & 31) == 0) red[t >> 5] = amax;
+    __syncthreads();
+    amax = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+    const float sc = __fdiv_rn(amax, 127.0f);
+    auto emit = [&](int ci, const Chunk16& c) {
+        uint32_t out[4] = {0u, 0u, 0u, 0u};
+        if (amax > 0.f) {
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-                const uint32_t c = (uint32_t)(quant_i8(vals[i], sc) & 0xFF);
-                out[i >> 2] |= c << (8 * (i & 3));
+                const uint32_t q = (uint32_t)(quant_i8(c.v[i], sc) & 0xFF);
+                out[i >> 2] |= q << (8 * (i & 3));
             }
         }
-        if (ci < nchunks)
-            *reinterpret_cast<uint4*>(act + act_offset(r, k0, Fp / kGroup, RB)) = make_uint4(out[0], out[1], out[2], out[3]);
+        *reinterpret_cast<uint4*>(act + act_offset(r, ci * 16, G, RB)) = make_uint4(out[0], out[1], out[2], out[3]);
+    };
+#pragma unroll
+    for (int c = 0; c < kRowCache; ++c) {
+        const int ci = t + c * 128;
+        if (ci < nch) {
+            if (row == nullptr) {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) cache[c].v[i] = 0.f;
+            }
+            emit(ci, cache[c]);
+        }
     }
-    if (lane == 0) s[r] = sc;
+    for (int ci = t + kRowCache * 128; ci < nch; ci += 128) {
+        Chunk16 tmp;
+        if (row != nullptr) load_chunk(row, len, ci * 16, tmp);
+        else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) tmp.v[i] = 0.f;
+        }
+        emit(ci, tmp);
+    }
+    if (t == 0) s[r] = sc;
+}
+
+// x rows (bf16) -> INT8 rows in expert-grouped order
+__global__ void __launch_bounds__(128) act_scatter_kernel(const uint16_t* __restrict__ x, int H, int k,
+                                                          const int* __restrict__ row_src,
+                                                          const int* __restrict__ poffs, int E, int RB,
+                                                          int8_t* __restrict__ act, float* __restrict__ s) {
+    const int r = blockIdx.x;
+    if (r >= __ldg(poffs + E)) return;
+    const int src = row_src[r];
+    quant_row_cta<uint16_t>(src < 0 ? nullptr : x + (size_t)(src / k) * H, H, r, RB, act, s);
+}
+
+// h rows (fp32, SwiGLU output of the up GEMM) -> INT8 rows for the down GEMM
+__global__ void __launch_bounds__(128) requant_kernel(const float* __restrict__ h, int ldh, int F,
+                                                      const int* __restrict__ row_src, const int* __restrict__ poffs,
+                                                      int E, int RB, int8_t* __restrict__ act, float* __restrict__ s) {
+    const int r = blockIdx.x;
+    if (r >= __ldg(poffs + E)) return;
+    quant_row_cta<float>(row_src[r] < 0 ? nullptr : h + (size_t)r * ldh, F, r, RB, act, s);
 }
 
 // ---------------------------------------------------------------------------
@@ -469,45 +547,51 @@ __global__ void __launch_bounds__(256) requant_kernel(const float* __restrict__ 
 __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ y2, int H, const int* __restrict__ inv,
                                                       const float* __restrict__ w, int T, int k,
                                                       uint16_t* __restrict__ out) {
-    const int cols8 = (H + 7) >> 3;
-    const size_t idx = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (idx >= (size_t)T * cols8) return;
-    const int t = (int)(idx / cols8);
-    const int c0 = (int)(idx % cols8) * 8;
-    float acc[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+    __shared__ int rows[32];
+    __shared__ float wts[32];
+    const int t = blockIdx.x;
+    if (threadIdx.x < k) {
+        rows[threadIdx.x] = inv[(size_t)t * k + threadIdx.x];
+        wts[threadIdx.x] = w[(size_t)t * k + threadIdx.x];
+    }
+    __syncthreads();
     const bool vec = (H & 7) == 0;
-    for (int j = 0; j < k; ++j) {
-        const int rr = inv[(size_t)t * k + j];
-        if (rr < 0) continue;
-        const float wt = w[(size_t)t * k + j];
-        const float* row = y2 + (size_t)rr * H + c0;
+    for (int c0 = threadIdx.x * 8; c0 < H; c0 += blockDim.x * 8) {
+        float acc[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+#pragma unroll 4
+        for (int j = 0; j < k; ++j) {
+            const int rr = rows[j];
+            if (rr < 0) continue;
+            const float wt = wts[j];
+            const float* row = y2 + (size_t)rr * H + c0;
+            if (vec) {
+                const float4 a = *reinterpret_cast<const float4*>(row);
+                const float4 b = *reinterpret_cast<const float4*>(row + 4);
+                acc[0] = fmaf(wt, a.x, acc[0]); acc[1] = fmaf(wt, a.y, acc[1]);
+                acc[2] = fmaf(wt, a.z, acc[2]); acc[3] = fmaf(wt, a.w, acc[3]);
+                acc[4] = fmaf(wt, b.x, acc[4]); acc[5] = fmaf(wt, b.y, acc[5]);
+                acc[6] = fmaf(wt, b.z, acc[6]); acc[7] = fmaf(wt, b.w, acc[7]);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    if (c0 + i < H) acc[i] = fmaf(wt, row[i], acc[i]);
+            }
+        }
+        uint16_t* o = out + (size_t)t * H + c0;
         if (vec) {
-            const float4 a = *reinterpret_cast<const float4*>(row);
-            const float4 b = *reinterpret_cast<const float4*>(row + 4);
-            acc[0] = fmaf(wt, a.x, acc[0]); acc[1] = fmaf(wt, a.y, acc[1]);
-            acc[2] = fmaf(wt, a.z, acc[2]); acc[3] = fmaf(wt, a.w, acc[3]);
-            acc[4] = fmaf(wt, b.x, acc[4]); acc[5] = fmaf(wt, b.y, acc[5]);
-            acc[6] = fmaf(wt, b.z, acc[6]); acc[7] = fmaf(wt, b.w, acc[7]);
+            uint32_t pk[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                pk[i] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(acc[2 * i])) |
+                        ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(acc[2 * i + 1])) << 16);
+            *reinterpret_cast<uint4*>(o) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
         } else {
 #pragma unroll
             for (int i = 0; i < 8; ++i)
-                if (c0 + i < H) acc[i] = fmaf(wt, row[i], acc[i]);
+                if (c0 + i < H) o[i] = __bfloat16_as_ushort(__float2bfloat16_rn(acc[i]));
         }
-    }
-    uint16_t* o = out + (size_t)t * H + c0;
-    if (vec) {
-        uint32_t pk[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-            pk[i] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(acc[2 * i])) |
-                    ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(acc[2 * i + 1])) << 16);
-        *reinterpret_cast<uint4*>(o) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-    } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-            if (c0 + i < H) o[i] = __bfloat16_as_ushort(__float2bfloat16_rn(acc[i]));
     }
 }
 
@@ -552,9 +636,26 @@ cudaError_t launch_route_topk(const uint16_t* logits, int T, int E, int k, int32
     return cudaGetLastError();
 }
 
+int perm_launch_count(int nslots) { return nslots <= kPermSmallSlots ? 1 : 3; }
+
 cudaError_t launch_perm(const int32_t* ids, int nslots, int E, int tile_tokens, int* chist, int nchunk, int* counts,
                         int* offs, int* poffs, int* mtstart, int4* mt_tab, int* perm, int* inv, int* row_src,
                         uint32_t* err, cudaStream_t stream) {
+    if (nslots <= kPermSmallSlots) {
+        const size_t smem = (size_t)35 * E * sizeof(int);
+        static int attr_done[64] = {0};
+        int dev = 0;
+        cudaGetDevice(&dev);
+        if (dev < 0 || dev >= 64 || !attr_done[dev]) {
+            const cudaError_t e = cudaFuncSetAttribute(perm_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                       35 * kMaxExperts * (int)sizeof(int));
+            if (e != cudaSuccess) return e;
+            if (dev >= 0 && dev < 64) attr_done[dev] = 1;
+        }
+        perm_small_kernel<<<1, 1024, smem, stream>>>(ids, nslots, E, tile_tokens, counts, offs, poffs, mtstart, mt_tab,
+                                                     perm, inv, row_src, err);
+        return cudaGetLastError();
+    }
     perm_hist_kernel<<<nchunk, kPermChunk, 0, stream>>>(ids, nslots, E, chist, err);
     perm_scan_kernel<<<1, 1024, 0, stream>>>(chist, nchunk, E, tile_tokens, counts, offs, poffs, mtstart, mt_tab,
                                              row_src);
@@ -564,21 +665,22 @@ cudaError_t launch_perm(const int32_t* ids, int nslots, int E, int tile_tokens, 
 
 cudaError_t launch_act_scatter(const uint16_t* x, int H, int k, const int* row_src, const int* poffs, int E,
                                int rows_cap, int rb, int8_t* act, float* s, cudaStream_t stream) {
-    act_scatter_kernel<<<ceil_div(rows_cap, 8), 256, 0, stream>>>(x, H, k, row_src, poffs, E, rb, act, s);
+    if (rows_cap == 0) return cudaSuccess;
+    act_scatter_kernel<<<rows_cap, 128, 0, stream>>>(x, H, k, row_src, poffs, E, rb, act, s);
     return cudaGetLastError();
 }
 
 cudaError_t launch_requant(const float* h, int ldh, int F, const int* row_src, const int* poffs, int E,
                            int rows_cap, int rb, int8_t* act, float* s, cudaStream_t stream) {
-    requant_kernel<<<ceil_div(rows_cap, 8), 256, 0, stream>>>(h, ldh, F, row_src, poffs, E, rb, act, s);
+    if (rows_cap == 0) return cudaSuccess;
+    requant_kernel<<<rows_cap, 128, 0, stream>>>(h, ldh, F, row_src, poffs, E, rb, act, s);
     return cudaGetLastError();
 }
 
 cudaError_t launch_combine(const float* y2, int H, const int* inv, const float* w, int T, int k, uint16_t* out,
                            cudaStream_t stream) {
-    const size_t n = (size_t)T * ((H + 7) / 8);
-    if (n == 0) return cudaSuccess;
-    combine_kernel<<<(unsigned)((n + 255) / 256), 256, 0, stream>>>(y2, H, inv, w, T, k, out);
+    if (T == 0) return cudaSuccess;
+    combine_kernel<<<T, 256, 0, stream>>>(y2, H, inv, w, T, k, out);
     return cudaGetLastError();
 }
 

@@ -45,8 +45,9 @@ cudaError_t launch_route_topk(const uint16_t* logits, int T, int E, int k, int32
 cudaError_t launch_perm(const int32_t* ids, int nslots, int E, int tile_tokens, int* chist, int nchunk, int* counts,
                         int* offs, int* poffs, int* mtstart, int4* mt_tab, int* perm, int* inv, int* row_src,
                         uint32_t* err, cudaStream_t stream);
-// capacity of the row-tile table for a layer (tiles of at least 32 rows)
-inline int mt_tab_capacity(int nslots, int E) { return nslots / 32 + E + 1; }
+// capacity of the row-tile table for a layer: sum over experts of ceil(count / tile)
+// <= nslots / tile + E, with tiles of at least 16 rows
+inline int mt_tab_capacity(int nslots, int E) { return nslots / 16 + E + 1; }
 cudaError_t launch_act_scatter(const uint16_t* x, int H, int k, const int* row_src, const int* poffs, int E,
                                int rows_cap, int rb, int8_t* act, float* s, cudaStream_t stream);
 cudaError_t launch_requant(const float* h, int ldh, int F, const int* row_src, const int* poffs, int E,
@@ -56,6 +57,8 @@ cudaError_t launch_combine(const float* y2, int H, const int* inv, const float* 
 cudaError_t launch_dense_prep(const int8_t* qa, int M, int Kp, int tile_tokens, int rb, int8_t* act, int4* mt_tab,
                               int* n_mtiles, cudaStream_t stream);
 
-constexpr int kPermChunk = 256;  // slots per permutation chunk
+constexpr int kPermChunk = 256;       // slots per permutation chunk (multi-CTA path)
+constexpr int kPermSmallSlots = 16384;  // up to this many slots the permutation runs in one CTA
+int perm_launch_count(int nslots);
 
 }  // namespace w4a8
