@@ -190,7 +190,7 @@ int moe_forward_impl(const void* packed_up, const void* packed_down, int E, int 
     }
     {
         ProfScope p(W4A8_KERNEL_ACT_QUANT, 1, st);
-        W4A8_TRY(launch_act_scatter(x, H, k, row_src, poffs, E, L.R, rb, act1, s1, st));
+        W4A8_TRY(launch_act_scatter(x, T, H, k, inv, offs, poffs, E, rb, act1, s1, st));
     }
 
     GemmArgs up{};

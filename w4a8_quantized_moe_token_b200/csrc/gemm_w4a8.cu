@@ -86,7 +86,7 @@ struct Cfg {
     static_assert(kDCol0 + ND * BN <= kTmemCols, "tensor memory over-subscribed");
     static_assert(kNSC >= NA + ND, "scale ring too small");
     static_assert(NS % 2 == 0, "the two producers own the stages of one parity each");
-    static_assert(kCW % 64 == 0, "epilogue column split (batches of 64)");
+    static_assert(kCW % 16 == 0 && (kCW <= 64 || kCW % 64 == 0), "epilogue column split");
     static_assert(MAGIC_, "accumulators are preloaded with 1.5 * 2^23");
     // shared memory carve-up
     static constexpr int kOffB = 0;  // 1024-aligned (128-byte swizzle atoms)
@@ -376,76 +376,88 @@ __global__ void __launch_bounds__(C::kThreads, 1) gemm_w4a8_kernel(const GemmArg
                 {
                     // wide tiles: one step per pass, magic-constant accumulators
                     const int b = j % ND;
+                    // the converters publish the step's scales well before its MMAs finish
+                    if (!wait_bar(SCFULL_BAR(j % kNSC), (j / kNSC) & 1u, abort_flag, a.err)) { ok = false; break; }
+                    const float sc = sc_ring[(j % kNSC) * kTileRows + r];
                     if (!wait_bar(DFULL_BAR(b), (j / ND) & 1u, abort_flag, a.err)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t taddr = tmem_base + lane_base + C::kDCol0 + (uint32_t)b * BN + col0;
-                    if (!wait_bar(SCFULL_BAR(j % kNSC), (j / kNSC) & 1u, abort_flag, a.err)) { ok = false; break; }
-                    const float sc = sc_ring[(j % kNSC) * kTileRows + r];
-                    // batches of kLdB columns: kLdB/16 loads, one wait, fold (the partials
+                    // batches of kLdB columns: kLdB/16 loads and one wait; the accumulator
+                    // columns get their constant back and the buffer is released to the MMA
+                    // warps before the fold, which then runs from registers (the partials
                     // instance keeps its batches small so that it needs no spill)
-                    constexpr int kLdB = kPartials ? 16 : 64;
+                    constexpr int kLdB = kPartials ? 16 : (kCW < 64 ? kCW : 64);
+                    constexpr int kNB = kCW / kLdB;
 #pragma unroll
-                    for (int rd = 0; rd < kCW / kLdB; ++rd) {
+                    for (int rd = 0; rd < kNB; ++rd) {
                         const int m0 = col0 + rd * kLdB;
-                        if (m0 < nb) {
-                            uint32_t v[kLdB];
+                        uint32_t v[kLdB];
 #pragma unroll
-                            for (int c = 0; c < kLdB / 16; ++c)
-                                if (m0 + c * 16 < nb)
-                                    tmem_ld16(taddr + rd * kLdB + c * 16, *reinterpret_cast<uint32_t(*)[16]>(&v[c * 16]));
-                            tmem_ld_wait();
-                            if (kPartials && n_out < a.nvalid) {
-                                int32_t* pp = a.partials + ((size_t)(it.row0 + m0) * a.nvalid + n_out) * G + g;
-                                const size_t pstride = (size_t)a.nvalid * G;
+                        for (int c = 0; c < kLdB / 16; ++c)
+                            if (m0 + c * 16 < nb)
+                                tmem_ld16(taddr + rd * kLdB + c * 16, *reinterpret_cast<uint32_t(*)[16]>(&v[c * 16]));
+                        tmem_ld_wait();
 #pragma unroll
-                                for (int i = 0; i < kLdB; ++i)
-                                    if (m0 + i < it.nrows) pp[i * pstride] = (int32_t)(v[i] - kMagicBits);
-                            }
-#pragma unroll
-                            for (int c = 0; c < kLdB / 16; ++c)
-                                if (m0 + c * 16 < nb) {
-#pragma unroll
-                                    for (int i = 0; i < 16; i += 2)
-                                        fold2_magic(acc[rd * kLdB + c * 16 + i], acc[rd * kLdB + c * 16 + i + 1], sc,
-                                                    v[c * 16 + i], v[c * 16 + i + 1]);
-                                }
+                        for (int c = 0; c < kLdB / 16; ++c)
+                            if (m0 + c * 16 < nb) tmem_st16_const(taddr + rd * kLdB + c * 16, kMagicBits);
+                        if (rd == kNB - 1) {
+                            tmem_st_wait();
+                            tc_fence_before();
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive(DEMPTY_BAR(b));
                         }
-                    }
+                        if (kPartials && n_out < a.nvalid) {
+                            int32_t* pp = a.partials + ((size_t)(it.row0 + m0) * a.nvalid + n_out) * G + g;
+                            const size_t pstride = (size_t)a.nvalid * G;
 #pragma unroll
-                    for (int c = 0; c < kCW / 16; ++c)
-                        if (col0 + c * 16 < nb) tmem_st16_const(taddr + c * 16, kMagicBits);
-                    tmem_st_wait();
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(DEMPTY_BAR(b));
+                            for (int i = 0; i < kLdB; ++i)
+                                if (m0 + i < it.nrows) pp[i * pstride] = (int32_t)(v[i] - kMagicBits);
+                        }
+#pragma unroll
+                        for (int c = 0; c < kLdB / 16; ++c)
+                            if (m0 + c * 16 < nb) {
+#pragma unroll
+                                for (int i = 0; i < 16; i += 2)
+                                    fold2_magic(acc[rd * kLdB + c * 16 + i], acc[rd * kLdB + c * 16 + i + 1], sc,
+                                                v[c * 16 + i], v[c * 16 + i + 1]);
+                            }
+                    }
                     ++j;
                     ++g;
                 }
             }
             if (!ok) break;
             const float* sap = a.act_scale + it.row0 + col0;
+            const int ncol = it.nrows - col0;
             if (a.mode != 1) {
-                if (n_out < a.nvalid) {
-                    float* op = a.out + (size_t)(it.row0 + col0) * a.ldo + n_out;
-#pragma unroll
-                    for (int i = 0; i < kCW; ++i) {
-                        if (col0 + i < it.nrows) *op = acc[i] * __ldg(sap + i);
-                        op += a.ldo;
-                    }
-                }
-            } else {
-                // SwiGLU: even tile rows hold gate channel f, odd rows the matching up channel
-                const int f = it.nt * (kTileRows / 2) + (r >> 1);
-                const bool valid = ((r & 1) == 0) && f < a.nvalid;
-                float* op = a.out + (size_t)(it.row0 + col0) * a.ldo + f;
+                const bool valid = n_out < a.nvalid;
+                float* op = a.out + (size_t)(it.row0 + col0) * a.ldo + (valid ? n_out : 0);
 #pragma unroll
                 for (int i = 0; i < kCW; ++i) {
-                    if (col0 + i < it.nrows) {
-                        const float y = acc[i] * __ldg(sap + i);
-                        const float yo = __shfl_xor_sync(0xffffffffu, y, 1);
-                        if (valid) *op = silu_mul(y, yo);
-                    }
+                    if (valid && i < ncol) *op = acc[i] * __ldg(sap + i);
                     op += a.ldo;
+                }
+            } else {
+                // SwiGLU: even tile rows hold gate channel f, odd rows the matching up
+                // channel.  Per pair of tokens (i, i+1) the lanes of a pair swap one value:
+                // the even lane finishes token i, the odd lane token i+1.
+                const int f = it.nt * (kTileRows / 2) + (r >> 1);
+                const int odd = r & 1;
+                const bool valid = f < a.nvalid;
+                float* op = a.out + (size_t)(it.row0 + col0 + odd) * a.ldo + f;
+                float sa[kCW / 2];
+#pragma unroll
+                for (int i = 0; i < kCW; i += 2) sa[i / 2] = i + odd < ncol ? __ldg(sap + i + odd) : 0.f;
+#pragma unroll
+                for (int i = 0; i < kCW; i += 2) {
+                    // even lane: own gate_i, needs the partner's up_i; odd lane: own up_{i+1},
+                    // needs the partner's gate_{i+1}
+                    const float send = odd ? acc[i] : acc[i + 1];
+                    const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
+                    const float g = (odd ? recv : acc[i]) * sa[i / 2];
+                    const float u = (odd ? acc[i + 1] : recv) * sa[i / 2];
+                    if (valid && i + odd < ncol) *op = silu_mul(g, u);
+                    op += 2 * (size_t)a.ldo;
                 }
             }
         }

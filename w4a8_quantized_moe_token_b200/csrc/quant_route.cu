@@ -455,7 +455,7 @@ __device__ __forceinline__ void load_chunk(const float* row, int len, int k0, Ch
     }
 }
 
-template <typename TIn>
+template <int kCache, typename TIn>
 __device__ __forceinline__ void quant_row_cta(const TIn* row, int len, int r, int RB, int8_t* __restrict__ act,
                                               float* __restrict__ s) {
     __shared__ float red[4];
@@ -463,11 +463,11 @@ __device__ __forceinline__ void quant_row_cta(const TIn* row, int len, int r, in
     const int nch = Kp / 16;
     const int G = Kp / kGroup;
     const int t = threadIdx.x;
-    Chunk16 cache[kRowCache];
+    Chunk16 cache[kCache];
     float amax = 0.f;
     if (row != nullptr) {
 #pragma unroll
-        for (int c = 0; c < kRowCache; ++c) {
+        for (int c = 0; c < kCache; ++c) {
             const int ci = t + c * 128;
             if (ci < nch) {
                 load_chunk(row, len, ci * 16, cache[c]);
@@ -475,7 +475,7 @@ __device__ __forceinline__ void quant_row_cta(const TIn* row, int len, int r, in
                 for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(cache[c].v[i]));
             }
         }
-        for (int ci = t + kRowCache * 128; ci < nch; ci += 128) {
+        for (int ci = t + kCache * 128; ci < nch; ci += 128) {
             Chunk16 tmp;
             load_chunk(row, len, ci * 16, tmp);
 #pragma unroll
@@ -499,7 +499,7 @@ __device__ __forceinline__ void quant_row_cta(const TIn* row, int len, int r, in
         *reinterpret_cast<uint4*>(act + act_offset(r, ci * 16, G, RB)) = make_uint4(out[0], out[1], out[2], out[3]);
     };
 #pragma unroll
-    for (int c = 0; c < kRowCache; ++c) {
+    for (int c = 0; c < kCache; ++c) {
         const int ci = t + c * 128;
         if (ci < nch) {
             if (row == nullptr) {
@@ -509,7 +509,7 @@ __device__ __forceinline__ void quant_row_cta(const TIn* row, int len, int r, in
             emit(ci, cache[c]);
         }
     }
-    for (int ci = t + kRowCache * 128; ci < nch; ci += 128) {
+    for (int ci = t + kCache * 128; ci < nch; ci += 128) {
         Chunk16 tmp;
         if (row != nullptr) load_chunk(row, len, ci * 16, tmp);
         else {
@@ -521,24 +521,93 @@ __device__ __forceinline__ void quant_row_cta(const TIn* row, int len, int r, in
     if (t == 0) s[r] = sc;
 }
 
-// x rows (bf16) -> INT8 rows in expert-grouped order
-__global__ void __launch_bounds__(128) act_scatter_kernel(const uint16_t* __restrict__ x, int H, int k,
-                                                          const int* __restrict__ row_src,
-                                                          const int* __restrict__ poffs, int E, int RB,
+// x rows (bf16) -> INT8 rows in expert-grouped order.  CTA t < T quantises token t
+// once (one read of x) and writes the codes to each of its k grouped rows; CTA T + e
+// writes zero codes and scale 0 into the pad rows of expert e.
+__global__ void __launch_bounds__(128) act_scatter_kernel(const uint16_t* __restrict__ x, int T, int H, int k,
+                                                          const int* __restrict__ inv,
+                                                          const int* __restrict__ offs,
+                                                          const int* __restrict__ poffs, int RB,
                                                           int8_t* __restrict__ act, float* __restrict__ s) {
-    const int r = blockIdx.x;
-    if (r >= __ldg(poffs + E)) return;
-    const int src = row_src[r];
-    quant_row_cta<uint16_t>(src < 0 ? nullptr : x + (size_t)(src / k) * H, H, r, RB, act, s);
+    const int Kp = round_up(H, kGroup);
+    const int nch = Kp / 16;
+    const int G = Kp / kGroup;
+    const int t = threadIdx.x;
+    if ((int)blockIdx.x >= T) {
+        const int e = (int)blockIdx.x - T;
+        const int r0 = __ldg(poffs + e) + (__ldg(offs + e + 1) - __ldg(offs + e));
+        const int r1 = __ldg(poffs + e + 1);
+        for (int r = r0; r < r1; ++r) {
+            for (int ci = t; ci < nch; ci += 128)
+                *reinterpret_cast<uint4*>(act + act_offset(r, ci * 16, G, RB)) = make_uint4(0u, 0u, 0u, 0u);
+            if (t == 0) s[r] = 0.f;
+        }
+        return;
+    }
+    const int tok = blockIdx.x;
+    const uint16_t* row = x + (size_t)tok * H;
+    __shared__ int dst[32];
+    __shared__ float red[4];
+    if (t < k) dst[t] = __ldg(inv + (size_t)tok * k + t);
+    Chunk16 cache[kRowCache];
+    float amax = 0.f;
+#pragma unroll
+    for (int c = 0; c < kRowCache; ++c) {
+        const int ci = t + c * 128;
+        if (ci < nch) {
+            load_chunk(row, H, ci * 16, cache[c]);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(cache[c].v[i]));
+        }
+    }
+    for (int ci = t + kRowCache * 128; ci < nch; ci += 128) {
+        Chunk16 tmp;
+        load_chunk(row, H, ci * 16, tmp);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(tmp.v[i]));
+    }
+    amax = warp_max(amax);
+    if ((t & 31) == 0) red[t >> 5] = amax;
+    __syncthreads();
+    amax = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+    const float sc = __fdiv_rn(amax, 127.0f);
+    auto emit = [&](int ci, const Chunk16& c) {
+        uint32_t out[4] = {0u, 0u, 0u, 0u};
+        if (amax > 0.f) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const uint32_t q = (uint32_t)(quant_i8(c.v[i], sc) & 0xFF);
+                out[i >> 2] |= q << (8 * (i & 3));
+            }
+        }
+        const uint4 o = make_uint4(out[0], out[1], out[2], out[3]);
+        for (int j = 0; j < k; ++j) {
+            const int r = dst[j];
+            if (r >= 0) *reinterpret_cast<uint4*>(act + act_offset(r, ci * 16, G, RB)) = o;
+        }
+    };
+#pragma unroll
+    for (int c = 0; c < kRowCache; ++c) {
+        const int ci = t + c * 128;
+        if (ci < nch) emit(ci, cache[c]);
+    }
+    for (int ci = t + kRowCache * 128; ci < nch; ci += 128) {
+        Chunk16 tmp;
+        load_chunk(row, H, ci * 16, tmp);
+        emit(ci, tmp);
+    }
+    if (t < k && dst[t] >= 0) s[dst[t]] = sc;
 }
 
 // h rows (fp32, SwiGLU output of the up GEMM) -> INT8 rows for the down GEMM
+// (kCache chunks of 16 per thread stay in registers: 1 covers F <= 2048)
+template <int kCache>
 __global__ void __launch_bounds__(128) requant_kernel(const float* __restrict__ h, int ldh, int F,
                                                       const int* __restrict__ row_src, const int* __restrict__ poffs,
                                                       int E, int RB, int8_t* __restrict__ act, float* __restrict__ s) {
     const int r = blockIdx.x;
     if (r >= __ldg(poffs + E)) return;
-    quant_row_cta<float>(row_src[r] < 0 ? nullptr : h + (size_t)r * ldh, F, r, RB, act, s);
+    quant_row_cta<kCache, float>(row_src[r] < 0 ? nullptr : h + (size_t)r * ldh, F, r, RB, act, s);
 }
 
 // ---------------------------------------------------------------------------
@@ -663,17 +732,20 @@ cudaError_t launch_perm(const int32_t* ids, int nslots, int E, int tile_tokens, 
     return cudaGetLastError();
 }
 
-cudaError_t launch_act_scatter(const uint16_t* x, int H, int k, const int* row_src, const int* poffs, int E,
-                               int rows_cap, int rb, int8_t* act, float* s, cudaStream_t stream) {
-    if (rows_cap == 0) return cudaSuccess;
-    act_scatter_kernel<<<rows_cap, 128, 0, stream>>>(x, H, k, row_src, poffs, E, rb, act, s);
+cudaError_t launch_act_scatter(const uint16_t* x, int T, int H, int k, const int* inv, const int* offs,
+                               const int* poffs, int E, int rb, int8_t* act, float* s, cudaStream_t stream) {
+    if (T == 0) return cudaSuccess;
+    act_scatter_kernel<<<T + E, 128, 0, stream>>>(x, T, H, k, inv, offs, poffs, rb, act, s);
     return cudaGetLastError();
 }
 
 cudaError_t launch_requant(const float* h, int ldh, int F, const int* row_src, const int* poffs, int E,
                            int rows_cap, int rb, int8_t* act, float* s, cudaStream_t stream) {
     if (rows_cap == 0) return cudaSuccess;
-    requant_kernel<<<rows_cap, 128, 0, stream>>>(h, ldh, F, row_src, poffs, E, rb, act, s);
+    if (F <= 128 * 16)
+        requant_kernel<1><<<rows_cap, 128, 0, stream>>>(h, ldh, F, row_src, poffs, E, rb, act, s);
+    else
+        requant_kernel<kRowCache><<<rows_cap, 128, 0, stream>>>(h, ldh, F, row_src, poffs, E, rb, act, s);
     return cudaGetLastError();
 }
 

@@ -48,8 +48,8 @@ cudaError_t launch_perm(const int32_t* ids, int nslots, int E, int tile_tokens, 
 // capacity of the row-tile table for a layer: sum over experts of ceil(count / tile)
 // <= nslots / tile + E, with tiles of at least 16 rows
 inline int mt_tab_capacity(int nslots, int E) { return nslots / 16 + E + 1; }
-cudaError_t launch_act_scatter(const uint16_t* x, int H, int k, const int* row_src, const int* poffs, int E,
-                               int rows_cap, int rb, int8_t* act, float* s, cudaStream_t stream);
+cudaError_t launch_act_scatter(const uint16_t* x, int T, int H, int k, const int* inv, const int* offs,
+                               const int* poffs, int E, int rb, int8_t* act, float* s, cudaStream_t stream);
 cudaError_t launch_requant(const float* h, int ldh, int F, const int* row_src, const int* poffs, int E,
                            int rows_cap, int rb, int8_t* act, float* s, cudaStream_t stream);
 cudaError_t launch_combine(const float* y2, int H, const int* inv, const float* w, int T, int k, uint16_t* out,
