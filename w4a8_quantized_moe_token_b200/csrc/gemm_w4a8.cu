@@ -157,18 +157,25 @@ __device__ __forceinline__ void tmem_st16_const(uint32_t taddr, uint32_t v) {
         : "memory");
 }
 
-// acc0/acc1 += s * (x0 - 1.5*2^23, x1 - 1.5*2^23) with packed fp32x2 arithmetic
-__device__ __forceinline__ void fold2_magic(float& acc0, float& acc1, float s, uint32_t x0, uint32_t x1) {
-    asm("{\n\t.reg .b64 a, x, m, sc;\n\t"
-        "mov.b64 a, {%0, %1};\n\t"
-        "mov.b64 x, {%2, %3};\n\t"
-        "mov.b64 m, {%4, %4};\n\t"
-        "mov.b64 sc, {%5, %5};\n\t"
-        "sub.rn.f32x2 x, x, m;\n\t"
-        "fma.rn.f32x2 a, sc, x, a;\n\t"
-        "mov.b64 {%0, %1}, a;\n\t}"
-        : "+f"(acc0), "+f"(acc1)
-        : "r"(x0), "r"(x1), "f"(kMagicF), "f"(s));
+// a packed pair of accumulators (low word: even column) += sc * (x - 1.5*2^23) with
+// fp32x2 arithmetic: acc2 += sc2 * (x - m2), sc2 and m2 holding the value twice
+__device__ __forceinline__ void fold2_packed(uint64_t& acc2, uint64_t sc2, uint64_t m2, uint32_t x0, uint32_t x1) {
+    asm("{\n\t.reg .b64 x;\n\t"
+        "mov.b64 x, {%1, %2};\n\t"
+        "sub.rn.f32x2 x, x, %3;\n\t"
+        "fma.rn.f32x2 %0, %4, x, %0;\n\t}"
+        : "+l"(acc2)
+        : "r"(x0), "r"(x1), "l"(m2), "l"(sc2));
+}
+
+__device__ __forceinline__ uint64_t splat2(float v) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %1};" : "=l"(r) : "f"(v));
+    return r;
+}
+
+__device__ __forceinline__ void unpack2(uint64_t p, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(p));
 }
 
 __device__ __forceinline__ float silu_mul(float g, float u) { return __fdividef(g, 1.0f + __expf(-g)) * u; }
@@ -366,10 +373,10 @@ __global__ void __launch_bounds__(C::kThreads, 1) gemm_w4a8_kernel(const GemmArg
         bool ok = true;
         for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
             const Item it = decode_item<BN>(u, a);
-            const int nb = round_up(it.nrows, 16);
-            float acc[kCW];
+            uint64_t acc2[kCW / 2];  // column pairs, packed fp32x2
 #pragma unroll
-            for (int i = 0; i < kCW; ++i) acc[i] = 0.f;
+            for (int i = 0; i < kCW / 2; ++i) acc2[i] = 0ull;
+            const uint64_t m2 = splat2(kMagicF);
             const int n_out = (a.mode == 1) ? -1 : it.nt * kTileRows + r;
             int g = 0;
             while (g < G) {
@@ -378,14 +385,16 @@ __global__ void __launch_bounds__(C::kThreads, 1) gemm_w4a8_kernel(const GemmArg
                     const int b = j % ND;
                     // the converters publish the step's scales well before its MMAs finish
                     if (!wait_bar(SCFULL_BAR(j % kNSC), (j / kNSC) & 1u, abort_flag, a.err)) { ok = false; break; }
-                    const float sc = sc_ring[(j % kNSC) * kTileRows + r];
+                    const uint64_t sc2 = splat2(sc_ring[(j % kNSC) * kTileRows + r]);
                     if (!wait_bar(DFULL_BAR(b), (j / ND) & 1u, abort_flag, a.err)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t taddr = tmem_base + lane_base + C::kDCol0 + (uint32_t)b * BN + col0;
                     // batches of kLdB columns: kLdB/16 loads and one wait; the accumulator
                     // columns get their constant back and the buffer is released to the MMA
                     // warps before the fold, which then runs from registers (the partials
-                    // instance keeps its batches small so that it needs no spill)
+                    // instance keeps its batches small so that it needs no spill).  Columns
+                    // past the tile's tokens are never written by the MMAs: they hold the
+                    // constant, so they read as partial 0 and need no test.
                     constexpr int kLdB = kPartials ? 16 : (kCW < 64 ? kCW : 64);
                     constexpr int kNB = kCW / kLdB;
 #pragma unroll
@@ -394,12 +403,10 @@ __global__ void __launch_bounds__(C::kThreads, 1) gemm_w4a8_kernel(const GemmArg
                         uint32_t v[kLdB];
 #pragma unroll
                         for (int c = 0; c < kLdB / 16; ++c)
-                            if (m0 + c * 16 < nb)
-                                tmem_ld16(taddr + rd * kLdB + c * 16, *reinterpret_cast<uint32_t(*)[16]>(&v[c * 16]));
+                            tmem_ld16(taddr + rd * kLdB + c * 16, *reinterpret_cast<uint32_t(*)[16]>(&v[c * 16]));
                         tmem_ld_wait();
 #pragma unroll
-                        for (int c = 0; c < kLdB / 16; ++c)
-                            if (m0 + c * 16 < nb) tmem_st16_const(taddr + rd * kLdB + c * 16, kMagicBits);
+                        for (int c = 0; c < kLdB / 16; ++c) tmem_st16_const(taddr + rd * kLdB + c * 16, kMagicBits);
                         if (rd == kNB - 1) {
                             tmem_st_wait();
                             tc_fence_before();
@@ -414,19 +421,17 @@ __global__ void __launch_bounds__(C::kThreads, 1) gemm_w4a8_kernel(const GemmArg
                                 if (m0 + i < it.nrows) pp[i * pstride] = (int32_t)(v[i] - kMagicBits);
                         }
 #pragma unroll
-                        for (int c = 0; c < kLdB / 16; ++c)
-                            if (m0 + c * 16 < nb) {
-#pragma unroll
-                                for (int i = 0; i < 16; i += 2)
-                                    fold2_magic(acc[rd * kLdB + c * 16 + i], acc[rd * kLdB + c * 16 + i + 1], sc,
-                                                v[c * 16 + i], v[c * 16 + i + 1]);
-                            }
+                        for (int i = 0; i < kLdB; i += 2)
+                            fold2_packed(acc2[(rd * kLdB + i) / 2], sc2, m2, v[i], v[i + 1]);
                     }
                     ++j;
                     ++g;
                 }
             }
             if (!ok) break;
+            float acc[kCW];
+#pragma unroll
+            for (int i = 0; i < kCW; i += 2) unpack2(acc2[i / 2], acc[i], acc[i + 1]);
             const float* sap = a.act_scale + it.row0 + col0;
             const int ncol = it.nrows - col0;
             if (a.mode != 1) {
