@@ -296,6 +296,18 @@ __global__ void __launch_bounds__(C::kThreads, 1) gemm_w4a8_kernel(const GemmArg
         const int cg = warp >> 2;         // converter group: takes the steps with j % NCG == cg
         const int r = threadIdx.x & 127;  // tile row = TMEM lane
         const int nsteps = ((total - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x) * G;
+        // The tensor-memory store of step j completes while step j + NCG is fetched and
+        // converted; step j is signalled just before step j + NCG's store.
+        int prev = -1;  // step stored but not yet signalled
+        auto signal = [&](int jp) {
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(CONV_BAR(jp % NA));
+                mbar_arrive(SCFULL_BAR(jp % kNSC));
+            }
+        };
         for (int j = cg; j < nsteps; j += C::NCG) {
             const int s = j % NS;
             const int x = j % NA;
@@ -306,8 +318,7 @@ __global__ void __launch_bounds__(C::kThreads, 1) gemm_w4a8_kernel(const GemmArg
 #pragma unroll
             for (int c = 0; c < 4; ++c) w[c] = *reinterpret_cast<const uint4*>(blk + code_chunk_offset(r, c));
             const int zp = (int)__half2float(reinterpret_cast<const __half*>(blk + kZpOff)[r]);
-            const int slot = j % kNSC;
-            sc_ring[slot * kTileRows + r] = __half2float(reinterpret_cast<const __half*>(blk + kScaleOff)[r]);
+            sc_ring[(j % kNSC) * kTileRows + r] = __half2float(reinterpret_cast<const __half*>(blk + kScaleOff)[r]);
             uint32_t v[32];
             {
                 // signed INT8 (code - zp): byte-wise (code + 128 - zp) ^ 128, no carries
@@ -323,15 +334,11 @@ __global__ void __launch_bounds__(C::kThreads, 1) gemm_w4a8_kernel(const GemmArg
                     }
                 }
             }
+            if (prev >= 0) signal(prev);
             tmem_st32(tmem_base + lane_base + C::kACol0 + (uint32_t)x * 32u, v);
-            tmem_st_wait();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(CONV_BAR(x));
-                mbar_arrive(SCFULL_BAR(slot));
-            }
+            prev = j;
         }
+        if (prev >= 0) signal(prev);
     } else if (warp >= C::kMmaWarp0) {
         // ---------------- MMA issue: warp mi takes the steps with j % 2 == mi ----------------
         const int mi = warp - C::kMmaWarp0;
@@ -369,6 +376,8 @@ __global__ void __launch_bounds__(C::kThreads, 1) gemm_w4a8_kernel(const GemmArg
         const int eh = (warp - C::kEpiWarp0) >> 2;  // epilogue warpgroup: columns [eh*kCW, eh*kCW + kCW)
         const int r = q * 32 + lane;                 // tile row = TMEM lane
         const int col0 = eh * kCW;
+        const int nsteps = ((total - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x) * G;
+        float sc4[4] = {0.f, 0.f, 0.f, 0.f};
         uint32_t j = 0;
         bool ok = true;
         for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
@@ -378,54 +387,69 @@ __global__ void __launch_bounds__(C::kThreads, 1) gemm_w4a8_kernel(const GemmArg
             for (int i = 0; i < kCW / 2; ++i) acc2[i] = 0ull;
             const uint64_t m2 = splat2(kMagicF);
             const int n_out = (a.mode == 1) ? -1 : it.nt * kTileRows + r;
-            int g = 0;
-            while (g < G) {
-                {
-                    // wide tiles: one step per pass, magic-constant accumulators
-                    const int b = j % ND;
-                    // the converters publish the step's scales well before its MMAs finish
-                    if (!wait_bar(SCFULL_BAR(j % kNSC), (j / kNSC) & 1u, abort_flag, a.err)) { ok = false; break; }
-                    const uint64_t sc2 = splat2(sc_ring[(j % kNSC) * kTileRows + r]);
-                    if (!wait_bar(DFULL_BAR(b), (j / ND) & 1u, abort_flag, a.err)) { ok = false; break; }
-                    tc_fence_after();
-                    const uint32_t taddr = tmem_base + lane_base + C::kDCol0 + (uint32_t)b * BN + col0;
-                    // batches of kLdB columns: kLdB/16 loads and one wait; the accumulator
-                    // columns get their constant back and the buffer is released to the MMA
-                    // warps before the fold, which then runs from registers (the partials
-                    // instance keeps its batches small so that it needs no spill).  Columns
-                    // past the tile's tokens are never written by the MMAs: they hold the
-                    // constant, so they read as partial 0 and need no test.
-                    constexpr int kLdB = kPartials ? 16 : (kCW < 64 ? kCW : 64);
-                    constexpr int kNB = kCW / kLdB;
+            for (int g = 0; g < G; ++g, ++j) {
+                const int b = j % ND;
+                // the scales come in blocks of four steps: one wait on the last step of
+                // the block (of each converter group, which work in step order) covers all four
+                if ((j & 3u) == 0) {
+                    const uint32_t jl = min(j + 3u, (uint32_t)nsteps - 1u);
 #pragma unroll
-                    for (int rd = 0; rd < kNB; ++rd) {
-                        const int m0 = col0 + rd * kLdB;
-                        uint32_t v[kLdB];
+                    for (int d = 0; d < C::NCG; ++d) {
+                        const uint32_t jj = jl - (uint32_t)d;
+                        if (jj >= j && !wait_bar(SCFULL_BAR(jj % kNSC), (jj / kNSC) & 1u, abort_flag, a.err)) ok = false;
+                    }
+                    if (!ok) break;
 #pragma unroll
-                        for (int c = 0; c < kLdB / 16; ++c)
-                            tmem_ld16(taddr + rd * kLdB + c * 16, *reinterpret_cast<uint32_t(*)[16]>(&v[c * 16]));
+                    for (int d = 0; d < 4; ++d) sc4[d] = sc_ring[((j + d) % kNSC) * kTileRows + r];
+                } else {
+#pragma unroll
+                    for (int d = 0; d < 3; ++d) sc4[d] = sc4[d + 1];
+                }
+                const uint64_t sc2 = splat2(sc4[0]);
+                if (!wait_bar(DFULL_BAR(b), (j / ND) & 1u, abort_flag, a.err)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t taddr = tmem_base + lane_base + C::kDCol0 + (uint32_t)b * BN + col0;
+                // Columns past the tile's tokens are never written by the MMAs: they hold
+                // the constant, so they read as partial 0 and need no test.
+                if constexpr (!kPartials) {
+                    // two loads of the warp's columns, the constant goes back, the buffer is
+                    // released to the MMA warps, then the fold runs from registers
+                    static_assert(kCW == 64, "64 columns per epilogue thread");
+                    uint32_t v[64];
+                    tmem_ld32(taddr, v);
+                    tmem_ld32(taddr + 32, v + 32);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) tmem_st16_const(taddr + c * 16, kMagicBits);
+                    tmem_st_wait();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(DEMPTY_BAR(b));
+#pragma unroll
+                    for (int i = 0; i < 64; i += 2) fold2_packed(acc2[i / 2], sc2, m2, v[i], v[i + 1]);
+                } else {
+                    // the INT32-partials output: batches of 16 columns (no spill)
+#pragma unroll
+                    for (int rd = 0; rd < kCW / 16; ++rd) {
+                        const int m0 = col0 + rd * 16;
+                        uint32_t v[16];
+                        tmem_ld16(taddr + rd * 16, v);
                         tmem_ld_wait();
-#pragma unroll
-                        for (int c = 0; c < kLdB / 16; ++c) tmem_st16_const(taddr + rd * kLdB + c * 16, kMagicBits);
-                        if (rd == kNB - 1) {
-                            tmem_st_wait();
-                            tc_fence_before();
-                            __syncwarp();
-                            if (lane == 0) mbar_arrive(DEMPTY_BAR(b));
-                        }
-                        if (kPartials && n_out < a.nvalid) {
+                        tmem_st16_const(taddr + rd * 16, kMagicBits);
+                        if (n_out < a.nvalid) {
                             int32_t* pp = a.partials + ((size_t)(it.row0 + m0) * a.nvalid + n_out) * G + g;
                             const size_t pstride = (size_t)a.nvalid * G;
 #pragma unroll
-                            for (int i = 0; i < kLdB; ++i)
+                            for (int i = 0; i < 16; ++i)
                                 if (m0 + i < it.nrows) pp[i * pstride] = (int32_t)(v[i] - kMagicBits);
                         }
 #pragma unroll
-                        for (int i = 0; i < kLdB; i += 2)
-                            fold2_packed(acc2[(rd * kLdB + i) / 2], sc2, m2, v[i], v[i + 1]);
+                        for (int i = 0; i < 16; i += 2) fold2_packed(acc2[(rd * 16 + i) / 2], sc2, m2, v[i], v[i + 1]);
                     }
-                    ++j;
-                    ++g;
+                    tmem_st_wait();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(DEMPTY_BAR(b));
                 }
             }
             if (!ok) break;
