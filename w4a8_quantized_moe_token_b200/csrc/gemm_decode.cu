@@ -392,26 +392,39 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
                 }
             }
             if (!ok) break;
+            // token scales: all loads before the stores (the compiler may not move a load
+            // across a store it cannot prove disjoint)
             const float* sap = a.act_scale + it.row0;
-            if (a.mode != 1) {
-                if (n_out < a.nvalid) {
-                    float* op = a.out + (size_t)it.row0 * a.ldo + n_out;
+            float sa[BN];
 #pragma unroll
-                    for (int i = 0; i < BN; ++i)
-                        if (i < it.nrows) op[(size_t)i * a.ldo] = acc[i] * __ldg(sap + i);
-                }
-            } else {
-                // SwiGLU: even tile rows hold gate channel f, odd rows the matching up channel
-                const int f = it.nt * (kTileRows / 2) + (r >> 1);
-                const bool valid = ((r & 1) == 0) && f < a.nvalid;
-                float* op = a.out + (size_t)it.row0 * a.ldo + f;
+            for (int i = 0; i < BN; ++i) sa[i] = i < it.nrows ? __ldg(sap + i) : 0.f;
+            if (a.mode != 1) {
+                const bool valid = n_out < a.nvalid;
+                float* op = a.out + (size_t)it.row0 * a.ldo + (valid ? n_out : 0);
 #pragma unroll
                 for (int i = 0; i < BN; ++i) {
-                    if (i < it.nrows) {
-                        const float y = acc[i] * __ldg(sap + i);
-                        const float yo = __shfl_xor_sync(0xffffffffu, y, 1);
-                        if (valid) op[(size_t)i * a.ldo] = silu_mul(y, yo);
-                    }
+                    if (valid && i < it.nrows) *op = acc[i] * sa[i];
+                    op += a.ldo;
+                }
+            } else {
+                // SwiGLU: even tile rows hold gate channel f, odd rows the matching up
+                // channel.  Per pair of tokens (i, i+1) the lanes of a pair swap one value:
+                // the even lane finishes token i, the odd lane token i+1.
+                const int f = it.nt * (kTileRows / 2) + (r >> 1);
+                const int odd = r & 1;
+                const bool valid = f < a.nvalid;
+                float* op = a.out + (size_t)(it.row0 + odd) * a.ldo + f;
+#pragma unroll
+                for (int i = 0; i < BN; i += 2) {
+                    // even lane: own gate_i, needs the partner's up_i; odd lane: own up_{i+1},
+                    // needs the partner's gate_{i+1}
+                    const float send = odd ? acc[i] : acc[i + 1];
+                    const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
+                    const float si = odd ? sa[i + 1] : sa[i];
+                    const float g = (odd ? recv : acc[i]) * si;
+                    const float u = (odd ? acc[i + 1] : recv) * si;
+                    if (valid && i + odd < it.nrows) *op = silu_mul(g, u);
+                    op += 2 * (size_t)a.ldo;
                 }
             }
         }

@@ -459,12 +459,20 @@ __global__ void __launch_bounds__(C::kThreads, 1) gemm_w4a8_kernel(const GemmArg
             const float* sap = a.act_scale + it.row0 + col0;
             const int ncol = it.nrows - col0;
             if (a.mode != 1) {
+                // token scales in halves of 32, all loads of a half before its stores (the
+                // compiler may not move a load across a store it cannot prove disjoint)
                 const bool valid = n_out < a.nvalid;
                 float* op = a.out + (size_t)(it.row0 + col0) * a.ldo + (valid ? n_out : 0);
 #pragma unroll
-                for (int i = 0; i < kCW; ++i) {
-                    if (valid && i < ncol) *op = acc[i] * __ldg(sap + i);
-                    op += a.ldo;
+                for (int h0 = 0; h0 < kCW; h0 += 32) {
+                    float sa[32];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) sa[i] = h0 + i < ncol ? __ldg(sap + h0 + i) : 0.f;
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        if (valid && h0 + i < ncol) *op = acc[h0 + i] * sa[i];
+                        op += a.ldo;
+                    }
                 }
             } else {
                 // SwiGLU: even tile rows hold gate channel f, odd rows the matching up
