@@ -17,16 +17,14 @@
 //                        (contiguous in the packed layout) and one of its token rows
 //                        (contiguous in the 16-row-block activation layout);
 //   2 converter groups : (alternate steps) each thread expands one weight row's codes
-//                        to unsigned INT8 (raw 4-bit codes 0..15: a mask and a
-//                        multiply-high per 8 codes), stores them to a tensor-memory A
-//                        slot, publishes the row's scale and zero point, and sums each
-//                        token's 128 INT8 codes per group (S, with dp4a);
-//   2 MMA warps        : (alternate steps) per group 4 x tcgen05.mma.kind::i8 u8 x s8,
+//                        to signed INT8 (code - zp, byte-wise without carries), stores
+//                        them to a tensor-memory A slot and publishes the row's scales;
+//   2 MMA warps        : (both on every step, two groups each) per group 4 x
+//                        tcgen05.mma.kind::i8 s8 x s8,
 //                        M=128 weight rows, N=16 tokens, K=32, into the group's own
 //                        INT32 accumulator (preloaded with 1.5 * 2^23, see below);
-//   1 epilogue group   : reads the partials, removes the zero point exactly
-//                        (P = sum a*c - zp * S), acc += scale * P in fp32 (packed
-//                        fp32x2), then applies the token scale and stores.
+//   1 epilogue group   : reads the partials, acc += scale * P in fp32 (packed fp32x2),
+//                        then applies the token scale and stores.
 // The accumulators start at the bit pattern 0x4B400000 (1.5 * 2^23): the MMAs add
 // the partial (|P| < 2^22), so the bits read back as fp32 are exactly 1.5 * 2^23 + P,
 // and one packed fp32 subtraction yields P without an int -> float conversion.
@@ -46,7 +44,7 @@ constexpr int BN = 16;    // tokens per tile (one 16-row block)
 constexpr int NS = 4;     // shared-memory stages
 constexpr int NA = 2;     // tensor-memory A slots (GPS x 32 columns each)
 constexpr int ND = 4;     // tensor-memory accumulators (GPS x BN columns each)
-constexpr int NSC = 8;    // side-information ring slots (>= NA + ND)
+constexpr int NSC = 8;    // scale ring slots (>= NA + ND)
 constexpr int kAStage = GPS * kBlockBytes;  // weight blocks of one step
 constexpr int kBStage = GPS * BN * 128;     // token rows of one step
 constexpr int kACols = GPS * 32;
@@ -55,8 +53,9 @@ constexpr uint32_t kACol0 = 0;
 constexpr uint32_t kDCol0 = NA * kACols;
 constexpr uint32_t kTmemCols = 512;
 static_assert(kDCol0 + ND * kDCols <= kTmemCols, "tensor memory over-subscribed");
-static_assert(NSC >= NA + ND, "side-information ring too small");
+static_assert(NSC >= NA + ND, "scale ring too small");
 static_assert(NS % 2 == 0, "the two producers own the stages of one parity each");
+static_assert(GPS % 2 == 0, "the two MMA warps split the groups of a step");
 
 // warps: 0-7 converters (2 groups), 8-11 epilogue, 12 producer 0, 13-14 MMA, 15 producer 1
 constexpr int kThreads = 512;
@@ -68,10 +67,8 @@ static_assert(128 * (2 * kRegConv + kRegCtrl + kRegEpi) <= kRegLaunch * kThreads
 // shared memory carve-up (offsets from a 1024-aligned base)
 constexpr int kOffB = 0;
 constexpr int kOffA = kOffB + NS * kBStage;
-constexpr int kOffSc = kOffA + NS * kAStage;      // ring: fp32 scale   [NSC][GPS][128]
-constexpr int kOffZp = kOffSc + NSC * GPS * 128 * 4;  // ring: zero point  [NSC][GPS][128]
-constexpr int kOffS = kOffZp + NSC * GPS * 128 * 4;   // ring: group sums  [NSC][GPS][BN]
-constexpr int kOffBar = kOffS + NSC * GPS * BN * 4;
+constexpr int kOffSc = kOffA + NS * kAStage;  // ring: fp32 scale [NSC][GPS][128]
+constexpr int kOffBar = kOffSc + NSC * GPS * 128 * 4;
 // full[NS] empty[NS] conv[NA] aempty[NA] dfull[ND] dempty[ND] side[NSC] final[2]
 constexpr int kNumBars = 2 * NS + 2 * NA + 2 * ND + NSC + 2;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
@@ -131,24 +128,27 @@ __device__ __forceinline__ void tmem_st16_const(uint32_t taddr, uint32_t v) {
         : "memory");
 }
 
-// (a0, a1) += s * ((x0, x1) - 1.5*2^23 - zp * (S0, S1)), packed fp32x2.  With x the
-// bits of 1.5*2^23 + P_raw, the subtraction and the zero-point term are exact (all
-// values are integers below 2^24), so the fold sees the exact INT32 partial.
-__device__ __forceinline__ void fold2_zp(float& a0, float& a1, float s, float nzp, uint32_t x0, uint32_t x1, float s0,
-                                         float s1) {
-    asm("{\n\t.reg .b64 a, x, m, sc, z, sg;\n\t"
-        "mov.b64 a, {%0, %1};\n\t"
-        "mov.b64 x, {%2, %3};\n\t"
-        "mov.b64 m, {%4, %4};\n\t"
-        "mov.b64 sc, {%5, %5};\n\t"
-        "mov.b64 z, {%6, %6};\n\t"
-        "mov.b64 sg, {%7, %8};\n\t"
-        "sub.rn.f32x2 x, x, m;\n\t"
-        "fma.rn.f32x2 x, z, sg, x;\n\t"
-        "fma.rn.f32x2 a, sc, x, a;\n\t"
-        "mov.b64 {%0, %1}, a;\n\t}"
-        : "+f"(a0), "+f"(a1)
-        : "r"(x0), "r"(x1), "f"(kMagicF), "f"(s), "f"(nzp), "f"(s0), "f"(s1));
+// a packed pair of accumulators (low word: even column) += sc * (x - 1.5*2^23) with
+// fp32x2 arithmetic: acc2 += sc2 * (x - m2), sc2 and m2 holding the value twice.  With
+// x the bits of 1.5*2^23 + P, the subtraction is exact, so the fold sees the exact
+// INT32 partial.
+__device__ __forceinline__ void fold2_packed(uint64_t& acc2, uint64_t sc2, uint64_t m2, uint32_t x0, uint32_t x1) {
+    asm("{\n\t.reg .b64 x;\n\t"
+        "mov.b64 x, {%1, %2};\n\t"
+        "sub.rn.f32x2 x, x, %3;\n\t"
+        "fma.rn.f32x2 %0, %4, x, %0;\n\t}"
+        : "+l"(acc2)
+        : "r"(x0), "r"(x1), "l"(m2), "l"(sc2));
+}
+
+__device__ __forceinline__ uint64_t splat2(float v) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %1};" : "=l"(r) : "f"(v));
+    return r;
+}
+
+__device__ __forceinline__ void unpack2(uint64_t p, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(p));
 }
 
 __device__ __forceinline__ float silu_mul(float g, float u) { return __fdividef(g, 1.0f + __expf(-g)) * u; }
@@ -162,10 +162,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
     const int lane = threadIdx.x & 31;
 
     const uint8_t* smA = smem + kOffA;
-    const uint8_t* smB = smem + kOffB;
     float* sc_ring = reinterpret_cast<float*>(smem + kOffSc);
-    float* zp_ring = reinterpret_cast<float*>(smem + kOffZp);
-    float* s_ring = reinterpret_cast<float*>(smem + kOffS);
     const uint32_t sA = base_addr + kOffA, sB = base_addr + kOffB;
     const uint32_t bar0 = base_addr + kOffBar;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
@@ -174,14 +171,14 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
     if (threadIdx.x == 0) {
         for (int s = 0; s < NS; ++s) {
             mbar_init(FULL_BAR(s), 1);
-            mbar_init(EMPTY_BAR(s), 1);
+            mbar_init(EMPTY_BAR(s), 2);  // commits of both MMA warps
         }
         for (int x = 0; x < NA; ++x) {
             mbar_init(CONV_BAR(x), 4);
-            mbar_init(AEMPTY_BAR(x), 1);
+            mbar_init(AEMPTY_BAR(x), 2);
         }
         for (int b = 0; b < ND; ++b) {
-            mbar_init(DFULL_BAR(b), 1);
+            mbar_init(DFULL_BAR(b), 2);
             mbar_init(DEMPTY_BAR(b), 4);
         }
         for (int i = 0; i < NSC; ++i) mbar_init(SIDE_BAR(i), 4);
@@ -243,26 +240,33 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
             __syncwarp();
         } else {
             // ---------------- MMA issuers ----------------
+            // Both warps take every step, warp mi issuing the MMAs of groups 2mi and
+            // 2mi+1: the issue rate of tcgen05.mma is a per-thread limit, so splitting a
+            // step halves the time its A slot stays busy.  Each warp commits to the
+            // step's barriers (two arrivals each), also when it had no group to issue.
             const int mi = cw - 1;
             if (lane == 0) {
                 uint32_t j = 0;
                 bool ok = true;
-                const uint32_t idesc = idesc_i8(128, BN, false);
+                const uint32_t idesc = idesc_i8(128, BN);
                 for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
                     for (int t = 0; t < steps_per_item; ++t, ++j) {
-                        if ((int)(j & 1u) != mi) continue;
                         const int ng = min(GPS, G - t * GPS);
                         const int s = j % NS, x = j % NA, b = j % ND;
                         if (!wait_bar(CONV_BAR(x), (j / NA) & 1u, abort_flag, a.err)) { ok = false; break; }
                         if (!wait_bar(DEMPTY_BAR(b), ((j / ND) & 1u) ^ 1u, abort_flag, a.err)) { ok = false; break; }
                         tc_fence_after();
-                        for (int gq = 0; gq < ng; ++gq) {
-                            const uint32_t dt = tmem_base + kDCol0 + (uint32_t)(b * kDCols + gq * BN);
-                            const uint32_t at = tmem_base + kACol0 + (uint32_t)(x * kACols + gq * 32);
-                            const uint32_t sb = sB + s * kBStage + gq * BN * 128;
 #pragma unroll
-                            for (int kk = 0; kk < 4; ++kk)
-                                mma_i8_ts(dt, at + kk * 8, smem_desc_sw128(sb + kk * 32), idesc, 1u);
+                        for (int gh = 0; gh < GPS / 2; ++gh) {
+                            const int gq = mi * (GPS / 2) + gh;
+                            if (gq < ng) {
+                                const uint32_t dt = tmem_base + kDCol0 + (uint32_t)(b * kDCols + gq * BN);
+                                const uint32_t at = tmem_base + kACol0 + (uint32_t)(x * kACols + gq * 32);
+                                const uint32_t sb = sB + s * kBStage + gq * BN * 128;
+#pragma unroll
+                                for (int kk = 0; kk < 4; ++kk)
+                                    mma_i8_ts(dt, at + kk * 8, smem_desc_sw128(sb + kk * 32), idesc, 1u);
+                            }
                         }
                         tc_commit(EMPTY_BAR(s));
                         tc_commit(AEMPTY_BAR(x));
@@ -279,8 +283,6 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegConv));
         const int cg = warp >> 2;
         const int r = threadIdx.x & 127;
-        // group sums: this thread adds half (64 bytes) of token m's row in group gs
-        const int gs = r >> 5, m = (r & 31) >> 1, half = r & 1;
         uint32_t m28;
         asm volatile("mov.u32 %0, 0x10000000;" : "=r"(m28));  // x * 2^28 >> 32 = x >> 4, on the FMA pipe
         const int nsteps = ((total - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x) * steps_per_item;
@@ -295,8 +297,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
                 uint4 w[4];
 #pragma unroll
                 for (int c = 0; c < 4; ++c) w[c] = *reinterpret_cast<const uint4*>(blk + code_chunk_offset(r, c));
+                const int zp = (int)__half2float(reinterpret_cast<const __half*>(blk + kZpOff)[r]);
                 sc_ring[(slot * GPS + gq) * 128 + r] = __half2float(reinterpret_cast<const __half*>(blk + kScaleOff)[r]);
-                zp_ring[(slot * GPS + gq) * 128 + r] = __half2float(reinterpret_cast<const __half*>(blk + kZpOff)[r]);
+                // signed INT8 (code - zp): byte-wise (code + 128 - zp) ^ 128, no carries
+                const uint32_t nz = (uint32_t)(0x80 - zp) * 0x01010101u;
                 uint32_t v[32];
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
@@ -304,27 +308,11 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
 #pragma unroll
                     for (int qq = 0; qq < 4; ++qq) {
                         const int i = 4 * c + qq;  // word i holds K = 8i .. 8i+7 of the group
-                        v[2 * i] = xw[qq] & 0x0F0F0F0Fu;
-                        v[2 * i + 1] = __umulhi(xw[qq], m28) & 0x0F0F0F0Fu;
+                        v[2 * i] = ((xw[qq] & 0x0F0F0F0Fu) + nz) ^ 0x80808080u;
+                        v[2 * i + 1] = ((__umulhi(xw[qq], m28) & 0x0F0F0F0Fu) + nz) ^ 0x80808080u;
                     }
                 }
                 tmem_st32(tmem_base + lane_base + kACol0 + (uint32_t)(x * kACols + gq * 32), v);
-            }
-            if (gs < ng) {
-                // S[gs][m] = sum of token m's 128 INT8 codes of group gs (the swizzle only
-                // permutes the 16-byte chunks inside the row, so the row sum is unaffected)
-                const uint4* rowp = reinterpret_cast<const uint4*>(smB + s * kBStage + gs * BN * 128 + m * 128 + half * 64);
-                int sum = 0;
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const uint4 b4 = rowp[c];
-                    sum = __dp4a((int)b4.x, 0x01010101, sum);
-                    sum = __dp4a((int)b4.y, 0x01010101, sum);
-                    sum = __dp4a((int)b4.z, 0x01010101, sum);
-                    sum = __dp4a((int)b4.w, 0x01010101, sum);
-                }
-                sum += __shfl_xor_sync(0xffffffffu, sum, 1);
-                if (half == 0) s_ring[(slot * GPS + gs) * BN + m] = (float)sum;
             }
             tmem_st_wait();
             tc_fence_before();
@@ -342,9 +330,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
         bool ok = true;
         for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
             const Item it = decode_item(u, a);
-            float acc[BN];
+            uint64_t acc2[BN / 2];  // token pairs, packed fp32x2
 #pragma unroll
-            for (int i = 0; i < BN; ++i) acc[i] = 0.f;
+            for (int i = 0; i < BN / 2; ++i) acc2[i] = 0ull;
+            const uint64_t m2 = splat2(kMagicF);
             const int n_out = (a.mode == 1) ? -1 : it.nt * kTileRows + r;
             for (int t = 0; t < steps_per_item; ++t, ++j) {
                 const int ng = min(GPS, G - t * GPS);
@@ -368,30 +357,23 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
 #pragma unroll
                 for (int gq = 0; gq < GPS; ++gq) {
                     if (gq < ng) {
-                        const float sc = sc_ring[(slot * GPS + gq) * 128 + r];
-                        const float zpf = zp_ring[(slot * GPS + gq) * 128 + r];
-                        const float4* sp = reinterpret_cast<const float4*>(s_ring + (slot * GPS + gq) * BN);
-                        float sg[BN];
-#pragma unroll
-                        for (int i = 0; i < BN / 4; ++i) {
-                            const float4 f4 = sp[i];
-                            sg[4 * i] = f4.x; sg[4 * i + 1] = f4.y; sg[4 * i + 2] = f4.z; sg[4 * i + 3] = f4.w;
-                        }
+                        const uint64_t sc2 = splat2(sc_ring[(slot * GPS + gq) * 128 + r]);
                         if (a.partials != nullptr && n_out < a.nvalid) {
                             int32_t* pp = a.partials + ((size_t)it.row0 * a.nvalid + n_out) * G + t * GPS + gq;
                             const size_t pstride = (size_t)a.nvalid * G;
 #pragma unroll
                             for (int i = 0; i < BN; ++i)
-                                if (i < it.nrows)
-                                    pp[i * pstride] = (int32_t)(v[gq][i] - kMagicBits) - (int32_t)zpf * (int32_t)sg[i];
+                                if (i < it.nrows) pp[i * pstride] = (int32_t)(v[gq][i] - kMagicBits);
                         }
 #pragma unroll
-                        for (int i = 0; i < BN; i += 2)
-                            fold2_zp(acc[i], acc[i + 1], sc, -zpf, v[gq][i], v[gq][i + 1], sg[i], sg[i + 1]);
+                        for (int i = 0; i < BN; i += 2) fold2_packed(acc2[i / 2], sc2, m2, v[gq][i], v[gq][i + 1]);
                     }
                 }
             }
             if (!ok) break;
+            float acc[BN];
+#pragma unroll
+            for (int i = 0; i < BN; i += 2) unpack2(acc2[i / 2], acc[i], acc[i + 1]);
             // token scales: all loads before the stores (the compiler may not move a load
             // across a store it cannot prove disjoint)
             const float* sap = a.act_scale + it.row0;
