@@ -12,7 +12,7 @@
 // bandwidth; so one pipeline step here carries GPS = 4 consecutive K groups of a tile
 // (35 KB of weights, 16 MMAs), paying the synchronisation once per 4 groups.
 //
-// Roles (one persistent CTA per SM, 16 warps):
+// Roles (one persistent CTA per SM, 20 warps):
 //   2 producer warps   : (alternate steps) one 1-D bulk copy of the step's weight blocks
 //                        (contiguous in the packed layout) and one of its token rows
 //                        (contiguous in the 16-row-block activation layout);
@@ -23,8 +23,10 @@
 //                        tcgen05.mma.kind::i8 s8 x s8,
 //                        M=128 weight rows, N=16 tokens, K=32, into the group's own
 //                        INT32 accumulator (preloaded with 1.5 * 2^23, see below);
-//   1 epilogue group   : reads the partials, acc += scale * P in fp32 (packed fp32x2),
-//                        then applies the token scale and stores.
+//   2 epilogue groups  : each reads the partials of two of the step's groups and folds
+//                        acc += scale * P in fp32 (packed fp32x2); at the end of a tile
+//                        group 1 passes its sums to group 0, which applies the token
+//                        scale and stores.
 // The accumulators start at the bit pattern 0x4B400000 (1.5 * 2^23): the MMAs add
 // the partial (|P| < 2^22), so the bits read back as fp32 are exactly 1.5 * 2^23 + P,
 // and one packed fp32 subtraction yields P without an int -> float conversion.
@@ -57,20 +59,23 @@ static_assert(NSC >= NA + ND, "scale ring too small");
 static_assert(NS % 2 == 0, "the two producers own the stages of one parity each");
 static_assert(GPS % 2 == 0, "the two MMA warps split the groups of a step");
 
-// warps: 0-7 converters (2 groups), 8-11 epilogue, 12 producer 0, 13-14 MMA, 15 producer 1
-constexpr int kThreads = 512;
-constexpr int kEpiWarp0 = 8, kCtrlWarp0 = 12;
-constexpr int kRegLaunch = 128;  // 65536 / 512
-constexpr int kRegConv = 96, kRegCtrl = 48, kRegEpi = 200;
-static_assert(128 * (2 * kRegConv + kRegCtrl + kRegEpi) <= kRegLaunch * kThreads, "register split");
+// warps: 0-7 converters (2 groups), 8-15 epilogue (2 groups), 16 producer 0, 17-18 MMA,
+// 19 producer 1
+constexpr int kThreads = 640;
+constexpr int kEpiWarp0 = 8, kCtrlWarp0 = 16;
+constexpr int kRegLaunch = 96;  // 65536 / 640, rounded down to the allocation unit
+constexpr int kRegConv = 88, kRegCtrl = 48, kRegEpi = 128;
+static_assert(128 * (2 * kRegConv + kRegCtrl + 2 * kRegEpi) <= kRegLaunch * kThreads, "register split");
 
 // shared memory carve-up (offsets from a 1024-aligned base)
 constexpr int kOffB = 0;
 constexpr int kOffA = kOffB + NS * kBStage;
 constexpr int kOffSc = kOffA + NS * kAStage;  // ring: fp32 scale [NSC][GPS][128]
-constexpr int kOffBar = kOffSc + NSC * GPS * 128 * 4;
+constexpr int kOffX = kOffSc + NSC * GPS * 128 * 4;  // epilogue exchange: [2][128][BN] fp32
+constexpr int kOffBar = kOffX + 2 * 128 * BN * 4;
 // full[NS] empty[NS] conv[NA] aempty[NA] dfull[ND] dempty[ND] side[NSC] final[2]
-constexpr int kNumBars = 2 * NS + 2 * NA + 2 * ND + NSC + 2;
+// xfull[2] xempty[2]
+constexpr int kNumBars = 2 * NS + 2 * NA + 2 * ND + NSC + 2 + 4;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr int kSmemBytes = kOffMisc + 16 + 1024;
 static_assert(kSmemBytes <= 227 * 1024, "shared memory over-subscribed");
@@ -83,6 +88,8 @@ static_assert(kSmemBytes <= 227 * 1024, "shared memory over-subscribed");
 #define DEMPTY_BAR(b) (bar0 + 8u * (uint32_t)(2 * NS + 2 * NA + ND + (b)))
 #define SIDE_BAR(i) (bar0 + 8u * (uint32_t)(2 * NS + 2 * NA + 2 * ND + (i)))
 #define FINAL_BAR(m) (bar0 + 8u * (uint32_t)(2 * NS + 2 * NA + 2 * ND + NSC + (m)))
+#define XFULL_BAR(p) (bar0 + 8u * (uint32_t)(2 * NS + 2 * NA + 2 * ND + NSC + 2 + (p)))
+#define XEMPTY_BAR(p) (bar0 + 8u * (uint32_t)(2 * NS + 2 * NA + 2 * ND + NSC + 4 + (p)))
 
 struct Item {
     int e, nt, row0, nrows;
@@ -179,11 +186,15 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
         }
         for (int b = 0; b < ND; ++b) {
             mbar_init(DFULL_BAR(b), 2);
-            mbar_init(DEMPTY_BAR(b), 4);
+            mbar_init(DEMPTY_BAR(b), 8);  // the 8 epilogue warps
         }
         for (int i = 0; i < NSC; ++i) mbar_init(SIDE_BAR(i), 4);
         mbar_init(FINAL_BAR(0), 1);
         mbar_init(FINAL_BAR(1), 1);
+        for (int p = 0; p < 2; ++p) {
+            mbar_init(XFULL_BAR(p), 4);   // epilogue group 1 has written its sums
+            mbar_init(XEMPTY_BAR(p), 4);  // epilogue group 0 has read them
+        }
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -197,8 +208,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
     const uint32_t tmem_base = *tmem_slot;
     const int q = warp & 3;
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
-    const bool is_epi = warp >= kEpiWarp0 && warp < kCtrlWarp0;
-    if (is_epi) {
+    if (warp >= kEpiWarp0 && warp < kEpiWarp0 + 4) {
         for (int c = 0; c < ND * kDCols / 16; ++c) tmem_st16_const(tmem_base + lane_base + kDCol0 + c * 16, kMagicBits);
         tmem_st_wait();
     }
@@ -324,11 +334,18 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
         }
     } else {
         // ---------------- epilogue ----------------
+        // Two groups of 4 warps: group eh folds the step's K groups 2eh and 2eh+1 into
+        // its own sums; at the end of a tile group 1 hands its sums to group 0 through
+        // shared memory (double-buffered, with bounded mbarrier waits), and group 0
+        // adds them and stores the tile.
         asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegEpi));
+        const int eh = (warp - kEpiWarp0) >> 2;
         const int r = q * 32 + lane;
+        float* xbuf = reinterpret_cast<float*>(smem + kOffX);
         uint32_t j = 0;
+        uint32_t nit = 0;  // tiles done by this CTA
         bool ok = true;
-        for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
+        for (int u = blockIdx.x; u < total && ok; u += gridDim.x, ++nit) {
             const Item it = decode_item(u, a);
             uint64_t acc2[BN / 2];  // token pairs, packed fp32x2
 #pragma unroll
@@ -341,21 +358,22 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
                 if (!wait_bar(DFULL_BAR(b), (j / ND) & 1u, abort_flag, a.err)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t taddr = tmem_base + lane_base + kDCol0 + (uint32_t)(b * kDCols);
-                uint32_t v[GPS][BN];
+                uint32_t v[GPS / 2][BN];
 #pragma unroll
-                for (int gq = 0; gq < GPS; ++gq)
-                    if (gq < ng) tmem_ld16(taddr + gq * BN, v[gq]);
+                for (int gh = 0; gh < GPS / 2; ++gh)
+                    if (eh * (GPS / 2) + gh < ng) tmem_ld16(taddr + (eh * (GPS / 2) + gh) * BN, v[gh]);
                 tmem_ld_wait();
 #pragma unroll
-                for (int gq = 0; gq < GPS; ++gq)
-                    if (gq < ng) tmem_st16_const(taddr + gq * BN, kMagicBits);
+                for (int gh = 0; gh < GPS / 2; ++gh)
+                    if (eh * (GPS / 2) + gh < ng) tmem_st16_const(taddr + (eh * (GPS / 2) + gh) * BN, kMagicBits);
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(DEMPTY_BAR(b));
                 if (!wait_bar(SIDE_BAR(slot), (j / NSC) & 1u, abort_flag, a.err)) { ok = false; break; }
 #pragma unroll
-                for (int gq = 0; gq < GPS; ++gq) {
+                for (int gh = 0; gh < GPS / 2; ++gh) {
+                    const int gq = eh * (GPS / 2) + gh;
                     if (gq < ng) {
                         const uint64_t sc2 = splat2(sc_ring[(slot * GPS + gq) * 128 + r]);
                         if (a.partials != nullptr && n_out < a.nvalid) {
@@ -363,17 +381,39 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
                             const size_t pstride = (size_t)a.nvalid * G;
 #pragma unroll
                             for (int i = 0; i < BN; ++i)
-                                if (i < it.nrows) pp[i * pstride] = (int32_t)(v[gq][i] - kMagicBits);
+                                if (i < it.nrows) pp[i * pstride] = (int32_t)(v[gh][i] - kMagicBits);
                         }
 #pragma unroll
-                        for (int i = 0; i < BN; i += 2) fold2_packed(acc2[i / 2], sc2, m2, v[gq][i], v[gq][i + 1]);
+                        for (int i = 0; i < BN; i += 2) fold2_packed(acc2[i / 2], sc2, m2, v[gh][i], v[gh][i + 1]);
                     }
                 }
             }
             if (!ok) break;
+            const int xp = nit & 1;
+            const uint32_t xpar = (nit >> 1) & 1u;
+            float* xrow = xbuf + (xp * 128 + r) * BN;
+            if (eh == 1) {
+                // hand the sums to group 0 and go on with the next tile
+                if (!wait_bar(XEMPTY_BAR(xp), xpar ^ 1u, abort_flag, a.err)) { ok = false; break; }
+#pragma unroll
+                for (int i = 0; i < BN / 2; ++i) reinterpret_cast<uint64_t*>(xrow)[i] = acc2[i];
+                __syncwarp();
+                if (lane == 0) mbar_arrive(XFULL_BAR(xp));
+                continue;
+            }
+            if (!wait_bar(XFULL_BAR(xp), xpar, abort_flag, a.err)) { ok = false; break; }
             float acc[BN];
 #pragma unroll
-            for (int i = 0; i < BN; i += 2) unpack2(acc2[i / 2], acc[i], acc[i + 1]);
+            for (int i = 0; i < BN; i += 2) {
+                float o0, o1;
+                unpack2(reinterpret_cast<const uint64_t*>(xrow)[i / 2], o0, o1);
+                unpack2(acc2[i / 2], acc[i], acc[i + 1]);
+                acc[i] += o0;
+                acc[i + 1] += o1;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(XEMPTY_BAR(xp));
+
             // token scales: all loads before the stores (the compiler may not move a load
             // across a store it cannot prove disjoint)
             const float* sap = a.act_scale + it.row0;
@@ -427,6 +467,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
 #undef DEMPTY_BAR
 #undef SIDE_BAR
 #undef FINAL_BAR
+#undef XFULL_BAR
+#undef XEMPTY_BAR
 
 }  // namespace
 
