@@ -58,6 +58,9 @@ static_assert(kDCol0 + ND * kDCols <= kTmemCols, "tensor memory over-subscribed"
 static_assert(NSC >= NA + ND, "scale ring too small");
 static_assert(NS % 2 == 0, "the two producers own the stages of one parity each");
 static_assert(GPS % 2 == 0, "the two MMA warps split the groups of a step");
+// one "MMA of step j done" barrier per j % NS serves the stage ring, the A slots and
+// the accumulators: their rings must step together
+static_assert(ND == NS && NS % NA == 0, "shared completion ring");
 
 // warps: 0-7 converters (2 groups), 8-15 epilogue (2 groups), 16 producer 0, 17-18 MMA,
 // 19 producer 1
@@ -73,7 +76,7 @@ constexpr int kOffA = kOffB + NS * kBStage;
 constexpr int kOffSc = kOffA + NS * kAStage;  // ring: fp32 scale [NSC][GPS][128]
 constexpr int kOffX = kOffSc + NSC * GPS * 128 * 4;  // epilogue exchange: [2][128][BN] fp32
 constexpr int kOffBar = kOffX + 2 * 128 * BN * 4;
-// full[NS] empty[NS] conv[NA] aempty[NA] dfull[ND] dempty[ND] side[NSC] final[2]
+// full[NS] empty[NS] conv[NA] (unused: NA + ND) dempty[ND] side[NSC] final[2]
 // xfull[2] xempty[2]
 constexpr int kNumBars = 2 * NS + 2 * NA + 2 * ND + NSC + 2 + 4;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
@@ -83,8 +86,8 @@ static_assert(kSmemBytes <= 227 * 1024, "shared memory over-subscribed");
 #define FULL_BAR(s) (bar0 + 8u * (uint32_t)(s))
 #define EMPTY_BAR(s) (bar0 + 8u * (uint32_t)(NS + (s)))
 #define CONV_BAR(x) (bar0 + 8u * (uint32_t)(2 * NS + (x)))
-#define AEMPTY_BAR(x) (bar0 + 8u * (uint32_t)(2 * NS + NA + (x)))
-#define DFULL_BAR(b) (bar0 + 8u * (uint32_t)(2 * NS + 2 * NA + (b)))
+// (slots 2 NS + NA .. 2 NS + 2 NA + ND - 1 are unused: the MMA completion of a step is
+// the EMPTY barrier of its stage)
 #define DEMPTY_BAR(b) (bar0 + 8u * (uint32_t)(2 * NS + 2 * NA + ND + (b)))
 #define SIDE_BAR(i) (bar0 + 8u * (uint32_t)(2 * NS + 2 * NA + 2 * ND + (i)))
 #define FINAL_BAR(m) (bar0 + 8u * (uint32_t)(2 * NS + 2 * NA + 2 * ND + NSC + (m)))
@@ -178,14 +181,13 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
     if (threadIdx.x == 0) {
         for (int s = 0; s < NS; ++s) {
             mbar_init(FULL_BAR(s), 1);
-            mbar_init(EMPTY_BAR(s), 2);  // commits of both MMA warps
+            mbar_init(EMPTY_BAR(s), 2);  // MMA of step j (j % NS == s) done: both MMA warps commit
         }
         for (int x = 0; x < NA; ++x) {
             mbar_init(CONV_BAR(x), 4);
-            mbar_init(AEMPTY_BAR(x), 2);
+
         }
         for (int b = 0; b < ND; ++b) {
-            mbar_init(DFULL_BAR(b), 2);
             mbar_init(DEMPTY_BAR(b), 8);  // the 8 epilogue warps
         }
         for (int i = 0; i < NSC; ++i) mbar_init(SIDE_BAR(i), 4);
@@ -278,9 +280,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
                                     mma_i8_ts(dt, at + kk * 8, smem_desc_sw128(sb + kk * 32), idesc, 1u);
                             }
                         }
+                        // one commit tells the producer (stage s free), the converters (A
+                        // slot free) and the epilogue (accumulators ready) at once
                         tc_commit(EMPTY_BAR(s));
-                        tc_commit(AEMPTY_BAR(x));
-                        tc_commit(DFULL_BAR(b));
                     }
                 }
                 tc_commit(FINAL_BAR(mi));
@@ -301,7 +303,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
             const int ng = min(GPS, G - t * GPS);
             const int s = j % NS, x = j % NA, slot = j % NSC;
             if (!wait_bar(FULL_BAR(s), (j / NS) & 1u, abort_flag, a.err)) break;
-            if (!wait_bar(AEMPTY_BAR(x), ((j / NA) & 1u) ^ 1u, abort_flag, a.err)) break;
+            // A slot x was last read by the MMAs of step j - NA
+            if (j >= NA && !wait_bar(EMPTY_BAR((j - NA) % NS), ((j - NA) / NS) & 1u, abort_flag, a.err)) break;
             for (int gq = 0; gq < ng; ++gq) {
                 const uint8_t* blk = smA + s * kAStage + gq * kBlockBytes;
                 uint4 w[4];
@@ -355,7 +358,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
             for (int t = 0; t < steps_per_item; ++t, ++j) {
                 const int ng = min(GPS, G - t * GPS);
                 const int b = j % ND, slot = j % NSC;
-                if (!wait_bar(DFULL_BAR(b), (j / ND) & 1u, abort_flag, a.err)) { ok = false; break; }
+                if (!wait_bar(EMPTY_BAR(j % NS), (j / NS) & 1u, abort_flag, a.err)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t taddr = tmem_base + lane_base + kDCol0 + (uint32_t)(b * kDCols);
                 uint32_t v[GPS / 2][BN];
@@ -462,8 +465,6 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
 #undef FULL_BAR
 #undef EMPTY_BAR
 #undef CONV_BAR
-#undef AEMPTY_BAR
-#undef DFULL_BAR
 #undef DEMPTY_BAR
 #undef SIDE_BAR
 #undef FINAL_BAR
