@@ -84,6 +84,28 @@ def gemm_accounting(W):
             "kernel_bytes": {"gemm_dense": wb + M * padded(K) * 2 + M * N * 4.0, "act_quant": M * K * 2.0 + M * K}}
 
 
+def load_traffic(workload: str, kernel: str):
+    """DRAM bytes per launch of `kernel` on `workload` from a committed ncu capture
+    (profiles/dram_traffic.json), or None when there is none or when any source file
+    the kernel is built from has changed since the counters were taken."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "dram_traffic.json")) as f:
+            entry = json.load(f).get(workload)
+    except (OSError, ValueError):
+        return None
+    if not entry or entry.get("kernel") != kernel:
+        return None
+    for rel, digest in entry.get("sources", {}).items():
+        try:
+            with open(os.path.join(ROOT, rel), "rb") as f:
+                if hashlib.sha256(f.read()).hexdigest() != digest:
+                    return None
+        except OSError:
+            return None
+    return float(entry["dram_bytes_per_launch"])
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -384,6 +406,7 @@ class OracleSample:
             qa, sa = O.quantize_act(self.x)
             return O.w4a8_linear(qa, sa, *self.qw)
         n = self.tokens if n is None else n
+        self._ensure_experts(n)  # a no-op once the sample's experts are quantised
         if self.logits is not None:
             O.route_topk(self.logits[:n], W.topk)
         return O.moe_forward(self.x[:n], self.ids[:n], self.w[:n], self.experts, W.E, W.F)
@@ -536,7 +559,7 @@ def main(argv=None):
     else:
         roof = {"bound": "hbm", "achieved": byt / (per_launch_ms / 1e3) / 1e9, "peak": hbm, "unit": "GB/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = None
+    roof["traffic"] = load_traffic(W.name, dom)
     roof["kernel"] = dom
     roof["peak_source"] = (f"{peaks['source']}: " + ("MEASURED_PEAKS hbm_gbs" if roof["bound"] == "hbm" else
                            "bf16_tflops x 2 (nominal int8/bf16 ratio)"))
