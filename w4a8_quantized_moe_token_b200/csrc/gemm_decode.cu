@@ -17,13 +17,16 @@
 //                        (contiguous in the packed layout) and one of its token rows
 //                        (contiguous in the 16-row-block activation layout);
 //   2 converter groups : (alternate steps) each thread expands one weight row's codes
-//                        to signed INT8 (code - zp, byte-wise without carries), stores
-//                        them to a tensor-memory A slot and publishes the row's scales;
+//                        to unsigned INT8 (the raw 4-bit codes: a mask and a
+//                        multiply-high per 8 codes), stores them to a tensor-memory A
+//                        slot, publishes the row's scale and zero point, and sums each
+//                        token's 128 INT8 codes per group (S, with dp4a);
 //   2 MMA warps        : (both on every step, two groups each) per group 4 x
-//                        tcgen05.mma.kind::i8 s8 x s8,
+//                        tcgen05.mma.kind::i8 u8 x s8,
 //                        M=128 weight rows, N=16 tokens, K=32, into the group's own
 //                        INT32 accumulator (preloaded with 1.5 * 2^23, see below);
-//   2 epilogue groups  : each reads the partials of two of the step's groups and folds
+//   2 epilogue groups  : each reads the partials of two of the step's groups, removes
+//                        the zero point exactly (P = sum a*c - zp * S) and folds
 //                        acc += scale * P in fp32 (packed fp32x2); at the end of a tile
 //                        group 1 passes its sums to group 0, which applies the token
 //                        scale and stores.
@@ -73,8 +76,10 @@ static_assert(128 * (2 * kRegConv + kRegCtrl + 2 * kRegEpi) <= kRegLaunch * kThr
 // shared memory carve-up (offsets from a 1024-aligned base)
 constexpr int kOffB = 0;
 constexpr int kOffA = kOffB + NS * kBStage;
-constexpr int kOffSc = kOffA + NS * kAStage;  // ring: fp32 scale [NSC][GPS][128]
-constexpr int kOffX = kOffSc + NSC * GPS * 128 * 4;  // epilogue exchange: [2][128][BN] fp32
+constexpr int kOffSc = kOffA + NS * kAStage;          // ring: fp32 scale       [NSC][GPS][128]
+constexpr int kOffZp = kOffSc + NSC * GPS * 128 * 4;  // ring: fp32 zero point  [NSC][GPS][128]
+constexpr int kOffS = kOffZp + NSC * GPS * 128 * 4;   // ring: token group sums [NSC][GPS][BN]
+constexpr int kOffX = kOffS + NSC * GPS * BN * 4;     // epilogue exchange: [2][128][BN] fp32
 constexpr int kOffBar = kOffX + 2 * 128 * BN * 4;
 // full[NS] empty[NS] conv[NA] (unused: NA + ND) dempty[ND] side[NSC] final[2]
 // xfull[2] xempty[2]
@@ -138,17 +143,26 @@ __device__ __forceinline__ void tmem_st16_const(uint32_t taddr, uint32_t v) {
         : "memory");
 }
 
-// a packed pair of accumulators (low word: even column) += sc * (x - 1.5*2^23) with
-// fp32x2 arithmetic: acc2 += sc2 * (x - m2), sc2 and m2 holding the value twice.  With
-// x the bits of 1.5*2^23 + P, the subtraction is exact, so the fold sees the exact
-// INT32 partial.
-__device__ __forceinline__ void fold2_packed(uint64_t& acc2, uint64_t sc2, uint64_t m2, uint32_t x0, uint32_t x1) {
+// a packed pair of accumulators (low word: even token) += sc * P with the zero point
+// removed, in fp32x2 arithmetic: acc2 += sc2 * ((x - m2) + nzp2 * s2), where x holds
+// the bits of 1.5*2^23 + sum a*c, m2 = 1.5*2^23 twice, nzp2 = -zp twice and s2 the two
+// tokens' code sums S; all values are integers below 2^24, so P = sum a*c - zp*S comes
+// out exact
+__device__ __forceinline__ void fold2_packed_zp(uint64_t& acc2, uint64_t sc2, uint64_t m2, uint64_t nzp2, uint64_t s2,
+                                                uint32_t x0, uint32_t x1) {
     asm("{\n\t.reg .b64 x;\n\t"
         "mov.b64 x, {%1, %2};\n\t"
         "sub.rn.f32x2 x, x, %3;\n\t"
-        "fma.rn.f32x2 %0, %4, x, %0;\n\t}"
+        "fma.rn.f32x2 x, %4, %5, x;\n\t"
+        "fma.rn.f32x2 %0, %6, x, %0;\n\t}"
         : "+l"(acc2)
-        : "r"(x0), "r"(x1), "l"(m2), "l"(sc2));
+        : "r"(x0), "r"(x1), "l"(m2), "l"(nzp2), "l"(s2), "l"(sc2));
+}
+
+__device__ __forceinline__ uint64_t pack2(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
 }
 
 __device__ __forceinline__ uint64_t splat2(float v) {
@@ -173,6 +187,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
 
     const uint8_t* smA = smem + kOffA;
     float* sc_ring = reinterpret_cast<float*>(smem + kOffSc);
+    float* zp_ring = reinterpret_cast<float*>(smem + kOffZp);
+    float* s_ring = reinterpret_cast<float*>(smem + kOffS);
+    const uint8_t* smB = smem + kOffB;
     const uint32_t sA = base_addr + kOffA, sB = base_addr + kOffB;
     const uint32_t bar0 = base_addr + kOffBar;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
@@ -260,7 +277,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
             if (lane == 0) {
                 uint32_t j = 0;
                 bool ok = true;
-                const uint32_t idesc = idesc_i8(128, BN);
+                const uint32_t idesc = idesc_i8(128, BN, false);  // u8 codes x s8 tokens
                 for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
                     for (int t = 0; t < steps_per_item; ++t, ++j) {
                         const int ng = min(GPS, G - t * GPS);
@@ -295,6 +312,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegConv));
         const int cg = warp >> 2;
         const int r = threadIdx.x & 127;
+        // group sums: this thread adds half (64 bytes) of token m's row in group gs
+        const int gs = r >> 5, m = (r & 31) >> 1, half = r & 1;
         uint32_t m28;
         asm volatile("mov.u32 %0, 0x10000000;" : "=r"(m28));  // x * 2^28 >> 32 = x >> 4, on the FMA pipe
         const int nsteps = ((total - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x) * steps_per_item;
@@ -310,10 +329,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
                 uint4 w[4];
 #pragma unroll
                 for (int c = 0; c < 4; ++c) w[c] = *reinterpret_cast<const uint4*>(blk + code_chunk_offset(r, c));
-                const int zp = (int)__half2float(reinterpret_cast<const __half*>(blk + kZpOff)[r]);
                 sc_ring[(slot * GPS + gq) * 128 + r] = __half2float(reinterpret_cast<const __half*>(blk + kScaleOff)[r]);
-                // signed INT8 (code - zp): byte-wise (code + 128 - zp) ^ 128, no carries
-                const uint32_t nz = (uint32_t)(0x80 - zp) * 0x01010101u;
+                zp_ring[(slot * GPS + gq) * 128 + r] = __half2float(reinterpret_cast<const __half*>(blk + kZpOff)[r]);
                 uint32_t v[32];
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
@@ -321,11 +338,27 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
 #pragma unroll
                     for (int qq = 0; qq < 4; ++qq) {
                         const int i = 4 * c + qq;  // word i holds K = 8i .. 8i+7 of the group
-                        v[2 * i] = ((xw[qq] & 0x0F0F0F0Fu) + nz) ^ 0x80808080u;
-                        v[2 * i + 1] = ((__umulhi(xw[qq], m28) & 0x0F0F0F0Fu) + nz) ^ 0x80808080u;
+                        v[2 * i] = xw[qq] & 0x0F0F0F0Fu;
+                        v[2 * i + 1] = __umulhi(xw[qq], m28) & 0x0F0F0F0Fu;
                     }
                 }
                 tmem_st32(tmem_base + lane_base + kACol0 + (uint32_t)(x * kACols + gq * 32), v);
+            }
+            if (gs < ng) {
+                // S[gs][m] = sum of token m's 128 INT8 codes of group gs (the swizzle only
+                // permutes the 16-byte chunks inside the row, so the row sum is unaffected)
+                const uint4* rowp = reinterpret_cast<const uint4*>(smB + s * kBStage + gs * BN * 128 + m * 128 + half * 64);
+                int sum = 0;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const uint4 b4 = rowp[c];
+                    sum = __dp4a((int)b4.x, 0x01010101, sum);
+                    sum = __dp4a((int)b4.y, 0x01010101, sum);
+                    sum = __dp4a((int)b4.z, 0x01010101, sum);
+                    sum = __dp4a((int)b4.w, 0x01010101, sum);
+                }
+                sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+                if (half == 0) s_ring[(slot * GPS + gs) * BN + m] = (float)sum;
             }
             tmem_st_wait();
             tc_fence_before();
@@ -378,16 +411,27 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
                 for (int gh = 0; gh < GPS / 2; ++gh) {
                     const int gq = eh * (GPS / 2) + gh;
                     if (gq < ng) {
+                        const float zpf = zp_ring[(slot * GPS + gq) * 128 + r];
                         const uint64_t sc2 = splat2(sc_ring[(slot * GPS + gq) * 128 + r]);
+                        const uint64_t nzp2 = splat2(-zpf);
+                        const float4* sp = reinterpret_cast<const float4*>(s_ring + (slot * GPS + gq) * BN);
+                        float sg[BN];
+#pragma unroll
+                        for (int i = 0; i < BN / 4; ++i) {
+                            const float4 f4 = sp[i];
+                            sg[4 * i] = f4.x; sg[4 * i + 1] = f4.y; sg[4 * i + 2] = f4.z; sg[4 * i + 3] = f4.w;
+                        }
                         if (a.partials != nullptr && n_out < a.nvalid) {
                             int32_t* pp = a.partials + ((size_t)it.row0 * a.nvalid + n_out) * G + t * GPS + gq;
                             const size_t pstride = (size_t)a.nvalid * G;
 #pragma unroll
                             for (int i = 0; i < BN; ++i)
-                                if (i < it.nrows) pp[i * pstride] = (int32_t)(v[gh][i] - kMagicBits);
+                                if (i < it.nrows)
+                                    pp[i * pstride] = (int32_t)(v[gh][i] - kMagicBits) - (int32_t)zpf * (int32_t)sg[i];
                         }
 #pragma unroll
-                        for (int i = 0; i < BN; i += 2) fold2_packed(acc2[i / 2], sc2, m2, v[gh][i], v[gh][i + 1]);
+                        for (int i = 0; i < BN; i += 2)
+                            fold2_packed_zp(acc2[i / 2], sc2, m2, nzp2, pack2(sg[i], sg[i + 1]), v[gh][i], v[gh][i + 1]);
                     }
                 }
             }
