@@ -34,7 +34,8 @@ its reason in the design notes):
   R11 softmax routing: top-k experts by logit (ties -> lower id), gate weight = the
       softmax probability over all E experts, not renormalised;
   R12 tokens inside an expert's segment keep their slot order (t * k + j ascending);
-  R14 h enters the requantisation as fp32.
+  R14 h enters the requantisation as fp32;
+  R18 symmetric INT4 variant: q clamped to [-7, 7], stored as code q + 8 with zero point 8.
 
 Parity status: every function below is pinned by tests/test_oracle_pins.py
 against values the pages print, closed forms, brute force or an independent
@@ -48,6 +49,8 @@ import numpy as np
 GROUP = 128  # [P2] §2.1: one scale and one zero point per 128 weights along K
 INT4_MAX = 15  # [P2] §2.2: 2^4 - 1
 INT8_QMAX = 127  # [P3] §2.1: 2^(b-1) - 1 for b = 8 (symmetric)
+INT4_SYM_QMAX = 7  # [P3] §2.1: 2^(b-1) - 1 for b = 4 (symmetric weights)
+INT4_SYM_ZP = 8  # the symmetric codes are stored as q + 8
 
 
 # --------------------------------------------------------------------------- #
@@ -105,6 +108,39 @@ def quantize_weights(w: np.ndarray):
         codes[:, g * GROUP:(g + 1) * GROUP] = np.clip(q, 0, INT4_MAX).astype(np.uint8)
         scale[:, g] = s16
         zp[:, g] = z.astype(np.float16)
+    return codes, scale, zp
+
+
+def quantize_weights_symmetric(w: np.ndarray):
+    """Group-wise symmetric INT4 of one weight matrix w [N][K] (the packer's
+    symmetric variant).
+
+    [P3] §2.1, symmetric form with b = 4, per group of 128 along K:
+        scale = max|weight| / (2^(4-1) - 1)
+        q     = clamp(round(weight / scale), -7, 7)
+    stored in the same format as the asymmetric scheme: code = q + 8 with a zero
+    point of 8, so (code - zp) * scale reproduces q * scale.  Readings R4-R6 as
+    above; R18: the clamp is the formula's own range [-(2^3 - 1), 2^3 - 1]; an fp16
+    scale that rounds to 0 is replaced by 1.
+
+    Returns codes uint8 [N][Kp] (values 1..15), scale float16 [N][G], zp float16 [N][G] (all 8).
+    """
+    w = pad_k(np.asarray(w, dtype=np.float32))
+    N, Kp = w.shape
+    G = Kp // GROUP
+    codes = np.zeros((N, Kp), dtype=np.uint8)
+    scale = np.zeros((N, G), dtype=np.float16)
+    zp = np.full((N, G), INT4_SYM_ZP, dtype=np.float16)
+    qmax = np.float32(INT4_SYM_QMAX)
+    for g in range(G):
+        v = w[:, g * GROUP:(g + 1) * GROUP]  # [N][128]
+        amax = np.abs(v).max(axis=1)
+        s16 = (amax / qmax).astype(np.float16)  # fp32 division, then fp16 RNE (R5, R6)
+        s16[s16 == 0] = np.float16(1.0)
+        sf = s16.astype(np.float32)
+        q = np.clip(np.rint(v / sf[:, None]), -qmax, qmax)  # R4, R6
+        codes[:, g * GROUP:(g + 1) * GROUP] = (q + INT4_SYM_ZP).astype(np.uint8)
+        scale[:, g] = s16
     return codes, scale, zp
 
 
@@ -297,11 +333,13 @@ def round_to_bf16(x: np.ndarray) -> np.ndarray:
 # the whole layer
 # --------------------------------------------------------------------------- #
 class QuantExpert:
-    """Quantised weights of one expert: up [2F][Hp] (gate|up rows) and down [H][Fp]."""
+    """Quantised weights of one expert: up [2F][Hp] (gate|up rows) and down [H][Fp]
+    (asymmetric INT4, or the symmetric variant)."""
 
-    def __init__(self, w_up: np.ndarray, w_down: np.ndarray):
-        self.up = quantize_weights(w_up)
-        self.down = quantize_weights(w_down)
+    def __init__(self, w_up: np.ndarray, w_down: np.ndarray, symmetric: bool = False):
+        quant = quantize_weights_symmetric if symmetric else quantize_weights
+        self.up = quant(w_up)
+        self.down = quant(w_down)
 
 
 def expert_forward(xq, xs, qe: QuantExpert, F: int, stages: dict | None = None):

@@ -125,6 +125,46 @@ def test_asym_int4_roundtrip_bound():
     assert codes.max() <= 15
 
 
+def test_sym_int4_closed_form():
+    # [P3] section 2.1 symmetric form with b = 4: scale = max|w| / 7.  Group max 0.7 ->
+    # scale fp16(0.1) = 0.0999755859375; 0.35 / 0.09998 = 3.5009 -> 4 (code 12);
+    # -0.35 -> -4 (code 4); 0.2 -> 2.0005 -> 2 (code 10); 0.7 -> 7.0017 -> 7 (code 15);
+    # -0.7 -> -7 (code 1); 0 -> 0 (code 8 = the zero point, exact)
+    w = _group_with([0.7, -0.35, 0.35, 0.2, 0.0, -0.7])
+    codes, scale, zp = O.quantize_weights_symmetric(w)
+    assert float(scale[0, 0]) == float(np.float16(np.float32(0.7) / np.float32(7.0)))
+    assert float(scale[0, 0]) == 0.0999755859375
+    assert float(zp[0, 0]) == 8.0
+    assert list(codes[0, :6]) == [15, 4, 12, 10, 8, 1]
+    deq = O.dequantize_weights(codes, scale, zp)
+    assert deq[0, 4] == 0.0 and np.all(deq[0, 6:] == 0.0)  # zero and the padding are exact
+    assert abs(deq[0, 3] - 0.2) <= float(scale[0, 0]) / 2
+
+
+def test_sym_int4_roundtrip_bound_and_symmetry():
+    rng = np.random.default_rng(11)
+    w = synth.bf16_round((rng.standard_normal((32, 256)) * 0.02).astype(np.float32))
+    codes, scale, zp = O.quantize_weights_symmetric(w)
+    assert codes.min() >= 1 and codes.max() <= 15 and np.all(zp == 8)
+    deq = O.dequantize_weights(codes, scale, zp)
+    sc = np.repeat(scale.astype(np.float64), 128, axis=1)
+    assert np.all(np.abs(w - deq) <= sc / 2 * (1 + 1e-3))
+    # the scheme is odd-symmetric: -w gives the mirrored codes and the same scales
+    c2, s2, _ = O.quantize_weights_symmetric(-w)
+    assert np.array_equal(s2, scale) and np.array_equal(c2.astype(int) - 8, -(codes.astype(int) - 8))
+    # the largest magnitude of every group lands on +-7
+    q = codes.astype(int) - 8
+    for g in range(2):
+        blk = w[:, g * 128:(g + 1) * 128]
+        i = np.abs(blk).argmax(axis=1)
+        assert np.all(np.abs(q[np.arange(32), g * 128 + i]) == 7)
+
+
+def test_sym_int4_degenerate_group():
+    codes, scale, zp = O.quantize_weights_symmetric(np.zeros((2, 128), np.float32))
+    assert np.all(scale == np.float16(1.0)) and np.all(zp == 8) and np.all(codes == 8)
+
+
 def test_quantize_uses_fp16_scale_for_codes():
     # reconstructing the codes from the stored fp16 scale + zp reproduces them (R5)
     rng = np.random.default_rng(3)
