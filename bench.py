@@ -177,9 +177,18 @@ def dev_bf16(a, device):
     return torch.from_numpy(synth.bf16_bits(a).view(np.int16)).view(torch.bfloat16).to(device)
 
 
+# weight scheme of the packer: asymmetric INT4 (default) or the symmetric variant
+SYMMETRIC = False
+
+
+def weights_desc():
+    return "int4 g128 sym (fp16 scale, zero point 8)" if SYMMETRIC else "int4 g128 asym (fp16 scale+zp)"
+
+
 def pack_experts(B, torch, W, seed, device):
     """Pack every expert's up (gate|up) and down weights on the device, one expert at a time."""
     E, H, F = W.E, W.H, W.F
+    flag = B.W4A8_PACK_SYMMETRIC if SYMMETRIC else 0
     up = B.empty_aligned(B.w4a8_packed_bytes(E, 2 * F, H, B.W4A8_LAYOUT_GATEUP), device)
     dn = B.empty_aligned(B.w4a8_packed_bytes(E, H, F, B.W4A8_LAYOUT_PLAIN), device)
     su = (up.numel() - 256) // E
@@ -189,7 +198,7 @@ def pack_experts(B, torch, W, seed, device):
     for which, (buf, tmp, stride, rows, cols, layout) in (("up", (up, tu, su, 2 * F, H, 1)),
                                                            ("down", (dn, td, sd, H, F, 0))):
         for e, w in synth.expert_weights_parallel(seed, E, which, rows, cols):
-            B.w4a8_pack_weights(dev_bf16(w, device), layout, tmp)
+            B.w4a8_pack_weights(dev_bf16(w, device), layout | flag, tmp)
             buf[256 + e * stride:256 + (e + 1) * stride].copy_(tmp[256:])
     torch.cuda.synchronize(device)
     return up, dn
@@ -299,7 +308,7 @@ class GemmStep:
         x, w = synth.dense_gemm_inputs(seed, W.M, W.K, W.N)
         self.x = dev_bf16(x, device)
         self.packed = B.empty_aligned(B.w4a8_packed_bytes(1, W.N, W.K, 0), device)
-        B.w4a8_pack_weights(dev_bf16(w, device), 0, self.packed)
+        B.w4a8_pack_weights(dev_bf16(w, device), B.W4A8_PACK_SYMMETRIC if SYMMETRIC else 0, self.packed)
         Kp = padded(W.K)
         self.q = torch.empty((W.M, Kp), dtype=torch.int8, device=device)
         self.s = torch.empty(W.M, dtype=torch.float32, device=device)
@@ -363,7 +372,7 @@ class OracleSample:
         self.O, self.W, self.seed = O, W, seed
         if W.kind == "gemm":
             x, w = synth.dense_gemm_inputs(seed, W.M, W.K, W.N)
-            self.x, self.qw = x, O.quantize_weights(w)
+            self.x, self.qw = x, (O.quantize_weights_symmetric if SYMMETRIC else O.quantize_weights)(w)
             self.tokens = W.M
             self.sample_desc = f"all {W.M} rows"
             return
@@ -392,7 +401,8 @@ class OracleSample:
             if e not in self.experts:
                 W = self.W
                 self.experts[e] = self.O.QuantExpert(synth.expert_weight(self.seed, e, "up", 2 * W.F, W.H),
-                                                     synth.expert_weight(self.seed, e, "down", W.H, W.F))
+                                                     synth.expert_weight(self.seed, e, "down", W.H, W.F),
+                                                     SYMMETRIC)
 
     def _time(self, n):
         self._ensure_experts(n)
@@ -458,7 +468,7 @@ def config_of(W, l2):
         c = {"workload": W.name, "M": W.M, "K": W.K, "N": W.N}
     else:
         c = {"workload": W.name, "T": W.T, "E": W.E, "topk": W.topk, "H": W.H, "F": W.F, "routing": W.routing}
-    c.update({"weights": "int4 g128 asym (fp16 scale+zp)", "acts": "int8 per-token", "l2": l2,
+    c.update({"weights": weights_desc(), "acts": "int8 per-token", "l2": l2,
               "parallelism": "replicas (no cross-GPU exchange)"})
     return c
 
@@ -473,7 +483,11 @@ def main(argv=None):
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--cpu-baseline-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--weights", choices=["asym", "sym"], default="asym",
+                    help="packer scheme: asymmetric INT4 (default) or the symmetric variant")
     args = ap.parse_args(argv)
+    global SYMMETRIC
+    SYMMETRIC = args.weights == "sym"
     W = synth.WORKLOADS[args.workload]
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

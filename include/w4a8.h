@@ -64,14 +64,29 @@ typedef enum {
  *                     GEMM's epilogue.                                            */
 enum { W4A8_LAYOUT_PLAIN = 0, W4A8_LAYOUT_GATEUP = 1 };
 
+/* Quantisation scheme flag, OR-ed into the `layout` argument of w4a8_packed_bytes
+ * and w4a8_pack_weights.
+ * Without it (the default): asymmetric INT4 per 128-wide group along K (the
+ *   «Kimi 2.7 Moe 从 4 bit 存储到 INT8 拆解» page, section 2.2): scale = (max - min)/15
+ *   over the group's range widened to contain 0, stored as fp16 and used for the
+ *   codes; zero_point = round(-min/scale); code = clamp(round(w/scale) + zp, 0, 15).
+ * W4A8_PACK_SYMMETRIC: symmetric INT4 (the LLM quantisation primer at
+ *   hotelren.com/news/5982361, section 2.1, with b = 4): scale = max|w|/7 (fp16),
+ *   q = clamp(round(w/scale), -7, 7), stored as code q + 8 with zero point 8.
+ * Both write the same tiled format, so w4a8_gemm and w4a8_moe_forward take either.
+ * Rounding is half to even; divisions are correctly rounded fp32; an fp16 scale
+ * that rounds to 0 is replaced by 1.                                              */
+enum { W4A8_PACK_SYMMETRIC = 0x100 };
+
 /* Bytes of a packed weight buffer for E matrices of shape [N][K] in `layout`:
  * a 256-byte header, then one 8704-byte block per (matrix, 128-row tile, 128-wide
  * K group): 8192 bytes of 4-bit codes, 128 fp16 scales, 128 fp16 zero points.
  * K is padded to a multiple of 128 (zero weights).  Returns 0 for invalid shapes
- * (GATEUP needs an even N). */
+ * (GATEUP needs an even N) or an unknown flag; W4A8_PACK_SYMMETRIC may be set. */
 size_t w4a8_packed_bytes(int E, int N, int K, int layout);
 
 /* Quantise and pack E weight matrices  (a1: the offline conversion step).
+ *   layout      : W4A8_LAYOUT_PLAIN or W4A8_LAYOUT_GATEUP, optionally | W4A8_PACK_SYMMETRIC.
  *   w_bf16      : device, bf16 [E][N][K], row-major (nn.Linear orientation).
  *   packed      : device, w4a8_packed_bytes(E,N,K,layout) bytes (256-B aligned),
  *                 the tiled layout consumed by w4a8_gemm / w4a8_moe_forward.

@@ -29,8 +29,10 @@ def bf16_to_f32(t):
 class Layer:
     """One synthetic MoE layer, packed on the GPU, with lazily quantised oracle experts."""
 
-    def __init__(self, T, E, k, H, F, routing="uniform", seed=0, zipf_s=1.1, outlier=0.0):
+    def __init__(self, T, E, k, H, F, routing="uniform", seed=0, zipf_s=1.1, outlier=0.0, symmetric=False):
         self.T, self.E, self.k, self.H, self.F, self.seed = T, E, k, H, F, seed
+        self.symmetric = symmetric
+        flag = B.W4A8_PACK_SYMMETRIC if symmetric else 0
         self.x = synth.activations(seed, T, H, outlier, 20.0)
         if routing == "softmax":
             self.logits = synth.router_logits(seed, T, E)
@@ -50,8 +52,8 @@ class Layer:
         tmp_up = B.empty_aligned(B.w4a8_packed_bytes(1, 2 * F, H, 1))
         tmp_dn = B.empty_aligned(B.w4a8_packed_bytes(1, H, F, 0))
         for e in range(E):
-            B.w4a8_pack_weights(dev_bf16(self.w_up(e)), B.W4A8_LAYOUT_GATEUP, tmp_up)
-            B.w4a8_pack_weights(dev_bf16(self.w_down(e)), B.W4A8_LAYOUT_PLAIN, tmp_dn)
+            B.w4a8_pack_weights(dev_bf16(self.w_up(e)), B.W4A8_LAYOUT_GATEUP | flag, tmp_up)
+            B.w4a8_pack_weights(dev_bf16(self.w_down(e)), B.W4A8_LAYOUT_PLAIN | flag, tmp_dn)
             self.packed_up[256 + e * up_stride:256 + (e + 1) * up_stride].copy_(tmp_up[256:])
             self.packed_down[256 + e * dn_stride:256 + (e + 1) * dn_stride].copy_(tmp_dn[256:])
         torch.cuda.synchronize()
@@ -69,7 +71,7 @@ class Layer:
     def experts(self):
         for e in np.unique(self.ids):
             if e not in self._experts:
-                self._experts[int(e)] = O.QuantExpert(self.w_up(int(e)), self.w_down(int(e)))
+                self._experts[int(e)] = O.QuantExpert(self.w_up(int(e)), self.w_down(int(e)), self.symmetric)
         return self._experts
 
     def run(self, use_router=False):
@@ -162,6 +164,16 @@ SMALL = [
 @pytest.mark.parametrize("T,E,k,H,F,routing", SMALL)
 def test_moe_small_stages_and_output(T, E, k, H, F, routing):
     L = Layer(T, E, k, H, F, routing, seed=T + E)
+    out = L.run()
+    check_stages(L, out)
+    ref = O.moe_forward(L.x, L.ids, L.w, L.experts(), E, F)
+    assert_close(out, ref, what="out")
+
+
+@pytest.mark.parametrize("T,E,k,H,F,routing", [(300, 4, 2, 512, 256, "uniform"), (64, 32, 4, 256, 256, "zipf")])
+def test_moe_symmetric_weights_stages_and_output(T, E, k, H, F, routing):
+    """The symmetric INT4 variant of the packer through the whole layer (wide and decode tiles)."""
+    L = Layer(T, E, k, H, F, routing, seed=T + E + 1, symmetric=True)
     out = L.run()
     check_stages(L, out)
     ref = O.moe_forward(L.x, L.ids, L.w, L.experts(), E, F)

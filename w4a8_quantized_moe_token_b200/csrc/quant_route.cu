@@ -35,9 +35,10 @@ __device__ __forceinline__ float warp_sum(float v) {
 // a1: weight quantisation + packing.  One block per (group g, tile t, matrix e);
 // thread r quantises tiled row r's 128 weights of group g.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(128) pack_kernel(const uint16_t* __restrict__ w, int N, int K, int layout, int NT,
-                                                   int G, uint8_t* __restrict__ blocks, uint8_t* __restrict__ codes_out,
-                                                   uint16_t* __restrict__ scale_out, uint16_t* __restrict__ zp_out) {
+__global__ void __launch_bounds__(128) pack_kernel(const uint16_t* __restrict__ w, int N, int K, int layout, int sym,
+                                                   int NT, int G, uint8_t* __restrict__ blocks,
+                                                   uint8_t* __restrict__ codes_out, uint16_t* __restrict__ scale_out,
+                                                   uint16_t* __restrict__ zp_out) {
     const int g = blockIdx.x, t = blockIdx.y, e = blockIdx.z;
     const int r = threadIdx.x;
     int src;
@@ -74,26 +75,44 @@ __global__ void __launch_bounds__(128) pack_kernel(const uint16_t* __restrict__ 
 #pragma unroll
         for (int i = 0; i < kGroup; ++i) v[i] = 0.f;
     }
-    // range widened to contain 0
-    float mn = 0.f, mx = 0.f;
-#pragma unroll
-    for (int i = 0; i < kGroup; ++i) {
-        mn = fminf(mn, v[i]);
-        mx = fmaxf(mx, v[i]);
-    }
-    // scale = (max - min) / (2^4 - 1), stored as fp16; the fp16 value is the one used
-    const float s32 = __fdiv_rn(__fsub_rn(mx, mn), 15.0f);
-    __half sh = __float2half_rn(s32);
-    if (__half2float(sh) == 0.f) sh = __float2half_rn(1.0f);
-    const float shf = __half2float(sh);
-    // zero_point = round(-min / scale)
-    const int zp = (int)fminf(fmaxf(rintf(__fdiv_rn(-mn, shf)), 0.f), 15.f);
-    // index = clamp(round(w / scale) + zero_point, 0, 15)
+    __half sh;
+    int zp;
     uint32_t code[kGroup];
+    if (!sym) {
+        // range widened to contain 0
+        float mn = 0.f, mx = 0.f;
 #pragma unroll
-    for (int i = 0; i < kGroup; ++i) {
-        const int c = (int)rintf(__fdiv_rn(v[i], shf)) + zp;
-        code[i] = (uint32_t)min(max(c, 0), 15);
+        for (int i = 0; i < kGroup; ++i) {
+            mn = fminf(mn, v[i]);
+            mx = fmaxf(mx, v[i]);
+        }
+        // scale = (max - min) / (2^4 - 1), stored as fp16; the fp16 value is the one used
+        sh = __float2half_rn(__fdiv_rn(__fsub_rn(mx, mn), 15.0f));
+        if (__half2float(sh) == 0.f) sh = __float2half_rn(1.0f);
+        const float shf = __half2float(sh);
+        // zero_point = round(-min / scale)
+        zp = (int)fminf(fmaxf(rintf(__fdiv_rn(-mn, shf)), 0.f), 15.f);
+        // index = clamp(round(w / scale) + zero_point, 0, 15)
+#pragma unroll
+        for (int i = 0; i < kGroup; ++i) {
+            const int c = (int)rintf(__fdiv_rn(v[i], shf)) + zp;
+            code[i] = (uint32_t)min(max(c, 0), 15);
+        }
+    } else {
+        // symmetric (b = 4): scale = max|w| / (2^3 - 1), q = clamp(round(w / scale), -7, 7),
+        // stored as code q + 8 with zero point 8
+        float amax = 0.f;
+#pragma unroll
+        for (int i = 0; i < kGroup; ++i) amax = fmaxf(amax, fabsf(v[i]));
+        sh = __float2half_rn(__fdiv_rn(amax, 7.0f));
+        if (__half2float(sh) == 0.f) sh = __float2half_rn(1.0f);
+        const float shf = __half2float(sh);
+        zp = 8;
+#pragma unroll
+        for (int i = 0; i < kGroup; ++i) {
+            const int q = (int)rintf(__fdiv_rn(v[i], shf));
+            code[i] = (uint32_t)(min(max(q, -7), 7) + 8);
+        }
     }
     // tiled block: word i (K = 8i..8i+7): byte b = code[8i+b] | code[8i+4+b] << 4
     uint8_t* blk = blocks + ((size_t)(e * NT + t) * G + g) * kBlockBytes;
@@ -140,7 +159,7 @@ __global__ void __launch_bounds__(128) pack_kernel(const uint16_t* __restrict__ 
         PackHeader* h = reinterpret_cast<PackHeader*>(blocks - kHeaderBytes);
         h->magic = kPackMagic;
         h->version = 1;
-        h->layout = (uint32_t)layout;
+        h->layout = (uint32_t)layout | (sym ? 0x100u : 0u);
         h->E = gridDim.z;
         h->N = (uint32_t)N;
         h->K = (uint32_t)K;
@@ -685,12 +704,13 @@ __global__ void __launch_bounds__(256) dense_prep_kernel(const int8_t* __restric
 }  // namespace
 
 // ------------------------------- launchers ---------------------------------
-cudaError_t launch_pack(const uint16_t* w, int E, int N, int K, int layout, uint8_t* packed, uint8_t* codes,
-                        uint16_t* scale, uint16_t* zp, cudaStream_t stream) {
+cudaError_t launch_pack(const uint16_t* w, int E, int N, int K, int layout, bool symmetric, uint8_t* packed,
+                        uint8_t* codes, uint16_t* scale, uint16_t* zp, cudaStream_t stream) {
     const int G = ceil_div(K, kGroup);
     const int NT = layout == 1 ? ceil_div(N / 2, kTileRows / 2) : ceil_div(N, kTileRows);
     dim3 grid(G, NT, E);
-    pack_kernel<<<grid, 128, 0, stream>>>(w, N, K, layout, NT, G, packed + kHeaderBytes, codes, scale, zp);
+    pack_kernel<<<grid, 128, 0, stream>>>(w, N, K, layout, symmetric ? 1 : 0, NT, G, packed + kHeaderBytes, codes,
+                                          scale, zp);
     return cudaGetLastError();
 }
 
