@@ -35,7 +35,9 @@ its reason in the design notes):
       softmax probability over all E experts, not renormalised;
   R12 tokens inside an expert's segment keep their slot order (t * k + j ascending);
   R14 h enters the requantisation as fp32;
-  R18 symmetric INT4 variant: q clamped to [-7, 7], stored as code q + 8 with zero point 8.
+  R18 symmetric INT4 variant: q clamped to [-7, 7], stored as code q + 8 with zero point 8;
+  R19 percentile-clipped variant: per group the 0.1th and 99.9th percentiles by linear
+      interpolation at q * (n - 1), in fp32 with fractions fp32(0.127) and fp32(0.873).
 
 Parity status: every function below is pinned by tests/test_oracle_pins.py
 against values the pages print, closed forms, brute force or an independent
@@ -75,7 +77,25 @@ def pad_k(a: np.ndarray) -> np.ndarray:
 # --------------------------------------------------------------------------- #
 # a1: weight quantisation and packing  ([P2] §2.1, §2.2)
 # --------------------------------------------------------------------------- #
-def quantize_weights(w: np.ndarray):
+# R19: the 0.1th / 99.9th percentiles of a 128-value group, by linear interpolation
+# between order statistics at position q * (n - 1): 0.127 and 126.873
+PCT_LO_FRAC = np.float32(0.127)
+PCT_HI_FRAC = np.float32(0.873)
+
+
+def group_range_percentile(v: np.ndarray):
+    """Clipped range of each row of v [N][128] (fp32): the 0.1th and 99.9th
+    percentiles ([P2] §2.2: a percentile filters outliers better than min/max; R19:
+    linear interpolation at position q * (n - 1), evaluated in fp32 as
+    a + f * (b - a) with separate roundings)."""
+    srt = np.sort(np.asarray(v, dtype=np.float32), axis=1)
+    assert srt.shape[1] == GROUP
+    lo = srt[:, 0] + PCT_LO_FRAC * (srt[:, 1] - srt[:, 0])
+    hi = srt[:, 126] + PCT_HI_FRAC * (srt[:, 127] - srt[:, 126])
+    return lo.astype(np.float32), hi.astype(np.float32)
+
+
+def quantize_weights(w: np.ndarray, clip999: bool = False):
     """Group-wise asymmetric INT4 of one weight matrix w [N][K] (float32, bf16 values).
 
     [P2] §2.2, per group of 128 along K:
@@ -83,7 +103,9 @@ def quantize_weights(w: np.ndarray):
         zero_point = round(-min / scale)
         index      = clamp(round(weight / scale) + zero_point, 0, 15)
     with readings R2-R6 (min/max widened to contain 0; fp16 scale used for the
-    codes; round half to even; fp32 correctly rounded division).
+    codes; round half to even; fp32 correctly rounded division).  With clip999 the
+    range is the group's 0.1th..99.9th percentile instead of its min..max ([P2] §2.2,
+    R19); values outside it land on codes 0 or 15 through the clamp.
 
     Returns codes uint8 [N][Kp] (values 0..15), scale float16 [N][G], zp float16 [N][G].
     """
@@ -96,8 +118,12 @@ def quantize_weights(w: np.ndarray):
     f15 = np.float32(INT4_MAX)
     for g in range(G):
         v = w[:, g * GROUP:(g + 1) * GROUP]  # [N][128]
-        mn = np.minimum(v.min(axis=1), np.float32(0))  # R3
-        mx = np.maximum(v.max(axis=1), np.float32(0))  # R3
+        if clip999:
+            lo, hi = group_range_percentile(v)
+        else:
+            lo, hi = v.min(axis=1), v.max(axis=1)
+        mn = np.minimum(lo, np.float32(0))  # R3
+        mx = np.maximum(hi, np.float32(0))  # R3
         s32 = (mx - mn) / f15  # fp32 division
         s16 = s32.astype(np.float16)  # round to nearest even fp16 (R5)
         s16[s16 == 0] = np.float16(1.0)  # R3: degenerate (all-zero) group
@@ -336,8 +362,12 @@ class QuantExpert:
     """Quantised weights of one expert: up [2F][Hp] (gate|up rows) and down [H][Fp]
     (asymmetric INT4, or the symmetric variant)."""
 
-    def __init__(self, w_up: np.ndarray, w_down: np.ndarray, symmetric: bool = False):
-        quant = quantize_weights_symmetric if symmetric else quantize_weights
+    def __init__(self, w_up: np.ndarray, w_down: np.ndarray, symmetric: bool = False, clip999: bool = False):
+        if symmetric:
+            quant = quantize_weights_symmetric
+        else:
+            def quant(w):
+                return quantize_weights(w, clip999)
         self.up = quant(w_up)
         self.down = quant(w_down)
 

@@ -165,6 +165,43 @@ def test_sym_int4_degenerate_group():
     assert np.all(scale == np.float16(1.0)) and np.all(zp == 8) and np.all(codes == 8)
 
 
+def test_percentile_range_closed_form_and_numpy():
+    # one outlier in a group: sorted tail ... 0.1, 1.0 -> 99.9th percentile
+    # = 0.1 + 0.873 * (1.0 - 0.1) = 0.8857 (position 0.999 * 127 = 126.873)
+    rng = np.random.default_rng(5)
+    v = synth.bf16_round((rng.uniform(-0.1, 0.1, size=(1, 128))).astype(np.float32))
+    v[0, :2] = [-0.1, -0.1]
+    v[0, 2] = 0.1
+    v[0, 3] = 1.0
+    v = np.clip(v, -0.1, 1.0)
+    lo, hi = O.group_range_percentile(v)
+    assert abs(float(hi[0]) - (0.1 + 0.873 * 0.9)) < 1e-6
+    assert float(lo[0]) == np.float32(-0.1)  # the two lowest are equal
+    # against numpy's percentile (linear interpolation) on random groups
+    w = (rng.standard_normal((64, 128)) * 0.02).astype(np.float32)
+    lo, hi = O.group_range_percentile(w)
+    np.testing.assert_allclose(lo, np.percentile(w.astype(np.float64), 0.1, axis=1), rtol=1e-6, atol=1e-9)
+    np.testing.assert_allclose(hi, np.percentile(w.astype(np.float64), 99.9, axis=1), rtol=1e-6, atol=1e-9)
+
+
+def test_clip999_codes_and_outlier():
+    rng = np.random.default_rng(9)
+    w = synth.bf16_round((rng.standard_normal((8, 256)) * 0.02).astype(np.float32))
+    w[2, 5] = 0.5  # an outlier far beyond the group's second largest value
+    w = synth.bf16_round(w)
+    c0, s0, z0 = O.quantize_weights(w)
+    c1, s1, z1 = O.quantize_weights(w, clip999=True)
+    # the clipped range is inside the min..max range: scales never grow
+    assert np.all(s1.astype(np.float32) <= s0.astype(np.float32))
+    # the outlier's group gets a much tighter scale and the outlier sits on code 15
+    assert float(s1[2, 0]) < float(s0[2, 0])
+    assert c1[2, 5] == 15
+    # reconstruct the codes from the stored scale and zero point (R5)
+    sf = np.repeat(s1.astype(np.float32), 128, axis=1)
+    z = np.repeat(z1.astype(np.float32), 128, axis=1)
+    assert np.array_equal(np.clip(np.rint(w / sf) + z, 0, 15).astype(np.uint8), c1)
+
+
 def test_quantize_uses_fp16_scale_for_codes():
     # reconstructing the codes from the stored fp16 scale + zp reproduces them (R5)
     rng = np.random.default_rng(3)
