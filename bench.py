@@ -177,18 +177,30 @@ def dev_bf16(a, device):
     return torch.from_numpy(synth.bf16_bits(a).view(np.int16)).view(torch.bfloat16).to(device)
 
 
-# weight scheme of the packer: asymmetric INT4 (default) or the symmetric variant
-SYMMETRIC = False
+# weight scheme of the packer: asymmetric INT4 (default), symmetric, or asymmetric on the
+# 0.1th..99.9th percentile range
+SCHEME = "asym"
 
 
 def weights_desc():
-    return "int4 g128 sym (fp16 scale, zero point 8)" if SYMMETRIC else "int4 g128 asym (fp16 scale+zp)"
+    return {"asym": "int4 g128 asym (fp16 scale+zp)", "sym": "int4 g128 sym (fp16 scale, zero point 8)",
+            "clip999": "int4 g128 asym on the 0.1..99.9 percentile range (fp16 scale+zp)"}[SCHEME]
+
+
+def scheme_flag(B):
+    return {"asym": 0, "sym": B.W4A8_PACK_SYMMETRIC, "clip999": B.W4A8_PACK_CLIP999}[SCHEME]
+
+
+def oracle_quant(O):
+    if SCHEME == "sym":
+        return O.quantize_weights_symmetric
+    return lambda w: O.quantize_weights(w, clip999=SCHEME == "clip999")
 
 
 def pack_experts(B, torch, W, seed, device):
     """Pack every expert's up (gate|up) and down weights on the device, one expert at a time."""
     E, H, F = W.E, W.H, W.F
-    flag = B.W4A8_PACK_SYMMETRIC if SYMMETRIC else 0
+    flag = scheme_flag(B)
     up = B.empty_aligned(B.w4a8_packed_bytes(E, 2 * F, H, B.W4A8_LAYOUT_GATEUP), device)
     dn = B.empty_aligned(B.w4a8_packed_bytes(E, H, F, B.W4A8_LAYOUT_PLAIN), device)
     su = (up.numel() - 256) // E
@@ -308,7 +320,7 @@ class GemmStep:
         x, w = synth.dense_gemm_inputs(seed, W.M, W.K, W.N)
         self.x = dev_bf16(x, device)
         self.packed = B.empty_aligned(B.w4a8_packed_bytes(1, W.N, W.K, 0), device)
-        B.w4a8_pack_weights(dev_bf16(w, device), B.W4A8_PACK_SYMMETRIC if SYMMETRIC else 0, self.packed)
+        B.w4a8_pack_weights(dev_bf16(w, device), scheme_flag(B), self.packed)
         Kp = padded(W.K)
         self.q = torch.empty((W.M, Kp), dtype=torch.int8, device=device)
         self.s = torch.empty(W.M, dtype=torch.float32, device=device)
@@ -372,7 +384,7 @@ class OracleSample:
         self.O, self.W, self.seed = O, W, seed
         if W.kind == "gemm":
             x, w = synth.dense_gemm_inputs(seed, W.M, W.K, W.N)
-            self.x, self.qw = x, (O.quantize_weights_symmetric if SYMMETRIC else O.quantize_weights)(w)
+            self.x, self.qw = x, oracle_quant(O)(w)
             self.tokens = W.M
             self.sample_desc = f"all {W.M} rows"
             return
@@ -402,7 +414,7 @@ class OracleSample:
                 W = self.W
                 self.experts[e] = self.O.QuantExpert(synth.expert_weight(self.seed, e, "up", 2 * W.F, W.H),
                                                      synth.expert_weight(self.seed, e, "down", W.H, W.F),
-                                                     SYMMETRIC)
+                                                     symmetric=SCHEME == "sym", clip999=SCHEME == "clip999")
 
     def _time(self, n):
         self._ensure_experts(n)
@@ -483,11 +495,12 @@ def main(argv=None):
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--cpu-baseline-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--weights", choices=["asym", "sym"], default="asym",
-                    help="packer scheme: asymmetric INT4 (default) or the symmetric variant")
+    ap.add_argument("--weights", choices=["asym", "sym", "clip999"], default="asym",
+                    help="packer scheme: asymmetric INT4 (default), symmetric, or asymmetric on the "
+                         "0.1th..99.9th percentile range")
     args = ap.parse_args(argv)
-    global SYMMETRIC
-    SYMMETRIC = args.weights == "sym"
+    global SCHEME
+    SCHEME = args.weights
     W = synth.WORKLOADS[args.workload]
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

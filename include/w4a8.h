@@ -73,20 +73,27 @@ enum { W4A8_LAYOUT_PLAIN = 0, W4A8_LAYOUT_GATEUP = 1 };
  * W4A8_PACK_SYMMETRIC: symmetric INT4 (the LLM quantisation primer at
  *   hotelren.com/news/5982361, section 2.1, with b = 4): scale = max|w|/7 (fp16),
  *   q = clamp(round(w/scale), -7, 7), stored as code q + 8 with zero point 8.
- * Both write the same tiled format, so w4a8_gemm and w4a8_moe_forward take either.
- * Rounding is half to even; divisions are correctly rounded fp32; an fp16 scale
- * that rounds to 0 is replaced by 1.                                              */
-enum { W4A8_PACK_SYMMETRIC = 0x100 };
+ * W4A8_PACK_CLIP999: asymmetric as the default, but over the range from the group's
+ *   0.1th to its 99.9th percentile (same page, section 2.2: a percentile keeps
+ *   outliers from stretching the range), each by linear interpolation between the
+ *   two nearest order statistics (positions 0.127 and 126.873 of the 128 sorted
+ *   values) evaluated in fp32 as a + f*(b - a), f = 0.127f / 0.873f; values outside
+ *   the range land on codes 0 / 15 through the clamp.
+ * At most one flag may be set.  All write the same tiled format, so w4a8_gemm and
+ * w4a8_moe_forward take any of them.  Rounding is half to even; divisions are
+ * correctly rounded fp32; an fp16 scale that rounds to 0 is replaced by 1.         */
+enum { W4A8_PACK_SYMMETRIC = 0x100, W4A8_PACK_CLIP999 = 0x200 };
 
 /* Bytes of a packed weight buffer for E matrices of shape [N][K] in `layout`:
  * a 256-byte header, then one 8704-byte block per (matrix, 128-row tile, 128-wide
  * K group): 8192 bytes of 4-bit codes, 128 fp16 scales, 128 fp16 zero points.
  * K is padded to a multiple of 128 (zero weights).  Returns 0 for invalid shapes
- * (GATEUP needs an even N) or an unknown flag; W4A8_PACK_SYMMETRIC may be set. */
+ * (GATEUP needs an even N) or an unknown flag combination; one of
+ * W4A8_PACK_SYMMETRIC, W4A8_PACK_CLIP999 may be set. */
 size_t w4a8_packed_bytes(int E, int N, int K, int layout);
 
 /* Quantise and pack E weight matrices  (a1: the offline conversion step).
- *   layout      : W4A8_LAYOUT_PLAIN or W4A8_LAYOUT_GATEUP, optionally | W4A8_PACK_SYMMETRIC.
+ *   layout      : W4A8_LAYOUT_PLAIN or W4A8_LAYOUT_GATEUP, optionally | one scheme flag.
  *   w_bf16      : device, bf16 [E][N][K], row-major (nn.Linear orientation).
  *   packed      : device, w4a8_packed_bytes(E,N,K,layout) bytes (256-B aligned),
  *                 the tiled layout consumed by w4a8_gemm / w4a8_moe_forward.

@@ -51,7 +51,9 @@ def test_packed_bytes_accounting(lib):
     assert lib.w4a8_packed_bytes(1, 3, 128, 1) == 0  # odd N for gate|up
     # the symmetric scheme flag keeps the format (and size); unknown flags are refused
     assert lib.w4a8_packed_bytes(8, 2048, 2048, 1 | 0x100) == lib.w4a8_packed_bytes(8, 2048, 2048, 1)
-    assert lib.w4a8_packed_bytes(1, 256, 512, 0x200) == 0
+    assert lib.w4a8_packed_bytes(1, 256, 512, 0x200) == lib.w4a8_packed_bytes(1, 256, 512, 0)
+    assert lib.w4a8_packed_bytes(1, 256, 512, 0x300) == 0  # two scheme flags
+    assert lib.w4a8_packed_bytes(1, 256, 512, 0x400) == 0  # unknown flag
     assert lib.w4a8_packed_bytes(0, 128, 128, 0) == 0
     # per weight: 0.5 byte of codes + 4 bytes per 128-group of scale and zero point
     blk = 8704

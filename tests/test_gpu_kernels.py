@@ -63,19 +63,26 @@ def test_quant_act_worked_example():
     assert int(q[0, 0]) == int(qo[0, 0])
 
 
-@pytest.mark.parametrize("sym", [False, True])
+SCHEMES = {"asym": (0, O.quantize_weights),
+           "sym": (B.W4A8_PACK_SYMMETRIC, O.quantize_weights_symmetric),
+           "clip999": (B.W4A8_PACK_CLIP999, lambda w: O.quantize_weights(w, clip999=True))}
+
+
+@pytest.mark.parametrize("scheme", sorted(SCHEMES))
 @pytest.mark.parametrize("E,N,K,layout", [(2, 256, 512, 0), (3, 200, 200, 0), (2, 384, 256, 1), (1, 130, 1000, 1),
                                           (4, 128, 128, 0)])
-def test_pack_bit_exact(E, N, K, layout, sym):
+def test_pack_bit_exact(E, N, K, layout, scheme):
     rng = np.random.default_rng(E * 1000 + N + K)
     w = synth.bf16_round((rng.standard_normal((E, N, K)) * 0.02).astype(np.float32))
     w[0, 0, :] = 0.0  # degenerate group
     w[0, 1, :128] += 0.3  # skewed group
+    w[-1, -1, 0] = 0.4  # an outlier
+    w[-1, -2, 1:3] = -0.25  # two equal low outliers
     w = synth.bf16_round(w)
-    packed, codes, scale, zp = pack_on_gpu(w, layout | (B.W4A8_PACK_SYMMETRIC if sym else 0))
+    flag, quant = SCHEMES[scheme]
+    packed, codes, scale, zp = pack_on_gpu(w, layout | flag)
     codes_h, scale_h, zp_h = codes.cpu().numpy(), scale.cpu().numpy(), zp.cpu().numpy()
     dc, ds, dz = decode_packed(packed.cpu().numpy(), E, N, K, layout)
-    quant = O.quantize_weights_symmetric if sym else O.quantize_weights
     for e in range(E):
         c, sc, z = quant(w[e])
         assert np.array_equal(codes_h[e], O.pack_nibbles(c)), f"canonical bytes, expert {e}"
@@ -101,11 +108,12 @@ def test_route_topk():
 
 
 # --------------------------------------------------------------------------- #
-def run_dense_gemm(M, N, K, seed=0, sym=False):
+def run_dense_gemm(M, N, K, seed=0, scheme="asym"):
     x, w = synth.dense_gemm_inputs(seed, M, K, N)
     qa, sa = O.quantize_act(x)
-    codes, scale, zp = (O.quantize_weights_symmetric if sym else O.quantize_weights)(w)
-    packed, _, _, _ = pack_on_gpu(w[None], B.W4A8_PACK_SYMMETRIC if sym else 0, canonical=False)
+    flag, quant = SCHEMES[scheme]
+    codes, scale, zp = quant(w)
+    packed, _, _, _ = pack_on_gpu(w[None], flag, canonical=False)
     G = O.padded_k(K) // 128
     qa_d = torch.from_numpy(qa).cuda()
     sa_d = torch.from_numpy(sa).cuda()
@@ -125,10 +133,12 @@ def test_dense_gemm_16x512x256_partials_bit_exact():
     assert_close(y, yo, max_rel=1e-4, mae_rel=1e-5, what="y")
 
 
+@pytest.mark.parametrize("scheme", ["sym", "clip999"])
 @pytest.mark.parametrize("M,N,K", [(16, 256, 512), (300, 100, 640)])
-def test_dense_gemm_symmetric_weights_partials_bit_exact(M, N, K):
-    """Symmetric INT4 weights (zero point 8) through both GEMM kernels (M <= 16: decode tiles)."""
-    y, part, acc, yo = run_dense_gemm(M, N, K, seed=7 + M, sym=True)
+def test_dense_gemm_other_schemes_partials_bit_exact(M, N, K, scheme):
+    """Symmetric (zero point 8) and percentile-clipped weights through both GEMM kernels
+    (M <= 16: decode tiles)."""
+    y, part, acc, yo = run_dense_gemm(M, N, K, seed=7 + M, scheme=scheme)
     assert np.array_equal(part.astype(np.int64), acc)
     assert_close(y, yo, max_rel=1e-4, mae_rel=1e-5, what="y")
 

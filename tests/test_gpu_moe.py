@@ -29,10 +29,10 @@ def bf16_to_f32(t):
 class Layer:
     """One synthetic MoE layer, packed on the GPU, with lazily quantised oracle experts."""
 
-    def __init__(self, T, E, k, H, F, routing="uniform", seed=0, zipf_s=1.1, outlier=0.0, symmetric=False):
+    def __init__(self, T, E, k, H, F, routing="uniform", seed=0, zipf_s=1.1, outlier=0.0, scheme="asym"):
         self.T, self.E, self.k, self.H, self.F, self.seed = T, E, k, H, F, seed
-        self.symmetric = symmetric
-        flag = B.W4A8_PACK_SYMMETRIC if symmetric else 0
+        self.scheme = scheme
+        flag = {"asym": 0, "sym": B.W4A8_PACK_SYMMETRIC, "clip999": B.W4A8_PACK_CLIP999}[scheme]
         self.x = synth.activations(seed, T, H, outlier, 20.0)
         if routing == "softmax":
             self.logits = synth.router_logits(seed, T, E)
@@ -71,7 +71,9 @@ class Layer:
     def experts(self):
         for e in np.unique(self.ids):
             if e not in self._experts:
-                self._experts[int(e)] = O.QuantExpert(self.w_up(int(e)), self.w_down(int(e)), self.symmetric)
+                self._experts[int(e)] = O.QuantExpert(self.w_up(int(e)), self.w_down(int(e)),
+                                                      symmetric=self.scheme == "sym",
+                                                      clip999=self.scheme == "clip999")
         return self._experts
 
     def run(self, use_router=False):
@@ -170,10 +172,12 @@ def test_moe_small_stages_and_output(T, E, k, H, F, routing):
     assert_close(out, ref, what="out")
 
 
+@pytest.mark.parametrize("scheme", ["sym", "clip999"])
 @pytest.mark.parametrize("T,E,k,H,F,routing", [(300, 4, 2, 512, 256, "uniform"), (64, 32, 4, 256, 256, "zipf")])
-def test_moe_symmetric_weights_stages_and_output(T, E, k, H, F, routing):
-    """The symmetric INT4 variant of the packer through the whole layer (wide and decode tiles)."""
-    L = Layer(T, E, k, H, F, routing, seed=T + E + 1, symmetric=True)
+def test_moe_other_weight_schemes_stages_and_output(T, E, k, H, F, routing, scheme):
+    """The symmetric and percentile-clipped packer variants through the whole layer
+    (wide and decode tiles)."""
+    L = Layer(T, E, k, H, F, routing, seed=T + E + 1, scheme=scheme)
     out = L.run()
     check_stages(L, out)
     ref = O.moe_forward(L.x, L.ids, L.w, L.experts(), E, F)

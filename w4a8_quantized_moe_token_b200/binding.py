@@ -19,6 +19,7 @@ LIB_PATH = os.path.join(_HERE, "libw4a8.so")
 W4A8_LAYOUT_PLAIN = 0
 W4A8_LAYOUT_GATEUP = 1
 W4A8_PACK_SYMMETRIC = 0x100  # OR into the layout: symmetric INT4 (scale = max|w|/7, codes q + 8, zero point 8)
+W4A8_PACK_CLIP999 = 0x200  # OR into the layout: asymmetric INT4 over the 0.1th..99.9th percentile range
 
 DUMP = {
     "counts": 0, "offs": 1, "perm": 2, "inv": 3, "poffs": 4, "act1": 5, "s1": 6,

@@ -275,7 +275,8 @@ W4A8_EXPORT const char* w4a8_status_string(int status) {
 
 W4A8_EXPORT size_t w4a8_packed_bytes(int E, int N, int K, int layout) {
     if (E < 1 || N < 1 || K < 1) return 0;
-    if ((layout & ~0xFF) != 0 && (layout & ~0xFF) != W4A8_PACK_SYMMETRIC) return 0;
+    const int flags = layout & ~0xFF;
+    if (flags != 0 && flags != W4A8_PACK_SYMMETRIC && flags != W4A8_PACK_CLIP999) return 0;
     layout &= 0xFF;  // the scheme flag does not change the size
     if (layout != W4A8_LAYOUT_PLAIN && layout != W4A8_LAYOUT_GATEUP) return 0;
     if (layout == W4A8_LAYOUT_GATEUP && (N & 1)) return 0;
@@ -294,8 +295,8 @@ W4A8_EXPORT int w4a8_pack_weights(const void* w_bf16, int E, int N, int K, int l
         (zp_f16_opt && !aligned(zp_f16_opt, 2)))
         return W4A8_EALIGN;
     if (packed_bytes < need) return W4A8_ENOSPACE;
-    const bool symmetric = (layout & W4A8_PACK_SYMMETRIC) != 0;
-    return to_status(launch_pack(static_cast<const uint16_t*>(w_bf16), E, N, K, layout & 0xFF, symmetric,
+    const int scheme = (layout & W4A8_PACK_SYMMETRIC) ? 1 : (layout & W4A8_PACK_CLIP999) ? 2 : 0;
+    return to_status(launch_pack(static_cast<const uint16_t*>(w_bf16), E, N, K, layout & 0xFF, scheme,
                                  static_cast<uint8_t*>(packed), codes_opt, scale_f16_opt, zp_f16_opt,
                                  static_cast<cudaStream_t>(stream)));
 }

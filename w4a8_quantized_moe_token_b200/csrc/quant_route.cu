@@ -35,6 +35,7 @@ __device__ __forceinline__ float warp_sum(float v) {
 // a1: weight quantisation + packing.  One block per (group g, tile t, matrix e);
 // thread r quantises tiled row r's 128 weights of group g.
 // ---------------------------------------------------------------------------
+// sym: 0 asymmetric min/max, 1 symmetric, 2 asymmetric on the 0.1th..99.9th percentile range
 __global__ void __launch_bounds__(128) pack_kernel(const uint16_t* __restrict__ w, int N, int K, int layout, int sym,
                                                    int NT, int G, uint8_t* __restrict__ blocks,
                                                    uint8_t* __restrict__ codes_out, uint16_t* __restrict__ scale_out,
@@ -78,14 +79,33 @@ __global__ void __launch_bounds__(128) pack_kernel(const uint16_t* __restrict__ 
     __half sh;
     int zp;
     uint32_t code[kGroup];
-    if (!sym) {
-        // range widened to contain 0
-        float mn = 0.f, mx = 0.f;
+    if (sym != 1) {
+        float lo, hi;
+        if (sym == 2) {
+            // the 0.1th and 99.9th percentiles of the group: linear interpolation
+            // between the order statistics around positions 0.127 and 126.873, so
+            // only the two smallest and the two largest values are needed
+            float a0 = v[0], a1 = INFINITY, b0 = v[0], b1 = -INFINITY;  // a0 <= a1 smallest, b0 >= b1 largest
 #pragma unroll
-        for (int i = 0; i < kGroup; ++i) {
-            mn = fminf(mn, v[i]);
-            mx = fmaxf(mx, v[i]);
+            for (int i = 1; i < kGroup; ++i) {
+                a1 = fminf(a1, fmaxf(v[i], a0));
+                a0 = fminf(a0, v[i]);
+                b1 = fmaxf(b1, fminf(v[i], b0));
+                b0 = fmaxf(b0, v[i]);
+            }
+            lo = __fadd_rn(a0, __fmul_rn(0.127f, __fsub_rn(a1, a0)));
+            hi = __fadd_rn(b1, __fmul_rn(0.873f, __fsub_rn(b0, b1)));
+        } else {
+            lo = v[0];
+            hi = v[0];
+#pragma unroll
+            for (int i = 1; i < kGroup; ++i) {
+                lo = fminf(lo, v[i]);
+                hi = fmaxf(hi, v[i]);
+            }
         }
+        // range widened to contain 0
+        const float mn = fminf(lo, 0.f), mx = fmaxf(hi, 0.f);
         // scale = (max - min) / (2^4 - 1), stored as fp16; the fp16 value is the one used
         sh = __float2half_rn(__fdiv_rn(__fsub_rn(mx, mn), 15.0f));
         if (__half2float(sh) == 0.f) sh = __float2half_rn(1.0f);
@@ -159,7 +179,7 @@ __global__ void __launch_bounds__(128) pack_kernel(const uint16_t* __restrict__ 
         PackHeader* h = reinterpret_cast<PackHeader*>(blocks - kHeaderBytes);
         h->magic = kPackMagic;
         h->version = 1;
-        h->layout = (uint32_t)layout | (sym ? 0x100u : 0u);
+        h->layout = (uint32_t)layout | (sym == 1 ? 0x100u : sym == 2 ? 0x200u : 0u);
         h->E = gridDim.z;
         h->N = (uint32_t)N;
         h->K = (uint32_t)K;
@@ -704,13 +724,12 @@ __global__ void __launch_bounds__(256) dense_prep_kernel(const int8_t* __restric
 }  // namespace
 
 // ------------------------------- launchers ---------------------------------
-cudaError_t launch_pack(const uint16_t* w, int E, int N, int K, int layout, bool symmetric, uint8_t* packed,
+cudaError_t launch_pack(const uint16_t* w, int E, int N, int K, int layout, int scheme, uint8_t* packed,
                         uint8_t* codes, uint16_t* scale, uint16_t* zp, cudaStream_t stream) {
     const int G = ceil_div(K, kGroup);
     const int NT = layout == 1 ? ceil_div(N / 2, kTileRows / 2) : ceil_div(N, kTileRows);
     dim3 grid(G, NT, E);
-    pack_kernel<<<grid, 128, 0, stream>>>(w, N, K, layout, symmetric ? 1 : 0, NT, G, packed + kHeaderBytes, codes,
-                                          scale, zp);
+    pack_kernel<<<grid, 128, 0, stream>>>(w, N, K, layout, scheme, NT, G, packed + kHeaderBytes, codes, scale, zp);
     return cudaGetLastError();
 }
 

@@ -35,7 +35,8 @@ inline int act_block_rows(int tile_tokens, int rows_cap) { return tile_tokens ==
 cudaError_t launch_gemm(const GemmArgs& a, int tile_tokens, int num_ctas, cudaStream_t stream);
 cudaError_t launch_gemm_decode(const GemmArgs& a, int num_ctas, cudaStream_t stream);
 
-cudaError_t launch_pack(const uint16_t* w, int E, int N, int K, int layout, bool symmetric, uint8_t* packed,
+// scheme: 0 asymmetric (min/max), 1 symmetric, 2 asymmetric on the 0.1th..99.9th percentiles
+cudaError_t launch_pack(const uint16_t* w, int E, int N, int K, int layout, int scheme, uint8_t* packed,
                         uint8_t* codes, uint16_t* scale, uint16_t* zp, cudaStream_t stream);
 cudaError_t launch_quant_act(const uint16_t* x, int T, int K, int8_t* q, float* s, cudaStream_t stream);
 cudaError_t launch_route_topk(const uint16_t* logits, int T, int E, int k, int32_t* ids, float* w,
