@@ -37,7 +37,10 @@ its reason in the design notes):
   R14 h enters the requantisation as fp32;
   R18 symmetric INT4 variant: q clamped to [-7, 7], stored as code q + 8 with zero point 8;
   R19 percentile-clipped variant: per group the 0.1th and 99.9th percentiles by linear
-      interpolation at q * (n - 1), in fp32 with fractions fp32(0.127) and fp32(0.873).
+      interpolation at q * (n - 1), in fp32 with fractions fp32(0.127) and fp32(0.873);
+  R20 INT8 KV cache: static symmetric per-head scale max|x|/127 over the calibration
+      values (0 for an all-zero head, which then quantises to 0); dequantisation rounds
+      the fp32 product q * scale once to bf16.
 
 Parity status: every function below is pinned by tests/test_oracle_pins.py
 against values the pages print, closed forms, brute force or an independent
@@ -422,3 +425,37 @@ def token_forward(t: int, x, ids, w, experts: dict, F: int) -> np.ndarray:
         y2 = expert_forward(xq, xs, experts[int(ids[t, j])], F)[0]
         out = out + float(w[t, j]) * y2
     return round_to_bf16(out)
+
+
+# --------------------------------------------------------------------------- #
+# INT8 KV cache with static per-head scales (the next W4A8 deployment step)
+# --------------------------------------------------------------------------- #
+def kv_calibrate(x: np.ndarray) -> np.ndarray:
+    """Static per-head scales of a KV cache from calibration data x [T][H][D] (fp32,
+    bf16 values).
+
+    [P1] §5 (deployment): the attention KV cache is quantised to INT8 statically,
+    with per-head scales fixed from a little calibration data; [P3] §2.1 symmetric
+    form: scale = max|x| / 127 over the head's calibration values (fp32 division).
+    A head whose calibration values are all zero gets scale 0 (R20).
+    """
+    x = np.asarray(x, dtype=np.float32)
+    amax = np.abs(x).max(axis=(0, 2)) if x.shape[0] else np.zeros(x.shape[1], np.float32)
+    return (amax.astype(np.float32) / np.float32(INT8_QMAX)).astype(np.float32)
+
+
+def kv_quantize(x: np.ndarray, scale: np.ndarray) -> np.ndarray:
+    """q[t, h, d] = clamp(round(x / scale[h]), -127, 127), fp32 division, round half to
+    even (R4, R6, R7); values beyond the calibrated range saturate; scale 0 -> q = 0."""
+    x = np.asarray(x, dtype=np.float32)
+    s = np.asarray(scale, dtype=np.float32)[None, :, None]
+    safe = np.where(s > 0, s, np.float32(1))
+    q = np.clip(np.rint(x / safe), -INT8_QMAX, INT8_QMAX)
+    return np.where(s > 0, q, 0).astype(np.int8)
+
+
+def kv_dequantize(q: np.ndarray, scale: np.ndarray) -> np.ndarray:
+    """x'[t, h, d] = bf16(q * scale[h]): the fp32 product rounded once to bf16 (RNE),
+    returned as float32 values (R20)."""
+    y = np.asarray(q, dtype=np.float32) * np.asarray(scale, dtype=np.float32)[None, :, None]
+    return round_to_bf16(y.astype(np.float64)).astype(np.float32)

@@ -461,3 +461,44 @@ def test_round_to_bf16_against_library_rounding():
     assert np.array_equal(O.round_to_bf16(v), ref)
     assert O.round_to_bf16(np.array([1.0 + 2.0 ** -8]))[0] == 1.0  # tie to even
     assert O.round_to_bf16(np.array([1.0 + 3 * 2.0 ** -8]))[0] == 1.0 + 2.0 ** -6
+
+
+# --------------------------------------------------------------------------- #
+# INT8 KV cache (static per-head scales)
+# --------------------------------------------------------------------------- #
+def test_kv_int8_worked_example_per_head():
+    # the primer's worked example per head: calibrated range 0.5 -> s = 0.5/127,
+    # 0.2 -> 51 -> 51 * s = 0.20079 (bf16: 0.2001953125... rounding of 0.2007874)
+    x = np.zeros((2, 2, 4), np.float32)
+    x[0, 0] = [0.5, -0.5, 0.2, 0.0]
+    x[1, 1] = [1.0, 0.2, -0.2, 0.1]
+    s = O.kv_calibrate(x)
+    assert s[0] == np.float32(0.5) / np.float32(127) and s[1] == np.float32(1.0) / np.float32(127)
+    q = O.kv_quantize(x, s)
+    assert list(q[0, 0]) == [127, -127, 51, 0]
+    assert list(q[1, 1]) == [127, 25, -25, 13]  # 25.4 -> 25 (page: "25 or 26"), 12.7 -> 13
+    dq = O.kv_dequantize(q, s)
+    assert dq[0, 0, 2] == np.float32(synth.bf16_round(np.array([51 * (0.5 / 127)], np.float32))[0])
+    assert abs(dq[0, 0, 2] - 0.2) < 2e-3
+
+
+def test_kv_int8_roundtrip_saturation_and_zero_head():
+    rng = np.random.default_rng(21)
+    calib = synth.bf16_round(rng.standard_normal((64, 4, 32)).astype(np.float32))
+    calib[:, 3] = 0.0  # an all-zero head
+    s = O.kv_calibrate(calib)
+    assert s[3] == 0
+    x = synth.bf16_round(rng.standard_normal((16, 4, 32)).astype(np.float32) * 0.5)
+    x[0, 0, 0] = 100.0  # beyond the calibrated range: saturates
+    q = O.kv_quantize(x, s)
+    assert q[0, 0, 0] == 127 and np.all(q[:, 3] == 0)
+    dq = O.kv_dequantize(q, s)
+    inside = np.abs(x) <= (127 * s)[None, :, None]
+    sc = np.broadcast_to(s[None, :, None], x.shape)
+    # half a step of quantisation plus the bf16 rounding of the result
+    err = np.abs(dq - x)
+    assert np.all(err[inside] <= sc[inside] / 2 + np.abs(x[inside]) * 2.0 ** -8 + 1e-12)
+    # the brute-force definition, element by element, on a few values
+    for (t, h, d) in [(1, 0, 3), (5, 2, 31), (15, 1, 0)]:
+        ref = max(-127, min(127, int(np.rint(np.float32(x[t, h, d]) / s[h]))))
+        assert q[t, h, d] == ref
