@@ -454,6 +454,19 @@ def run_reference(args, W):
     world, rank, _ = dist_env()
     if rank != 0:
         return 0
+    if W.kind == "kv":
+        target = max(0.5, min(10.0, 150.0 / max(1, args.steps + args.warmup)))
+        H, D = W.extra["heads"], W.extra["head_dim"]
+        vals = [kv_oracle_sample(W, args.seed, target) for _ in range(args.steps)]
+        value = statistics.mean(v[0] for v in vals) * 6 * H * D / 1e9
+        line = {"impl": "reference", "metric": KV_METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": kv_config(W),
+                "cpu_baseline": {"value": value, "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
+                                 "sample": vals[0][1]},
+                "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return 0
     target = max(0.5, min(10.0, 150.0 / max(1, args.steps + args.warmup)))
     S = OracleSample(W, args.seed, target)
     for _ in range(args.warmup):
@@ -483,6 +496,132 @@ def config_of(W, l2):
     c.update({"weights": weights_desc(), "acts": "int8 per-token", "l2": l2,
               "parallelism": "replicas (no cross-GPU exchange)"})
     return c
+
+
+KV_METRIC = "INT8 KV cache (static per-head scales): quantise + dequantise, GB/s on 1 B200; % of HBM roofline"
+
+
+def kv_config(W):
+    x = W.extra
+    return {"workload": W.name, "T": W.T, "heads": x["heads"], "head_dim": x["head_dim"],
+            "calib_tokens": x["calib_tokens"], "kv": "bf16 -> int8 (per-head static scale) -> bf16",
+            "l2": "flushed before every timed step (256 MiB write, outside the timed span)",
+            "parallelism": "replicas (no cross-GPU exchange)"}
+
+
+def kv_oracle_sample(W, seed, target_s):
+    """The oracle's quantise + dequantise on a bounded token sample (tokens/s, sample text)."""
+    from oracle import w4a8_oracle as O
+    H, D = W.extra["heads"], W.extra["head_dim"]
+    calib = synth.kv_cache(seed, min(W.T, W.extra["calib_tokens"]), H, D)
+    s = O.kv_calibrate(calib)
+    n = min(W.T, 256)
+    x = synth.kv_cache(seed, n, H, D)
+    t0 = time.perf_counter()
+    O.kv_dequantize(O.kv_quantize(x, s), s)
+    per_tok = (time.perf_counter() - t0) / n
+    n = int(max(1, min(W.T, target_s / max(per_tok, 1e-9))))
+    x = synth.kv_cache(seed, n, H, D)
+    t0 = time.perf_counter()
+    O.kv_dequantize(O.kv_quantize(x, s), s)
+    t = time.perf_counter() - t0
+    return n / t, f"{n} of {W.T} tokens"
+
+
+def run_kv(args, W, torch, B, device, world, rank):
+    """Time the INT8 KV cache round trip (w4a8_kv_quant + w4a8_kv_dequant of the whole
+    cache) per step; the calibration is offline (static scales), done once before."""
+    H, D, T = W.extra["heads"], W.extra["head_dim"], W.T
+    x_h = synth.kv_cache(args.seed, T, H, D)
+    calib = dev_bf16(x_h[:W.extra["calib_tokens"]], device)
+    x = dev_bf16(x_h, device)
+    scale = torch.empty(H, dtype=torch.float32, device=device)
+    q = torch.empty((T, H, D), dtype=torch.int8, device=device)
+    y = torch.empty((T, H, D), dtype=torch.bfloat16, device=device)
+    B.w4a8_kv_calibrate(calib, scale)
+
+    def step():
+        B.w4a8_kv_quant(x, scale, q)
+        B.w4a8_kv_dequant(q, scale, y)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    sampler = ClockSampler(torch.cuda.current_device())
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    sampler.start()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.zero_()
+        ev[i][0].record()
+        B.w4a8_kv_quant(x, scale, q)
+        ev[i][1].record()
+        B.w4a8_kv_dequant(q, scale, y)
+        ev[i][2].record()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    sampler.stop()
+    qms = sum(e[0].elapsed_time(e[1]) for e in ev) / args.steps
+    dms = sum(e[1].elapsed_time(e[2]) for e in ev) / args.steps
+    ms_t = torch.tensor([qms + dms], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(ms_t, op=torch.distributed.ReduceOp.MAX)
+    ms = float(ms_t.item())
+    n = T * H * D
+    qbytes, dbytes = 3 * n, 3 * n  # bf16 in + int8 out; int8 in + bf16 out
+    # end to end: host cache in, round trip, host cache out
+    xh = torch.from_numpy(synth.bf16_bits(x_h).view(np.int16)).view(torch.bfloat16).pin_memory()
+    yh = torch.empty((T, H, D), dtype=torch.bfloat16).pin_memory()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for _ in range(args.warmup):
+        x.copy_(xh, non_blocking=True)
+        step()
+        yh.copy_(y, non_blocking=True)
+    torch.cuda.synchronize()
+    a.record()
+    for _ in range(args.steps):
+        x.copy_(xh, non_blocking=True)
+        step()
+        yh.copy_(y, non_blocking=True)
+    b.record()
+    torch.cuda.synchronize()
+    e2e_ms = a.elapsed_time(b) / args.steps
+    peaks = load_peaks()
+    hbm = float(peaks["hbm_gbs"])
+    dom, dom_ms, dom_b = ("kv_dequant", dms, dbytes) if dms >= qms else ("kv_quant", qms, qbytes)
+    roof = {"bound": "hbm", "achieved": dom_b / (dom_ms / 1e3) / 1e9, "peak": hbm, "unit": "GB/s"}
+    roof["frac"] = roof["achieved"] / hbm
+    roof["traffic"] = load_traffic(W.name, dom)
+    roof["kernel"] = dom
+    roof["peak_source"] = f"{peaks['source']}: MEASURED_PEAKS hbm_gbs"
+    total_bytes = (qbytes + dbytes) * world
+    line = {
+        "metric": KV_METRIC, "value": total_bytes / (ms / 1e3) / 1e9, "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "int8", "data": "synthetic", "config": kv_config(W),
+        "tokens_per_s": T * world / (ms / 1e3),
+        "roofline": roof,
+        "kernels": {"kv_quant": {"launches": args.steps, "ms_per_step": qms, "gbs": qbytes / (qms / 1e3) / 1e9},
+                    "kv_dequant": {"launches": args.steps, "ms_per_step": dms, "gbs": dbytes / (dms / 1e3) / 1e9}},
+        "gpu_launches": 2 * args.steps,
+        "e2e": {"value": total_bytes / (e2e_ms / 1e3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": 2 * n,
+                "d2h_bytes_per_step": 2 * n},
+        "clocks": sampler.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tps, desc = kv_oracle_sample(W, args.seed, args.cpu_baseline_seconds)
+        line["cpu_baseline"] = {"value": tps * 6 * H * D / 1e9, "unit": "GB/s", "cores": blas_threads(),
+                                "kind": "oracle", "sample": desc}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    return 0
 
 
 def main(argv=None):
@@ -521,6 +660,8 @@ def main(argv=None):
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
 
+    if W.kind == "kv":
+        return run_kv(args, W, torch, B, device, world, rank)
     step = (GemmStep if W.kind == "gemm" else MoeStep)(B, torch, W, args.seed + rank * 0, device)
     for _ in range(args.warmup):
         step()

@@ -244,6 +244,25 @@ enum {
 int w4a8_profile_start(void);
 int w4a8_profile_stop(int* launches, float* total_ms, int n);
 
+/* INT8 KV cache with static per-head scales (the Kimi 2.7T MoE W4A8 article,
+ * hotelren.com/news/5173946, section 5: the attention KV cache is quantised to INT8
+ * statically, one scale per head fixed from a little calibration data; the scale is
+ * the symmetric form of the LLM quantisation primer, section 2.1).
+ * Layout: x [T][H][D] bf16 row-major (token, head, channel); q [T][H][D] int8;
+ * scale [H] fp32.  D must be a multiple of 16 (16 <= D), 1 <= H <= 1024; x, q 16-byte
+ * aligned, scale 4-byte aligned (W4A8_EUNSUPPORTED / W4A8_EALIGN otherwise).
+ * Device pointers owned by the caller; asynchronous on `stream`.
+ *
+ * w4a8_kv_calibrate: scale[h] = max|x[:, h, :]| / 127 over the calibration tokens
+ *   (correctly rounded fp32 division); 0 for a head whose values are all zero (and
+ *   for T = 0).
+ * w4a8_kv_quant:     q = clamp(round(x / scale[h]), -127, 127), fp32 division, round
+ *   half to even; values beyond the calibrated range saturate; scale 0 -> q = 0.
+ * w4a8_kv_dequant:   x = bf16(q * scale[h]), the fp32 product rounded once (RNE). */
+int w4a8_kv_calibrate(const void* x_bf16, int T, int H, int D, float* scale, void* stream);
+int w4a8_kv_quant(const void* x_bf16, int T, int H, int D, const float* scale, int8_t* q, void* stream);
+int w4a8_kv_dequant(const int8_t* q, int T, int H, int D, const float* scale, void* x_bf16, void* stream);
+
 /* Human-readable name of a w4a8_status value. */
 const char* w4a8_status_string(int status);
 

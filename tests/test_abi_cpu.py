@@ -80,6 +80,15 @@ def test_host_validation_without_gpu(lib):
     assert lib.w4a8_moe_forward(fake, fake, 8, 256, 128, fake, 4, fake, fake, 9, fake, fake, 1 << 40, None) == EINVAL
     assert lib.w4a8_gemm(fake, fake, 4, fake, 256, 512, fake, None, fake, 8, None) == ENOSPACE
     assert lib.w4a8_last_device_error(None, None) == EINVAL
+    # INT8 KV cache
+    assert lib.w4a8_kv_quant(fake, 4, 8, 100, fake, fake, None) == EUNSUPPORTED  # D % 16
+    assert lib.w4a8_kv_quant(fake, 4, 2000, 128, fake, fake, None) == EUNSUPPORTED  # too many heads
+    assert lib.w4a8_kv_quant(fake, 4, 0, 128, fake, fake, None) == EINVAL
+    assert lib.w4a8_kv_quant(fake, 0, 8, 128, None, None, None) == 0  # nothing to do
+    assert lib.w4a8_kv_quant(vp((1 << 20) + 8), 4, 8, 128, fake, fake, None) == EALIGN
+    assert lib.w4a8_kv_dequant(fake, 4, 8, 128, None, fake, None) == EINVAL
+    assert lib.w4a8_kv_calibrate(fake, 4, 8, 128, None, None) == EINVAL
+    assert lib.w4a8_kv_calibrate(fake, 4, 8, 128, vp((1 << 20) + 2), None) == EALIGN
 
 
 def test_moe_workspace_regions(lib):

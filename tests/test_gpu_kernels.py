@@ -42,6 +42,11 @@ def test_quant_act_bit_exact(T, K, outl):
     if T > 3:
         x[2] = 0.0  # an all-zero row
         x[3, ::7] = 0.5  # ties at x/s = k + 0.5 are possible
+        # a row with max 1.0 (s = 1/127): +-0.5 and +-1.5 * 2^-k land within a few ulp of
+        # half-integers, the quantiser's slow (exact division) path
+        x[T - 1] = 0.0
+        x[T - 1, 0] = 1.0
+        x[T - 1, 1:9] = [0.5, -0.5, 0.75, -0.25, 0.125, 1.0, -1.0, 0.0625]
     q = torch.empty((T, O.padded_k(K)), dtype=torch.int8, device="cuda")
     s = torch.empty(T, dtype=torch.float32, device="cuda")
     B.w4a8_quant_act(dev_bf16(x), q, s)

@@ -33,6 +33,9 @@ _SIGS = {
     "w4a8_packed_bytes": ([_c_int, _c_int, _c_int, _c_int], _c_size),
     "w4a8_pack_weights": ([_vp, _c_int, _c_int, _c_int, _c_int, _vp, _c_size, _vp, _vp, _vp, _vp], _c_int),
     "w4a8_quant_act": ([_vp, _c_int, _c_int, _vp, _vp, _vp], _c_int),
+    "w4a8_kv_calibrate": ([_vp, _c_int, _c_int, _c_int, _vp, _vp], _c_int),
+    "w4a8_kv_quant": ([_vp, _c_int, _c_int, _c_int, _vp, _vp, _vp], _c_int),
+    "w4a8_kv_dequant": ([_vp, _c_int, _c_int, _c_int, _vp, _vp, _vp], _c_int),
     "w4a8_route_topk": ([_vp, _c_int, _c_int, _c_int, _vp, _vp, _vp], _c_int),
     "w4a8_moe_workspace_bytes": ([_c_int] * 5, _c_size),
     "w4a8_moe_host_workspace_bytes": ([_c_int] * 5, _c_size),
@@ -135,6 +138,32 @@ def w4a8_quant_act(x: torch.Tensor, q: torch.Tensor, s: torch.Tensor):
     _dev(s, torch.float32, "s")
     T, K = x.shape
     _check(lib().w4a8_quant_act(_ptr(x), T, K, _ptr(q), _ptr(s), _stream()), "w4a8_quant_act")
+
+
+def w4a8_kv_calibrate(x: torch.Tensor, scale: torch.Tensor):
+    """x: bf16 [T][H][D] calibration values; scale: float32 [H] (written)."""
+    _dev(x, torch.bfloat16, "x")
+    _dev(scale, torch.float32, "scale")
+    T, H, D = x.shape
+    _check(lib().w4a8_kv_calibrate(_ptr(x), T, H, D, _ptr(scale), _stream()), "w4a8_kv_calibrate")
+
+
+def w4a8_kv_quant(x: torch.Tensor, scale: torch.Tensor, q: torch.Tensor):
+    """x: bf16 [T][H][D]; scale: float32 [H]; q: int8 [T][H][D] (written)."""
+    _dev(x, torch.bfloat16, "x")
+    _dev(scale, torch.float32, "scale")
+    _dev(q, torch.int8, "q")
+    T, H, D = x.shape
+    _check(lib().w4a8_kv_quant(_ptr(x), T, H, D, _ptr(scale), _ptr(q), _stream()), "w4a8_kv_quant")
+
+
+def w4a8_kv_dequant(q: torch.Tensor, scale: torch.Tensor, x: torch.Tensor):
+    """q: int8 [T][H][D]; scale: float32 [H]; x: bf16 [T][H][D] (written)."""
+    _dev(q, torch.int8, "q")
+    _dev(scale, torch.float32, "scale")
+    _dev(x, torch.bfloat16, "x")
+    T, H, D = q.shape
+    _check(lib().w4a8_kv_dequant(_ptr(q), T, H, D, _ptr(scale), _ptr(x), _stream()), "w4a8_kv_dequant")
 
 
 def w4a8_route_topk(logits: torch.Tensor, k: int, ids: torch.Tensor, w: torch.Tensor):

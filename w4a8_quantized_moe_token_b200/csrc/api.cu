@@ -301,6 +301,45 @@ W4A8_EXPORT int w4a8_pack_weights(const void* w_bf16, int E, int N, int K, int l
                                  static_cast<cudaStream_t>(stream)));
 }
 
+namespace {
+int kv_check(int T, int H, int D) {
+    if (T < 0 || H < 1 || D < 16) return W4A8_EINVAL;
+    if (D % 16 != 0 || H > kv_max_heads()) return W4A8_EUNSUPPORTED;
+    return W4A8_OK;
+}
+}  // namespace
+
+W4A8_EXPORT int w4a8_kv_calibrate(const void* x_bf16, int T, int H, int D, float* scale, void* stream) {
+    const int c = kv_check(T, H, D);
+    if (c != W4A8_OK) return c;
+    if (scale == nullptr || (T > 0 && x_bf16 == nullptr)) return W4A8_EINVAL;
+    if (!aligned(x_bf16, 16) || !aligned(scale, 4)) return W4A8_EALIGN;
+    return to_status(launch_kv_calibrate(static_cast<const uint16_t*>(x_bf16), T, H, D, scale, sm_count(),
+                                         static_cast<cudaStream_t>(stream)));
+}
+
+W4A8_EXPORT int w4a8_kv_quant(const void* x_bf16, int T, int H, int D, const float* scale, int8_t* q,
+                              void* stream) {
+    const int c = kv_check(T, H, D);
+    if (c != W4A8_OK) return c;
+    if (T == 0) return W4A8_OK;
+    if (x_bf16 == nullptr || scale == nullptr || q == nullptr) return W4A8_EINVAL;
+    if (!aligned(x_bf16, 16) || !aligned(q, 16) || !aligned(scale, 4)) return W4A8_EALIGN;
+    return to_status(launch_kv_quant(static_cast<const uint16_t*>(x_bf16), T, H, D, scale, q, sm_count(),
+                                     static_cast<cudaStream_t>(stream)));
+}
+
+W4A8_EXPORT int w4a8_kv_dequant(const int8_t* q, int T, int H, int D, const float* scale, void* x_bf16,
+                                void* stream) {
+    const int c = kv_check(T, H, D);
+    if (c != W4A8_OK) return c;
+    if (T == 0) return W4A8_OK;
+    if (x_bf16 == nullptr || scale == nullptr || q == nullptr) return W4A8_EINVAL;
+    if (!aligned(x_bf16, 16) || !aligned(q, 16) || !aligned(scale, 4)) return W4A8_EALIGN;
+    return to_status(launch_kv_dequant(q, T, H, D, scale, static_cast<uint16_t*>(x_bf16), sm_count(),
+                                       static_cast<cudaStream_t>(stream)));
+}
+
 W4A8_EXPORT int w4a8_quant_act(const void* x_bf16, int T, int K, int8_t* q, float* s, void* stream) {
     if (T < 0 || K < 1) return W4A8_EINVAL;
     if (T == 0) return W4A8_OK;

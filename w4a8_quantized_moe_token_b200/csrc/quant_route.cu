@@ -204,10 +204,11 @@ __global__ void __launch_bounds__(256) quant_act_kernel(const uint16_t* __restri
     for (int k = lane; k < K; k += 32) amax = fmaxf(amax, fabsf(bf16_to_f32(xr[k])));
     amax = warp_max(amax);
     const float sc = __fdiv_rn(amax, 127.0f);
+    const float rinv = __fdiv_rn(1.0f, sc);
     int8_t* qr = q + (size_t)row * Kp;
     for (int k = lane; k < Kp; k += 32) {
         int c = 0;
-        if (k < K && amax > 0.f) c = quant_i8(bf16_to_f32(xr[k]), sc);
+        if (k < K && amax > 0.f) c = quant_i8_fast(bf16_to_f32(xr[k]), sc, rinv);
         qr[k] = (int8_t)c;
     }
     if (lane == 0) s[row] = sc;
@@ -526,12 +527,13 @@ __device__ __forceinline__ void quant_row_cta(const TIn* row, int len, int r, in
     __syncthreads();
     amax = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
     const float sc = __fdiv_rn(amax, 127.0f);
+    const float rinv = __fdiv_rn(1.0f, sc);
     auto emit = [&](int ci, const Chunk16& c) {
         uint32_t out[4] = {0u, 0u, 0u, 0u};
         if (amax > 0.f) {
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-                const uint32_t q = (uint32_t)(quant_i8(c.v[i], sc) & 0xFF);
+                const uint32_t q = (uint32_t)(quant_i8_fast(c.v[i], sc, rinv) & 0xFF);
                 out[i >> 2] |= q << (8 * (i & 3));
             }
         }
@@ -610,12 +612,13 @@ __global__ void __launch_bounds__(128) act_scatter_kernel(const uint16_t* __rest
     __syncthreads();
     amax = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
     const float sc = __fdiv_rn(amax, 127.0f);
+    const float rinv = __fdiv_rn(1.0f, sc);
     auto emit = [&](int ci, const Chunk16& c) {
         uint32_t out[4] = {0u, 0u, 0u, 0u};
         if (amax > 0.f) {
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-                const uint32_t q = (uint32_t)(quant_i8(c.v[i], sc) & 0xFF);
+                const uint32_t q = (uint32_t)(quant_i8_fast(c.v[i], sc, rinv) & 0xFF);
                 out[i >> 2] |= q << (8 * (i & 3));
             }
         }

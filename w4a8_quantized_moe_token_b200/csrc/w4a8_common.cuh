@@ -206,4 +206,19 @@ __device__ __forceinline__ int quant_i8(float x, float s) {
     return (int)r;
 }
 
+// The same code, bit for bit, with a multiply by inv = RN(1/s) in the common case.
+// With v = x/s exact, d = RN(v) (what quant_i8 rounds) and y = RN(x * inv):
+// |y - d| <= 3 * 2^-24 * |v| < 2.3e-5 for |v| < 128, so rint(y) and rint(d) can only
+// differ when y is that close to a half-integer (a rounding boundary, including the
+// ties that rint(d) sends to even); those values, and a y that is not finite, take
+// the exact division.  Beyond |v| = 128 both saturate to +-127.
+__device__ __forceinline__ int quant_i8_fast(float x, float s, float inv) {
+    const float y = __fmul_rn(x, inv);
+    const float f = __fsub_rn(y, floorf(y));
+    if (!(fabsf(y) <= 1.0e30f) || fabsf(__fsub_rn(f, 0.5f)) <= 6.103515625e-05f) return quant_i8(x, s);
+    float r = rintf(y);
+    r = fminf(fmaxf(r, -127.0f), 127.0f);
+    return (int)r;
+}
+
 }  // namespace w4a8

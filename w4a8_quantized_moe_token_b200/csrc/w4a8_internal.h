@@ -62,4 +62,13 @@ constexpr int kPermChunk = 256;       // slots per permutation chunk (multi-CTA 
 constexpr int kPermSmallSlots = 16384;  // up to this many slots the permutation runs in one CTA
 int perm_launch_count(int nslots);
 
+// INT8 KV cache (kv_int8.cu)
+int kv_max_heads();
+cudaError_t launch_kv_calibrate(const uint16_t* x, int T, int H, int D, float* scale, int sm_count,
+                                cudaStream_t stream);
+cudaError_t launch_kv_quant(const uint16_t* x, int T, int H, int D, const float* scale, int8_t* q, int sm_count,
+                            cudaStream_t stream);
+cudaError_t launch_kv_dequant(const int8_t* q, int T, int H, int D, const float* scale, uint16_t* x, int sm_count,
+                              cudaStream_t stream);
+
 }  // namespace w4a8

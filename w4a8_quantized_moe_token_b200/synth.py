@@ -23,7 +23,7 @@ from dataclasses import dataclass, field
 import numpy as np
 
 # tags that separate the random streams of the different tensors
-_TAG_X, _TAG_W_UP, _TAG_W_DOWN, _TAG_LOGITS, _TAG_IDS, _TAG_WTS, _TAG_OUTL, _TAG_RANK, _TAG_DENSE_W = range(9)
+_TAG_X, _TAG_W_UP, _TAG_W_DOWN, _TAG_LOGITS, _TAG_IDS, _TAG_WTS, _TAG_OUTL, _TAG_RANK, _TAG_DENSE_W, _TAG_KV = range(10)
 
 WEIGHT_STD = 0.02
 
@@ -33,7 +33,7 @@ class Workload:
     """One synthetic layer: a dense GEMM or a MoE expert FFN."""
 
     name: str
-    kind: str  # "gemm" | "moe"
+    kind: str  # "gemm" | "moe" | "kv"
     # dense GEMM
     M: int = 0
     K: int = 0
@@ -59,6 +59,9 @@ WORKLOADS = {
     "large_decode": Workload("large_decode", "moe", E=384, topk=8, T=256, H=7168, F=2048,
                              routing="zipf", zipf_s=1.1),
     "prefill": Workload("prefill", "moe", E=384, topk=8, T=16384, H=7168, F=2048, routing="uniform"),
+    # INT8 KV cache of one attention layer: 32768 tokens x 8 KV heads x 128 channels,
+    # static per-head scales calibrated on the first 1024 tokens
+    "kv_int8": Workload("kv_int8", "kv", T=32768, extra={"heads": 8, "head_dim": 128, "calib_tokens": 1024}),
 }
 
 
@@ -134,6 +137,14 @@ def dense_gemm_inputs(seed: int, M: int, K: int, N: int):
     x = normal_bf16(_rng(seed, _TAG_X), (M, K))
     w = normal_bf16(_rng(seed, _TAG_DENSE_W), (N, K), WEIGHT_STD)
     return x, w
+
+
+def kv_cache(seed: int, T: int, H: int, D: int) -> np.ndarray:
+    """Keys or values of one attention layer [T][H][D]: N(0,1) times a seeded
+    per-head magnitude in [0.5, 4), in bf16 (heads differ in range, as the per-head
+    scales assume)."""
+    mag = _rng(seed, _TAG_KV, 0).uniform(0.5, 4.0, size=(1, H, 1)).astype(np.float32)
+    return bf16_round(normal_bf16(_rng(seed, _TAG_KV, 1), (T, H, D)) * mag)
 
 
 def router_logits(seed: int, T: int, E: int) -> np.ndarray:
