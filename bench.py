@@ -443,6 +443,19 @@ class OracleSample:
 
 
 # --------------------------------------------------------------------------- #
+def max_over_ranks(x: float, torch, device, world: int) -> float:
+    """The largest of every rank's x (the job's time is its slowest rank's)."""
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank: float, world: int, max_ms: float) -> float:
+    """Whole-job throughput: the units all ranks processed over the slowest rank's time."""
+    return units_per_rank * world / (max_ms / 1e3)
+
+
 def dist_env():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -567,10 +580,7 @@ def run_kv(args, W, torch, B, device, world, rank):
     sampler.stop()
     qms = sum(e[0].elapsed_time(e[1]) for e in ev) / args.steps
     dms = sum(e[1].elapsed_time(e[2]) for e in ev) / args.steps
-    ms_t = torch.tensor([qms + dms], dtype=torch.float64, device=device)
-    if world > 1:
-        torch.distributed.all_reduce(ms_t, op=torch.distributed.ReduceOp.MAX)
-    ms = float(ms_t.item())
+    ms = max_over_ranks(qms + dms, torch, device, world)
     n = T * H * D
     qbytes, dbytes = 3 * n, 3 * n  # bf16 in + int8 out; int8 in + bf16 out
     # end to end: host cache in, round trip, host cache out
@@ -600,7 +610,7 @@ def run_kv(args, W, torch, B, device, world, rank):
     roof["peak_source"] = f"{peaks['source']}: MEASURED_PEAKS hbm_gbs"
     total_bytes = (qbytes + dbytes) * world
     line = {
-        "metric": KV_METRIC, "value": total_bytes / (ms / 1e3) / 1e9, "unit": "GB/s", "n_gpus": world,
+        "metric": KV_METRIC, "value": whole_job_rate(qbytes + dbytes, world, ms) / 1e9, "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "int8", "data": "synthetic", "config": kv_config(W),
         "tokens_per_s": T * world / (ms / 1e3),
@@ -692,16 +702,10 @@ def main(argv=None):
     prof = B.w4a8_profile_stop()
     assert B.w4a8_last_device_error(step.ws) == 0, "device error during the timed steps"
     ms = sum(a.elapsed_time(b) for a, b in zip(starts, ends)) / args.steps
-    ms_t = torch.tensor([ms], dtype=torch.float64, device=device)
-    if world > 1:
-        torch.distributed.all_reduce(ms_t, op=torch.distributed.ReduceOp.MAX)
-    ms_max = float(ms_t.item())
+    ms_max = max_over_ranks(ms, torch, device, world)
 
     e2e_ms, h2d, d2h = step.e2e(args.steps, args.warmup)
-    e2e_t = torch.tensor([e2e_ms], dtype=torch.float64, device=device)
-    if world > 1:
-        torch.distributed.all_reduce(e2e_t, op=torch.distributed.ReduceOp.MAX)
-    e2e_ms = float(e2e_t.item())
+    e2e_ms = max_over_ranks(e2e_ms, torch, device, world)
 
     acct = step.acct
     tokens = (W.T if W.kind == "moe" else W.M) * world
@@ -741,7 +745,7 @@ def main(argv=None):
 
     line = {
         "metric": METRIC,
-        "value": tokens / sec,
+        "value": whole_job_rate(tokens // world, world, ms_max),
         "unit": "tokens/s",
         "n_gpus": world,
         "steps": args.steps,
@@ -759,7 +763,7 @@ def main(argv=None):
         "roofline": roof,
         "kernels": kernels,
         "gpu_launches": sum(v["launches"] for v in kernels.values()),
-        "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+        "e2e": {"value": whole_job_rate(tokens // world, world, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "clocks": sampler.summary(),
     }
