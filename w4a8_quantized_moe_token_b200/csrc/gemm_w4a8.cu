@@ -56,12 +56,10 @@ constexpr long long kWaitLimitCycles = 4000000000ll;  // ~2 s: a bounded wait
 //   BN    : tokens per tile at most (MMA N <= BN)
 //   NS    : shared-memory stages        NA : tensor-memory A slots
 //   ND    : INT32 accumulators          NEPI: epilogue warpgroups (split the columns)
-//   MAGIC : accumulator pre-load (see above)
 //   NCG   : converter warpgroups (they take alternate steps)
-template <int BN_, int NS_, int NA_, int ND_, int NEPI_, bool MAGIC_, int NCG_>
+template <int BN_, int NS_, int NA_, int ND_, int NEPI_, int NCG_>
 struct Cfg {
     static constexpr int BN = BN_, NS = NS_, NA = NA_, ND = ND_, NEPI = NEPI_, NCG = NCG_;
-    static constexpr bool kMagic = MAGIC_;
     static constexpr int kNSC = 32;       // scale ring slots (>= NA + ND)
     static constexpr int kCW = BN / NEPI;  // accumulator columns per epilogue thread
     // warpgroups: NCG converter groups, NEPI epilogue groups, 1 control group
@@ -87,7 +85,6 @@ struct Cfg {
     static_assert(kNSC >= NA + ND, "scale ring too small");
     static_assert(NS % 2 == 0, "the two producers own the stages of one parity each");
     static_assert(kCW % 16 == 0 && (kCW <= 64 || kCW % 64 == 0), "epilogue column split");
-    static_assert(MAGIC_, "accumulators are preloaded with 1.5 * 2^23");
     // shared memory carve-up
     static constexpr int kOffB = 0;  // 1024-aligned (128-byte swizzle atoms)
     static constexpr int kOffA = kOffB + NS * kBStageBytes;
@@ -516,7 +513,7 @@ __global__ void __launch_bounds__(C::kThreads, 1) gemm_w4a8_kernel(const GemmArg
 #undef SCFULL_BAR
 #undef FINAL_BAR
 
-using CfgLarge = Cfg<128, 8, 4, 3, 2, true, 1>;  // many tokens per expert
+using CfgLarge = Cfg<128, 8, 4, 3, 2, 1>;  // many tokens per expert
 
 template <class C, bool kPartials>
 cudaError_t launch_cfg(const GemmArgs& a, int num_ctas, cudaStream_t stream) {
