@@ -473,7 +473,8 @@ def run_reference(args, W):
         vals = [kv_oracle_sample(W, args.seed, target) for _ in range(args.steps)]
         value = statistics.mean(v[0] for v in vals) * 6 * H * D / 1e9
         line = {"impl": "reference", "metric": KV_METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
-                "steps": args.steps, "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True,
+                "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": statistics.mean(v[2] for v in vals) * 1e3, "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": kv_config(W),
                 "cpu_baseline": {"value": value, "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
                                  "sample": vals[0][1]},
@@ -538,7 +539,7 @@ def kv_oracle_sample(W, seed, target_s):
     t0 = time.perf_counter()
     O.kv_dequantize(O.kv_quantize(x, s), s)
     t = time.perf_counter() - t0
-    return n / t, f"{n} of {W.T} tokens"
+    return n / t, f"{n} of {W.T} tokens", t
 
 
 def run_kv(args, W, torch, B, device, world, rank):
@@ -623,7 +624,7 @@ def run_kv(args, W, torch, B, device, world, rank):
         "clocks": sampler.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        tps, desc = kv_oracle_sample(W, args.seed, args.cpu_baseline_seconds)
+        tps, desc, _ = kv_oracle_sample(W, args.seed, args.cpu_baseline_seconds)
         line["cpu_baseline"] = {"value": tps * 6 * H * D / 1e9, "unit": "GB/s", "cores": blas_threads(),
                                 "kind": "oracle", "sample": desc}
     if rank == 0:
