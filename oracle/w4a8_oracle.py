@@ -40,7 +40,9 @@ its reason in the design notes):
       interpolation at q * (n - 1), in fp32 with fractions fp32(0.127) and fp32(0.873);
   R20 INT8 KV cache: static symmetric per-head scale max|x|/127 over the calibration
       values (0 for an all-zero head, which then quantises to 0); dequantisation rounds
-      the fp32 product q * scale once to bf16.
+      the fp32 product q * scale once to bf16;
+  R21 W4A16 comparison layer: activations unquantised bf16, h rounded to bf16 between
+      the projections.
 
 Parity status: every function below is pinned by tests/test_oracle_pins.py
 against values the pages print, closed forms, brute force or an independent
@@ -459,3 +461,39 @@ def kv_dequantize(q: np.ndarray, scale: np.ndarray) -> np.ndarray:
     returned as float32 values (R20)."""
     y = np.asarray(q, dtype=np.float32) * np.asarray(scale, dtype=np.float32)[None, :, None]
     return round_to_bf16(y.astype(np.float64)).astype(np.float32)
+
+
+# --------------------------------------------------------------------------- #
+# W4A16: the same INT4 weights with 16-bit activations (the comparison point)
+# --------------------------------------------------------------------------- #
+def w4a16_linear(x, codes, scale, zp) -> np.ndarray:
+    """y[m, n] = sum_k x[m, k] * (code[n, k] - zp[n, g(k)]) * scale[n, g(k)]  (fp64).
+
+    [P2] §1 and §3.3: W4A16 keeps the 4-bit weights but multiplies with 16-bit
+    activations (no activation quantisation); x [M][K] holds bf16 values.
+    """
+    x = pad_k(np.asarray(x, dtype=np.float32)).astype(np.float64)
+    return x @ dequantize_weights(codes, scale, zp).T
+
+
+def w4a16_expert_forward(x, qe: QuantExpert, F: int) -> np.ndarray:
+    """One expert with 16-bit activations: up GEMM -> SwiGLU -> h rounded to bf16
+    (R21: the activations between the projections stay 16-bit) -> down GEMM."""
+    h = round_to_bf16(swiglu(w4a16_linear(x, *qe.up), F))
+    return w4a16_linear(h, *qe.down)
+
+
+def moe_forward_w4a16(x, ids, w, experts: dict, E: int, F: int):
+    """The MoE expert FFN with W4A16 experts (same routing, permutation and combine
+    as moe_forward), output rounded to bf16."""
+    x = np.asarray(x, dtype=np.float32)
+    T, H = x.shape
+    k = ids.shape[1]
+    counts, offs, perm, inv = permute(ids, E)
+    y2 = np.zeros((T * k, H), dtype=np.float64)
+    for e in range(E):
+        if counts[e] == 0:
+            continue
+        tok = perm[offs[e]:offs[e + 1]] // k
+        y2[offs[e]:offs[e + 1]] = w4a16_expert_forward(x[tok], experts[e], F)[:, :H]
+    return round_to_bf16(combine(y2, w, inv, T, k))

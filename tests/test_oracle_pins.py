@@ -502,3 +502,51 @@ def test_kv_int8_roundtrip_saturation_and_zero_head():
     for (t, h, d) in [(1, 0, 3), (5, 2, 31), (15, 1, 0)]:
         ref = max(-127, min(127, int(np.rint(np.float32(x[t, h, d]) / s[h]))))
         assert q[t, h, d] == ref
+
+
+# --------------------------------------------------------------------------- #
+# W4A16 comparison layer
+# --------------------------------------------------------------------------- #
+def test_w4a16_linear_brute_force():
+    rng = np.random.default_rng(31)
+    x = synth.bf16_round(rng.standard_normal((3, 200)).astype(np.float32))
+    w = synth.bf16_round((rng.standard_normal((4, 200)) * 0.02).astype(np.float32))
+    codes, scale, zp = O.quantize_weights(w)
+    y = O.w4a16_linear(x, codes, scale, zp)
+    for m in range(3):
+        for n in range(4):
+            ref = 0.0
+            for kk in range(200):
+                g = kk // 128
+                ref += float(x[m, kk]) * (int(codes[n, kk]) - float(zp[n, g])) * float(scale[n, g])
+            assert abs(y[m, n] - ref) <= 1e-12 * max(1.0, abs(ref))
+
+
+def test_w4a16_reduces_to_w4a8_on_int8_exact_activations():
+    # rows that are exactly s * q with q in [-127, 127] (the row maximum at 127) and s a
+    # power of two are quantised by the activation quantiser without loss, so the
+    # W4A16 layer (fp64 matmul on dequantised weights) and the W4A8 layer (exact INT32
+    # group partials, then the fold) must agree
+    rng = np.random.default_rng(32)
+    q = rng.integers(-127, 128, size=(5, 256))
+    q[:, 0] = 127
+    s = np.float32(2.0 ** -6)
+    x = (q.astype(np.float32) * s).astype(np.float32)
+    w = synth.bf16_round((rng.standard_normal((8, 256)) * 0.02).astype(np.float32))
+    codes, scale, zp = O.quantize_weights(w)
+    qa, sa = O.quantize_act(x)
+    assert np.array_equal(qa[:, :256], q) and np.all(sa == s)  # lossless
+    np.testing.assert_allclose(O.w4a16_linear(x, codes, scale, zp), O.w4a8_linear(qa, sa, codes, scale, zp),
+                               rtol=1e-12, atol=1e-15)
+
+
+def test_w4a16_layer_single_expert_top1():
+    rng = np.random.default_rng(33)
+    T, H, F = 6, 256, 128
+    x = synth.bf16_round(rng.standard_normal((T, H)).astype(np.float32))
+    qe = O.QuantExpert(synth.bf16_round((rng.standard_normal((2 * F, H)) * 0.02).astype(np.float32)),
+                       synth.bf16_round((rng.standard_normal((H, F)) * 0.02).astype(np.float32)))
+    ids = np.zeros((T, 1), np.int32)
+    out = O.moe_forward_w4a16(x, ids, np.ones((T, 1)), {0: qe}, 1, F)
+    direct = O.round_to_bf16(O.w4a16_expert_forward(x, qe, F))
+    assert np.array_equal(out, direct)
