@@ -17,6 +17,9 @@
  *     (weight scale of the group) x (token scale).
  * "round" is round-half-to-even everywhere; the min/max range of a weight group
  * is widened to contain 0; an fp16 scale that rounds to 0 is stored as 1.
+ * The packer also offers a symmetric INT4 scheme and a percentile-clipped range
+ * (W4A8_PACK_SYMMETRIC, W4A8_PACK_CLIP999) in the same packed format, and the
+ * library carries an INT8 KV cache with static per-head scales (w4a8_kv_*).
  *
  * Conventions for every entry point:
  *   - pointers are DEVICE pointers owned by the caller unless a parameter says
