@@ -63,16 +63,16 @@ INT4_SYM_ZP = 8  # the symmetric codes are stored as q + 8
 # --------------------------------------------------------------------------- #
 # shapes
 # --------------------------------------------------------------------------- #
-def padded_k(K: int) -> int:
+def padded_k(K: int, group: int = GROUP) -> int:
     """K rounded up to a whole number of groups ([P2] §2.1: pad the matrix to a
     multiple of the group size at conversion time)."""
-    return ((K + GROUP - 1) // GROUP) * GROUP
+    return ((K + group - 1) // group) * group
 
 
-def pad_k(a: np.ndarray) -> np.ndarray:
+def pad_k(a: np.ndarray, group: int = GROUP) -> np.ndarray:
     """Zero-pad the last axis to padded_k ([P2] §2.1)."""
     K = a.shape[-1]
-    Kp = padded_k(K)
+    Kp = padded_k(K, group)
     if Kp == K:
         return a
     pad = [(0, 0)] * (a.ndim - 1) + [(0, Kp - K)]
@@ -100,7 +100,7 @@ def group_range_percentile(v: np.ndarray):
     return lo.astype(np.float32), hi.astype(np.float32)
 
 
-def quantize_weights(w: np.ndarray, clip999: bool = False):
+def quantize_weights(w: np.ndarray, clip999: bool = False, group: int = GROUP):
     """Group-wise asymmetric INT4 of one weight matrix w [N][K] (float32, bf16 values).
 
     [P2] §2.2, per group of 128 along K:
@@ -110,19 +110,22 @@ def quantize_weights(w: np.ndarray, clip999: bool = False):
     with readings R2-R6 (min/max widened to contain 0; fp16 scale used for the
     codes; round half to even; fp32 correctly rounded division).  With clip999 the
     range is the group's 0.1th..99.9th percentile instead of its min..max ([P2] §2.2,
-    R19); values outside it land on codes 0 or 15 through the clamp.
+    R19); values outside it land on codes 0 or 15 through the clamp.  `group` is the
+    number of weights per group along K ([P1] §5 names 128 or 256; [P2] §2.1 trades
+    accuracy against the scale storage; 128 unless stated).
 
     Returns codes uint8 [N][Kp] (values 0..15), scale float16 [N][G], zp float16 [N][G].
     """
-    w = pad_k(np.asarray(w, dtype=np.float32))
+    assert not clip999 or group == GROUP, "the percentile positions are those of 128-value groups"
+    w = pad_k(np.asarray(w, dtype=np.float32), group)
     N, Kp = w.shape
-    G = Kp // GROUP
+    G = Kp // group
     codes = np.zeros((N, Kp), dtype=np.uint8)
     scale = np.zeros((N, G), dtype=np.float16)
     zp = np.zeros((N, G), dtype=np.float16)
     f15 = np.float32(INT4_MAX)
     for g in range(G):
-        v = w[:, g * GROUP:(g + 1) * GROUP]  # [N][128]
+        v = w[:, g * group:(g + 1) * group]  # [N][group]
         if clip999:
             lo, hi = group_range_percentile(v)
         else:
@@ -136,13 +139,13 @@ def quantize_weights(w: np.ndarray, clip999: bool = False):
         # R4, R6; the zero point is an integer index offset, so -0.0 is stored as 0
         z = np.clip(np.rint(-mn / sf), 0, INT4_MAX) + np.float32(0)
         q = np.rint(v / sf[:, None]) + z[:, None]
-        codes[:, g * GROUP:(g + 1) * GROUP] = np.clip(q, 0, INT4_MAX).astype(np.uint8)
+        codes[:, g * group:(g + 1) * group] = np.clip(q, 0, INT4_MAX).astype(np.uint8)
         scale[:, g] = s16
         zp[:, g] = z.astype(np.float16)
     return codes, scale, zp
 
 
-def quantize_weights_symmetric(w: np.ndarray):
+def quantize_weights_symmetric(w: np.ndarray, group: int = GROUP):
     """Group-wise symmetric INT4 of one weight matrix w [N][K] (the packer's
     symmetric variant).
 
@@ -156,29 +159,31 @@ def quantize_weights_symmetric(w: np.ndarray):
 
     Returns codes uint8 [N][Kp] (values 1..15), scale float16 [N][G], zp float16 [N][G] (all 8).
     """
-    w = pad_k(np.asarray(w, dtype=np.float32))
+    w = pad_k(np.asarray(w, dtype=np.float32), group)
     N, Kp = w.shape
-    G = Kp // GROUP
+    G = Kp // group
     codes = np.zeros((N, Kp), dtype=np.uint8)
     scale = np.zeros((N, G), dtype=np.float16)
     zp = np.full((N, G), INT4_SYM_ZP, dtype=np.float16)
     qmax = np.float32(INT4_SYM_QMAX)
     for g in range(G):
-        v = w[:, g * GROUP:(g + 1) * GROUP]  # [N][128]
+        v = w[:, g * group:(g + 1) * group]  # [N][group]
         amax = np.abs(v).max(axis=1)
         s16 = (amax / qmax).astype(np.float16)  # fp32 division, then fp16 RNE (R5, R6)
         s16[s16 == 0] = np.float16(1.0)
         sf = s16.astype(np.float32)
         q = np.clip(np.rint(v / sf[:, None]), -qmax, qmax)  # R4, R6
-        codes[:, g * GROUP:(g + 1) * GROUP] = (q + INT4_SYM_ZP).astype(np.uint8)
+        codes[:, g * group:(g + 1) * group] = (q + INT4_SYM_ZP).astype(np.uint8)
         scale[:, g] = s16
     return codes, scale, zp
 
 
 def dequantize_weights(codes: np.ndarray, scale: np.ndarray, zp: np.ndarray) -> np.ndarray:
-    """weight ~= (index - zero_point) * scale  ([P2] §2.1), in fp64, shape [N][Kp]."""
-    sc = np.repeat(scale.astype(np.float64), GROUP, axis=1)
-    z = np.repeat(zp.astype(np.float64), GROUP, axis=1)
+    """weight ~= (index - zero_point) * scale  ([P2] §2.1), in fp64, shape [N][Kp]
+    (the group size is Kp / G)."""
+    group = codes.shape[1] // scale.shape[1]
+    sc = np.repeat(scale.astype(np.float64), group, axis=1)
+    z = np.repeat(zp.astype(np.float64), group, axis=1)
     return (codes.astype(np.float64) - z) * sc
 
 
@@ -203,14 +208,15 @@ def unpack_nibbles(packed: np.ndarray) -> np.ndarray:
 # --------------------------------------------------------------------------- #
 # a2 / a6: per-token symmetric INT8 ([P3] §2.1, [P1] §4.3 step 3)
 # --------------------------------------------------------------------------- #
-def quantize_act(x: np.ndarray):
+def quantize_act(x: np.ndarray, group: int = GROUP):
     """Dynamic per-token symmetric INT8 of x [T][K] (fp32 values).
 
     [P3] §2.1 symmetric form: scale = max|x| / (2^(b-1) - 1), q = round(x / scale),
     computed per token at run time ([P1] §4.3).  fp32 arithmetic, round half to even,
     codes clamped to [-127, 127] (R7).  A row of zeros gets scale 0 and codes 0.
 
-    Returns q int8 [T][Kp] (zero padded) and s float32 [T].
+    Returns q int8 [T][Kp] (zero padded to a whole number of weight groups) and
+    s float32 [T].
     """
     x = np.asarray(x, dtype=np.float32)
     T = x.shape[0]
@@ -221,7 +227,7 @@ def quantize_act(x: np.ndarray):
     if nz.any():
         r = np.rint(x[nz] / s[nz][:, None])
         q[nz] = np.clip(r, -INT8_QMAX, INT8_QMAX).astype(np.int8)
-    return pad_k(q), s
+    return pad_k(q, group), s
 
 
 # --------------------------------------------------------------------------- #
@@ -296,12 +302,14 @@ def group_partials(qa: np.ndarray, codes: np.ndarray, zp: np.ndarray) -> np.ndar
     qa = np.asarray(qa)
     M, Kp = qa.shape
     N = codes.shape[0]
-    G = Kp // GROUP
+    G = zp.shape[1]
+    group = Kp // G  # 128 unless the weights were quantised with another group size
+    assert group * G == Kp and codes.shape[1] == Kp
     acc = np.zeros((M, N, G), dtype=np.int64)
     for g in range(G):
-        sl = slice(g * GROUP, (g + 1) * GROUP)
-        a = qa[:, sl].astype(np.float64)  # [M][128]
-        wq = codes[:, sl].astype(np.float64) - zp[:, g].astype(np.float64)[:, None]  # [N][128]
+        sl = slice(g * group, (g + 1) * group)
+        a = qa[:, sl].astype(np.float64)  # [M][group]
+        wq = codes[:, sl].astype(np.float64) - zp[:, g].astype(np.float64)[:, None]  # [N][group]
         acc[:, :, g] = np.rint(a @ wq.T).astype(np.int64)
     return acc
 

@@ -320,6 +320,37 @@ def test_linear_equals_dequantized_matmul():
     assert rms(y - exact) < 0.2 * rms(exact)
 
 
+@pytest.mark.parametrize("group", [64, 256])
+def test_other_group_sizes(group):
+    # [P1] section 5 names group sizes 128 or 256; [P2] section 2.1 trades accuracy
+    # against scale storage.  Brute-force partials, the dequantised formulation, the
+    # half-step bound, padding to the group and the storage accounting per group size.
+    rng = np.random.default_rng(group)
+    K = 300
+    Kp = O.padded_k(K, group)
+    assert Kp == -(-K // group) * group
+    x = synth.bf16_round(rng.standard_normal((3, K)).astype(np.float32))
+    w = synth.bf16_round((rng.standard_normal((5, K)) * 0.02).astype(np.float32))
+    qa, sa = O.quantize_act(x, group)
+    codes, scale, zp = O.quantize_weights(w, group=group)
+    assert codes.shape == (5, Kp) and scale.shape == (5, Kp // group) and qa.shape == (3, Kp)
+    deq = O.dequantize_weights(codes, scale, zp)
+    sc = np.repeat(scale.astype(np.float64), group, axis=1)
+    assert np.all(np.abs(O.pad_k(w, group) - deq) <= sc / 2 * (1 + 1e-3))
+    assert np.all(deq[:, K:] == 0.0)  # padding is exact
+    acc = O.group_partials(qa, codes, zp)
+    for m, n, g in [(0, 0, 0), (2, 4, Kp // group - 1), (1, 2, 0)]:
+        ref = sum(int(qa[m, kk]) * (int(codes[n, kk]) - int(zp[n, g])) for kk in range(g * group, (g + 1) * group))
+        assert acc[m, n, g] == ref
+    y = O.w4a8_linear(qa, sa, codes, scale, zp)
+    ref = (qa.astype(np.float64) * sa.astype(np.float64)[:, None]) @ deq.T
+    np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-15)
+    # 4 bytes of fp16 scale + zero point per group: 4 / group bytes per weight
+    assert scale.nbytes + zp.nbytes == 4 * codes.size // group
+    cs, ss, zs = O.quantize_weights_symmetric(w, group)
+    assert ss.shape == scale.shape and np.all(zs == 8) and cs.max() <= 15
+
+
 # --------------------------------------------------------------------------- #
 # routing and permutation
 # --------------------------------------------------------------------------- #
