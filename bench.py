@@ -2,6 +2,11 @@
 """Benchmark of the W4A8 MoE expert FFN on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload toy_moe] [--impl ours|reference]
+                    [--weights asym|sym|clip999] [--no-cpu-baseline]
+
+Workloads: dense_gemm, toy_moe (default), decode, large_decode, prefill (MoE
+layers) and kv_int8 (the INT8 KV cache round trip, reported in GB/s).  --weights
+selects the packer's scheme (asymmetric INT4, symmetric, or the percentile range).
 
 One step = one forward of the whole hot path (routing when the workload routes
 from logits, permutation, INT8 activation quant, up GEMM + SwiGLU, requant, down
