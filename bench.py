@@ -1,12 +1,21 @@
 #!/usr/bin/env python
 """Benchmark of the W4A8 MoE expert FFN on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload toy_moe] [--impl ours|reference]
-                    [--weights asym|sym|clip999] [--no-cpu-baseline]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload prefill] [--impl ours|reference]
+                    [--weights asym|sym|clip999] [--no-cpu-baseline] [--no-extra]
 
-Workloads: dense_gemm, toy_moe (default), decode, large_decode, prefill (MoE
-layers) and kv_int8 (the INT8 KV cache round trip, reported in GB/s).  --weights
-selects the packer's scheme (asymmetric INT4, symmetric, or the percentile range).
+Workloads: dense_gemm, toy_moe, decode, large_decode, prefill (the default: the
+largest MoE layer, 384 experts, top-8, 16384 tokens, hidden 7168, expert ffn 2048,
+INT8-tensor-bound) and kv_int8 (the INT8 KV cache round trip, reported in GB/s).
+--weights selects the packer's scheme (asymmetric INT4, symmetric, or the
+percentile range).  On one GPU the default run also times the two HBM-bound decode
+layers (large_decode reusing the packed 384-expert weights, and decode) and reports
+each under "extra" with its own step time, roofline and kernel table (--no-extra
+skips them).
+
+The INT8 tensor-core peak that tensor-bound kernels are compared with is measured
+in the same run, before the timed steps: torch._int_mm (cuBLASLt) on 8192^3 INT8
+operands, best of 10, CUDA events, with the SM clock sampled meanwhile.
 
 One step = one forward of the whole hot path (routing when the workload routes
 from logits, permutation, INT8 activation quant, up GEMM + SwiGLU, requant, down
@@ -41,7 +50,7 @@ from w4a8_quantized_moe_token_b200 import synth  # noqa: E402
 
 METRIC = "W4A8 MoE FFN tokens/s, TOPS and weight GB/s on 1 B200; % of HBM / INT8 roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
-INT8_OVER_BF16 = 4.5 / 2.25  # nominal dense INT8 / BF16 tensor peak ratio on B200
+INT8_OVER_BF16 = 4.5 / 2.25  # nominal dense INT8 / BF16 tensor peak ratio on B200 (used only if the measurement fails)
 
 
 # --------------------------------------------------------------------------- #
@@ -222,7 +231,7 @@ def pack_experts(B, torch, W, seed, device):
 
 
 class MoeStep:
-    def __init__(self, B, torch, W, seed, device):
+    def __init__(self, B, torch, W, seed, device, packed=None):
         self.B, self.torch, self.W, self.device = B, torch, W, device
         inp = synth.moe_inputs(W, seed)
         self.x_host = inp["x"]
@@ -242,37 +251,17 @@ class MoeStep:
             self.ids.copy_(torch.from_numpy(inp["ids"]))
             self.w.copy_(torch.from_numpy(inp["wts"]))
         self.logits_host = inp.get("logits")
-        self.packed_up, self.packed_down = pack_experts(B, torch, W, seed, device)
+        self.packed_up, self.packed_down = packed if packed is not None else pack_experts(B, torch, W, seed, device)
         self.out = torch.empty((T, H), dtype=torch.bfloat16, device=device)
         self.ws = B.empty_aligned(B.w4a8_moe_workspace_bytes(T, E, k, H, F), device)
         self.acct = moe_accounting(W, self.ids_host)
-        self.route_ms = 0.0
-        self.route_launches = 0
-        self.timing_route = False
 
     def __call__(self):
         B, W = self.B, self.W
         if self.logits is not None:
-            if self.timing_route:
-                a = self.torch.cuda.Event(enable_timing=True)
-                b = self.torch.cuda.Event(enable_timing=True)
-                a.record()
             B.w4a8_route_topk(self.logits, W.topk, self.ids, self.w)
-            if self.timing_route:
-                b.record()
-                self._route_events.append((a, b))
-                self.route_launches += 1
         B.w4a8_moe_forward(self.packed_up, self.packed_down, W.E, W.H, W.F, self.x, self.ids, self.w, self.out,
                            self.ws)
-
-    def start_route_timing(self):
-        self._route_events = []
-        self.route_launches = 0
-        self.timing_route = True
-
-    def stop_route_timing(self):
-        self.timing_route = False
-        self.route_ms = sum(a.elapsed_time(b) for a, b in self._route_events)
 
     def e2e(self, steps, warmup):
         """Same metric through the public API with HOST inputs/outputs: per step the
@@ -290,18 +279,13 @@ class MoeStep:
             def step():
                 B.w4a8_moe_forward_host(self.packed_up, self.packed_down, E, H, F, x_h, ids_h, w_h, out_h, ws)
         else:
+            # routed on the device from the router logits: one C-ABI call with host buffers
             lg_h = torch.from_numpy(synth.bf16_bits(self.logits_host).view(np.int16)).view(torch.bfloat16).pin_memory()
-            x_d = torch.empty_like(self.x)
-            lg_d = torch.empty_like(self.logits)
+            ws = B.empty_aligned(B.w4a8_moe_host_workspace_bytes(T, E, k, H, F), self.device)
             h2d = x_h.numel() * 2 + lg_h.numel() * 2
 
             def step():
-                x_d.copy_(x_h, non_blocking=True)
-                lg_d.copy_(lg_h, non_blocking=True)
-                B.w4a8_route_topk(lg_d, k, self.ids, self.w)
-                B.w4a8_moe_forward(self.packed_up, self.packed_down, E, H, F, x_d, self.ids, self.w, self.out,
-                                   self.ws)
-                out_h.copy_(self.out, non_blocking=True)
+                B.w4a8_moe_forward_logits_host(self.packed_up, self.packed_down, E, H, F, x_h, lg_h, k, out_h, ws)
         for _ in range(warmup):
             step()
         torch.cuda.synchronize()
@@ -332,17 +316,10 @@ class GemmStep:
         self.y = torch.empty((W.M, W.N), dtype=torch.float32, device=device)
         self.ws = B.empty_aligned(B.w4a8_gemm_workspace_bytes(W.M, W.N, W.K), device)
         self.acct = gemm_accounting(W)
-        self.route_ms, self.route_launches = 0.0, 0
 
     def __call__(self):
         self.B.w4a8_quant_act(self.x, self.q, self.s)
         self.B.w4a8_gemm(self.q, self.s, self.packed, self.W.N, self.W.K, self.y, self.ws)
-
-    def start_route_timing(self):
-        pass
-
-    def stop_route_timing(self):
-        pass
 
     def e2e(self, steps, warmup):
         torch = self.torch
@@ -384,9 +361,10 @@ class OracleSample:
     """The oracle forward on a bounded token sample of the workload (weights
     quantised once beforehand, untimed -- the GPU step excludes packing too)."""
 
-    def __init__(self, W, seed, target_s):
+    def __init__(self, W, seed, target_s, max_experts=16):
         from oracle import w4a8_oracle as O
         self.O, self.W, self.seed = O, W, seed
+        self.reps = 1
         if W.kind == "gemm":
             x, w = synth.dense_gemm_inputs(seed, W.M, W.K, W.N)
             self.x, self.qw = x, oracle_quant(O)(w)
@@ -401,13 +379,22 @@ class OracleSample:
         else:
             self.logits = None
             self.ids, self.w = inp["ids"], inp["wts"].astype(np.float64)
-        # size the token sample: time a few tokens, scale to the target
+        # size the token sample: time a few tokens, scale to the target.  Every expert a
+        # sampled token touches must be quantised first (about a second each for the
+        # 384-expert layers), so the sample is also capped at max_experts experts; a
+        # sample smaller than the target is run `reps` times per timing.
         self.experts = {}
-        n = min(W.T, 8)
+        cap = 1
+        while cap < W.T and self._touched(cap + 1) <= max_experts:
+            cap += 1
+        n = min(cap, 8)
         t = self._time(n)
         per_tok = t / n
-        self.tokens = int(max(1, min(W.T, target_s / max(per_tok, 1e-6))))
-        self.sample_desc = f"{self.tokens} of {W.T} tokens ({self._touched(self.tokens)} experts)"
+        self.tokens = int(max(1, min(cap, target_s / max(per_tok, 1e-6))))
+        self._ensure_experts(self.tokens)
+        self.reps = int(max(1, round(target_s / max(per_tok * self.tokens, 1e-6))))
+        self.sample_desc = (f"{self.tokens} of {W.T} tokens ({self._touched(self.tokens)} experts)"
+                            + (f", run {self.reps} times per timing" if self.reps > 1 else ""))
 
     def _touched(self, n):
         return int(np.unique(self.ids[:n]).size)
@@ -438,13 +425,14 @@ class OracleSample:
             O.route_topk(self.logits[:n], W.topk)
         return O.moe_forward(self.x[:n], self.ids[:n], self.w[:n], self.experts, W.E, W.F)
 
-    def timed(self, reps=1):
+    def timed(self):
+        """Seconds per forward of the token sample (averaged over self.reps runs)."""
         if self.W.kind != "gemm":
             self._ensure_experts(self.tokens)
         t0 = time.perf_counter()
-        for _ in range(reps):
+        for _ in range(self.reps):
             self.run()
-        return (time.perf_counter() - t0) / reps
+        return (time.perf_counter() - t0) / self.reps
 
 
 # --------------------------------------------------------------------------- #
@@ -486,7 +474,7 @@ def run_reference(args, W):
                 "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
         print(json.dumps(line), flush=True)
         return 0
-    target = max(0.5, min(10.0, 150.0 / max(1, args.steps + args.warmup)))
+    target = max(0.5, min(10.0, 100.0 / max(1, args.steps + args.warmup)))
     S = OracleSample(W, args.seed, target)
     for _ in range(args.warmup):
         S.run()
@@ -640,16 +628,134 @@ def run_kv(args, W, torch, B, device, world, rank):
     return 0
 
 
+def measure_int8_peak(torch, device, n=8192, reps=10):
+    """Dense INT8 tensor-core throughput of a library GEMM on this GPU: torch._int_mm
+    (cuBLASLt, int8 x int8 -> int32) on n^3 operands, best of `reps` CUDA-event timed
+    calls after warm-up, with the SM clock sampled meanwhile.  TOPS = 2 n^3 / time."""
+    info = {"method": f"torch._int_mm int8 {n}^3 (cuBLASLt), best of {reps}, CUDA events"}
+    try:
+        a = torch.randint(-127, 128, (n, n), dtype=torch.int8, device=device)
+        b = torch.randint(-127, 128, (n, n), dtype=torch.int8, device=device).t()  # column-major operand
+        for _ in range(3):
+            torch._int_mm(a, b)
+        torch.cuda.synchronize()
+        sampler = ClockSampler(torch.cuda.current_device(), period=0.002)
+        sampler.start()
+        best = float("inf")
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            torch._int_mm(a, b)
+            e1.record()
+            e1.synchronize()
+            best = min(best, e0.elapsed_time(e1))
+        sampler.stop()
+        del a, b
+        info.update({"tops": 2.0 * n ** 3 / (best / 1e3) / 1e12, "ms": best, "clocks": sampler.summary()})
+    except Exception as ex:  # recorded, and the nominal ratio is used instead
+        info.update({"tops": None, "error": f"{type(ex).__name__}: {ex}"[:200]})
+    return info
+
+
+def time_steps(step, B, torch, device, world, steps, warmup):
+    """Warm up, then time `steps` steps with CUDA events on the launching stream (L2
+    flushed before each, outside the timed span), the library's per-kernel event
+    profiler and NVML clock samples over the same region.  Returns (max-over-ranks
+    ms per step, {kernel kind: (launches, total ms)}, clock summary)."""
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    sampler = ClockSampler(torch.cuda.current_device())
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    B.w4a8_profile_start()
+    sampler.start()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    for i in range(steps):
+        flush.zero_()
+        starts[i].record()
+        step()
+        ends[i].record()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    sampler.stop()
+    prof = B.w4a8_profile_stop()
+    assert B.w4a8_last_device_error(step.ws) == 0, "device error during the timed steps"
+    ms = sum(a.elapsed_time(b) for a, b in zip(starts, ends)) / steps
+    return max_over_ranks(ms, torch, device, world), prof, sampler.summary()
+
+
+def kernel_table(prof, acct, steps):
+    kernels = {}
+    for kind, (n, tot) in prof.items():
+        if n:
+            kernels[kind] = {"launches": n, "ms_per_step": tot / steps}
+    for kind, v in kernels.items():
+        kb = acct["kernel_bytes"].get(kind, 0.0)
+        ko = acct["kernel_ops"].get(kind, 0.0)
+        t = v["ms_per_step"] * steps / v["launches"] / 1e3
+        v["gbs"] = kb / t / 1e9 if t > 0 else None
+        if ko:
+            v["tops"] = ko / t / 1e12 if t > 0 else None
+    return kernels
+
+
+def roofline_of(kernel, kernels, acct, steps, peaks, workload):
+    """Roofline of one kernel: algorithmic ops (tensor-bound) or bytes (HBM-bound) per
+    launch over its average event-timed launch duration, against the measured peak."""
+    hbm, i8 = peaks["hbm_gbs"], peaks["int8_tops"]
+    per_launch_ms = kernels[kernel]["ms_per_step"] * steps / kernels[kernel]["launches"]
+    ops = acct["kernel_ops"].get(kernel, 0.0)
+    byt = acct["kernel_bytes"].get(kernel, 0.0)
+    ridge = i8 * 1e12 / (hbm * 1e9)
+    if ops and ops / max(byt, 1) > ridge:
+        roof = {"bound": "tensor", "achieved": ops / (per_launch_ms / 1e3) / 1e12, "peak": i8, "unit": "TFLOP/s",
+                "peak_source": peaks["int8_source"]}
+    else:
+        roof = {"bound": "hbm", "achieved": byt / (per_launch_ms / 1e3) / 1e9, "peak": hbm, "unit": "GB/s",
+                "peak_source": f"{peaks['source']}: MEASURED_PEAKS hbm_gbs (copy bandwidth)"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = load_traffic(workload, kernel)
+    roof["kernel"] = kernel
+    roof["ms_per_launch"] = per_launch_ms
+    return roof
+
+
+def moe_summary(W, step, ms, prof, clocks, steps, peaks, world):
+    acct = step.acct
+    kernels = kernel_table(prof, acct, steps)
+    dom = max((k for k in kernels if k.startswith("gemm")), key=lambda k: kernels[k]["ms_per_step"])
+    tokens = (W.T if W.kind == "moe" else W.M) * world
+    sec = ms / 1e3
+    return {
+        "value": whole_job_rate(tokens // world, world, ms), "unit": "tokens/s", "ms_per_step": ms,
+        "tops": acct["ops"] * world / sec / 1e12,
+        "weight_gbs": acct["weight_bytes"] * world / sec / 1e9,
+        "touched_experts": acct["touched_experts"],
+        "roofline": roofline_of(dom, kernels, acct, steps, peaks, W.name),
+        "rooflines": {k: roofline_of(k, kernels, acct, steps, peaks, W.name)
+                      for k in kernels if k.startswith("gemm") and k != dom},
+        "kernels": kernels,
+        "gpu_launches": sum(v["launches"] for v in kernels.values()),
+        "clocks": clocks,
+    }
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(synth.WORKLOADS), default="toy_moe")
+    ap.add_argument("--workload", choices=sorted(synth.WORKLOADS), default="prefill")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--cpu-baseline-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true", help="do not also time the decode layers")
     ap.add_argument("--weights", choices=["asym", "sym", "clip999"], default="asym",
                     help="packer scheme: asymmetric INT4 (default), symmetric, or asymmetric on the "
                          "0.1th..99.9th percentile range")
@@ -678,80 +784,28 @@ def main(argv=None):
 
     if W.kind == "kv":
         return run_kv(args, W, torch, B, device, world, rank)
-    step = (GemmStep if W.kind == "gemm" else MoeStep)(B, torch, W, args.seed + rank * 0, device)
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
-    sampler = ClockSampler(torch.cuda.current_device())
 
-    def barrier():
-        if world > 1:
-            torch.distributed.barrier()
+    peaks = load_peaks()
+    i8 = measure_int8_peak(torch, device)
+    if i8.get("tops"):
+        peaks["int8_tops"] = i8["tops"]
+        peaks["int8_source"] = "measured in this run: " + i8["method"]
+    else:
+        peaks["int8_tops"] = float(peaks["bf16_tflops"]) * INT8_OVER_BF16
+        peaks["int8_source"] = "bf16_tflops x 2 (nominal int8/bf16 ratio; the measurement failed)"
+    peaks["hbm_gbs"] = float(peaks["hbm_gbs"])
 
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    B.w4a8_profile_start()
-    step.start_route_timing()
-    sampler.start()
-    barrier()
-    torch.cuda.synchronize()
-    for i in range(args.steps):
-        flush.zero_()
-        starts[i].record()
-        step()
-        ends[i].record()
-    torch.cuda.synchronize()
-    barrier()
-    sampler.stop()
-    step.stop_route_timing()
-    prof = B.w4a8_profile_stop()
-    assert B.w4a8_last_device_error(step.ws) == 0, "device error during the timed steps"
-    ms = sum(a.elapsed_time(b) for a, b in zip(starts, ends)) / args.steps
-    ms_max = max_over_ranks(ms, torch, device, world)
+    step = (GemmStep if W.kind == "gemm" else MoeStep)(B, torch, W, args.seed, device)
+    ms_max, prof, clocks = time_steps(step, B, torch, device, world, args.steps, args.warmup)
+    summ = moe_summary(W, step, ms_max, prof, clocks, args.steps, peaks, world)
 
     e2e_ms, h2d, d2h = step.e2e(args.steps, args.warmup)
     e2e_ms = max_over_ranks(e2e_ms, torch, device, world)
-
-    acct = step.acct
     tokens = (W.T if W.kind == "moe" else W.M) * world
-    sec = ms_max / 1e3
-    peaks = load_peaks()
-    hbm = float(peaks["hbm_gbs"])
-    i8 = float(peaks["bf16_tflops"]) * INT8_OVER_BF16
-
-    # per-kernel table and the dominant kernel's roofline
-    kernels = {}
-    for kind, (n, tot) in prof.items():
-        if n:
-            kernels[kind] = {"launches": n, "ms_per_step": tot / args.steps}
-    if step.route_launches:
-        kernels["route"] = {"launches": step.route_launches, "ms_per_step": step.route_ms / args.steps}
-    dom = max(kernels, key=lambda k: kernels[k]["ms_per_step"])
-    per_launch_ms = kernels[dom]["ms_per_step"] * args.steps / kernels[dom]["launches"]
-    ops = acct["kernel_ops"].get(dom, 0.0)
-    byt = acct["kernel_bytes"].get(dom, 0.0)
-    ridge = i8 * 1e12 / (hbm * 1e9)
-    if ops and ops / max(byt, 1) > ridge:
-        roof = {"bound": "tensor", "achieved": ops / (per_launch_ms / 1e3) / 1e12, "peak": i8, "unit": "TFLOP/s"}
-    else:
-        roof = {"bound": "hbm", "achieved": byt / (per_launch_ms / 1e3) / 1e9, "peak": hbm, "unit": "GB/s"}
-    roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = load_traffic(W.name, dom)
-    roof["kernel"] = dom
-    roof["peak_source"] = (f"{peaks['source']}: " + ("MEASURED_PEAKS hbm_gbs" if roof["bound"] == "hbm" else
-                           "bf16_tflops x 2 (nominal int8/bf16 ratio)"))
-    for kind, v in kernels.items():
-        kb = acct["kernel_bytes"].get(kind, 0.0)
-        ko = acct["kernel_ops"].get(kind, 0.0)
-        t = v["ms_per_step"] * args.steps / v["launches"] / 1e3
-        v["gbs"] = kb / t / 1e9 if t > 0 else None
-        if ko:
-            v["tops"] = ko / t / 1e12 if t > 0 else None
 
     line = {
         "metric": METRIC,
-        "value": whole_job_rate(tokens // world, world, ms_max),
+        "value": summ["value"],
         "unit": "tokens/s",
         "n_gpus": world,
         "steps": args.steps,
@@ -763,16 +817,38 @@ def main(argv=None):
         "dtype": "int8",
         "data": "synthetic",
         "config": config_of(W, "flushed before every timed step (256 MiB write, outside the timed span)"),
-        "tops": acct["ops"] * world / sec / 1e12,
-        "weight_gbs": acct["weight_bytes"] * world / sec / 1e9,
-        "touched_experts": acct["touched_experts"],
-        "roofline": roof,
-        "kernels": kernels,
-        "gpu_launches": sum(v["launches"] for v in kernels.values()),
+        "tops": summ["tops"],
+        "weight_gbs": summ["weight_gbs"],
+        "touched_experts": summ["touched_experts"],
+        "roofline": summ["roofline"],
+        "rooflines": summ["rooflines"],
+        "kernels": summ["kernels"],
+        "gpu_launches": summ["gpu_launches"],
         "e2e": {"value": whole_job_rate(tokens // world, world, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
-        "clocks": sampler.summary(),
+        "clocks": summ["clocks"],
+        "int8_peak": i8,
     }
+
+    # the HBM-bound decode layers, timed in the same run (one GPU only)
+    if world == 1 and not args.no_extra and W.name == "prefill":
+        extra = {}
+        shared = (step.packed_up, step.packed_down)
+        for name in ("large_decode", "decode"):
+            Wx = synth.WORKLOADS[name]
+            same = (Wx.E, Wx.H, Wx.F) == (W.E, W.H, W.F)
+            sx = MoeStep(B, torch, Wx, args.seed, device, packed=shared if same else None)
+            msx, profx, clx = time_steps(sx, B, torch, device, world, args.steps, args.warmup)
+            ex = moe_summary(Wx, sx, msx, profx, clx, args.steps, peaks, world)
+            e2x, h2x, d2x = sx.e2e(args.steps, args.warmup)
+            ex["e2e"] = {"value": Wx.T / (e2x / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2x,
+                         "d2h_bytes_per_step": d2x}
+            ex["config"] = config_of(Wx, "flushed before every timed step (256 MiB write, outside the timed span)")
+            extra[name] = ex
+            del sx
+            torch.cuda.empty_cache()
+        line["extra"] = extra
+
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         S = OracleSample(W, args.seed, args.cpu_baseline_seconds)
         t = S.timed()

@@ -115,7 +115,11 @@ int w4a8_pack_weights(const void* w_bf16, int E, int N, int K, int layout,
  *   s      : device, float [T]; s = max|x|/127 (0 for an all-zero row, with q = 0). */
 int w4a8_quant_act(const void* x_bf16, int T, int K, int8_t* q, float* s, void* stream);
 
-/* Top-k softmax routing  (a3; the router stays in 16-bit float).
+/* Top-k softmax routing  (a3).  The Kimi 2.7T MoE W4A8 article (hotelren.com
+ * 5173946), section 5.2: the router is not quantised; it reads 16-bit logits and
+ * picks each token's experts, whose gate weights scale the expert outputs in the
+ * combine (section 4.3, step 4).  The selection and weights follow the plainest
+ * softmax gating, which the pages do not spell out.
  *   logits_bf16 : device, bf16 [T][E];  1 <= k <= min(E, 32), E <= 1024.
  *   ids         : device, int32 [T][k]: the k largest logits, largest first, ties
  *                 to the lower expert id.
@@ -131,6 +135,12 @@ size_t w4a8_moe_workspace_bytes(int T, int E, int k, int H, int F);
  *   out[t] = sum_j w[t][j] * Down_e( SwiGLU( Up_e( x[t] ) ) ),  e = ids[t][j],
  * with x quantised per token to INT8, Up/Down W4A8 GEMMs (INT32 per-group
  * partials), h = silu(gate) * up requantised per token to INT8 before Down.
+ * Source: the Kimi 2.7T MoE W4A8 article (hotelren.com 5173946), section 4.3: the
+ * activations are quantised per token at run time, the INT4 weights are expanded
+ * inside the kernel and multiplied in INT8 with INT32 accumulation, the result is
+ * scaled back and the input of the next projection is quantised again; section 5.1:
+ * tokens are grouped by expert before the expert GEMMs; «Kimi 2.7 Moe 从 4 bit 存储到
+ * INT8 拆解» (pptc.cn), section 3.2: INT8 x INT8 products accumulate in INT32.
  *   packed_up   : from w4a8_pack_weights(E, 2F, H, W4A8_LAYOUT_GATEUP).
  *   packed_down : from w4a8_pack_weights(E, H, F, W4A8_LAYOUT_PLAIN).
  *   x_bf16      : device bf16 [T][H].   ids: device int32 [T][k] (0 <= id < E;
@@ -153,12 +163,26 @@ int w4a8_moe_forward_host(const void* packed_up, const void* packed_down, int E,
                           const float* w_host, int k, void* out_bf16_host,
                           void* ws, size_t ws_bytes, void* stream);
 
+/* The layer routed from router logits, with HOST buffers: x_bf16_host [T][H] and
+ * logits_bf16_host [T][E] (bf16) are copied into the workspace, the experts are
+ * chosen on the device exactly as w4a8_route_topk does, the layer runs as in
+ * w4a8_moe_forward and out_bf16_host [T][H] is copied back, all on `stream`.
+ * Same workspace as w4a8_moe_forward_host; asynchronous like it. */
+int w4a8_moe_forward_logits_host(const void* packed_up, const void* packed_down, int E, int H, int F,
+                                 const void* x_bf16_host, int T, const void* logits_bf16_host, int k,
+                                 void* out_bf16_host, void* ws, size_t ws_bytes, void* stream);
+
 /* Workspace bytes needed by w4a8_gemm. */
 size_t w4a8_gemm_workspace_bytes(int M, int N, int K);
 
 /* One dense W4A8 linear layer  (a5 on a single weight matrix):
  *   y[m][n] = sa[m] * sum_g scale[n][g] * acc[m][n][g],
  *   acc[m][n][g] = sum_{k in group g} qa[m][k] * (code[n][k] - zp[n][g])   (INT32).
+ * Source: «Kimi 2.7 Moe 从 4 bit 存储到 INT8 拆解» (pptc.cn), section 3.2: the INT4
+ * weights become INT8 values (code - zero point), INT8 x INT8 products accumulate in
+ * INT32, and the integer result is scaled back to floating point by the weight scale
+ * (one per 128-wide group, section 2.1) and the token scale; the Kimi 2.7T MoE W4A8
+ * article (hotelren.com 5173946), section 4.3, steps 2-4.
  *   qa          : device int8 [M][Kp] (as written by w4a8_quant_act), sa: float [M].
  *   packed      : from w4a8_pack_weights(1, N, K, W4A8_LAYOUT_PLAIN).
  *   y           : device float [M][N].
@@ -188,6 +212,12 @@ int w4a8_gemm(const int8_t* qa, const float* sa, int M, const void* packed, int 
  *   - The device error word lives in that array and is not readable by the caller. */
 int w4a8_gemm_noalloc(const int8_t* qa, const float* sa, int M, const void* packed, int N, int K,
                       float* y, int32_t* partials_opt, void* stream);
+
+/* The device error word of the last w4a8_gemm_noalloc call on the current device
+ * (the same bits as w4a8_last_device_error): synchronises `stream`, then reads the
+ * word from the library's scratch array.  Read it before the next noalloc call,
+ * which clears it. */
+int w4a8_gemm_noalloc_last_error(void* stream);
 
 /* Intermediate results kept in a w4a8_moe_forward workspace, for stage tests. */
 enum {
@@ -227,7 +257,8 @@ int w4a8_debug_dump(const void* ws, int T, int E, int k, int H, int F, int what,
 int w4a8_last_device_error(const void* ws, void* stream);
 
 /* Per-kernel device timing, for benchmarks.  After w4a8_profile_start(), every
- * w4a8_moe_forward / w4a8_moe_forward_host / w4a8_gemm call made from the same
+ * w4a8_quant_act / w4a8_route_topk / w4a8_moe_forward / w4a8_moe_forward_host /
+ * w4a8_moe_forward_logits_host / w4a8_gemm call made from the same
  * host thread records a pair of CUDA events around each kernel kind it launches
  * (on the call's stream).  w4a8_profile_stop() waits for those events, writes
  * per kind the number of kernel launches and their summed device milliseconds
@@ -242,10 +273,24 @@ enum {
     W4A8_KERNEL_GEMM_DOWN = 4, /* grouped W4A8 GEMM, down projection            */
     W4A8_KERNEL_COMBINE = 5,   /* weighted sum of the k expert outputs          */
     W4A8_KERNEL_GEMM_DENSE = 6,/* w4a8_gemm (re-layout + GEMM, 2 launches)      */
-    W4A8_KERNEL_KINDS = 7
+    W4A8_KERNEL_ROUTE = 7,     /* top-k softmax routing                         */
+    W4A8_KERNEL_KINDS = 8
 };
 int w4a8_profile_start(void);
 int w4a8_profile_stop(int* launches, float* total_ms, int n);
+
+/* Test hook of the failure detection (no counterpart in the pages).  Every bounded
+ * wait inside the GEMM kernels gives up after a number of clock cycles (about 2 s by
+ * default), sets bit 0 of the device error word, drains what it issued, frees its
+ * tensor memory and returns.  While set on the calling host thread, this makes the
+ * GEMM launches of w4a8_moe_forward* and w4a8_gemm* use `wait_limit_cycles` (0 = the
+ * default) and, with flags = W4A8_DEBUG_SKIP_FIRST_COPY, has the first CTA issue no
+ * copy for its first pipeline step, so that the waits for it run out: the result of
+ * that call is undefined and its device error word has bit 0 set.  flags = 0 and
+ * wait_limit_cycles = 0 restore normal operation.  Returns W4A8_EINVAL for unknown
+ * flags or a negative limit. */
+enum { W4A8_DEBUG_SKIP_FIRST_COPY = 1 };
+int w4a8_debug_inject(unsigned int flags, long long wait_limit_cycles);
 
 /* INT8 KV cache with static per-head scales (the Kimi 2.7T MoE W4A8 article,
  * hotelren.com/news/5173946, section 5: the attention KV cache is quantised to INT8

@@ -119,3 +119,16 @@ def test_gemm_workspace(lib):
     assert lib.w4a8_gemm_workspace_bytes(16, 256, 512) >= 4 * 16 * 128
     assert lib.w4a8_gemm_workspace_bytes(0, 256, 512) > 0
     assert lib.w4a8_gemm_workspace_bytes(-1, 256, 512) == 0
+
+
+def test_debug_inject_validates_its_arguments(lib):
+    assert lib.w4a8_debug_inject(0x80, 0) == EINVAL  # unknown flag
+    assert lib.w4a8_debug_inject(0, -1) == EINVAL  # negative wait limit
+    assert lib.w4a8_debug_inject(1, 1000) == 0
+    assert lib.w4a8_debug_inject(0, 0) == 0  # back to normal operation
+
+
+def test_logits_host_forward_validates_on_the_host(lib):
+    # invalid shapes and a missing workspace are refused before any CUDA call
+    assert lib.w4a8_moe_forward_logits_host(None, None, 0, 256, 128, None, 4, None, 2, None, None, 0, None) == EINVAL
+    assert lib.w4a8_moe_forward_logits_host(None, None, 8, 256, 128, None, 4, None, 2, None, None, 0, None) == EINVAL

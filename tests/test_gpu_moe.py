@@ -241,3 +241,42 @@ def test_host_buffer_entry_point_matches_device_entry_point():
     B.w4a8_moe_forward_host(L.packed_up, L.packed_down, E, H, F, xh, idh, wh, outh, ws)
     torch.cuda.synchronize()
     assert np.array_equal(bf16_to_f32(outh), out_dev)
+
+
+def test_logits_host_entry_point_matches_router_and_device_entry_point():
+    L = Layer(37, 8, 3, 256, 128, "softmax", seed=5)
+    out_dev = L.run(use_router=True)
+    T, E, k, H, F = L.T, L.E, L.k, L.H, L.F
+    ws = B.empty_aligned(B.w4a8_moe_host_workspace_bytes(T, E, k, H, F))
+    xh = torch.from_numpy(synth.bf16_bits(L.x).view(np.int16)).view(torch.bfloat16).pin_memory()
+    lgh = torch.from_numpy(synth.bf16_bits(L.logits).view(np.int16)).view(torch.bfloat16).pin_memory()
+    outh = torch.empty((T, H), dtype=torch.bfloat16).pin_memory()
+    B.w4a8_moe_forward_logits_host(L.packed_up, L.packed_down, E, H, F, xh, lgh, k, outh, ws)
+    torch.cuda.synchronize()
+    assert B.w4a8_last_device_error(ws) == 0
+    assert np.array_equal(bf16_to_f32(outh), out_dev)
+
+
+def test_binding_rejects_undersized_buffers():
+    """The kernels trust the sizes they are given, so the binding checks every buffer
+    against the shapes before the call."""
+    M, N, K = 32, 256, 512
+    qa = torch.zeros((M, K), dtype=torch.int8, device="cuda")
+    sa = torch.ones(M, dtype=torch.float32, device="cuda")
+    packed = B.empty_aligned(B.w4a8_packed_bytes(1, N, K, 0))
+    ws = B.empty_aligned(B.w4a8_gemm_workspace_bytes(M, N, K))
+    with pytest.raises(B.W4A8Error):
+        B.w4a8_gemm(qa, sa, packed, N, K, torch.empty(M * N - 1, dtype=torch.float32, device="cuda"), ws)
+    with pytest.raises(B.W4A8Error):
+        B.w4a8_gemm(qa[:, :256], sa, packed, N, K, torch.empty((M, N), dtype=torch.float32, device="cuda"), ws)
+    with pytest.raises(B.W4A8Error):
+        B.w4a8_gemm(qa, sa[:M - 1], packed, N, K, torch.empty((M, N), dtype=torch.float32, device="cuda"), ws)
+    with pytest.raises(B.W4A8Error):
+        B.w4a8_gemm_noalloc(qa, sa, packed, N, K, torch.empty((M, N), dtype=torch.float32, device="cuda"),
+                            torch.empty((M, N, 3), dtype=torch.int32, device="cuda"))
+    L = Layer(8, 4, 2, 256, 128)
+    with pytest.raises(B.W4A8Error):  # out has the wrong shape
+        B.w4a8_moe_forward(L.packed_up, L.packed_down, 4, 256, 128, dev_bf16(L.x), torch.from_numpy(L.ids).cuda(),
+                           torch.from_numpy(L.w.astype(np.float32)).cuda(),
+                           torch.empty((8, 128), dtype=torch.bfloat16, device="cuda"),
+                           B.empty_aligned(B.w4a8_moe_workspace_bytes(8, 4, 2, 256, 128)))

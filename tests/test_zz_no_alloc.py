@@ -42,8 +42,17 @@ def test_noalloc_gemm_matches_workspace_gemm_on_consecutive_calls():
         p = torch.zeros((M, N, G), dtype=torch.int32, device="cuda")
         B.w4a8_gemm_noalloc(qa, sa, packed, N, K, y, p)
         torch.cuda.synchronize()
+        assert B.w4a8_gemm_noalloc_last_error() == 0
         assert torch.equal(p, p_ref)
         assert_close(y.cpu().numpy(), y_ref.cpu().numpy(), max_rel=1e-4, mae_rel=1e-5, what="y")
+        # and against the oracle on its own: exact INT32 partials, y within the GEMM tolerance
+        x, w = synth.dense_gemm_inputs(seed, M, K, N)
+        qo, so = O.quantize_act(x)
+        codes, scale, zp = O.quantize_weights(w)
+        acc = O.group_partials(qo, codes, zp)
+        assert np.array_equal(p.cpu().numpy().astype(np.int64), acc)
+        assert_close(y.cpu().numpy(), O.w4a8_linear(qo, so, codes, scale, zp, acc), max_rel=1e-4, mae_rel=1e-5,
+                     what="y vs oracle")
 
 
 def test_noalloc_gemm_rejects_sizes_beyond_its_scratch():

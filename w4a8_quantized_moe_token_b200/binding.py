@@ -48,6 +48,10 @@ _SIGS = {
     "w4a8_gemm_workspace_bytes": ([_c_int] * 3, _c_size),
     "w4a8_gemm": ([_vp, _vp, _c_int, _vp, _c_int, _c_int, _vp, _vp, _vp, _c_size, _vp], _c_int),
     "w4a8_gemm_noalloc": ([_vp, _vp, _c_int, _vp, _c_int, _c_int, _vp, _vp, _vp], _c_int),
+    "w4a8_gemm_noalloc_last_error": ([_vp], _c_int),
+    "w4a8_moe_forward_logits_host": ([_vp, _vp, _c_int, _c_int, _c_int, _vp, _c_int, _vp, _c_int, _vp, _vp,
+                                      _c_size, _vp], _c_int),
+    "w4a8_debug_inject": ([ctypes.c_uint, ctypes.c_longlong], _c_int),
     "w4a8_debug_region": ([_c_int] * 6 + [ctypes.POINTER(_c_size), ctypes.POINTER(_c_size)], _c_int),
     "w4a8_debug_dump": ([_vp] + [_c_int] * 6 + [_vp, _c_size, _vp], _c_int),
     "w4a8_last_device_error": ([_vp, _vp], _c_int),
@@ -55,7 +59,8 @@ _SIGS = {
     "w4a8_profile_stop": ([ctypes.POINTER(_c_int), ctypes.POINTER(ctypes.c_float), _c_int], _c_int),
 }
 
-KERNEL_KINDS = ["perm", "act_quant", "gemm_up", "requant", "gemm_down", "combine", "gemm_dense"]
+KERNEL_KINDS = ["perm", "act_quant", "gemm_up", "requant", "gemm_down", "combine", "gemm_dense", "route"]
+W4A8_DEBUG_SKIP_FIRST_COPY = 1
 
 _lib = None
 
@@ -104,8 +109,20 @@ def _ptr(t):
 def _dev(t, dtype, name):
     if not t.is_cuda:
         raise W4A8Error(f"{name} must be a CUDA tensor")
+    if t.device.index != torch.cuda.current_device():
+        raise W4A8Error(f"{name} is on {t.device}, not on the current device cuda:{torch.cuda.current_device()}")
     if t.dtype != dtype:
         raise W4A8Error(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def _need(cond, msg):
+    if not cond:
+        raise W4A8Error(msg)
+
+
+def padded_k(K: int) -> int:
+    """K rounded up to a whole number of 128-wide groups (the layout's row length)."""
+    return (K + 127) // 128 * 128
 
 
 # --------------------------------------------------------------------------- #
@@ -190,13 +207,27 @@ def w4a8_moe_act_block_rows(T, E, k) -> int:
     return lib().w4a8_moe_act_block_rows(T, E, k)
 
 
+def _moe_buffers(packed_up, packed_down, E, H, F, ws, host_ws=False):
+    _dev(packed_up, torch.uint8, "packed_up")
+    _dev(packed_down, torch.uint8, "packed_down")
+    _dev(ws, torch.uint8, "ws")
+    _need(packed_up.numel() >= w4a8_packed_bytes(E, 2 * F, H, W4A8_LAYOUT_GATEUP),
+          "packed_up is smaller than the packed gate|up weights of this layer")
+    _need(packed_down.numel() >= w4a8_packed_bytes(E, H, F, W4A8_LAYOUT_PLAIN),
+          "packed_down is smaller than the packed down weights of this layer")
+
+
 def w4a8_moe_forward(packed_up, packed_down, E, H, F, x, ids, w, out, ws):
     """x bf16 [T][H], ids int32 [T][k], w float32 [T][k], out bf16 [T][H], ws uint8 (cuda)."""
     _dev(x, torch.bfloat16, "x")
     _dev(ids, torch.int32, "ids")
     _dev(w, torch.float32, "w")
     _dev(out, torch.bfloat16, "out")
+    _moe_buffers(packed_up, packed_down, E, H, F, ws)
     T, k = ids.shape
+    _need(tuple(x.shape) == (T, H), f"x must be [T={T}][H={H}], got {tuple(x.shape)}")
+    _need(tuple(w.shape) == (T, k), f"w must be [T={T}][k={k}], got {tuple(w.shape)}")
+    _need(tuple(out.shape) == (T, H), f"out must be [T={T}][H={H}], got {tuple(out.shape)}")
     _check(lib().w4a8_moe_forward(_ptr(packed_up), _ptr(packed_down), E, H, F, _ptr(x), T, _ptr(ids), _ptr(w), k,
                                   _ptr(out), _ptr(ws), ws.numel(), _stream()), "w4a8_moe_forward")
 
@@ -206,21 +237,61 @@ def w4a8_moe_forward_host(packed_up, packed_down, E, H, F, x, ids, w, out, ws):
     for t, nm in ((x, "x"), (ids, "ids"), (w, "w"), (out, "out")):
         if t.is_cuda:
             raise W4A8Error(f"{nm} must be a host tensor")
+    _moe_buffers(packed_up, packed_down, E, H, F, ws)
     T, k = ids.shape
+    _need(x.dtype == torch.bfloat16 and tuple(x.shape) == (T, H), "x must be bf16 [T][H]")
+    _need(ids.dtype == torch.int32, "ids must be int32")
+    _need(w.dtype == torch.float32 and tuple(w.shape) == (T, k), "w must be float32 [T][k]")
+    _need(out.dtype == torch.bfloat16 and tuple(out.shape) == (T, H), "out must be bf16 [T][H]")
     _check(lib().w4a8_moe_forward_host(_ptr(packed_up), _ptr(packed_down), E, H, F, _ptr(x), T, _ptr(ids), _ptr(w),
                                        k, _ptr(out), _ptr(ws), ws.numel(), _stream()), "w4a8_moe_forward_host")
+
+
+def w4a8_moe_forward_logits_host(packed_up, packed_down, E, H, F, x, logits, k, out, ws):
+    """The layer routed on the device from bf16 router logits [T][E]; x, logits and
+    out are (pinned) HOST tensors; ws as for w4a8_moe_forward_host."""
+    for t, nm in ((x, "x"), (logits, "logits"), (out, "out")):
+        if t.is_cuda:
+            raise W4A8Error(f"{nm} must be a host tensor")
+    _moe_buffers(packed_up, packed_down, E, H, F, ws)
+    T = x.shape[0]
+    _need(x.dtype == torch.bfloat16 and tuple(x.shape) == (T, H), "x must be bf16 [T][H]")
+    _need(logits.dtype == torch.bfloat16 and tuple(logits.shape) == (T, E), "logits must be bf16 [T][E]")
+    _need(out.dtype == torch.bfloat16 and tuple(out.shape) == (T, H), "out must be bf16 [T][H]")
+    _check(lib().w4a8_moe_forward_logits_host(_ptr(packed_up), _ptr(packed_down), E, H, F, _ptr(x), T,
+                                              _ptr(logits), k, _ptr(out), _ptr(ws), ws.numel(), _stream()),
+           "w4a8_moe_forward_logits_host")
 
 
 def w4a8_gemm_workspace_bytes(M, N, K) -> int:
     return lib().w4a8_gemm_workspace_bytes(M, N, K)
 
 
-def w4a8_gemm(qa, sa, packed, N, K, y, ws, partials=None):
-    """qa int8 [M][Kp], sa float32 [M], y float32 [M][N], partials int32 [M][N][Kp/128] or None."""
+def _gemm_buffers(qa, sa, packed, N, K, y, partials):
+    """Check every buffer of a dense GEMM against its shape before the call: the
+    kernels trust the sizes they are given."""
     _dev(qa, torch.int8, "qa")
     _dev(sa, torch.float32, "sa")
     _dev(y, torch.float32, "y")
+    _dev(packed, torch.uint8, "packed")
+    _need(qa.dim() == 2, "qa must be [M][Kp]")
     M = qa.shape[0]
+    Kp = padded_k(K)
+    _need(tuple(qa.shape) == (M, Kp), f"qa must be [M][{Kp}] for K = {K}, got {tuple(qa.shape)}")
+    _need(sa.numel() >= M, f"sa needs {M} entries, has {sa.numel()}")
+    _need(y.numel() >= M * N, f"y needs {M * N} elements, has {y.numel()}")
+    _need(packed.numel() >= w4a8_packed_bytes(1, N, K, W4A8_LAYOUT_PLAIN),
+          "packed is smaller than the packed weights of an N x K matrix")
+    if partials is not None:
+        _dev(partials, torch.int32, "partials")
+        _need(partials.numel() >= M * N * (Kp // 128), f"partials needs {M * N * (Kp // 128)} elements")
+    return M
+
+
+def w4a8_gemm(qa, sa, packed, N, K, y, ws, partials=None):
+    """qa int8 [M][Kp], sa float32 [M], y float32 [M][N], partials int32 [M][N][Kp/128] or None."""
+    M = _gemm_buffers(qa, sa, packed, N, K, y, partials)
+    _dev(ws, torch.uint8, "ws")
     _check(lib().w4a8_gemm(_ptr(qa), _ptr(sa), M, _ptr(packed), N, K, _ptr(y), _ptr(partials), _ptr(ws), ws.numel(),
                            _stream()), "w4a8_gemm")
 
@@ -228,12 +299,23 @@ def w4a8_gemm(qa, sa, packed, N, K, y, ws, partials=None):
 def w4a8_gemm_noalloc(qa, sa, packed, N, K, y, partials=None):
     """w4a8_gemm without a caller workspace: the library's own fixed scratch array
     is used (for callers that cannot allocate; concurrent calls race)."""
-    _dev(qa, torch.int8, "qa")
-    _dev(sa, torch.float32, "sa")
-    _dev(y, torch.float32, "y")
-    M = qa.shape[0]
+    M = _gemm_buffers(qa, sa, packed, N, K, y, partials)
     _check(lib().w4a8_gemm_noalloc(_ptr(qa), _ptr(sa), M, _ptr(packed), N, K, _ptr(y), _ptr(partials), _stream()),
            "w4a8_gemm_noalloc")
+
+
+def w4a8_gemm_noalloc_last_error() -> int:
+    """Device error word of the last w4a8_gemm_noalloc call on the current device."""
+    r = lib().w4a8_gemm_noalloc_last_error(_stream())
+    if r < 0:
+        _check(r, "w4a8_gemm_noalloc_last_error")
+    return r
+
+
+def w4a8_debug_inject(flags: int = 0, wait_limit_cycles: int = 0):
+    """Test hook: bounded-wait limit and skipped-copy flag for the GEMM launches of
+    this host thread (0, 0 restores normal operation)."""
+    _check(lib().w4a8_debug_inject(flags, wait_limit_cycles), "w4a8_debug_inject")
 
 
 def w4a8_debug_region(T, E, k, H, F, what) -> tuple[int, int]:

@@ -47,7 +47,7 @@ int rows_capacity(int T, int E, int k) {
 enum Region {
     R_ERR, R_CHIST, R_COUNTS, R_OFFS, R_POFFS, R_MTSTART, R_MTTAB, R_PERM, R_INV, R_ROWSRC,
     R_ACT1, R_S1, R_H, R_ACT2, R_S2, R_Y2,
-    R_XIN, R_IDSIN, R_WIN, R_OUT,  // host-buffer variant only
+    R_XIN, R_IDSIN, R_WIN, R_OUT, R_LOGITS,  // host-buffer variants only
     R_COUNT
 };
 
@@ -89,6 +89,7 @@ bool moe_layout(int T, int E, int k, int H, int F, bool host_io, MoeLayout* L) {
     b[R_IDSIN] = host_io ? (size_t)L->nslots * 4 : 0;
     b[R_WIN] = host_io ? (size_t)L->nslots * 4 : 0;
     b[R_OUT] = host_io ? (size_t)T * H * 2 : 0;
+    b[R_LOGITS] = host_io ? (size_t)T * E * 2 : 0;
     size_t o = 0;
     for (int r = 0; r < R_COUNT; ++r) {
         L->off[r] = o;
@@ -99,6 +100,14 @@ bool moe_layout(int T, int E, int k, int H, int F, bool host_io, MoeLayout* L) {
 }
 
 int to_status(cudaError_t e) { return e == cudaSuccess ? W4A8_OK : W4A8_ECUDA; }
+
+thread_local DebugInject g_debug;
+
+// the test hook of w4a8_debug_inject, copied into every GEMM launch
+void apply_debug(GemmArgs& a) {
+    a.wait_limit = g_debug.wait_limit > 0 ? g_debug.wait_limit : kWaitLimitCycles;
+    a.debug = g_debug.flags;
+}
 
 // Optional per-kernel event timing (w4a8_profile_start / w4a8_profile_stop),
 // kept per host thread.
@@ -209,6 +218,7 @@ int moe_forward_impl(const void* packed_up, const void* packed_down, int E, int 
     up.nvalid = F;
     up.partials = nullptr;
     up.err = err;
+    apply_debug(up);
     {
         ProfScope p(W4A8_KERNEL_GEMM_UP, 1, st);
         W4A8_TRY(launch_gemm(up, tile, sm_count(), st));
@@ -345,6 +355,7 @@ W4A8_EXPORT int w4a8_quant_act(const void* x_bf16, int T, int K, int8_t* q, floa
     if (T == 0) return W4A8_OK;
     if (x_bf16 == nullptr || q == nullptr || s == nullptr) return W4A8_EINVAL;
     if (!aligned(x_bf16, 16) || !aligned(q, 16) || !aligned(s, 16)) return W4A8_EALIGN;
+    ProfScope prof(W4A8_KERNEL_ACT_QUANT, 1, static_cast<cudaStream_t>(stream));
     return to_status(launch_quant_act(static_cast<const uint16_t*>(x_bf16), T, K, q, s,
                                       static_cast<cudaStream_t>(stream)));
 }
@@ -356,6 +367,7 @@ W4A8_EXPORT int w4a8_route_topk(const void* logits_bf16, int T, int E, int k, in
     if (T == 0) return W4A8_OK;
     if (logits_bf16 == nullptr || ids == nullptr || w == nullptr) return W4A8_EINVAL;
     if (!aligned(logits_bf16, 16) || !aligned(ids, 16) || !aligned(w, 16)) return W4A8_EALIGN;
+    ProfScope prof(W4A8_KERNEL_ROUTE, 1, static_cast<cudaStream_t>(stream));
     return to_status(launch_route_topk(static_cast<const uint16_t*>(logits_bf16), T, E, k, ids, w,
                                        static_cast<cudaStream_t>(stream)));
 }
@@ -411,6 +423,32 @@ W4A8_EXPORT int w4a8_moe_forward_host(const void* packed_up, const void* packed_
     W4A8_TRY(cudaMemcpyAsync(x, x_bf16_host, L.bytes[R_XIN], cudaMemcpyHostToDevice, s));
     W4A8_TRY(cudaMemcpyAsync(ids, ids_host, L.bytes[R_IDSIN], cudaMemcpyHostToDevice, s));
     W4A8_TRY(cudaMemcpyAsync(w, w_host, L.bytes[R_WIN], cudaMemcpyHostToDevice, s));
+    const int r = moe_forward_impl(packed_up, packed_down, E, H, F, x, T, ids, w, k, out, ws, L, s);
+    if (r != W4A8_OK) return r;
+    W4A8_TRY(cudaMemcpyAsync(out_bf16_host, out, L.bytes[R_OUT], cudaMemcpyDeviceToHost, s));
+    return W4A8_OK;
+}
+
+W4A8_EXPORT int w4a8_moe_forward_logits_host(const void* packed_up, const void* packed_down, int E, int H, int F,
+                                             const void* x_bf16_host, int T, const void* logits_bf16_host, int k,
+                                             void* out_bf16_host, void* ws, size_t ws_bytes, void* stream) {
+    MoeLayout L;
+    const int st = check_moe_args(packed_up, packed_down, E, H, F, T, k, ws, ws_bytes, true, &L);
+    if (st != W4A8_OK) return st;
+    if (T == 0) return W4A8_OK;
+    if (x_bf16_host == nullptr || logits_bf16_host == nullptr || out_bf16_host == nullptr) return W4A8_EINVAL;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint16_t* x = at<uint16_t>(ws, L, R_XIN);
+    uint16_t* logits = at<uint16_t>(ws, L, R_LOGITS);
+    int32_t* ids = at<int32_t>(ws, L, R_IDSIN);
+    float* w = at<float>(ws, L, R_WIN);
+    uint16_t* out = at<uint16_t>(ws, L, R_OUT);
+    W4A8_TRY(cudaMemcpyAsync(x, x_bf16_host, L.bytes[R_XIN], cudaMemcpyHostToDevice, s));
+    W4A8_TRY(cudaMemcpyAsync(logits, logits_bf16_host, L.bytes[R_LOGITS], cudaMemcpyHostToDevice, s));
+    {
+        ProfScope p(W4A8_KERNEL_ROUTE, 1, s);
+        W4A8_TRY(launch_route_topk(logits, T, E, k, ids, w, s));
+    }
     const int r = moe_forward_impl(packed_up, packed_down, E, H, F, x, T, ids, w, k, out, ws, L, s);
     if (r != W4A8_OK) return r;
     W4A8_TRY(cudaMemcpyAsync(out_bf16_host, out, L.bytes[R_OUT], cudaMemcpyDeviceToHost, s));
@@ -482,6 +520,7 @@ W4A8_EXPORT int w4a8_gemm(const int8_t* qa, const float* sa, int M, const void* 
     a.nvalid = N;
     a.partials = partials_opt;
     a.err = err;
+    apply_debug(a);
     W4A8_TRY(launch_gemm(a, tile, sm_count(), s));
     return W4A8_OK;
 }
@@ -516,6 +555,13 @@ W4A8_EXPORT int w4a8_last_device_error(const void* ws, void* stream) {
     if (cudaMemcpyAsync(&v, ws, 4, cudaMemcpyDeviceToHost, s) != cudaSuccess) return W4A8_ECUDA;
     if (cudaStreamSynchronize(s) != cudaSuccess) return W4A8_ECUDA;
     return (int)v;
+}
+
+W4A8_EXPORT int w4a8_debug_inject(unsigned int flags, long long wait_limit_cycles) {
+    if ((flags & ~kDebugSkipFirstCopy) != 0 || wait_limit_cycles < 0) return W4A8_EINVAL;
+    g_debug.flags = flags;
+    g_debug.wait_limit = wait_limit_cycles;
+    return W4A8_OK;
 }
 
 W4A8_EXPORT int w4a8_profile_start(void) {

@@ -42,7 +42,6 @@ namespace {
 
 constexpr uint32_t kMagicBits = 0x4B400000u;  // 1.5 * 2^23
 constexpr float kMagicF = 12582912.0f;
-constexpr long long kWaitLimitCycles = 4000000000ll;  // ~2 s: a bounded wait
 
 constexpr int GPS = 4;    // K groups per pipeline step
 constexpr int BN = 16;    // tokens per tile (one 16-row block)
@@ -109,14 +108,15 @@ __device__ __forceinline__ Item decode_item(int u, const GemmArgs& a) {
     return Item{t.x, u - mt * a.NT, t.y, t.z};
 }
 
-__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag, uint32_t* err) {
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag, uint32_t* err,
+                                         long long limit) {
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     for (uint32_t n = 1;; ++n) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((n & 15u) == 0) {
             if (*abort_flag) return false;
-            if (clock64() - t0 > kWaitLimitCycles) {
+            if (clock64() - t0 > limit) {
                 *abort_flag = 1;
                 atomicOr(err, kErrTimeout);
                 return false;
@@ -125,10 +125,10 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
     }
 }
 
-__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint32_t* err) {
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint32_t* err, long long limit) {
     const long long t0 = clock64();
     while (!mbar_try_wait(bar, parity)) {
-        if (clock64() - t0 > kWaitLimitCycles) {
+        if (clock64() - t0 > limit) {
             atomicOr(err, kErrTimeout);
             return;
         }
@@ -257,14 +257,16 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
                         last = j + 1;
                         const int g0 = t * GPS, ng = min(GPS, G - g0);
                         const int s = j % NS;
-                        if (!wait_bar(EMPTY_BAR(s), ((j / NS) & 1u) ^ 1u, abort_flag, a.err)) { ok = false; break; }
+                        if (!wait_bar(EMPTY_BAR(s), ((j / NS) & 1u) ^ 1u, abort_flag, a.err, a.wait_limit)) { ok = false; break; }
+                        // test hook: leave the first step's stage empty, so that its consumers time out
+                        if (j == 0 && blockIdx.x == 0 && (a.debug & kDebugSkipFirstCopy)) continue;
                         mbar_arrive_expect_tx(FULL_BAR(s), (uint32_t)ng * (kBlockBytes + BN * 128));
                         bulk_g2s(sA + s * kAStage, wsrc + (size_t)g0 * kBlockBytes, ng * kBlockBytes, FULL_BAR(s));
                         bulk_g2s(sB + s * kBStage, bsrc + (size_t)g0 * BN * 128, ng * BN * 128, FULL_BAR(s));
                     }
                 }
                 for (uint32_t qq = (last > (uint32_t)NS ? last - NS : 0u); qq < last; ++qq)
-                    if ((int)(qq & 1u) == pi) drain_wait(FULL_BAR(qq % NS), (qq / NS) & 1u, a.err);
+                    if ((int)(qq & 1u) == pi) drain_wait(FULL_BAR(qq % NS), (qq / NS) & 1u, a.err, a.wait_limit);
             }
             __syncwarp();
         } else {
@@ -282,8 +284,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
                     for (int t = 0; t < steps_per_item; ++t, ++j) {
                         const int ng = min(GPS, G - t * GPS);
                         const int s = j % NS, x = j % NA, b = j % ND;
-                        if (!wait_bar(CONV_BAR(x), (j / NA) & 1u, abort_flag, a.err)) { ok = false; break; }
-                        if (!wait_bar(DEMPTY_BAR(b), ((j / ND) & 1u) ^ 1u, abort_flag, a.err)) { ok = false; break; }
+                        if (!wait_bar(CONV_BAR(x), (j / NA) & 1u, abort_flag, a.err, a.wait_limit)) { ok = false; break; }
+                        if (!wait_bar(DEMPTY_BAR(b), ((j / ND) & 1u) ^ 1u, abort_flag, a.err, a.wait_limit)) { ok = false; break; }
                         tc_fence_after();
 #pragma unroll
                         for (int gh = 0; gh < GPS / 2; ++gh) {
@@ -303,7 +305,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
                     }
                 }
                 tc_commit(FINAL_BAR(mi));
-                drain_wait(FINAL_BAR(mi), 0, a.err);
+                drain_wait(FINAL_BAR(mi), 0, a.err, a.wait_limit);
             }
             __syncwarp();
         }
@@ -321,9 +323,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
             const int t = j % steps_per_item;
             const int ng = min(GPS, G - t * GPS);
             const int s = j % NS, x = j % NA, slot = j % NSC;
-            if (!wait_bar(FULL_BAR(s), (j / NS) & 1u, abort_flag, a.err)) break;
+            if (!wait_bar(FULL_BAR(s), (j / NS) & 1u, abort_flag, a.err, a.wait_limit)) break;
             // A slot x was last read by the MMAs of step j - NA
-            if (j >= NA && !wait_bar(EMPTY_BAR((j - NA) % NS), ((j - NA) / NS) & 1u, abort_flag, a.err)) break;
+            if (j >= NA && !wait_bar(EMPTY_BAR((j - NA) % NS), ((j - NA) / NS) & 1u, abort_flag, a.err, a.wait_limit)) break;
             for (int gq = 0; gq < ng; ++gq) {
                 const uint8_t* blk = smA + s * kAStage + gq * kBlockBytes;
                 uint4 w[4];
@@ -391,7 +393,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
             for (int t = 0; t < steps_per_item; ++t, ++j) {
                 const int ng = min(GPS, G - t * GPS);
                 const int b = j % ND, slot = j % NSC;
-                if (!wait_bar(EMPTY_BAR(j % NS), (j / NS) & 1u, abort_flag, a.err)) { ok = false; break; }
+                if (!wait_bar(EMPTY_BAR(j % NS), (j / NS) & 1u, abort_flag, a.err, a.wait_limit)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t taddr = tmem_base + lane_base + kDCol0 + (uint32_t)(b * kDCols);
                 uint32_t v[GPS / 2][BN];
@@ -406,7 +408,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(DEMPTY_BAR(b));
-                if (!wait_bar(SIDE_BAR(slot), (j / NSC) & 1u, abort_flag, a.err)) { ok = false; break; }
+                if (!wait_bar(SIDE_BAR(slot), (j / NSC) & 1u, abort_flag, a.err, a.wait_limit)) { ok = false; break; }
 #pragma unroll
                 for (int gh = 0; gh < GPS / 2; ++gh) {
                     const int gq = eh * (GPS / 2) + gh;
@@ -441,14 +443,14 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
             float* xrow = xbuf + (xp * 128 + r) * BN;
             if (eh == 1) {
                 // hand the sums to group 0 and go on with the next tile
-                if (!wait_bar(XEMPTY_BAR(xp), xpar ^ 1u, abort_flag, a.err)) { ok = false; break; }
+                if (!wait_bar(XEMPTY_BAR(xp), xpar ^ 1u, abort_flag, a.err, a.wait_limit)) { ok = false; break; }
 #pragma unroll
                 for (int i = 0; i < BN / 2; ++i) reinterpret_cast<uint64_t*>(xrow)[i] = acc2[i];
                 __syncwarp();
                 if (lane == 0) mbar_arrive(XFULL_BAR(xp));
                 continue;
             }
-            if (!wait_bar(XFULL_BAR(xp), xpar, abort_flag, a.err)) { ok = false; break; }
+            if (!wait_bar(XFULL_BAR(xp), xpar, abort_flag, a.err, a.wait_limit)) { ok = false; break; }
             float acc[BN];
 #pragma unroll
             for (int i = 0; i < BN; i += 2) {

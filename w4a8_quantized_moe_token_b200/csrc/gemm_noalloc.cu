@@ -61,3 +61,11 @@ W4A8_EXPORT int w4a8_gemm_noalloc(const int8_t* qa, const float* sa, int M, cons
     if (r != W4A8_OK) return r;
     return w4a8_gemm(qa, sa, M, packed, N, K, y, partials_opt, scratch, w4a8::kNoAllocScratchBytes, stream);
 }
+
+W4A8_EXPORT int w4a8_gemm_noalloc_last_error(void* stream) {
+    void* scratch = nullptr;
+    const int r = w4a8::scratch_address(&scratch);
+    if (r != W4A8_OK) return r;
+    // the dense GEMM keeps its device error word in the first bytes of its workspace
+    return w4a8_last_device_error(scratch, stream);
+}

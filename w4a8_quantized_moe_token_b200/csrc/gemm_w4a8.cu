@@ -47,7 +47,6 @@ namespace {
 constexpr uint32_t kMagicBits = 0x4B400000u;  // 1.5 * 2^23
 constexpr float kMagicF = 12582912.0f;
 
-constexpr long long kWaitLimitCycles = 4000000000ll;  // ~2 s: a bounded wait
 #ifndef W4A8_BACKOFF
 #define W4A8_BACKOFF() ((void)0)
 #endif
@@ -118,7 +117,8 @@ __device__ __forceinline__ Item decode_item(int u, const GemmArgs& a) {
 
 // Bounded wait on an mbarrier phase.  Returns false (and flags the CTA and the
 // device error word) when the wait runs out or another role already gave up.
-__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag, uint32_t* err) {
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag, uint32_t* err,
+                                         long long limit) {
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     for (uint32_t n = 1;; ++n) {
@@ -126,7 +126,7 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
         if (mbar_try_wait(bar, parity)) return true;
         if ((n & 15u) == 0) {
             if (*abort_flag) return false;
-            if (clock64() - t0 > kWaitLimitCycles) {
+            if (clock64() - t0 > limit) {
                 *abort_flag = 1;
                 atomicOr(err, kErrTimeout);
                 return false;
@@ -136,10 +136,10 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
 }
 
 // wait without the abort bookkeeping, for draining at exit
-__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint32_t* err) {
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint32_t* err, long long limit) {
     const long long t0 = clock64();
     while (!mbar_try_wait(bar, parity)) {
-        if (clock64() - t0 > kWaitLimitCycles) {
+        if (clock64() - t0 > limit) {
             atomicOr(err, kErrTimeout);
             return;
         }
@@ -276,7 +276,9 @@ __global__ void __launch_bounds__(C::kThreads, 1) gemm_w4a8_kernel(const GemmArg
                     if ((int)(j & 1u) != pi) continue;
                     last = j + 1;
                     const int s = j % NS;
-                    if (!wait_bar(EMPTY_BAR(s), ((j / NS) & 1u) ^ 1u, abort_flag, a.err)) { ok = false; break; }
+                    if (!wait_bar(EMPTY_BAR(s), ((j / NS) & 1u) ^ 1u, abort_flag, a.err, a.wait_limit)) { ok = false; break; }
+                    // test hook: leave the first step's stage empty, so that its consumers time out
+                    if (j == 0 && blockIdx.x == 0 && (a.debug & kDebugSkipFirstCopy)) continue;
                     mbar_arrive_expect_tx(FULL_BAR(s), kBlockBytes + bbytes);
                     bulk_g2s(sA + s * kBlockBytes, wsrc + (size_t)g * kBlockBytes, kBlockBytes, FULL_BAR(s));
                     bulk_g2s(sB + s * C::kBStageBytes, asrc + (size_t)g * a.act_plane, bbytes, FULL_BAR(s));
@@ -284,7 +286,7 @@ __global__ void __launch_bounds__(C::kThreads, 1) gemm_w4a8_kernel(const GemmArg
             }
             // never leave the CTA with copies still landing in its shared memory
             for (uint32_t qq = (last > (uint32_t)NS ? last - NS : 0u); qq < last; ++qq)
-                if ((int)(qq & 1u) == pi) drain_wait(FULL_BAR(qq % NS), (qq / NS) & 1u, a.err);
+                if ((int)(qq & 1u) == pi) drain_wait(FULL_BAR(qq % NS), (qq / NS) & 1u, a.err, a.wait_limit);
         }
         __syncwarp();
     } else if (warp < C::kConvWarps) {
@@ -308,8 +310,8 @@ __global__ void __launch_bounds__(C::kThreads, 1) gemm_w4a8_kernel(const GemmArg
         for (int j = cg; j < nsteps; j += C::NCG) {
             const int s = j % NS;
             const int x = j % NA;
-            if (!wait_bar(FULL_BAR(s), (j / NS) & 1u, abort_flag, a.err)) break;
-            if (!wait_bar(AEMPTY_BAR(x), ((j / NA) & 1u) ^ 1u, abort_flag, a.err)) break;
+            if (!wait_bar(FULL_BAR(s), (j / NS) & 1u, abort_flag, a.err, a.wait_limit)) break;
+            if (!wait_bar(AEMPTY_BAR(x), ((j / NA) & 1u) ^ 1u, abort_flag, a.err, a.wait_limit)) break;
             const uint8_t* blk = smA + s * kBlockBytes;
             uint4 w[4];
 #pragma unroll
@@ -348,8 +350,8 @@ __global__ void __launch_bounds__(C::kThreads, 1) gemm_w4a8_kernel(const GemmArg
                 for (int g = 0; g < G; ++g, ++j) {
                     if ((int)(j & 1u) != mi) continue;
                     const int s = j % NS, x = j % NA, b = j % ND;
-                    if (!wait_bar(CONV_BAR(x), (j / NA) & 1u, abort_flag, a.err)) { ok = false; break; }
-                    if (!wait_bar(DEMPTY_BAR(b), ((j / ND) & 1u) ^ 1u, abort_flag, a.err)) { ok = false; break; }
+                    if (!wait_bar(CONV_BAR(x), (j / NA) & 1u, abort_flag, a.err, a.wait_limit)) { ok = false; break; }
+                    if (!wait_bar(DEMPTY_BAR(b), ((j / ND) & 1u) ^ 1u, abort_flag, a.err, a.wait_limit)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t dt = tmem_base + C::kDCol0 + (uint32_t)b * BN;
                     const uint32_t at = tmem_base + C::kACol0 + (uint32_t)x * 32u;
@@ -364,7 +366,7 @@ __global__ void __launch_bounds__(C::kThreads, 1) gemm_w4a8_kernel(const GemmArg
             }
             // every MMA this warp issued must be complete before tensor memory is freed
             tc_commit(FINAL_BAR(mi));
-            drain_wait(FINAL_BAR(mi), 0, a.err);
+            drain_wait(FINAL_BAR(mi), 0, a.err, a.wait_limit);
         }
         __syncwarp();
     } else {
@@ -393,7 +395,7 @@ __global__ void __launch_bounds__(C::kThreads, 1) gemm_w4a8_kernel(const GemmArg
 #pragma unroll
                     for (int d = 0; d < C::NCG; ++d) {
                         const uint32_t jj = jl - (uint32_t)d;
-                        if (jj >= j && !wait_bar(SCFULL_BAR(jj % kNSC), (jj / kNSC) & 1u, abort_flag, a.err)) ok = false;
+                        if (jj >= j && !wait_bar(SCFULL_BAR(jj % kNSC), (jj / kNSC) & 1u, abort_flag, a.err, a.wait_limit)) ok = false;
                     }
                     if (!ok) break;
 #pragma unroll
@@ -403,7 +405,7 @@ __global__ void __launch_bounds__(C::kThreads, 1) gemm_w4a8_kernel(const GemmArg
                     for (int d = 0; d < 3; ++d) sc4[d] = sc4[d + 1];
                 }
                 const uint64_t sc2 = splat2(sc4[0]);
-                if (!wait_bar(DFULL_BAR(b), (j / ND) & 1u, abort_flag, a.err)) { ok = false; break; }
+                if (!wait_bar(DFULL_BAR(b), (j / ND) & 1u, abort_flag, a.err, a.wait_limit)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t taddr = tmem_base + lane_base + C::kDCol0 + (uint32_t)b * BN + col0;
                 // Columns past the tile's tokens are never written by the MMAs: they hold

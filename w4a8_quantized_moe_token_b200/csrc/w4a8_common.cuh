@@ -28,6 +28,12 @@ constexpr int kMaxExperts = 1024;
 constexpr uint32_t kErrTimeout = 1u;
 constexpr uint32_t kErrBadExpert = 2u;
 
+// how long a bounded mbarrier wait may last before it gives up (clock cycles, ~2 s)
+constexpr long long kWaitLimitCycles = 4000000000ll;
+// debug word bit: CTA 0's producer issues no copy for its first pipeline step, so the
+// consumers' bounded waits run out (a test of the failure-detection path)
+constexpr uint32_t kDebugSkipFirstCopy = 1u;
+
 __host__ __device__ inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
 __host__ __device__ inline int round_up(int a, int b) { return ceil_div(a, b) * b; }
 

@@ -24,6 +24,15 @@ struct GemmArgs {
     int nvalid;               // valid output columns (N, or F for mode 1)
     int32_t* partials;        // mode 0 only, optional: exact INT32 partials [rows][nvalid][G]
     uint32_t* err;            // device error word
+    long long wait_limit;     // clock cycles a bounded wait may last (> 0; normally ~2 s)
+    uint32_t debug;           // test hook: bit 0 = CTA 0 issues no copy for its first step
+};
+
+// Test hook of the failure-detection path (w4a8_debug_inject): while set on the
+// calling host thread, GEMM launches get this wait limit and debug word.
+struct DebugInject {
+    uint32_t flags = 0;
+    long long wait_limit = 0;
 };
 
 // launchers (all asynchronous on `stream`); return the cudaGetLastError() of the launch

@@ -59,6 +59,12 @@ WORKLOADS = {
     "large_decode": Workload("large_decode", "moe", E=384, topk=8, T=256, H=7168, F=2048,
                              routing="zipf", zipf_s=1.1),
     "prefill": Workload("prefill", "moe", E=384, topk=8, T=16384, H=7168, F=2048, routing="uniform"),
+    # reduced layers of the same per-expert shapes, small enough for a full ncu capture:
+    # 16 experts with ~341 rows each (the prefill layer's mean), and 48 experts under
+    # the large decode layer's Zipf routing (~5 rows each)
+    "prefill_slice": Workload("prefill_slice", "moe", E=16, topk=8, T=682, H=7168, F=2048, routing="uniform"),
+    "large_decode_slice": Workload("large_decode_slice", "moe", E=48, topk=8, T=32, H=7168, F=2048,
+                                   routing="zipf", zipf_s=1.1),
     # INT8 KV cache of one attention layer: 32768 tokens x 8 KV heads x 128 channels,
     # static per-head scales calibrated on the first 1024 tokens
     "kv_int8": Workload("kv_int8", "kv", T=32768, extra={"heads": 8, "head_dim": 128, "calib_tokens": 1024}),
