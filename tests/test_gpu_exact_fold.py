@@ -54,7 +54,8 @@ def to_dev_bf16(a):
     return torch.from_numpy(synth.bf16_bits(a).view(np.int16)).view(torch.bfloat16).cuda()
 
 
-@pytest.mark.parametrize("M,N,K", [(300, 256, 640), (129, 384, 200), (17, 128, 1024), (16, 256, 512), (5, 128, 8192)])
+@pytest.mark.parametrize("M,N,K", [(300, 256, 640), (129, 384, 200), (17, 128, 1024), (16, 256, 512), (5, 128, 8192),
+                                   (40, 130, 256)])  # N % 4 != 0: rows not 16-byte aligned, direct stores
 def test_dense_gemm_without_partials_is_bit_exact(M, N, K):
     """M > 16: the wide-tile production instance (no partials buffer); M <= 16: the
     decode-tile kernel.  K = 8192 is the largest K (64 groups) for which the exact

@@ -30,9 +30,11 @@
 //                        acc += scale * P in fp32 (packed fp32x2); at the end of a tile
 //                        group 1 passes its sums to group 0, which applies the token
 //                        scale and stores.
-// The accumulators start at the bit pattern 0x4B400000 (1.5 * 2^23): the MMAs add
-// the partial (|P| < 2^22), so the bits read back as fp32 are exactly 1.5 * 2^23 + P,
-// and one packed fp32 subtraction yields P without an int -> float conversion.
+// Each MMA warp first resets its groups' accumulators to the bit pattern 0x4B400000
+// (1.5 * 2^23) with one bf16 MMA (mma_reset_acc); the INT8 MMAs add the partial
+// (|P| < 2^22), so the bits read back as fp32 are exactly 1.5 * 2^23 + P, and one packed
+// fp32 subtraction yields P without an int -> float conversion.  The epilogue only
+// reads the accumulators.
 #include "w4a8_common.cuh"
 #include "w4a8_internal.h"
 
@@ -40,7 +42,7 @@ namespace w4a8 {
 
 namespace {
 
-constexpr uint32_t kMagicBits = 0x4B400000u;  // 1.5 * 2^23
+constexpr uint32_t kMagicBits = 0x4B400000u;  // 1.5 * 2^23 (what the reset MMA writes)
 constexpr float kMagicF = 12582912.0f;
 
 constexpr int GPS = 4;    // K groups per pipeline step
@@ -48,7 +50,7 @@ constexpr int BN = 16;    // tokens per tile (one 16-row block)
 constexpr int NS = 4;     // shared-memory stages
 constexpr int NA = 2;     // tensor-memory A slots (GPS x 32 columns each)
 constexpr int ND = 4;     // tensor-memory accumulators (GPS x BN columns each)
-constexpr int NSC = 8;    // scale ring slots (>= NA + ND)
+constexpr int NSC = 6;    // scale ring slots (>= NA + ND)
 constexpr int kAStage = GPS * kBlockBytes;  // weight blocks of one step
 constexpr int kBStage = GPS * BN * 128;     // token rows of one step
 constexpr int kACols = GPS * 32;
@@ -79,7 +81,8 @@ constexpr int kOffSc = kOffA + NS * kAStage;          // ring: fp32 scale       
 constexpr int kOffZp = kOffSc + NSC * GPS * 128 * 4;  // ring: fp32 zero point  [NSC][GPS][128]
 constexpr int kOffS = kOffZp + NSC * GPS * 128 * 4;   // ring: token group sums [NSC][GPS][BN]
 constexpr int kOffX = kOffS + NSC * GPS * BN * 4;     // epilogue exchange: [2][128][BN] fp32
-constexpr int kOffBar = kOffX + 2 * 128 * BN * 4;
+constexpr int kOffReset = kOffX + 2 * 128 * BN * 4;   // the accumulator-reset operands
+constexpr int kOffBar = kOffReset + 2 * kResetTileBytes;
 // full[NS] empty[NS] conv[NA] (unused: NA + ND) dempty[ND] side[NSC] final[2]
 // xfull[2] xempty[2]
 constexpr int kNumBars = 2 * NS + 2 * NA + 2 * ND + NSC + 2 + 4;
@@ -133,14 +136,6 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint32
             return;
         }
     }
-}
-
-__device__ __forceinline__ void tmem_st16_const(uint32_t taddr, uint32_t v) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-        "{%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1};" ::"r"(taddr),
-        "r"(v)
-        : "memory");
 }
 
 // a packed pair of accumulators (low word: even token) += sc * P with the zero point
@@ -221,19 +216,14 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
         tmem_alloc(smem_u32(tmem_slot), kTmemCols);
         tmem_relinquish();
     }
+    fill_reset_tiles(smem + kOffReset);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    const uint32_t sReset = base_addr + kOffReset;
     const int q = warp & 3;
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
-    if (warp >= kEpiWarp0 && warp < kEpiWarp0 + 4) {
-        for (int c = 0; c < ND * kDCols / 16; ++c) tmem_st16_const(tmem_base + lane_base + kDCol0 + c * 16, kMagicBits);
-        tmem_st_wait();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
 
     const int total = a.NT * __ldg(a.n_mtiles);
     const int G = a.G;
@@ -247,7 +237,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
             const int pi = cw == 0 ? 0 : 1;
             if (lane == 0) {
                 uint32_t j = 0, last = 0;
-                bool ok = true;
+                bool ok = true, rdy = false;  // rdy: an early test found this step's stage free
                 for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
                     const Item it = decode_item(u, a);
                     const uint8_t* wsrc = a.wblocks + (size_t)(it.e * a.NT + it.nt) * G * kBlockBytes;
@@ -257,7 +247,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
                         last = j + 1;
                         const int g0 = t * GPS, ng = min(GPS, G - g0);
                         const int s = j % NS;
-                        if (!wait_bar(EMPTY_BAR(s), ((j / NS) & 1u) ^ 1u, abort_flag, a.err, a.wait_limit)) { ok = false; break; }
+                        if (!rdy && !wait_bar(EMPTY_BAR(s), ((j / NS) & 1u) ^ 1u, abort_flag, a.err, a.wait_limit)) { ok = false; break; }
+                        rdy = mbar_test(EMPTY_BAR((j + 2) % NS), (((j + 2) / NS) & 1u) ^ 1u);
                         // test hook: leave the first step's stage empty, so that its consumers time out
                         if (j == 0 && blockIdx.x == 0 && (a.debug & kDebugSkipFirstCopy)) continue;
                         mbar_arrive_expect_tx(FULL_BAR(s), (uint32_t)ng * (kBlockBytes + BN * 128));
@@ -275,18 +266,27 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
             // 2mi+1: the issue rate of tcgen05.mma is a per-thread limit, so splitting a
             // step halves the time its A slot stays busy.  Each warp commits to the
             // step's barriers (two arrivals each), also when it had no group to issue.
+            // the whole warp runs the loop (warp-uniform operands for tcgen05.mma); one
+            // elected thread issues
             const int mi = cw - 1;
-            if (lane == 0) {
+            {
                 uint32_t j = 0;
-                bool ok = true;
+                bool ok = true, conv_rdy = false, acc_rdy = false;  // early tests of this step's barriers
                 const uint32_t idesc = idesc_i8(128, BN, false);  // u8 codes x s8 tokens
                 for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
                     for (int t = 0; t < steps_per_item; ++t, ++j) {
                         const int ng = min(GPS, G - t * GPS);
                         const int s = j % NS, x = j % NA, b = j % ND;
-                        if (!wait_bar(CONV_BAR(x), (j / NA) & 1u, abort_flag, a.err, a.wait_limit)) { ok = false; break; }
-                        if (!wait_bar(DEMPTY_BAR(b), ((j / ND) & 1u) ^ 1u, abort_flag, a.err, a.wait_limit)) { ok = false; break; }
+                        if (!conv_rdy && !wait_bar(CONV_BAR(x), (j / NA) & 1u, abort_flag, a.err, a.wait_limit)) { ok = false; break; }
+                        if (!acc_rdy && !wait_bar(DEMPTY_BAR(b), ((j / ND) & 1u) ^ 1u, abort_flag, a.err, a.wait_limit)) { ok = false; break; }
+                        conv_rdy = mbar_test(CONV_BAR((j + 1) % NA), ((j + 1) / NA) & 1u);
+                        acc_rdy = mbar_test(DEMPTY_BAR((j + 1) % ND), (((j + 1) / ND) & 1u) ^ 1u);
                         tc_fence_after();
+                        if (elect_one()) {
+                        // reset this warp's groups' accumulators (32 columns), then add the partials
+                        if (mi * (GPS / 2) < ng)
+                            mma_reset_acc(tmem_base + kDCol0 + (uint32_t)(b * kDCols + mi * (GPS / 2) * BN), sReset,
+                                          (GPS / 2) * BN);
 #pragma unroll
                         for (int gh = 0; gh < GPS / 2; ++gh) {
                             const int gq = mi * (GPS / 2) + gh;
@@ -302,9 +302,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
                         // one commit tells the producer (stage s free), the converters (A
                         // slot free) and the epilogue (accumulators ready) at once
                         tc_commit(EMPTY_BAR(s));
+                        }
+                        __syncwarp();
                     }
                 }
-                tc_commit(FINAL_BAR(mi));
+                if (elect_one()) tc_commit(FINAL_BAR(mi));
+                __syncwarp();
                 drain_wait(FINAL_BAR(mi), 0, a.err, a.wait_limit);
             }
             __syncwarp();
@@ -319,13 +322,18 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
         uint32_t m28;
         asm volatile("mov.u32 %0, 0x10000000;" : "=r"(m28));  // x * 2^28 >> 32 = x >> 4, on the FMA pipe
         const int nsteps = ((total - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x) * steps_per_item;
+        bool full_rdy = false;  // an early test of this step's stage
         for (int j = cg; j < nsteps; j += 2) {
             const int t = j % steps_per_item;
             const int ng = min(GPS, G - t * GPS);
             const int s = j % NS, x = j % NA, slot = j % NSC;
-            if (!wait_bar(FULL_BAR(s), (j / NS) & 1u, abort_flag, a.err, a.wait_limit)) break;
+            if (!full_rdy && !wait_bar(FULL_BAR(s), (j / NS) & 1u, abort_flag, a.err, a.wait_limit)) break;
             // A slot x was last read by the MMAs of step j - NA
-            if (j >= NA && !wait_bar(EMPTY_BAR((j - NA) % NS), ((j - NA) / NS) & 1u, abort_flag, a.err, a.wait_limit)) break;
+            // (the MMAs of step j - NA can only finish after this group's previous step, so
+            // there is no earlier point at which to test for them)
+            if (j >= NA && !wait_bar(EMPTY_BAR((j - NA) % NS), ((j - NA) / NS) & 1u, abort_flag, a.err, a.wait_limit))
+                break;
+            full_rdy = mbar_test(FULL_BAR((j + 2) % NS), ((j + 2) / NS) & 1u);  // this group's next step
             for (int gq = 0; gq < ng; ++gq) {
                 const uint8_t* blk = smA + s * kAStage + gq * kBlockBytes;
                 uint4 w[4];
@@ -382,7 +390,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
         float* xbuf = reinterpret_cast<float*>(smem + kOffX);
         uint32_t j = 0;
         uint32_t nit = 0;  // tiles done by this CTA
-        bool ok = true;
+        bool ok = true, acc_rdy = false, side_rdy = false;  // early tests of this step's barriers
         for (int u = blockIdx.x; u < total && ok; u += gridDim.x, ++nit) {
             const Item it = decode_item(u, a);
             uint64_t acc2[BN / 2];  // token pairs, packed fp32x2
@@ -393,7 +401,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
             for (int t = 0; t < steps_per_item; ++t, ++j) {
                 const int ng = min(GPS, G - t * GPS);
                 const int b = j % ND, slot = j % NSC;
-                if (!wait_bar(EMPTY_BAR(j % NS), (j / NS) & 1u, abort_flag, a.err, a.wait_limit)) { ok = false; break; }
+                if (!acc_rdy && !wait_bar(EMPTY_BAR(j % NS), (j / NS) & 1u, abort_flag, a.err, a.wait_limit)) { ok = false; break; }
+                acc_rdy = mbar_test(EMPTY_BAR((j + 1) % NS), ((j + 1) / NS) & 1u);
                 tc_fence_after();
                 const uint32_t taddr = tmem_base + lane_base + kDCol0 + (uint32_t)(b * kDCols);
                 uint32_t v[GPS / 2][BN];
@@ -401,14 +410,11 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
                 for (int gh = 0; gh < GPS / 2; ++gh)
                     if (eh * (GPS / 2) + gh < ng) tmem_ld16(taddr + (eh * (GPS / 2) + gh) * BN, v[gh]);
                 tmem_ld_wait();
-#pragma unroll
-                for (int gh = 0; gh < GPS / 2; ++gh)
-                    if (eh * (GPS / 2) + gh < ng) tmem_st16_const(taddr + (eh * (GPS / 2) + gh) * BN, kMagicBits);
-                tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(DEMPTY_BAR(b));
-                if (!wait_bar(SIDE_BAR(slot), (j / NSC) & 1u, abort_flag, a.err, a.wait_limit)) { ok = false; break; }
+                if (!side_rdy && !wait_bar(SIDE_BAR(slot), (j / NSC) & 1u, abort_flag, a.err, a.wait_limit)) { ok = false; break; }
+                side_rdy = mbar_test(SIDE_BAR((j + 1) % NSC), ((j + 1) / NSC) & 1u);
 #pragma unroll
                 for (int gh = 0; gh < GPS / 2; ++gh) {
                     const int gq = eh * (GPS / 2) + gh;

@@ -32,11 +32,12 @@
 // many channels, so M=128 is always full and N shrinks to the tokens.
 //
 // This kernel serves layers with many tokens per expert (tiles of up to 128 tokens);
-// decode-shaped layers use gemm_decode.cu.  Every accumulator holds 0x4B400000 (the
-// fp32 bit pattern of 1.5 * 2^23) before its step's MMAs, which add the INT32 partial
-// P (|P| < 2^22) on top, so the result read as fp32 is exactly 1.5 * 2^23 + P and the
-// epilogue recovers P with one packed fp32 subtraction instead of an int -> float
-// conversion, then writes the constant back.
+// decode-shaped layers use gemm_decode.cu.  Every step starts with a bf16 MMA that
+// resets its accumulator to 0x4B400000 (the fp32 bit pattern of 1.5 * 2^23, see
+// mma_reset_acc); the step's INT8 MMAs add the INT32 partial P (|P| < 2^22) on top, so
+// the result read as fp32 is exactly 1.5 * 2^23 + P and the epilogue recovers P with
+// one packed fp32 subtraction instead of an int -> float conversion.  The epilogue
+// only reads the accumulator and releases it: no tensor-memory writes on the CUDA cores.
 #include "w4a8_common.cuh"
 #include "w4a8_internal.h"
 
@@ -44,7 +45,7 @@ namespace w4a8 {
 
 namespace {
 
-constexpr uint32_t kMagicBits = 0x4B400000u;  // 1.5 * 2^23
+constexpr uint32_t kMagicBits = 0x4B400000u;  // 1.5 * 2^23 (what the reset MMA writes)
 constexpr float kMagicF = 12582912.0f;
 
 #ifndef W4A8_BACKOFF
@@ -59,7 +60,7 @@ constexpr float kMagicF = 12582912.0f;
 template <int BN_, int NS_, int NA_, int ND_, int NEPI_, int NCG_>
 struct Cfg {
     static constexpr int BN = BN_, NS = NS_, NA = NA_, ND = ND_, NEPI = NEPI_, NCG = NCG_;
-    static constexpr int kNSC = 32;       // scale ring slots (>= NA + ND)
+    static constexpr int kNSC = 16;       // scale ring slots (>= NA + ND + 4)
     static constexpr int kCW = BN / NEPI;  // accumulator columns per epilogue thread
     // warpgroups: NCG converter groups, NEPI epilogue groups, 1 control group
     // (producer warp, two MMA warps, second producer warp)
@@ -81,16 +82,22 @@ struct Cfg {
     static constexpr uint32_t kACol0 = 0;
     static constexpr uint32_t kDCol0 = NA * 32;
     static_assert(kDCol0 + ND * BN <= kTmemCols, "tensor memory over-subscribed");
-    static_assert(kNSC >= NA + ND, "scale ring too small");
+    static_assert(kNSC >= NA + ND + 4, "scale ring too small");
     static_assert(NS % 2 == 0, "the two producers own the stages of one parity each");
     static_assert(kCW % 16 == 0 && (kCW <= 64 || kCW % 64 == 0), "epilogue column split");
     // shared memory carve-up
     static constexpr int kOffB = 0;  // 1024-aligned (128-byte swizzle atoms)
     static constexpr int kOffA = kOffB + NS * kBStageBytes;
     static constexpr int kOffSc = kOffA + NS * kBlockBytes;  // ring: fp32 scale per row
-    static constexpr int kOffBar = kOffSc + kNSC * kTileRows * 4;
-    // full[NS] empty[NS] conv[NA] aempty[NA] dfull[ND] dempty[ND] scfull[NSC] final[2]
-    static constexpr int kNumBars = 2 * NS + 2 * NA + 2 * ND + kNSC + 2;
+    static constexpr int kOffReset = kOffSc + kNSC * kTileRows * 4;  // the accumulator-reset operands
+    // output staging tile: fp32 [BN tokens][128 channels] (plain output) or
+    // [BN tokens][kStageH] (SwiGLU output, 64 channels + padding against bank conflicts)
+    static constexpr int kStageH = 80;
+    static constexpr int kOffStage = kOffReset + 2 * kResetTileBytes;
+    static constexpr int kOffSa = kOffStage + BN * kTileRows * 4;  // the tile's token scales
+    static constexpr int kOffBar = kOffSa + BN * 4;
+    // full[NS] empty[NS] conv[NA] aempty[NA] dfull[ND] dempty[ND] scfull[NSC] final[2] stage[2]
+    static constexpr int kNumBars = 2 * NS + 2 * NA + 2 * ND + kNSC + 2 + 2;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
     static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
     static_assert(kSmemBytes <= 227 * 1024, "shared memory over-subscribed");
@@ -146,16 +153,9 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint32
     }
 }
 
-__device__ __forceinline__ void tmem_st16_const(uint32_t taddr, uint32_t v) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-        "{%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1};" ::"r"(taddr),
-        "r"(v)
-        : "memory");
-}
-
 // a packed pair of accumulators (low word: even column) += sc * (x - 1.5*2^23) with
-// fp32x2 arithmetic: acc2 += sc2 * (x - m2), sc2 and m2 holding the value twice
+// fp32x2 arithmetic: acc2 += sc2 * (x - m2), sc2 and m2 holding the value twice; x holds
+// the INT32 partial P as the fp32 value 1.5 * 2^23 + P, so the subtraction is exact
 __device__ __forceinline__ void fold2_packed(uint64_t& acc2, uint64_t sc2, uint64_t m2, uint32_t x0, uint32_t x1) {
     asm("{\n\t.reg .b64 x;\n\t"
         "mov.b64 x, {%1, %2};\n\t"
@@ -186,6 +186,7 @@ __device__ __forceinline__ float silu_mul(float g, float u) { return __fdividef(
 #define DEMPTY_BAR(b) (bar0 + 8u * (uint32_t)(2 * NS + 2 * NA + ND + (b)))
 #define SCFULL_BAR(i) (bar0 + 8u * (uint32_t)(2 * NS + 2 * NA + 2 * ND + (i)))
 #define FINAL_BAR(m) (bar0 + 8u * (uint32_t)(2 * NS + 2 * NA + 2 * ND + kNSC + (m)))
+#define STAGE_BAR(m) (bar0 + 8u * (uint32_t)(2 * NS + 2 * NA + 2 * ND + kNSC + 2 + (m)))
 
 template <class C, bool kPartials>
 __global__ void __launch_bounds__(C::kThreads, 1) gemm_w4a8_kernel(const GemmArgs a) {
@@ -222,6 +223,8 @@ __global__ void __launch_bounds__(C::kThreads, 1) gemm_w4a8_kernel(const GemmArg
         for (int i = 0; i < kNSC; ++i) mbar_init(SCFULL_BAR(i), 4);
         mbar_init(FINAL_BAR(0), 1);
         mbar_init(FINAL_BAR(1), 1);
+        mbar_init(STAGE_BAR(0), 4 * C::NEPI);  // staging tile free, token scales written
+        mbar_init(STAGE_BAR(1), 4 * C::NEPI);  // staging tile written
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -229,27 +232,15 @@ __global__ void __launch_bounds__(C::kThreads, 1) gemm_w4a8_kernel(const GemmArg
         tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
         tmem_relinquish();
     }
+    fill_reset_tiles(smem + C::kOffReset);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    const uint32_t sReset = base_addr + C::kOffReset;
 
-    const bool is_epi = warp >= C::kEpiWarp0 && warp < C::kProdWarp;
     const int q = warp & 3;  // TMEM lane quarter of this warp
-
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
-    if (is_epi) {
-        const int eh = (warp - C::kEpiWarp0) >> 2;
-#pragma unroll
-        for (int b = 0; b < ND; ++b)
-#pragma unroll
-            for (int c = 0; c < kCW / 16; ++c)
-                tmem_st16_const(tmem_base + lane_base + C::kDCol0 + b * BN + eh * kCW + c * 16, kMagicBits);
-        tmem_st_wait();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
 
     const int total = a.NT * __ldg(a.n_mtiles);
     const int G = a.G;
@@ -266,7 +257,7 @@ __global__ void __launch_bounds__(C::kThreads, 1) gemm_w4a8_kernel(const GemmArg
         const int pi = warp == C::kProdWarp ? 0 : 1;
         if (lane == 0) {
             uint32_t j = 0, last = 0;
-            bool ok = true;
+            bool ok = true, rdy = false;  // rdy: an early test found this step's stage free
             for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
                 const Item it = decode_item<BN>(u, a);
                 const uint32_t bbytes = (uint32_t)round_up(it.nrows, 16) * 128u;
@@ -276,7 +267,8 @@ __global__ void __launch_bounds__(C::kThreads, 1) gemm_w4a8_kernel(const GemmArg
                     if ((int)(j & 1u) != pi) continue;
                     last = j + 1;
                     const int s = j % NS;
-                    if (!wait_bar(EMPTY_BAR(s), ((j / NS) & 1u) ^ 1u, abort_flag, a.err, a.wait_limit)) { ok = false; break; }
+                    if (!rdy && !wait_bar(EMPTY_BAR(s), ((j / NS) & 1u) ^ 1u, abort_flag, a.err, a.wait_limit)) { ok = false; break; }
+                    rdy = mbar_test(EMPTY_BAR((j + 2) % NS), (((j + 2) / NS) & 1u) ^ 1u);
                     // test hook: leave the first step's stage empty, so that its consumers time out
                     if (j == 0 && blockIdx.x == 0 && (a.debug & kDebugSkipFirstCopy)) continue;
                     mbar_arrive_expect_tx(FULL_BAR(s), kBlockBytes + bbytes);
@@ -307,11 +299,17 @@ __global__ void __launch_bounds__(C::kThreads, 1) gemm_w4a8_kernel(const GemmArg
                 mbar_arrive(SCFULL_BAR(jp % kNSC));
             }
         };
+        bool full_rdy = false, aslot_rdy = false;  // early tests of this step's barriers
         for (int j = cg; j < nsteps; j += C::NCG) {
             const int s = j % NS;
             const int x = j % NA;
-            if (!wait_bar(FULL_BAR(s), (j / NS) & 1u, abort_flag, a.err, a.wait_limit)) break;
-            if (!wait_bar(AEMPTY_BAR(x), ((j / NA) & 1u) ^ 1u, abort_flag, a.err, a.wait_limit)) break;
+            if (!full_rdy && !wait_bar(FULL_BAR(s), (j / NS) & 1u, abort_flag, a.err, a.wait_limit)) break;
+            if (!aslot_rdy && !wait_bar(AEMPTY_BAR(x), ((j / NA) & 1u) ^ 1u, abort_flag, a.err, a.wait_limit)) break;
+            {
+                const int jn = j + C::NCG;
+                full_rdy = mbar_test(FULL_BAR(jn % NS), (jn / NS) & 1u);
+                aslot_rdy = mbar_test(AEMPTY_BAR(jn % NA), ((jn / NA) & 1u) ^ 1u);
+            }
             const uint8_t* blk = smA + s * kBlockBytes;
             uint4 w[4];
 #pragma unroll
@@ -340,32 +338,42 @@ __global__ void __launch_bounds__(C::kThreads, 1) gemm_w4a8_kernel(const GemmArg
         if (prev >= 0) signal(prev);
     } else if (warp >= C::kMmaWarp0) {
         // ---------------- MMA issue: warp mi takes the steps with j % 2 == mi ----------------
+        // The whole warp runs the loop (its values stay warp-uniform, so the operands of
+        // tcgen05.mma need no per-instruction moves); one elected thread issues.
         const int mi = warp - C::kMmaWarp0;
-        if (lane == 0) {
+        {
             uint32_t j = 0;
-            bool ok = true;
+            bool ok = true, conv_rdy = false, acc_rdy = false;  // early tests of this step's barriers
             for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
                 const Item it = decode_item<BN>(u, a);
-                const uint32_t idesc = idesc_i8(128, round_up(it.nrows, 16));
+                const int ncols = round_up(it.nrows, 16);
+                const uint32_t idesc = idesc_i8(128, ncols);
                 for (int g = 0; g < G; ++g, ++j) {
                     if ((int)(j & 1u) != mi) continue;
                     const int s = j % NS, x = j % NA, b = j % ND;
-                    if (!wait_bar(CONV_BAR(x), (j / NA) & 1u, abort_flag, a.err, a.wait_limit)) { ok = false; break; }
-                    if (!wait_bar(DEMPTY_BAR(b), ((j / ND) & 1u) ^ 1u, abort_flag, a.err, a.wait_limit)) { ok = false; break; }
+                    if (!conv_rdy && !wait_bar(CONV_BAR(x), (j / NA) & 1u, abort_flag, a.err, a.wait_limit)) { ok = false; break; }
+                    if (!acc_rdy && !wait_bar(DEMPTY_BAR(b), ((j / ND) & 1u) ^ 1u, abort_flag, a.err, a.wait_limit)) { ok = false; break; }
+                    conv_rdy = mbar_test(CONV_BAR((j + 2) % NA), ((j + 2) / NA) & 1u);
+                    acc_rdy = mbar_test(DEMPTY_BAR((j + 2) % ND), (((j + 2) / ND) & 1u) ^ 1u);
                     tc_fence_after();
                     const uint32_t dt = tmem_base + C::kDCol0 + (uint32_t)b * BN;
                     const uint32_t at = tmem_base + C::kACol0 + (uint32_t)x * 32u;
                     const uint32_t sb = sB + s * C::kBStageBytes;
+                    if (elect_one()) {
+                        mma_reset_acc(dt, sReset, ncols);
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_i8_ts(dt, at + kk * 8, smem_desc_sw128(sb + kk * 32), idesc, 1u);
-                    tc_commit(EMPTY_BAR(s));
-                    tc_commit(AEMPTY_BAR(x));
-                    tc_commit(DFULL_BAR(b));
+                        for (int kk = 0; kk < 4; ++kk)
+                            mma_i8_ts(dt, at + kk * 8, smem_desc_sw128(sb + kk * 32), idesc, 1u);
+                        tc_commit(EMPTY_BAR(s));
+                        tc_commit(AEMPTY_BAR(x));
+                        tc_commit(DFULL_BAR(b));
+                    }
+                    __syncwarp();
                 }
             }
             // every MMA this warp issued must be complete before tensor memory is freed
-            tc_commit(FINAL_BAR(mi));
+            if (elect_one()) tc_commit(FINAL_BAR(mi));
+            __syncwarp();
             drain_wait(FINAL_BAR(mi), 0, a.err, a.wait_limit);
         }
         __syncwarp();
@@ -376,11 +384,23 @@ __global__ void __launch_bounds__(C::kThreads, 1) gemm_w4a8_kernel(const GemmArg
         const int r = q * 32 + lane;                 // tile row = TMEM lane
         const int col0 = eh * kCW;
         const int nsteps = ((total - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x) * G;
+        // The tile is written through a shared-memory staging tile and 1-D bulk copies
+        // (one output row per issuing thread), so the epilogue goes on with the next
+        // tile while the stores drain; this needs every output row to start on a
+        // 16-byte boundary.  Otherwise (a dense output with N % 4 != 0) it stores directly.
+        const bool staged = !kPartials && (a.ldo % 4 == 0) && (a.mode == 1 || a.nvalid % 4 == 0);
+        float* stage = reinterpret_cast<float*>(smem + C::kOffStage);
+        float* sa_s = reinterpret_cast<float*>(smem + C::kOffSa);
+        const int et = threadIdx.x - 32 * C::kEpiWarp0;  // epilogue thread 0 .. 128 * NEPI - 1
+        bool issued = false;                            // a bulk copy of this thread is in flight
+        uint32_t ntile = 0;
         float sc4[4] = {0.f, 0.f, 0.f, 0.f};
         uint32_t j = 0;
-        bool ok = true;
-        for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
+        bool ok = true, acc_rdy = false, sc_rdy = false;  // early tests of this step's barriers
+        for (int u = blockIdx.x; u < total && ok; u += gridDim.x, ++ntile) {
             const Item it = decode_item<BN>(u, a);
+            // the tile's token scales, loaded now and used at its end
+            const float my_sa = (staged && eh == 0 && r < it.nrows) ? __ldg(a.act_scale + it.row0 + r) : 0.f;
             uint64_t acc2[kCW / 2];  // column pairs, packed fp32x2
 #pragma unroll
             for (int i = 0; i < kCW / 2; ++i) acc2[i] = 0ull;
@@ -395,7 +415,9 @@ __global__ void __launch_bounds__(C::kThreads, 1) gemm_w4a8_kernel(const GemmArg
 #pragma unroll
                     for (int d = 0; d < C::NCG; ++d) {
                         const uint32_t jj = jl - (uint32_t)d;
-                        if (jj >= j && !wait_bar(SCFULL_BAR(jj % kNSC), (jj / kNSC) & 1u, abort_flag, a.err, a.wait_limit)) ok = false;
+                        if (jj >= j && !(sc_rdy && d == 0) &&
+                            !wait_bar(SCFULL_BAR(jj % kNSC), (jj / kNSC) & 1u, abort_flag, a.err, a.wait_limit))
+                            ok = false;
                     }
                     if (!ok) break;
 #pragma unroll
@@ -405,27 +427,34 @@ __global__ void __launch_bounds__(C::kThreads, 1) gemm_w4a8_kernel(const GemmArg
                     for (int d = 0; d < 3; ++d) sc4[d] = sc4[d + 1];
                 }
                 const uint64_t sc2 = splat2(sc4[0]);
-                if (!wait_bar(DFULL_BAR(b), (j / ND) & 1u, abort_flag, a.err, a.wait_limit)) { ok = false; break; }
+                if (!acc_rdy && !wait_bar(DFULL_BAR(b), (j / ND) & 1u, abort_flag, a.err, a.wait_limit)) { ok = false; break; }
+                // early tests for the next step (the scales of the next block of four when
+                // this step ends one)
+                acc_rdy = mbar_test(DFULL_BAR((j + 1) % ND), ((j + 1) / ND) & 1u);
+                if ((j & 3u) == 3u) {
+                    const uint32_t jl = min(j + 4u, (uint32_t)nsteps - 1u);
+                    sc_rdy = jl > j && mbar_test(SCFULL_BAR(jl % kNSC), (jl / kNSC) & 1u);
+                }
                 tc_fence_after();
                 const uint32_t taddr = tmem_base + lane_base + C::kDCol0 + (uint32_t)b * BN + col0;
-                // Columns past the tile's tokens are never written by the MMAs: they hold
-                // the constant, so they read as partial 0 and need no test.
+                // Columns past the tile's tokens (beyond the MMAs' N) hold stale values:
+                // they only reach outputs that are never stored.
                 if constexpr (!kPartials) {
-                    // two loads of the warp's columns, the constant goes back, the buffer is
-                    // released to the MMA warps, then the fold runs from registers
+                    // the first 32 columns are folded while the second 32 are loaded; the
+                    // buffer goes back to the MMA warps once both loads are complete
                     static_assert(kCW == 64, "64 columns per epilogue thread");
                     uint32_t v[64];
                     tmem_ld32(taddr, v);
-                    tmem_ld32(taddr + 32, v + 32);
                     tmem_ld_wait();
+                    tmem_ld32(taddr + 32, v + 32);
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) tmem_st16_const(taddr + c * 16, kMagicBits);
-                    tmem_st_wait();
+                    for (int i = 0; i < 32; i += 2) fold2_packed(acc2[i / 2], sc2, m2, v[i], v[i + 1]);
+                    tmem_ld_wait();
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(DEMPTY_BAR(b));
 #pragma unroll
-                    for (int i = 0; i < 64; i += 2) fold2_packed(acc2[i / 2], sc2, m2, v[i], v[i + 1]);
+                    for (int i = 32; i < 64; i += 2) fold2_packed(acc2[i / 2], sc2, m2, v[i], v[i + 1]);
                 } else {
                     // the INT32-partials output: batches of 16 columns (no spill)
 #pragma unroll
@@ -434,7 +463,6 @@ __global__ void __launch_bounds__(C::kThreads, 1) gemm_w4a8_kernel(const GemmArg
                         uint32_t v[16];
                         tmem_ld16(taddr + rd * 16, v);
                         tmem_ld_wait();
-                        tmem_st16_const(taddr + rd * 16, kMagicBits);
                         if (n_out < a.nvalid) {
                             int32_t* pp = a.partials + ((size_t)(it.row0 + m0) * a.nvalid + n_out) * G + g;
                             const size_t pstride = (size_t)a.nvalid * G;
@@ -445,7 +473,6 @@ __global__ void __launch_bounds__(C::kThreads, 1) gemm_w4a8_kernel(const GemmArg
 #pragma unroll
                         for (int i = 0; i < 16; i += 2) fold2_packed(acc2[(rd * 16 + i) / 2], sc2, m2, v[i], v[i + 1]);
                     }
-                    tmem_st_wait();
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(DEMPTY_BAR(b));
@@ -457,7 +484,60 @@ __global__ void __launch_bounds__(C::kThreads, 1) gemm_w4a8_kernel(const GemmArg
             for (int i = 0; i < kCW; i += 2) unpack2(acc2[i / 2], acc[i], acc[i + 1]);
             const float* sap = a.act_scale + it.row0 + col0;
             const int ncol = it.nrows - col0;
-            if (a.mode != 1) {
+            if (staged) {
+                // 1. this thread's previous copy has read the staging tile; publish the token
+                //    scales; all epilogue warps agree (bounded waits: an abort ends the loop)
+                if (issued) bulk_wait_read_all();
+                if (eh == 0) sa_s[r] = my_sa;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(STAGE_BAR(0));
+                if (!wait_bar(STAGE_BAR(0), ntile & 1u, abort_flag, a.err, a.wait_limit)) { ok = false; break; }
+                // 2. scaled (and SwiGLU-combined) results into the staging tile
+                if (a.mode != 1) {
+#pragma unroll
+                    for (int i = 0; i < kCW; i += 4) {
+                        const float4 s4 = *reinterpret_cast<const float4*>(sa_s + col0 + i);
+                        stage[(col0 + i) * kTileRows + r] = acc[i] * s4.x;
+                        stage[(col0 + i + 1) * kTileRows + r] = acc[i + 1] * s4.y;
+                        stage[(col0 + i + 2) * kTileRows + r] = acc[i + 2] * s4.z;
+                        stage[(col0 + i + 3) * kTileRows + r] = acc[i + 3] * s4.w;
+                    }
+                } else {
+                    // even tile rows hold gate channel f, odd rows the matching up channel;
+                    // per token pair (i, i+1) the lanes of a pair swap one value: the even
+                    // lane finishes token i, the odd lane token i+1
+                    const int odd = r & 1;
+                    float* srow = stage + (col0 + odd) * C::kStageH + (r >> 1);
+#pragma unroll
+                    for (int i = 0; i < kCW; i += 2) {
+                        const float send = odd ? acc[i] : acc[i + 1];
+                        const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
+                        const float si = sa_s[col0 + i + odd];
+                        const float g = (odd ? recv : acc[i]) * si;
+                        const float uu = (odd ? acc[i + 1] : recv) * si;
+                        srow[i * C::kStageH] = silu_mul(g, uu);
+                    }
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(STAGE_BAR(1));
+                if (!wait_bar(STAGE_BAR(1), ntile & 1u, abort_flag, a.err, a.wait_limit)) { ok = false; break; }
+                // 3. one bulk copy per token row of the tile, each by its own thread
+                if (et < it.nrows) {
+                    if (a.mode != 1) {
+                        const int n0 = it.nt * kTileRows;
+                        const int w = min(kTileRows, a.nvalid - n0);
+                        bulk_s2g(a.out + (size_t)(it.row0 + et) * a.ldo + n0,
+                                 smem_u32(stage + et * kTileRows), (uint32_t)w * 4u);
+                    } else {
+                        // all 64 channels: past F they land in the row's padding
+                        bulk_s2g(a.out + (size_t)(it.row0 + et) * a.ldo + it.nt * (kTileRows / 2),
+                                 smem_u32(stage + et * C::kStageH), (kTileRows / 2) * 4u);
+                    }
+                    bulk_commit();
+                    issued = true;
+                }
+            } else if (a.mode != 1) {
                 // token scales in halves of 32, all loads of a half before its stores (the
                 // compiler may not move a load across a store it cannot prove disjoint)
                 const bool valid = n_out < a.nvalid;
@@ -497,6 +577,7 @@ __global__ void __launch_bounds__(C::kThreads, 1) gemm_w4a8_kernel(const GemmArg
                 }
             }
         }
+        if (issued) bulk_wait_all();  // the output is complete before the CTA exits
     }
 
     __syncthreads();
@@ -514,8 +595,9 @@ __global__ void __launch_bounds__(C::kThreads, 1) gemm_w4a8_kernel(const GemmArg
 #undef DEMPTY_BAR
 #undef SCFULL_BAR
 #undef FINAL_BAR
+#undef STAGE_BAR
 
-using CfgLarge = Cfg<128, 8, 4, 3, 2, 1>;  // many tokens per expert
+using CfgLarge = Cfg<128, 6, 4, 3, 2, 1>;  // many tokens per expert
 
 template <class C, bool kPartials>
 cudaError_t launch_cfg(const GemmArgs& a, int num_ctas, cudaStream_t stream) {

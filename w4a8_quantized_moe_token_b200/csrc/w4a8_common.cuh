@@ -100,6 +100,33 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity, uin
     return ok != 0;
 }
 
+// Non-blocking test of an mbarrier phase (acquire semantics when it reports completion).
+// The result arrives with a latency of a few hundred cycles, so the pipelines test the
+// barrier of their next step early, while they work on the current one, and only fall
+// back to a blocking wait when that test found the phase incomplete.
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.b32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// one thread of the (converged) warp, the same one every time
+__device__ __forceinline__ bool elect_one() {
+    uint32_t pred = 0;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "elect.sync _|p, 0xffffffff;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(pred));
+    return pred != 0;
+}
+
 // 1-D bulk copy global -> shared (no tensor map, no multicast); completion is
 // reported to mbarrier `bar` as transaction bytes.  dst, src 16-B aligned, bytes % 16 == 0.
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
@@ -107,6 +134,22 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
         "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
         "l"(src), "r"(bytes), "r"(bar)
         : "memory");
+}
+
+// 1-D bulk copy shared -> global (no tensor map), tracked per issuing thread in a
+// bulk group.  dst, src 16-B aligned, bytes % 16 == 0.
+__device__ __forceinline__ void bulk_s2g(void* dst, uint32_t src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(src), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// wait until this thread's committed bulk copies have finished reading shared memory
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// wait until this thread's committed bulk copies are complete
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// make this thread's generic-proxy shared-memory writes visible to the async proxy
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 // ---- tcgen05 (5th-generation tensor core, tensor memory) ----
@@ -140,6 +183,65 @@ __device__ __forceinline__ void mma_i8_ts(uint32_t d_tmem, uint32_t a_tmem, uint
         "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
         "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T, bf16 x bf16 -> f32; M = 128, N from idesc, K = 16
+__device__ __forceinline__ void mma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Instruction descriptor for kind::f16 with bf16 A and B and an f32 D (bits 4-5 = 1,
+// bits 7-9 = 1, bits 10-12 = 1), both K-major, N >> 3 at bits 17-22, M >> 4 at 24-28.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// Shared-memory matrix descriptor without swizzling: 8-row x 16-byte core matrices,
+// `lbo` bytes apart along K and `sbo` bytes apart along M / N, descriptor version 1.
+__device__ __forceinline__ uint64_t smem_desc_noswz(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1u << 46;
+    return d;
+}
+
+// Accumulator reset by the tensor core.  The W4A8 GEMMs keep every INT32 accumulator
+// at the bit pattern 0x4B400000 (the fp32 value 1.5 * 2^23) before a K group's INT8
+// MMAs add the partial P on top, so that the bits read back as fp32 are exactly
+// 1.5 * 2^23 + P.  One bf16 MMA with accumulate = 0 writes that pattern into a whole
+// accumulator: A is all ones, B holds 1.5 * 2^19 everywhere, and the K = 16 products sum
+// to 16 * 1.5 * 2^19 = 1.5 * 2^23 exactly (every partial sum is a multiple of 1.5 * 2^19
+// below 2^24).  Both operands are uniform tiles, so the result does not depend on how
+// the descriptor's strides walk them; kResetTileBytes of each cover every address a
+// 128 x 16 operand with 128-byte strides can reach.
+constexpr int kResetTileBytes = 2304;
+constexpr uint32_t kResetOneBits = 0x3F80u;   // bf16 1.0
+constexpr uint32_t kResetBBits = 0x4940u;     // bf16 1.5 * 2^19
+constexpr uint32_t kResetStride = 128u;
+
+// fill the two reset operand tiles (A at `a`, B at `a + kResetTileBytes`); every thread
+// of the block takes part, then the writes are made visible to the tensor core
+__device__ __forceinline__ void fill_reset_tiles(uint8_t* a) {
+    uint32_t* w = reinterpret_cast<uint32_t*>(a);
+    for (int i = threadIdx.x; i < 2 * kResetTileBytes / 4; i += blockDim.x) {
+        const uint32_t h = i < kResetTileBytes / 4 ? kResetOneBits : kResetBBits;
+        w[i] = h | (h << 16);
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// the reset MMA for an accumulator of n columns (n a multiple of 16, 16..256) at d_tmem
+__device__ __forceinline__ void mma_reset_acc(uint32_t d_tmem, uint32_t reset_smem, int n) {
+    mma_bf16_ss(d_tmem, smem_desc_noswz(reset_smem, kResetStride, kResetStride),
+                smem_desc_noswz(reset_smem + kResetTileBytes, kResetStride, kResetStride), idesc_bf16(128, n), 0u);
 }
 
 // Instruction descriptor for kind::i8: D = s32 (bits 4-5 = 2), A = s8 or u8 (bits 7-9),
@@ -200,6 +302,26 @@ __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.
 
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// Named barrier over `nthreads` threads (whole warps) that also ORs a predicate across
+// them: every participant gets the same result.  A group of warps uses it to follow
+// one leader warp that did the group's mbarrier waits: mbarrier waits are costly (each
+// warp-level wait occupies the SM's barrier unit for tens of cycles, even on a phase
+// that has completed), a named barrier is not.  The leader passes "my wait failed"
+// as the predicate, so the whole group leaves together and no warp is left waiting
+// at a barrier that the others skipped.
+__device__ __forceinline__ bool named_bar_or(int id, int nthreads, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 q, %3, 0;\n\t"
+        "bar.red.or.pred p, %1, %2, q;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(r)
+        : "r"(id), "r"(nthreads), "r"((uint32_t)pred)
+        : "memory");
+    return r != 0;
 }
 
 // ---------------------------------------------------------------------------
