@@ -66,7 +66,9 @@ def packed_matrix_bytes(N, K):
     return N * Kp // 2 + N * (Kp // 128) * 4
 
 
-def moe_accounting(W, ids):
+def moe_accounting(W, ids, w4a16=False):
+    """Algorithmic ops and bytes per kernel kind.  w4a16: the comparison layer, whose
+    token rows (x and h) are bf16, 2 bytes per value, and which has no requant pass."""
     T, k, H, F = W.T, W.topk, W.H, W.F
     touched = int(np.unique(ids).size)
     slots = T * k
@@ -77,6 +79,17 @@ def moe_accounting(W, ids):
         "gemm_up": 2.0 * slots * 2 * F * H,
         "gemm_down": 2.0 * slots * H * F,
     }
+    if w4a16:
+        k_bytes = {
+            "perm": slots * 4 * 3.0,
+            "act_quant": T * H * 2.0 + slots * Hp * 2.0,
+            "gemm_up": up_w + slots * Hp * 2.0 + slots * F * 2.0,
+            "gemm_down": dn_w + slots * Fp * 2.0 + slots * H * 4.0,
+            "combine": slots * H * 4.0 + T * H * 2.0 + slots * 8,
+            "route": T * W.E * 2.0 + slots * 8,
+        }
+        return {"touched_experts": touched, "weight_bytes": up_w + dn_w, "ops": k_ops["gemm_up"] + k_ops["gemm_down"],
+                "kernel_ops": k_ops, "kernel_bytes": k_bytes}
     k_bytes = {
         "perm": slots * 4 * 3.0,
         "act_quant": T * H * 2.0 + slots * Hp + slots * 4,
@@ -231,8 +244,12 @@ def pack_experts(B, torch, W, seed, device):
 
 
 class MoeStep:
-    def __init__(self, B, torch, W, seed, device, packed=None):
+    """One forward of the MoE layer through w4a8_moe_forward (or, with w4a16=True,
+    through the W4A16 comparison layer w4a16_moe_forward on the same packed weights)."""
+
+    def __init__(self, B, torch, W, seed, device, packed=None, w4a16=False):
         self.B, self.torch, self.W, self.device = B, torch, W, device
+        self.w4a16 = w4a16
         inp = synth.moe_inputs(W, seed)
         self.x_host = inp["x"]
         T, E, k, H, F = W.T, W.E, W.topk, W.H, W.F
@@ -253,14 +270,16 @@ class MoeStep:
         self.logits_host = inp.get("logits")
         self.packed_up, self.packed_down = packed if packed is not None else pack_experts(B, torch, W, seed, device)
         self.out = torch.empty((T, H), dtype=torch.bfloat16, device=device)
-        self.ws = B.empty_aligned(B.w4a8_moe_workspace_bytes(T, E, k, H, F), device)
-        self.acct = moe_accounting(W, self.ids_host)
+        wsb = B.w4a16_moe_workspace_bytes if w4a16 else B.w4a8_moe_workspace_bytes
+        self.ws = B.empty_aligned(wsb(T, E, k, H, F), device)
+        self.acct = moe_accounting(W, self.ids_host, w4a16)
 
     def __call__(self):
         B, W = self.B, self.W
         if self.logits is not None:
             B.w4a8_route_topk(self.logits, W.topk, self.ids, self.w)
-        B.w4a8_moe_forward(self.packed_up, self.packed_down, W.E, W.H, W.F, self.x, self.ids, self.w, self.out,
+        fwd = B.w4a16_moe_forward if self.w4a16 else B.w4a8_moe_forward
+        fwd(self.packed_up, self.packed_down, W.E, W.H, W.F, self.x, self.ids, self.w, self.out,
                            self.ws)
 
     def e2e(self, steps, warmup):
@@ -830,6 +849,17 @@ def main(argv=None):
         "int8_peak": i8,
     }
 
+    # decode-shaped layers: the pages' comparison point, the same layer with W4A16
+    # experts (bf16 activations, same packed weights and routing)
+    if W.kind == "moe" and W.name != "prefill":
+        s16 = MoeStep(B, torch, W, args.seed, device, packed=(step.packed_up, step.packed_down), w4a16=True)
+        ms16, prof16, cl16 = time_steps(s16, B, torch, device, world, args.steps, args.warmup)
+        w16 = moe_summary(W, s16, ms16, prof16, cl16, args.steps, peaks, world)
+        line["w4a16"] = {k: w16[k] for k in ("value", "unit", "ms_per_step", "weight_gbs", "roofline", "kernels",
+                                             "gpu_launches", "clocks")}
+        line["w4a8_over_w4a16"] = summ["value"] / w16["value"]
+        del s16
+
     # the HBM-bound decode layers, timed in the same run (one GPU only)
     if world == 1 and not args.no_extra and W.name == "prefill":
         extra = {}
@@ -844,8 +874,16 @@ def main(argv=None):
             ex["e2e"] = {"value": Wx.T / (e2x / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2x,
                          "d2h_bytes_per_step": d2x}
             ex["config"] = config_of(Wx, "flushed before every timed step (256 MiB write, outside the timed span)")
+            # the pages' comparison point: the same layer with W4A16 experts (bf16
+            # activations, same packed weights and routing)
+            s16 = MoeStep(B, torch, Wx, args.seed, device, packed=(sx.packed_up, sx.packed_down), w4a16=True)
+            ms16, prof16, cl16 = time_steps(s16, B, torch, device, world, args.steps, args.warmup)
+            w16 = moe_summary(Wx, s16, ms16, prof16, cl16, args.steps, peaks, world)
+            ex["w4a16"] = {k: w16[k] for k in ("value", "unit", "ms_per_step", "weight_gbs", "roofline", "kernels",
+                                               "gpu_launches", "clocks")}
+            ex["w4a8_over_w4a16"] = ex["value"] / w16["value"]
             extra[name] = ex
-            del sx
+            del sx, s16
             torch.cuda.empty_cache()
         line["extra"] = extra
 

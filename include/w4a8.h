@@ -219,6 +219,36 @@ int w4a8_gemm_noalloc(const int8_t* qa, const float* sa, int M, const void* pack
  * which clears it. */
 int w4a8_gemm_noalloc_last_error(void* stream);
 
+/* ---- W4A16: the comparison point of the pages ----
+ * The same packed INT4 weights multiplied with 16-bit (bf16) activations that are
+ * never quantised: y[m][n] = sum_k x[m][k] * (code[n][k] - zp[n][g(k)]) * scale[n][g(k)].
+ * «Kimi 2.7 Moe 从 4 bit 存储到 INT8 拆解» (pptc.cn), section 1 (W4A16 keeps 16-bit
+ * activations; W4A8 decodes 20-40% faster) and section 3.3 (the W4A16 / W4A8 / W8A8
+ * table); the Kimi 2.7T MoE W4A8 article (hotelren.com 5173946), section 3.2 (W4A8
+ * over W4A16 on H100) and section 4.4.  Computed on the tensor core as bf16
+ * (code - zp) x bf16 x with one fp32 partial per 128-wide K group (every product is
+ * exact; the partial's sum is fp32), then acc += scale * partial in fp32.  The
+ * kernel uses 16-token tiles (the decode-shaped path): it is meant for decode-sized
+ * layers, where both schemes stream the same weight bytes.
+ *
+ * w4a16_gemm: x device bf16 [M][K] row-major (2-byte aligned), packed from
+ *   w4a8_pack_weights(1, N, K, W4A8_LAYOUT_PLAIN), y device float [M][N]; scratch
+ *   in ws (w4a16_gemm_workspace_bytes).  Error returns as w4a8_gemm. */
+size_t w4a16_gemm_workspace_bytes(int M, int N, int K);
+int w4a16_gemm(const void* x_bf16, int M, const void* packed, int N, int K, float* y, void* ws,
+               size_t ws_bytes, void* stream);
+
+/* w4a16_moe_forward: the MoE expert FFN with W4A16 experts, with the arguments and
+ * the routing, permutation and combine of w4a8_moe_forward: each token's bf16 row
+ * goes to its k experts, up GEMM (gate|up) -> SwiGLU -> h rounded to bf16 (the
+ * activations between the projections stay 16-bit) -> down GEMM -> weighted combine
+ * -> bf16.  Workspace from w4a16_moe_workspace_bytes; stages readable with
+ * w4a8_debug_dump(what | W4A8_DUMP_W4A16). */
+size_t w4a16_moe_workspace_bytes(int T, int E, int k, int H, int F);
+int w4a16_moe_forward(const void* packed_up, const void* packed_down, int E, int H, int F,
+                      const void* x_bf16, int T, const int32_t* ids, const float* w, int k,
+                      void* out_bf16, void* ws, size_t ws_bytes, void* stream);
+
 /* Intermediate results kept in a w4a8_moe_forward workspace, for stage tests. */
 enum {
     W4A8_DUMP_COUNTS = 0, /* int32 [E]      tokens routed to each expert             */
@@ -232,7 +262,13 @@ enum {
     W4A8_DUMP_ACT2 = 8,   /* int8, R x Fp: requantised h (tiled, see below)           */
     W4A8_DUMP_S2 = 9,     /* float [R]      scale of the requantised h rows           */
     W4A8_DUMP_Y2 = 10,    /* float [R][H]   down-projection output per padded row     */
-    W4A8_DUMP_ERR = 11    /* uint32 [1]     device error word                         */
+    W4A8_DUMP_ERR = 11,   /* uint32 [1]     device error word                         */
+    /* OR-ed into `what`: the region of a w4a16_moe_forward workspace.  There ACT1 holds
+     * the bf16 x rows and ACT2 the bf16 h rows, both tiled as below with 16-row blocks
+     * and 256 bytes per row and K group ([R/16][Kp/128][2][16][128 bytes]: the two
+     * 64-column halves of a group one after the other, each swizzled like the INT8
+     * rows); S1, H and S2 are empty. */
+    W4A8_DUMP_W4A16 = 0x100
 };
 /* R = w4a8_moe_rows_capacity(T,E,k).  Tiled INT8 rows: rows are grouped in blocks of
  * RB = w4a8_moe_act_block_rows(T,E,k) rows (16 for decode-shaped layers, whose mean

@@ -100,3 +100,38 @@ def untile_act(buf: np.ndarray, R: int, Kp: int, RB: int | None = None) -> np.nd
         for g in range(G):
             out.reshape(R // RB, RB, Kp)[:, :, g * 128 + c * 16:g * 128 + (c + 1) * 16] = p[:, g, i, phys]
     return out
+
+
+def untile_act16(buf: np.ndarray, R: int, Kp: int, RB: int = 16) -> np.ndarray:
+    """Tiled bf16 rows [R/RB][Kp/128][2][RB][128 bytes] (the two 64-column halves of a
+    K group one after the other, 16-byte chunk c of row i at chunk position c ^ (i & 7))
+    -> uint16 bf16 bits [R][Kp]."""
+    G = Kp // 128
+    p = np.asarray(buf, dtype=np.uint8)[:R * G * 256].reshape(R // RB, G, 2, RB, 8, 16)
+    out = np.zeros((R // RB, RB, Kp * 2), dtype=np.uint8)
+    i = np.arange(RB)
+    for g in range(G):
+        for hh in range(2):
+            for c in range(8):
+                b0 = g * 256 + hh * 128 + c * 16
+                out[:, :, b0:b0 + 16] = p[:, g, hh, i, c ^ (i & 7)]
+    return out.reshape(R, Kp * 2).view(np.uint16)
+
+
+def w4a16_error_bound(x, codes, scale, zp) -> np.ndarray:
+    """Largest error of the fp32 W4A16 GEMM against the exact result, per output.
+
+    Every product x * (code - zp) is exact in fp32 (8-bit by 5-bit significands), a
+    group's 128 products are summed in fp32 (at most 127 additions), the partial is
+    scaled (one rounding) and the G scaled partials are added (G roundings); with at
+    most 2^-23 relative error per operation (a truncating adder included) the error
+    is below (127 + G + 1) * 2^-23 * sum_k |x_k| * |w_k|."""
+    x = np.abs(np.asarray(x, dtype=np.float64))
+    G = scale.shape[1]
+    group = codes.shape[1] // G
+    Kp = codes.shape[1]
+    if x.shape[1] < Kp:
+        x = np.pad(x, ((0, 0), (0, Kp - x.shape[1])))
+    wabs = np.abs(codes.astype(np.float64) - np.repeat(zp.astype(np.float64), group, axis=1)) * \
+        np.repeat(scale.astype(np.float64), group, axis=1)
+    return (group - 1 + G + 1) * 2.0 ** -23 * (x @ wabs.T)

@@ -18,7 +18,7 @@ EINVAL, EALIGN, ENOSPACE, EUNSUPPORTED = -1, -2, -3, -5
 def header_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(w4a8_\w+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(w4a(?:8|16)_\w+)\s*\(", text)))
 
 
 @pytest.fixture(scope="module")
@@ -132,3 +132,28 @@ def test_logits_host_forward_validates_on_the_host(lib):
     # invalid shapes and a missing workspace are refused before any CUDA call
     assert lib.w4a8_moe_forward_logits_host(None, None, 0, 256, 128, None, 4, None, 2, None, None, 0, None) == EINVAL
     assert lib.w4a8_moe_forward_logits_host(None, None, 8, 256, 128, None, 4, None, 2, None, None, 0, None) == EINVAL
+
+
+def test_w4a16_workspaces_and_validation(lib):
+    T, E, k, H, F = 64, 64, 6, 4096, 1408
+    R = lib.w4a8_moe_rows_capacity(T, E, k)
+    total = lib.w4a16_moe_workspace_bytes(T, E, k, H, F)
+    regions = {}
+    for what in range(12):
+        off, nb = B.w4a8_debug_region(T, E, k, H, F, what | B.W4A8_DUMP_W4A16)
+        assert off % 256 == 0 and off + nb <= total
+        regions[what] = (off, nb)
+    # bf16 token rows: 256 bytes per row and K group; no INT8 scales, no fp32 h
+    assert regions[B.DUMP["act1"]][1] == (4096 // 128) * R * 256
+    assert regions[B.DUMP["act2"]][1] == 11 * R * 256  # Fp = 1408 -> 11 groups
+    assert regions[B.DUMP["s1"]][1] == regions[B.DUMP["h"]][1] == regions[B.DUMP["s2"]][1] == 0
+    assert regions[B.DUMP["y2"]][1] == R * H * 4
+    assert lib.w4a16_moe_workspace_bytes(T, E, 40, H, F) == 0  # k > 32
+    assert lib.w4a16_gemm_workspace_bytes(16, 256, 512) >= 4 * 16 * 256
+    assert lib.w4a16_gemm_workspace_bytes(-1, 256, 512) == 0
+    vp = ctypes.c_void_p
+    fake = vp(1 << 20)
+    assert lib.w4a16_gemm(fake, 4, fake, 256, 512, fake, fake, 8, None) == ENOSPACE
+    assert lib.w4a16_gemm(fake, 4, vp((1 << 20) + 16), 256, 512, fake, fake, 1 << 40, None) == EALIGN
+    assert lib.w4a16_moe_forward(fake, fake, 8, 256, 128, fake, 4, fake, fake, 2, fake, fake, 16, None) == ENOSPACE
+    assert lib.w4a16_moe_forward(fake, fake, 8, 256, 128, fake, 4, fake, fake, 9, fake, fake, 1 << 40, None) == EINVAL

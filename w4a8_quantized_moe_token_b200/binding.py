@@ -25,6 +25,7 @@ DUMP = {
     "counts": 0, "offs": 1, "perm": 2, "inv": 3, "poffs": 4, "act1": 5, "s1": 6,
     "h": 7, "act2": 8, "s2": 9, "y2": 10, "err": 11,
 }
+W4A8_DUMP_W4A16 = 0x100  # OR into a dump id: the region of a w4a16_moe_forward workspace
 
 _c_int, _c_size, _vp = ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p
 _SIGS = {
@@ -51,6 +52,11 @@ _SIGS = {
     "w4a8_gemm_noalloc_last_error": ([_vp], _c_int),
     "w4a8_moe_forward_logits_host": ([_vp, _vp, _c_int, _c_int, _c_int, _vp, _c_int, _vp, _c_int, _vp, _vp,
                                       _c_size, _vp], _c_int),
+    "w4a16_gemm_workspace_bytes": ([_c_int] * 3, _c_size),
+    "w4a16_gemm": ([_vp, _c_int, _vp, _c_int, _c_int, _vp, _vp, _c_size, _vp], _c_int),
+    "w4a16_moe_workspace_bytes": ([_c_int] * 5, _c_size),
+    "w4a16_moe_forward": ([_vp, _vp, _c_int, _c_int, _c_int, _vp, _c_int, _vp, _vp, _c_int, _vp, _vp, _c_size, _vp],
+                          _c_int),
     "w4a8_debug_inject": ([ctypes.c_uint, ctypes.c_longlong], _c_int),
     "w4a8_debug_region": ([_c_int] * 6 + [ctypes.POINTER(_c_size), ctypes.POINTER(_c_size)], _c_int),
     "w4a8_debug_dump": ([_vp] + [_c_int] * 6 + [_vp, _c_size, _vp], _c_int),
@@ -232,6 +238,26 @@ def w4a8_moe_forward(packed_up, packed_down, E, H, F, x, ids, w, out, ws):
                                   _ptr(out), _ptr(ws), ws.numel(), _stream()), "w4a8_moe_forward")
 
 
+def w4a16_moe_workspace_bytes(T, E, k, H, F) -> int:
+    return lib().w4a16_moe_workspace_bytes(T, E, k, H, F)
+
+
+def w4a16_moe_forward(packed_up, packed_down, E, H, F, x, ids, w, out, ws):
+    """The W4A16 comparison layer: same arguments as w4a8_moe_forward, bf16 token rows
+    into both projections; ws sized by w4a16_moe_workspace_bytes."""
+    _dev(x, torch.bfloat16, "x")
+    _dev(ids, torch.int32, "ids")
+    _dev(w, torch.float32, "w")
+    _dev(out, torch.bfloat16, "out")
+    _moe_buffers(packed_up, packed_down, E, H, F, ws)
+    T, k = ids.shape
+    _need(tuple(x.shape) == (T, H), f"x must be [T={T}][H={H}], got {tuple(x.shape)}")
+    _need(tuple(w.shape) == (T, k), f"w must be [T={T}][k={k}], got {tuple(w.shape)}")
+    _need(tuple(out.shape) == (T, H), f"out must be [T={T}][H={H}], got {tuple(out.shape)}")
+    _check(lib().w4a16_moe_forward(_ptr(packed_up), _ptr(packed_down), E, H, F, _ptr(x), T, _ptr(ids), _ptr(w), k,
+                                   _ptr(out), _ptr(ws), ws.numel(), _stream()), "w4a16_moe_forward")
+
+
 def w4a8_moe_forward_host(packed_up, packed_down, E, H, F, x, ids, w, out, ws):
     """Same as w4a8_moe_forward with x / ids / w / out in (pinned) HOST memory."""
     for t, nm in ((x, "x"), (ids, "ids"), (w, "w"), (out, "out")):
@@ -310,6 +336,24 @@ def w4a8_gemm_noalloc_last_error() -> int:
     if r < 0:
         _check(r, "w4a8_gemm_noalloc_last_error")
     return r
+
+
+def w4a16_gemm_workspace_bytes(M, N, K) -> int:
+    return lib().w4a16_gemm_workspace_bytes(M, N, K)
+
+
+def w4a16_gemm(x, packed, N, K, y, ws):
+    """x bf16 [M][K] (16-bit activations, not quantised), y float32 [M][N]."""
+    _dev(x, torch.bfloat16, "x")
+    _dev(y, torch.float32, "y")
+    _dev(packed, torch.uint8, "packed")
+    _dev(ws, torch.uint8, "ws")
+    _need(x.dim() == 2 and x.shape[1] == K, f"x must be [M][K={K}], got {tuple(x.shape)}")
+    M = x.shape[0]
+    _need(y.numel() >= M * N, f"y needs {M * N} elements, has {y.numel()}")
+    _need(packed.numel() >= w4a8_packed_bytes(1, N, K, W4A8_LAYOUT_PLAIN),
+          "packed is smaller than the packed weights of an N x K matrix")
+    _check(lib().w4a16_gemm(_ptr(x), M, _ptr(packed), N, K, _ptr(y), _ptr(ws), ws.numel(), _stream()), "w4a16_gemm")
 
 
 def w4a8_debug_inject(flags: int = 0, wait_limit_cycles: int = 0):

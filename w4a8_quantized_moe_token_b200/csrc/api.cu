@@ -57,7 +57,9 @@ struct MoeLayout {
     int nslots, nchunk, R, Hp, Fp, G1, G2;
 };
 
-bool moe_layout(int T, int E, int k, int H, int F, bool host_io, MoeLayout* L) {
+// w4a16: the W4A16 layer's workspace, in which ACT1 and ACT2 hold bf16 token rows
+// (act16_offset, 16-row blocks) and the INT8 scales and the fp32 h are absent
+bool moe_layout(int T, int E, int k, int H, int F, bool host_io, MoeLayout* L, bool w4a16 = false) {
     if (T < 0 || E < 1 || E > kMaxExperts || k < 1 || k > 32 || k > E || H < 1 || F < 1) return false;
     if ((long long)T * k >= (1ll << 31)) return false;
     L->nslots = T * k;
@@ -79,11 +81,12 @@ bool moe_layout(int T, int E, int k, int H, int F, bool host_io, MoeLayout* L) {
     b[R_PERM] = (size_t)L->nslots * 4;
     b[R_INV] = (size_t)L->nslots * 4;
     b[R_ROWSRC] = R * 4;
-    b[R_ACT1] = (size_t)L->G1 * R * 128;
-    b[R_S1] = R * 4;
-    b[R_H] = R * (size_t)L->Fp * 4;
-    b[R_ACT2] = (size_t)L->G2 * R * 128;
-    b[R_S2] = R * 4;
+    const size_t row_bytes = w4a16 ? 256 : 128;  // token row bytes per K group
+    b[R_ACT1] = (size_t)L->G1 * R * row_bytes;
+    b[R_S1] = w4a16 ? 0 : R * 4;
+    b[R_H] = w4a16 ? 0 : R * (size_t)L->Fp * 4;
+    b[R_ACT2] = (size_t)L->G2 * R * row_bytes;
+    b[R_S2] = w4a16 ? 0 : R * 4;
     b[R_Y2] = R * (size_t)H * 4;
     b[R_XIN] = host_io ? (size_t)T * H * 2 : 0;
     b[R_IDSIN] = host_io ? (size_t)L->nslots * 4 : 0;
@@ -250,9 +253,75 @@ int moe_forward_impl(const void* packed_up, const void* packed_down, int E, int 
     return W4A8_OK;
 }
 
+// The W4A16 comparison layer on the same packed weights: the same routing,
+// permutation and combine, 16-bit token rows into both projections (16-token tiles of
+// the decode-shaped kernel), h rounded to bf16 between them.
+int moe_forward_w4a16_impl(const void* packed_up, const void* packed_down, int E, int H, int F, const uint16_t* x,
+                           int T, const int32_t* ids, const float* w, int k, uint16_t* out, void* ws,
+                           const MoeLayout& L, cudaStream_t st) {
+    uint32_t* err = at<uint32_t>(ws, L, R_ERR);
+    W4A8_TRY(cudaMemsetAsync(err, 0, 16, st));
+    if (T == 0) return W4A8_OK;
+    int* mtstart = at<int>(ws, L, R_MTSTART);
+    int4* mt_tab = at<int4>(ws, L, R_MTTAB);
+    int* inv = at<int>(ws, L, R_INV);
+    float* y2 = at<float>(ws, L, R_Y2);
+    uint8_t* x16 = at<uint8_t>(ws, L, R_ACT1);
+    uint8_t* h16 = at<uint8_t>(ws, L, R_ACT2);
+    constexpr int tile = 16;
+    {
+        ProfScope p(W4A8_KERNEL_PERM, perm_launch_count(L.nslots), st);
+        W4A8_TRY(launch_perm(ids, L.nslots, E, tile, at<int>(ws, L, R_CHIST), L.nchunk, at<int>(ws, L, R_COUNTS),
+                             at<int>(ws, L, R_OFFS), at<int>(ws, L, R_POFFS), mtstart, mt_tab, at<int>(ws, L, R_PERM),
+                             inv, at<int>(ws, L, R_ROWSRC), err, st));
+    }
+    {
+        ProfScope p(W4A8_KERNEL_ACT_QUANT, 1, st);
+        W4A8_TRY(launch_act_gather_bf16(x, T, H, k, inv, x16, h16, F, st));
+    }
+    GemmArgs up{};
+    up.wblocks = static_cast<const uint8_t*>(packed_up) + kHeaderBytes;
+    up.NT = packed_tiles(2 * F, W4A8_LAYOUT_GATEUP);
+    up.G = L.G1;
+    up.act = reinterpret_cast<const int8_t*>(x16);
+    up.act_rb_stride = (size_t)L.G1 * tile * 256;
+    up.mt_tab = mt_tab;
+    up.n_mtiles = mtstart + E;
+    up.mode = 1;
+    up.nvalid = F;
+    up.out16 = h16;
+    up.out16_G = L.G2;
+    up.err = err;
+    apply_debug(up);
+    {
+        ProfScope p(W4A8_KERNEL_GEMM_UP, 1, st);
+        W4A8_TRY(launch_gemm_w4a16(up, sm_count(), st));
+    }
+    GemmArgs dn = up;
+    dn.wblocks = static_cast<const uint8_t*>(packed_down) + kHeaderBytes;
+    dn.NT = packed_tiles(H, W4A8_LAYOUT_PLAIN);
+    dn.G = L.G2;
+    dn.act = reinterpret_cast<const int8_t*>(h16);
+    dn.act_rb_stride = (size_t)L.G2 * tile * 256;
+    dn.mode = 2;
+    dn.out = y2;
+    dn.ldo = H;
+    dn.nvalid = H;
+    dn.out16 = nullptr;
+    {
+        ProfScope p(W4A8_KERNEL_GEMM_DOWN, 1, st);
+        W4A8_TRY(launch_gemm_w4a16(dn, sm_count(), st));
+    }
+    {
+        ProfScope p(W4A8_KERNEL_COMBINE, 1, st);
+        W4A8_TRY(launch_combine(y2, H, inv, w, T, k, out, st));
+    }
+    return W4A8_OK;
+}
+
 int check_moe_args(const void* packed_up, const void* packed_down, int E, int H, int F, int T, int k, void* ws,
-                   size_t ws_bytes, bool host_io, MoeLayout* L) {
-    if (!moe_layout(T, E, k, H, F, host_io, L)) {
+                   size_t ws_bytes, bool host_io, MoeLayout* L, bool w4a16 = false) {
+    if (!moe_layout(T, E, k, H, F, host_io, L, w4a16)) {
         if (E > kMaxExperts || k > 32) return W4A8_EUNSUPPORTED;
         return W4A8_EINVAL;
     }
@@ -406,6 +475,27 @@ W4A8_EXPORT int w4a8_moe_forward(const void* packed_up, const void* packed_down,
                             static_cast<uint16_t*>(out_bf16), ws, L, static_cast<cudaStream_t>(stream));
 }
 
+W4A8_EXPORT size_t w4a16_moe_workspace_bytes(int T, int E, int k, int H, int F) {
+    MoeLayout L;
+    if (!moe_layout(T, E, k, H, F, false, &L, true)) return 0;
+    return L.off[R_COUNT];
+}
+
+W4A8_EXPORT int w4a16_moe_forward(const void* packed_up, const void* packed_down, int E, int H, int F,
+                                  const void* x_bf16, int T, const int32_t* ids, const float* w, int k,
+                                  void* out_bf16, void* ws, size_t ws_bytes, void* stream) {
+    MoeLayout L;
+    const int st = check_moe_args(packed_up, packed_down, E, H, F, T, k, ws, ws_bytes, false, &L, true);
+    if (st != W4A8_OK) return st;
+    if (T > 0) {
+        if (x_bf16 == nullptr || ids == nullptr || w == nullptr || out_bf16 == nullptr) return W4A8_EINVAL;
+        if (!aligned(x_bf16, 16) || !aligned(ids, 16) || !aligned(w, 16) || !aligned(out_bf16, 16))
+            return W4A8_EALIGN;
+    }
+    return moe_forward_w4a16_impl(packed_up, packed_down, E, H, F, static_cast<const uint16_t*>(x_bf16), T, ids, w,
+                                  k, static_cast<uint16_t*>(out_bf16), ws, L, static_cast<cudaStream_t>(stream));
+}
+
 W4A8_EXPORT int w4a8_moe_forward_host(const void* packed_up, const void* packed_down, int E, int H, int F,
                                       const void* x_bf16_host, int T, const int32_t* ids_host, const float* w_host,
                                       int k, void* out_bf16_host, void* ws, size_t ws_bytes, void* stream) {
@@ -461,7 +551,7 @@ struct GemmLayout {
     size_t err, nmt, mttab, act, total;
     int Mp, G;
 };
-bool gemm_layout(int M, int N, int K, GemmLayout* L) {
+bool gemm_layout(int M, int N, int K, GemmLayout* L, bool bf16 = false) {
     if (M < 0 || N < 1 || K < 1) return false;
     L->Mp = round_up(M, kRowPad);
     L->G = ceil_div(K, kGroup);
@@ -469,7 +559,7 @@ bool gemm_layout(int M, int N, int K, GemmLayout* L) {
     L->err = o; o += align_up(16);
     L->nmt = o; o += align_up(4);
     L->mttab = o; o += align_up((size_t)(M / 16 + 2) * 16);
-    L->act = o; o += align_up((size_t)L->G * L->Mp * 128);
+    L->act = o; o += align_up((size_t)L->G * L->Mp * (bf16 ? 256 : 128));
     L->total = o;
     return true;
 }
@@ -525,9 +615,54 @@ W4A8_EXPORT int w4a8_gemm(const int8_t* qa, const float* sa, int M, const void* 
     return W4A8_OK;
 }
 
+W4A8_EXPORT size_t w4a16_gemm_workspace_bytes(int M, int N, int K) {
+    GemmLayout L;
+    if (!gemm_layout(M, N, K, &L, true)) return 0;
+    return L.total;
+}
+
+W4A8_EXPORT int w4a16_gemm(const void* x_bf16, int M, const void* packed, int N, int K, float* y, void* ws,
+                           size_t ws_bytes, void* stream) {
+    GemmLayout L;
+    if (!gemm_layout(M, N, K, &L, true)) return W4A8_EINVAL;
+    if (packed == nullptr || ws == nullptr) return W4A8_EINVAL;
+    if (!aligned(packed, kAlign) || !aligned(ws, kAlign)) return W4A8_EALIGN;
+    if (ws_bytes < L.total) return W4A8_ENOSPACE;
+    uint8_t* base = static_cast<uint8_t*>(ws);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint32_t* err = reinterpret_cast<uint32_t*>(base + L.err);
+    W4A8_TRY(cudaMemsetAsync(err, 0, 16, s));
+    if (M == 0) return W4A8_OK;
+    if (x_bf16 == nullptr || y == nullptr) return W4A8_EINVAL;
+    if (!aligned(x_bf16, 2) || !aligned(y, 4)) return W4A8_EALIGN;
+    int* n_mtiles = reinterpret_cast<int*>(base + L.nmt);
+    int4* mt_tab = reinterpret_cast<int4*>(base + L.mttab);
+    uint8_t* act = base + L.act;
+    ProfScope prof(W4A8_KERNEL_GEMM_DENSE, 2, s);
+    W4A8_TRY(launch_dense_prep_bf16(static_cast<const uint16_t*>(x_bf16), M, K, act, mt_tab, n_mtiles, s));
+    GemmArgs a{};
+    a.wblocks = static_cast<const uint8_t*>(packed) + kHeaderBytes;
+    a.NT = packed_tiles(N, W4A8_LAYOUT_PLAIN);
+    a.G = L.G;
+    a.act = reinterpret_cast<const int8_t*>(act);
+    a.act_rb_stride = (size_t)L.G * 16 * 256;
+    a.mt_tab = mt_tab;
+    a.n_mtiles = n_mtiles;
+    a.mode = 0;
+    a.out = y;
+    a.ldo = N;
+    a.nvalid = N;
+    a.err = err;
+    apply_debug(a);
+    W4A8_TRY(launch_gemm_w4a16(a, sm_count(), s));
+    return W4A8_OK;
+}
+
 W4A8_EXPORT int w4a8_debug_region(int T, int E, int k, int H, int F, int what, size_t* offset, size_t* bytes) {
     MoeLayout L;
-    if (!moe_layout(T, E, k, H, F, false, &L) || offset == nullptr || bytes == nullptr) return W4A8_EINVAL;
+    const bool w4a16 = (what & W4A8_DUMP_W4A16) != 0;
+    what &= ~W4A8_DUMP_W4A16;
+    if (!moe_layout(T, E, k, H, F, false, &L, w4a16) || offset == nullptr || bytes == nullptr) return W4A8_EINVAL;
     static const Region map[] = {R_COUNTS, R_OFFS, R_PERM, R_INV, R_POFFS, R_ACT1,
                                  R_S1,     R_H,    R_ACT2, R_S2,  R_Y2,    R_ERR};
     if (what < 0 || what >= (int)(sizeof(map) / sizeof(map[0]))) return W4A8_EINVAL;

@@ -45,26 +45,25 @@ namespace {
 constexpr uint32_t kMagicBits = 0x4B400000u;  // 1.5 * 2^23 (what the reset MMA writes)
 constexpr float kMagicF = 12582912.0f;
 
-constexpr int GPS = 4;    // K groups per pipeline step
+// Pipeline shape per operand kind.  W4A8: INT8 token rows (128 bytes per row and K
+// group), 4 groups per step.  W4A16: bf16 token rows (256 bytes per row and group);
+// a group's converted weights take 64 tensor-memory columns instead of 32, so a step
+// carries 2 groups and the rings are deeper (6 stages) to keep as many weight bytes
+// in flight.
+template <bool kBf16>
+struct DecCfg {
+    static constexpr int GPS = kBf16 ? 2 : 4;     // K groups per pipeline step
+    static constexpr int NS = kBf16 ? 6 : 4;      // shared-memory stages
+    static constexpr int NA = 2;                  // tensor-memory A slots
+    static constexpr int ND = NS;                 // tensor-memory accumulators (GPS x BN columns each)
+    static constexpr int NSC = kBf16 ? 8 : 6;     // scale ring slots (>= NA + ND)
+    static constexpr int kRowBytes = kBf16 ? 256 : 128;  // token row bytes per K group
+    static constexpr int kGCols = kBf16 ? 64 : 32;       // A columns per K group
+    static constexpr int kMmaK = kBf16 ? 16 : 32;        // K per MMA instruction
+};
+
 constexpr int BN = 16;    // tokens per tile (one 16-row block)
-constexpr int NS = 4;     // shared-memory stages
-constexpr int NA = 2;     // tensor-memory A slots (GPS x 32 columns each)
-constexpr int ND = 4;     // tensor-memory accumulators (GPS x BN columns each)
-constexpr int NSC = 6;    // scale ring slots (>= NA + ND)
-constexpr int kAStage = GPS * kBlockBytes;  // weight blocks of one step
-constexpr int kBStage = GPS * BN * 128;     // token rows of one step
-constexpr int kACols = GPS * 32;
-constexpr int kDCols = GPS * BN;
-constexpr uint32_t kACol0 = 0;
-constexpr uint32_t kDCol0 = NA * kACols;
 constexpr uint32_t kTmemCols = 512;
-static_assert(kDCol0 + ND * kDCols <= kTmemCols, "tensor memory over-subscribed");
-static_assert(NSC >= NA + ND, "scale ring too small");
-static_assert(NS % 2 == 0, "the two producers own the stages of one parity each");
-static_assert(GPS % 2 == 0, "the two MMA warps split the groups of a step");
-// one "MMA of step j done" barrier per j % NS serves the stage ring, the A slots and
-// the accumulators: their rings must step together
-static_assert(ND == NS && NS % NA == 0, "shared completion ring");
 
 // warps: 0-7 converters (2 groups), 8-15 epilogue (2 groups), 16 producer 0, 17-18 MMA,
 // 19 producer 1
@@ -74,21 +73,39 @@ constexpr int kRegLaunch = 96;  // 65536 / 640, rounded down to the allocation u
 constexpr int kRegConv = 88, kRegCtrl = 48, kRegEpi = 128;
 static_assert(128 * (2 * kRegConv + kRegCtrl + 2 * kRegEpi) <= kRegLaunch * kThreads, "register split");
 
-// shared memory carve-up (offsets from a 1024-aligned base)
-constexpr int kOffB = 0;
-constexpr int kOffA = kOffB + NS * kBStage;
-constexpr int kOffSc = kOffA + NS * kAStage;          // ring: fp32 scale       [NSC][GPS][128]
-constexpr int kOffZp = kOffSc + NSC * GPS * 128 * 4;  // ring: fp32 zero point  [NSC][GPS][128]
-constexpr int kOffS = kOffZp + NSC * GPS * 128 * 4;   // ring: token group sums [NSC][GPS][BN]
-constexpr int kOffX = kOffS + NSC * GPS * BN * 4;     // epilogue exchange: [2][128][BN] fp32
-constexpr int kOffReset = kOffX + 2 * 128 * BN * 4;   // the accumulator-reset operands
-constexpr int kOffBar = kOffReset + 2 * kResetTileBytes;
-// full[NS] empty[NS] conv[NA] (unused: NA + ND) dempty[ND] side[NSC] final[2]
-// xfull[2] xempty[2]
-constexpr int kNumBars = 2 * NS + 2 * NA + 2 * ND + NSC + 2 + 4;
-constexpr int kOffMisc = kOffBar + kNumBars * 8;
-constexpr int kSmemBytes = kOffMisc + 16 + 1024;
-static_assert(kSmemBytes <= 227 * 1024, "shared memory over-subscribed");
+template <bool kBf16>
+struct DecLayout {
+    using C = DecCfg<kBf16>;
+    static constexpr int GPS = C::GPS, NS = C::NS, NA = C::NA, ND = C::ND, NSC = C::NSC;
+    static constexpr int kAStage = GPS * kBlockBytes;        // weight blocks of one step
+    static constexpr int kBStage = GPS * BN * C::kRowBytes;  // token rows of one step
+    static constexpr int kACols = GPS * C::kGCols;
+    static constexpr int kDCols = GPS * BN;
+    static constexpr uint32_t kACol0 = 0;
+    static constexpr uint32_t kDCol0 = NA * kACols;
+    static_assert(kDCol0 + ND * kDCols <= kTmemCols, "tensor memory over-subscribed");
+    static_assert(NSC >= NA + ND, "scale ring too small");
+    static_assert(NS % 2 == 0, "the two producers own the stages of one parity each");
+    static_assert(GPS % 2 == 0, "the two MMA warps split the groups of a step");
+    // one "MMA of step j done" barrier per j % NS serves the stage ring, the A slots and
+    // the accumulators: their rings must step together
+    static_assert(ND == NS && NS % NA == 0, "shared completion ring");
+    // shared memory carve-up (offsets from a 1024-aligned base)
+    static constexpr int kOffB = 0;
+    static constexpr int kOffA = kOffB + NS * kBStage;
+    static constexpr int kOffSc = kOffA + NS * kAStage;          // ring: fp32 scale       [NSC][GPS][128]
+    static constexpr int kOffZp = kOffSc + NSC * GPS * 128 * 4;  // ring: fp32 zero point  [NSC][GPS][128]
+    static constexpr int kOffS = kOffZp + NSC * GPS * 128 * 4;   // ring: token group sums [NSC][GPS][BN]
+    static constexpr int kOffX = kOffS + NSC * GPS * BN * 4;     // epilogue exchange: [2][128][BN] fp32
+    static constexpr int kOffReset = kOffX + 2 * 128 * BN * 4;   // the accumulator-reset operands
+    static constexpr int kOffBar = kOffReset + 2 * kResetTileBytes;
+    // full[NS] empty[NS] conv[NA] (unused: NA + ND) dempty[ND] side[NSC] final[2]
+    // xfull[2] xempty[2]
+    static constexpr int kNumBars = 2 * NS + 2 * NA + 2 * ND + NSC + 2 + 4;
+    static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+    static constexpr int kSmemBytes = kOffMisc + 16 + 1024;
+    static_assert(kSmemBytes <= 227 * 1024, "shared memory over-subscribed");
+};
 
 #define FULL_BAR(s) (bar0 + 8u * (uint32_t)(s))
 #define EMPTY_BAR(s) (bar0 + 8u * (uint32_t)(NS + (s)))
@@ -154,6 +171,22 @@ __device__ __forceinline__ void fold2_packed_zp(uint64_t& acc2, uint64_t sc2, ui
         : "r"(x0), "r"(x1), "l"(m2), "l"(nzp2), "l"(s2), "l"(sc2));
 }
 
+// a packed pair of fp32 accumulators += sc * (d0, d1) (the W4A16 fold)
+__device__ __forceinline__ void fold2_f32(uint64_t& acc2, uint64_t sc2, uint32_t d0, uint32_t d1) {
+    asm("{\n\t.reg .b64 x;\n\t"
+        "mov.b64 x, {%1, %2};\n\t"
+        "fma.rn.f32x2 %0, %3, x, %0;\n\t}"
+        : "+l"(acc2)
+        : "r"(d0), "r"(d1), "l"(sc2));
+}
+
+// two bf16 values (128 + code) minus the packed offset nz2 = -(128 + zp): exact
+__device__ __forceinline__ uint32_t bf16x2_sub_offset(uint32_t v, uint32_t nz2) {
+    uint32_t r;
+    asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(v), "r"(0x3F803F80u), "r"(nz2));
+    return r;
+}
+
 __device__ __forceinline__ uint64_t pack2(float lo, float hi) {
     uint64_t r;
     asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
@@ -172,7 +205,15 @@ __device__ __forceinline__ void unpack2(uint64_t p, float& lo, float& hi) {
 
 __device__ __forceinline__ float silu_mul(float g, float u) { return __fdividef(g, 1.0f + __expf(-g)) * u; }
 
+template <bool kBf16>
 __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs a) {
+    using L = DecLayout<kBf16>;
+    constexpr int GPS = L::GPS, NS = L::NS, NA = L::NA, ND = L::ND, NSC = L::NSC;
+    constexpr int kAStage = L::kAStage, kBStage = L::kBStage, kACols = L::kACols, kDCols = L::kDCols;
+    constexpr uint32_t kACol0 = L::kACol0, kDCol0 = L::kDCol0;
+    constexpr int kRowBytes = DecCfg<kBf16>::kRowBytes, kGCols = DecCfg<kBf16>::kGCols;
+    constexpr int kOffA = L::kOffA, kOffB = L::kOffB, kOffSc = L::kOffSc, kOffZp = L::kOffZp, kOffS = L::kOffS;
+    constexpr int kOffX = L::kOffX, kOffReset = L::kOffReset, kOffBar = L::kOffBar, kOffMisc = L::kOffMisc;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
     const uint32_t base_addr = (raw_addr + 1023u) & ~1023u;
@@ -251,9 +292,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
                         rdy = mbar_test(EMPTY_BAR((j + 2) % NS), (((j + 2) / NS) & 1u) ^ 1u);
                         // test hook: leave the first step's stage empty, so that its consumers time out
                         if (j == 0 && blockIdx.x == 0 && (a.debug & kDebugSkipFirstCopy)) continue;
-                        mbar_arrive_expect_tx(FULL_BAR(s), (uint32_t)ng * (kBlockBytes + BN * 128));
+                        mbar_arrive_expect_tx(FULL_BAR(s), (uint32_t)ng * (kBlockBytes + BN * kRowBytes));
                         bulk_g2s(sA + s * kAStage, wsrc + (size_t)g0 * kBlockBytes, ng * kBlockBytes, FULL_BAR(s));
-                        bulk_g2s(sB + s * kBStage, bsrc + (size_t)g0 * BN * 128, ng * BN * 128, FULL_BAR(s));
+                        bulk_g2s(sB + s * kBStage, bsrc + (size_t)g0 * BN * kRowBytes, ng * BN * kRowBytes, FULL_BAR(s));
                     }
                 }
                 for (uint32_t qq = (last > (uint32_t)NS ? last - NS : 0u); qq < last; ++qq)
@@ -272,7 +313,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
             {
                 uint32_t j = 0;
                 bool ok = true, conv_rdy = false, acc_rdy = false;  // early tests of this step's barriers
-                const uint32_t idesc = idesc_i8(128, BN, false);  // u8 codes x s8 tokens
+                // u8 codes x s8 tokens, or bf16 (code - zp) x bf16 tokens
+                const uint32_t idesc = kBf16 ? idesc_bf16(128, BN) : idesc_i8(128, BN, false);
                 for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
                     for (int t = 0; t < steps_per_item; ++t, ++j) {
                         const int ng = min(GPS, G - t * GPS);
@@ -283,8 +325,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
                         acc_rdy = mbar_test(DEMPTY_BAR((j + 1) % ND), (((j + 1) / ND) & 1u) ^ 1u);
                         tc_fence_after();
                         if (elect_one()) {
-                        // reset this warp's groups' accumulators (32 columns), then add the partials
-                        if (mi * (GPS / 2) < ng)
+                        // W4A8: reset this warp's groups' INT32 accumulators to the magic
+                        // pattern, then add the partials.  W4A16: the first MMA of a group
+                        // overwrites its fp32 accumulator.
+                        if (!kBf16 && mi * (GPS / 2) < ng)
                             mma_reset_acc(tmem_base + kDCol0 + (uint32_t)(b * kDCols + mi * (GPS / 2) * BN), sReset,
                                           (GPS / 2) * BN);
 #pragma unroll
@@ -292,11 +336,21 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
                             const int gq = mi * (GPS / 2) + gh;
                             if (gq < ng) {
                                 const uint32_t dt = tmem_base + kDCol0 + (uint32_t)(b * kDCols + gq * BN);
-                                const uint32_t at = tmem_base + kACol0 + (uint32_t)(x * kACols + gq * 32);
-                                const uint32_t sb = sB + s * kBStage + gq * BN * 128;
+                                const uint32_t at = tmem_base + kACol0 + (uint32_t)(x * kACols + gq * kGCols);
+                                const uint32_t sb = sB + s * kBStage + gq * BN * kRowBytes;
+                                if constexpr (kBf16) {
+                                    // K = 16 per MMA: steps 0-3 in the group's first 64-column
+                                    // plane of token rows, 4-7 in the second
 #pragma unroll
-                                for (int kk = 0; kk < 4; ++kk)
-                                    mma_i8_ts(dt, at + kk * 8, smem_desc_sw128(sb + kk * 32), idesc, 1u);
+                                    for (int kk = 0; kk < 8; ++kk)
+                                        mma_bf16_ts(dt, at + kk * 8,
+                                                    smem_desc_sw128(sb + (kk >> 2) * BN * 128 + (kk & 3) * 32), idesc,
+                                                    kk > 0 ? 1u : 0u);
+                                } else {
+#pragma unroll
+                                    for (int kk = 0; kk < 4; ++kk)
+                                        mma_i8_ts(dt, at + kk * 8, smem_desc_sw128(sb + kk * 32), idesc, 1u);
+                                }
                             }
                         }
                         // one commit tells the producer (stage s free), the converters (A
@@ -340,6 +394,35 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
 #pragma unroll
                 for (int c = 0; c < 4; ++c) w[c] = *reinterpret_cast<const uint4*>(blk + code_chunk_offset(r, c));
                 sc_ring[(slot * GPS + gq) * 128 + r] = __half2float(reinterpret_cast<const __half*>(blk + kScaleOff)[r]);
+                if constexpr (kBf16) {
+                    // (code - zp) as bf16, exactly: the byte permute puts each code under
+                    // the bf16 bits 0x43, giving 128 + code, and one packed bf16 FMA
+                    // subtracts 128 + zp (the zero point is an integer 0..15); each 32-bit
+                    // tensor-memory column holds two consecutive K
+                    const int zi = __half2int_rn(reinterpret_cast<const __half*>(blk + kZpOff)[r]);
+                    const uint32_t nz2 = (0xC300u | (uint32_t)zi) * 0x10001u;  // -(128 + zp), twice
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {  // K 64hh .. 64hh + 63: chunks 2hh, 2hh + 1
+                        uint32_t v[32];
+#pragma unroll
+                        for (int cc = 0; cc < 2; ++cc) {
+                            const uint4 wc = w[2 * hh + cc];
+                            const uint32_t xw[4] = {wc.x, wc.y, wc.z, wc.w};
+#pragma unroll
+                            for (int qq = 0; qq < 4; ++qq) {
+                                const int i = 4 * cc + qq;  // K = 64hh + 8i .. 64hh + 8i + 7
+                                const uint32_t lo = xw[qq] & 0x0F0F0F0Fu;
+                                const uint32_t hi = __umulhi(xw[qq], m28) & 0x0F0F0F0Fu;
+                                v[4 * i] = bf16x2_sub_offset(__byte_perm(lo, 0x43434343u, 0x4140), nz2);
+                                v[4 * i + 1] = bf16x2_sub_offset(__byte_perm(lo, 0x43434343u, 0x4342), nz2);
+                                v[4 * i + 2] = bf16x2_sub_offset(__byte_perm(hi, 0x43434343u, 0x4140), nz2);
+                                v[4 * i + 3] = bf16x2_sub_offset(__byte_perm(hi, 0x43434343u, 0x4342), nz2);
+                            }
+                        }
+                        tmem_st32(tmem_base + lane_base + kACol0 + (uint32_t)(x * kACols + gq * kGCols + hh * 32), v);
+                    }
+                    continue;
+                }
                 zp_ring[(slot * GPS + gq) * 128 + r] = __half2float(reinterpret_cast<const __half*>(blk + kZpOff)[r]);
                 uint32_t v[32];
 #pragma unroll
@@ -354,10 +437,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
                 }
                 tmem_st32(tmem_base + lane_base + kACol0 + (uint32_t)(x * kACols + gq * 32), v);
             }
-            if (gs < ng) {
+            if (!kBf16 && gs < ng) {
                 // S[gs][m] = sum of token m's 128 INT8 codes of group gs (the swizzle only
                 // permutes the 16-byte chunks inside the row, so the row sum is unaffected)
-                const uint4* rowp = reinterpret_cast<const uint4*>(smB + s * kBStage + gs * BN * 128 + m * 128 + half * 64);
+                const uint4* rowp = reinterpret_cast<const uint4*>(smB + s * kBStage + gs * BN * kRowBytes + m * 128 + half * 64);
                 int sum = 0;
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
@@ -418,7 +501,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
 #pragma unroll
                 for (int gh = 0; gh < GPS / 2; ++gh) {
                     const int gq = eh * (GPS / 2) + gh;
-                    if (gq < ng) {
+                    if (kBf16 && gq < ng) {
+                        // fp32 partials: acc += scale * D
+                        const uint64_t sc2 = splat2(sc_ring[(slot * GPS + gq) * 128 + r]);
+#pragma unroll
+                        for (int i = 0; i < BN; i += 2) fold2_f32(acc2[i / 2], sc2, v[gh][i], v[gh][i + 1]);
+                    } else if (!kBf16 && gq < ng) {
                         const float zpf = zp_ring[(slot * GPS + gq) * 128 + r];
                         const uint64_t sc2 = splat2(sc_ring[(slot * GPS + gq) * 128 + r]);
                         const uint64_t nzp2 = splat2(-zpf);
@@ -474,7 +562,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
             const float* sap = a.act_scale + it.row0;
             float sa[BN];
 #pragma unroll
-            for (int i = 0; i < BN; ++i) sa[i] = i < it.nrows ? __ldg(sap + i) : 0.f;
+            for (int i = 0; i < BN; ++i) sa[i] = kBf16 ? 1.f : (i < it.nrows ? __ldg(sap + i) : 0.f);  // W4A16: no token scale
             if (a.mode != 1) {
                 const bool valid = n_out < a.nvalid;
                 float* op = a.out + (size_t)it.row0 * a.ldo + (valid ? n_out : 0);
@@ -500,8 +588,15 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
                     const float si = odd ? sa[i + 1] : sa[i];
                     const float g = (odd ? recv : acc[i]) * si;
                     const float u = (odd ? acc[i + 1] : recv) * si;
-                    if (valid && i + odd < it.nrows) *op = silu_mul(g, u);
-                    op += 2 * (size_t)a.ldo;
+                    if constexpr (kBf16) {
+                        // h rounded to bf16, straight into the down projection's token rows
+                        if (valid && i + odd < it.nrows)
+                            *reinterpret_cast<__nv_bfloat16*>(a.out16 + act16_offset(it.row0 + i + odd, f, a.out16_G, BN)) =
+                                __float2bfloat16_rn(silu_mul(g, u));
+                    } else {
+                        if (valid && i + odd < it.nrows) *op = silu_mul(g, u);
+                        op += 2 * (size_t)a.ldo;
+                    }
                 }
             }
         }
@@ -527,22 +622,35 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
 
 int gemm_decode_tile_tokens() { return BN; }
 
-cudaError_t launch_gemm_decode(const GemmArgs& a, int num_ctas, cudaStream_t stream) {
+namespace {
+template <bool kBf16>
+cudaError_t launch_decode(const GemmArgs& a, int num_ctas, cudaStream_t stream) {
+    constexpr int kSmem = DecLayout<kBf16>::kSmemBytes;
     static int attr_done[64] = {0};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64 || !attr_done[dev]) {
         // the register split assumes kRegLaunch registers per thread at launch
         cudaFuncAttributes fa;
-        cudaError_t e = cudaFuncGetAttributes(&fa, gemm_decode_kernel);
+        cudaError_t e = cudaFuncGetAttributes(&fa, gemm_decode_kernel<kBf16>);
         if (e != cudaSuccess) return e;
         if (fa.numRegs != kRegLaunch) return cudaErrorInvalidConfiguration;
-        e = cudaFuncSetAttribute(gemm_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+        e = cudaFuncSetAttribute(gemm_decode_kernel<kBf16>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
         if (e != cudaSuccess) return e;
         if (dev >= 0 && dev < 64) attr_done[dev] = 1;
     }
-    gemm_decode_kernel<<<num_ctas, kThreads, kSmemBytes, stream>>>(a);
+    gemm_decode_kernel<kBf16><<<num_ctas, kThreads, kSmem, stream>>>(a);
     return cudaGetLastError();
+}
+}  // namespace
+
+cudaError_t launch_gemm_decode(const GemmArgs& a, int num_ctas, cudaStream_t stream) {
+    return launch_decode<false>(a, num_ctas, stream);
+}
+
+cudaError_t launch_gemm_w4a16(const GemmArgs& a, int num_ctas, cudaStream_t stream) {
+    if (a.partials != nullptr || (a.mode == 1 && a.out16 == nullptr)) return cudaErrorInvalidValue;
+    return launch_decode<true>(a, num_ctas, stream);
 }
 
 }  // namespace w4a8

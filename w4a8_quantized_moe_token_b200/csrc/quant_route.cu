@@ -724,6 +724,70 @@ __global__ void __launch_bounds__(256) dense_prep_kernel(const int8_t* __restric
     *reinterpret_cast<uint4*>(act + act_offset(r, ci * 16, Kp / kGroup, RB)) = v;
 }
 
+// ---------------------------------------------------------------------------
+// W4A16 token rows: bf16 values copied (not quantised) into the tiled bf16 layout
+// of act16_offset, 16-row blocks, 8 values (16 bytes) per thread and step.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint4 load8_bf16(const uint16_t* row, int len, int k0) {
+    if ((len & 7) == 0 && k0 + 8 <= len) return *reinterpret_cast<const uint4*>(row + k0);
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t lo = k0 + 2 * i < len ? row[k0 + 2 * i] : 0u;
+        const uint32_t hi = k0 + 2 * i + 1 < len ? row[k0 + 2 * i + 1] : 0u;
+        w[i] = lo | (hi << 16);
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// CTA t copies token t's row to each of its k grouped rows (pad K columns zero) and
+// zeroes the pad columns [F, Fp) of the same rows of the h buffer, which the up
+// projection's epilogue leaves unwritten (chunks that straddle F are zeroed whole;
+// the epilogue writes their valid part afterwards, in stream order)
+__global__ void __launch_bounds__(128) act_gather_bf16_kernel(const uint16_t* __restrict__ x, int H, int k,
+                                                              const int* __restrict__ inv, uint8_t* __restrict__ x16,
+                                                              uint8_t* __restrict__ h16, int F) {
+    const int Hp = round_up(H, kGroup), G1 = Hp / kGroup;
+    const int Fp = round_up(F, kGroup), G2 = Fp / kGroup;
+    const int tok = blockIdx.x;
+    __shared__ int dst[32];
+    if ((int)threadIdx.x < k) dst[threadIdx.x] = __ldg(inv + (size_t)tok * k + threadIdx.x);
+    __syncthreads();
+    const uint16_t* row = x + (size_t)tok * H;
+    for (int ci = threadIdx.x; ci < Hp / 8; ci += blockDim.x) {
+        const uint4 v = load8_bf16(row, H, ci * 8);
+        for (int j = 0; j < k; ++j) {
+            const int r = dst[j];
+            if (r >= 0) *reinterpret_cast<uint4*>(x16 + act16_offset(r, ci * 8, G1, 16)) = v;
+        }
+    }
+    for (int ci = F / 8 + threadIdx.x; ci < Fp / 8; ci += blockDim.x) {
+        for (int j = 0; j < k; ++j) {
+            const int r = dst[j];
+            if (r >= 0) *reinterpret_cast<uint4*>(h16 + act16_offset(r, ci * 8, G2, 16)) = make_uint4(0u, 0u, 0u, 0u);
+        }
+    }
+}
+
+// dense W4A16 GEMM: x rows into the tiled bf16 layout (pad rows and columns zero),
+// described as one "expert" of 16-row tiles
+__global__ void __launch_bounds__(256) dense_prep_bf16_kernel(const uint16_t* __restrict__ x, int M, int K,
+                                                              uint8_t* __restrict__ act16, int4* mt_tab,
+                                                              int* n_mtiles) {
+    const int Kp = round_up(K, kGroup), G = Kp / kGroup;
+    const int Mp = round_up(M, kRowPad);
+    const int nch = Kp / 8;
+    const size_t idx = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int nmt = ceil_div(M, 16);
+    if (idx == 0) *n_mtiles = nmt;
+    if (idx < (size_t)nmt) mt_tab[idx] = make_int4(0, (int)idx * 16, min(16, M - (int)idx * 16), 0);
+    if (idx >= (size_t)Mp * nch) return;
+    const int r = (int)(idx / nch);
+    const int ci = (int)(idx % nch);
+    const uint4 v = r < M ? load8_bf16(x + (size_t)r * K, K, ci * 8) : make_uint4(0u, 0u, 0u, 0u);
+    *reinterpret_cast<uint4*>(act16 + act16_offset(r, ci * 8, G, 16)) = v;
+}
+
 }  // namespace
 
 // ------------------------------- launchers ---------------------------------
@@ -803,6 +867,20 @@ cudaError_t launch_dense_prep(const int8_t* qa, int M, int Kp, int tile_tokens, 
     const size_t n = (size_t)round_up(M, kRowPad) * (Kp / 16);
     dense_prep_kernel<<<(unsigned)((n + 255) / 256 + 1), 256, 0, stream>>>(qa, M, Kp, tile_tokens, rb, act, mt_tab,
                                                                           n_mtiles);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_dense_prep_bf16(const uint16_t* x, int M, int K, uint8_t* act16, int4* mt_tab, int* n_mtiles,
+                                   cudaStream_t stream) {
+    const size_t n = (size_t)round_up(M, kRowPad) * (round_up(K, kGroup) / 8);
+    dense_prep_bf16_kernel<<<(unsigned)((n + 255) / 256 + 1), 256, 0, stream>>>(x, M, K, act16, mt_tab, n_mtiles);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_act_gather_bf16(const uint16_t* x, int T, int H, int k, const int* inv, uint8_t* x16, uint8_t* h16,
+                                   int F, cudaStream_t stream) {
+    if (T == 0) return cudaSuccess;
+    act_gather_bf16_kernel<<<T, 128, 0, stream>>>(x, H, k, inv, x16, h16, F);
     return cudaGetLastError();
 }
 

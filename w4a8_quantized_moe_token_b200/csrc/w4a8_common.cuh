@@ -54,6 +54,15 @@ __host__ __device__ inline size_t act_offset(int r, int k, int G, int RB) {
     return ((size_t)(r / RB) * G + (size_t)(k >> 7)) * (size_t)RB * 128u + act_tiled_offset(r % RB, k & 127);
 }
 
+// Byte offset of (row r, column k) in a tiled bf16 token-row buffer: per block of RB
+// rows and 128-wide K group, two planes of 64 columns (128 bytes per row), each in the
+// swizzled arrangement of act_tiled_offset ([rows/RB][G][2][RB][128 bytes]).  A
+// 16-bit tensor-core step (K = 16, 32 bytes) then reads inside one plane.
+__host__ __device__ inline size_t act16_offset(int r, int k, int G, int RB) {
+    return (((size_t)(r / RB) * G + (size_t)(k >> 7)) * 2u + (size_t)((k >> 6) & 1)) * (size_t)RB * 128u +
+           act_tiled_offset(r % RB, (k & 63) * 2);
+}
+
 // Byte offset of 16-byte chunk c (K columns 32c..32c+31 of the group) of tiled row r
 // inside a code block: rows of 64 bytes, chunk swizzled with (r >> 1) & 3 so that
 // eight consecutive rows reading the same chunk hit distinct shared-memory banks.
@@ -193,6 +202,17 @@ __device__ __forceinline__ void mma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, ui
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem]^T, bf16 x bf16 -> f32; M = 128, N from idesc, K = 16
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
 

@@ -26,6 +26,10 @@ struct GemmArgs {
     uint32_t* err;            // device error word
     long long wait_limit;     // clock cycles a bounded wait may last (> 0; normally ~2 s)
     uint32_t debug;           // test hook: bit 0 = CTA 0 issues no copy for its first step
+    // W4A16 only (bf16 token rows, layout act16_offset): mode 1 writes h as bf16 into
+    // the tiled token rows of out16 (16-row blocks, out16_G K groups) instead of `out`
+    uint8_t* out16;
+    int out16_G;
 };
 
 // Test hook of the failure-detection path (w4a8_debug_inject): while set on the
@@ -43,6 +47,9 @@ int gemm_tile_tokens(int avg_tokens_per_expert);
 inline int act_block_rows(int tile_tokens, int rows_cap) { return tile_tokens == 16 ? 16 : rows_cap; }
 cudaError_t launch_gemm(const GemmArgs& a, int tile_tokens, int num_ctas, cudaStream_t stream);
 cudaError_t launch_gemm_decode(const GemmArgs& a, int num_ctas, cudaStream_t stream);
+// W4A16: the decode-tile kernel on bf16 token rows (act points at act16_offset rows with
+// 16-row blocks, act_rb_stride = G * 16 * 256); no partials; mode 1 needs out16
+cudaError_t launch_gemm_w4a16(const GemmArgs& a, int num_ctas, cudaStream_t stream);
 
 // scheme: 0 asymmetric (min/max), 1 symmetric, 2 asymmetric on the 0.1th..99.9th percentiles
 cudaError_t launch_pack(const uint16_t* w, int E, int N, int K, int layout, int scheme, uint8_t* packed,
@@ -66,6 +73,15 @@ cudaError_t launch_combine(const float* y2, int H, const int* inv, const float* 
                            cudaStream_t stream);
 cudaError_t launch_dense_prep(const int8_t* qa, int M, int Kp, int tile_tokens, int rb, int8_t* act, int4* mt_tab,
                               int* n_mtiles, cudaStream_t stream);
+// W4A16 token rows: x bf16 [M][K] -> tiled bf16 rows (16-row blocks, K padded with
+// zeros) described as one "expert" of 16-row tiles
+cudaError_t launch_dense_prep_bf16(const uint16_t* x, int M, int K, uint8_t* act16, int4* mt_tab, int* n_mtiles,
+                                   cudaStream_t stream);
+// W4A16 layer: each token's bf16 row copied to its k grouped rows (tiled, 16-row
+// blocks, pad K columns zero); the pad K columns [F, Fp) of the same rows of the h
+// buffer are zeroed too
+cudaError_t launch_act_gather_bf16(const uint16_t* x, int T, int H, int k, const int* inv, uint8_t* x16, uint8_t* h16,
+                                   int F, cudaStream_t stream);
 
 constexpr int kPermChunk = 256;       // slots per permutation chunk (multi-CTA path)
 constexpr int kPermSmallSlots = 16384;  // up to this many slots the permutation runs in one CTA
