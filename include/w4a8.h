@@ -82,17 +82,27 @@ enum { W4A8_LAYOUT_PLAIN = 0, W4A8_LAYOUT_GATEUP = 1 };
  *   two nearest order statistics (positions 0.127 and 126.873 of the 128 sorted
  *   values) evaluated in fp32 as a + f*(b - a), f = 0.127f / 0.873f; values outside
  *   the range land on codes 0 / 15 through the clamp.
- * At most one flag may be set.  All write the same tiled format, so w4a8_gemm and
+ * At most one of these may be set.  All write the same tiled format, so w4a8_gemm and
  * w4a8_moe_forward take any of them.  Rounding is half to even; divisions are
- * correctly rounded fp32; an fp16 scale that rounds to 0 is replaced by 1.         */
-enum { W4A8_PACK_SYMMETRIC = 0x100, W4A8_PACK_CLIP999 = 0x200 };
+ * correctly rounded fp32; an fp16 scale that rounds to 0 is replaced by 1.
+ * Group size flags (the same page, section 4.3: groups of 64, 128 and 256 weights
+ * were tried; the Kimi 2.7T MoE W4A8 article, hotelren.com 5173946, section 5: 128 or
+ * 256 is usual): W4A8_PACK_GROUP64 / W4A8_PACK_GROUP256 give each 64 / 256 weights
+ * along K their own scale and zero point instead of each 128 (with the asymmetric or
+ * the symmetric scheme; the percentile range is defined for 128-value groups only).
+ * Such weights are multiplied with w4a8_gemm_g / w4a8_moe_forward_g, which take the
+ * group size, and K is padded to a whole number of groups (and of 128).           */
+enum { W4A8_PACK_SYMMETRIC = 0x100, W4A8_PACK_CLIP999 = 0x200, W4A8_PACK_GROUP64 = 0x400,
+       W4A8_PACK_GROUP256 = 0x800 };
 
 /* Bytes of a packed weight buffer for E matrices of shape [N][K] in `layout`:
- * a 256-byte header, then one 8704-byte block per (matrix, 128-row tile, 128-wide
- * K group): 8192 bytes of 4-bit codes, 128 fp16 scales, 128 fp16 zero points.
- * K is padded to a multiple of 128 (zero weights).  Returns 0 for invalid shapes
- * (GATEUP needs an even N) or an unknown flag combination; one of
- * W4A8_PACK_SYMMETRIC, W4A8_PACK_CLIP999 may be set. */
+ * a 256-byte header, then one block per (matrix, 128-row tile, 128-wide K plane):
+ * 8192 bytes of 4-bit codes, then 128 fp16 scales and 128 fp16 zero points of the
+ * plane's group (8704 bytes).  Group 64: the plane holds two groups, and the scales
+ * and zero points of the second follow those of the first (9216 bytes).  Group 256:
+ * both planes of a group carry its scales and zero points (8704 bytes).  K is padded
+ * to a multiple of 128 and of the group (zero weights).  Returns 0 for invalid shapes
+ * (GATEUP needs an even N) or an unknown flag combination. */
 size_t w4a8_packed_bytes(int E, int N, int K, int layout);
 
 /* Quantise and pack E weight matrices  (a1: the offline conversion step).
@@ -152,6 +162,15 @@ int w4a8_moe_forward(const void* packed_up, const void* packed_down, int E, int 
                      const void* x_bf16, int T, const int32_t* ids, const float* w, int k,
                      void* out_bf16, void* ws, size_t ws_bytes, void* stream);
 
+/* w4a8_moe_forward for experts packed with another group size (group = 64, 128 or
+ * 256, both projections packed with it); the token rows are padded to whole groups.
+ * Workspace from w4a8_moe_workspace_bytes_g; stages readable with w4a8_debug_dump(what
+ * | W4A8_DUMP_GROUP64 or W4A8_DUMP_GROUP256).  Returns W4A8_EINVAL for another group. */
+size_t w4a8_moe_workspace_bytes_g(int T, int E, int k, int H, int F, int group);
+int w4a8_moe_forward_g(const void* packed_up, const void* packed_down, int E, int H, int F, int group,
+                       const void* x_bf16, int T, const int32_t* ids, const float* w, int k,
+                       void* out_bf16, void* ws, size_t ws_bytes, void* stream);
+
 /* Same as w4a8_moe_forward, but x_bf16, ids, w and out_bf16 are HOST buffers
  * (pinned memory recommended): they are copied to / from the workspace on
  * `stream` with cudaMemcpyAsync before and after the forward.  Needs
@@ -189,6 +208,15 @@ size_t w4a8_gemm_workspace_bytes(int M, int N, int K);
  *   partials_opt: device int32 [M][N][Kp/128] or NULL -- the exact INT32 partials. */
 int w4a8_gemm(const int8_t* qa, const float* sa, int M, const void* packed, int N, int K,
               float* y, int32_t* partials_opt, void* ws, size_t ws_bytes, void* stream);
+
+/* w4a8_gemm for weights packed with another group size (group = 64, 128 or 256, as
+ * packed): one INT32 partial per group, partials_opt int32 [M][N][Kp/group], where Kp
+ * is K padded to a multiple of 128 and of the group; qa as for w4a8_gemm ([M][K
+ * rounded up to 128], the row padding to Kp is implicit zeros).  Workspace from
+ * w4a8_gemm_workspace_bytes_g.  Returns W4A8_EINVAL for another group. */
+size_t w4a8_gemm_workspace_bytes_g(int M, int N, int K, int group);
+int w4a8_gemm_g(const int8_t* qa, const float* sa, int M, const void* packed, int N, int K, int group,
+                float* y, int32_t* partials_opt, void* ws, size_t ws_bytes, void* stream);
 
 /* w4a8_gemm for callers that cannot allocate device memory.  (The pages describe
  * no such variant: it exists for integration, not for the method.)
@@ -268,7 +296,11 @@ enum {
      * and 256 bytes per row and K group ([R/16][Kp/128][2][16][128 bytes]: the two
      * 64-column halves of a group one after the other, each swizzled like the INT8
      * rows); S1, H and S2 are empty. */
-    W4A8_DUMP_W4A16 = 0x100
+    W4A8_DUMP_W4A16 = 0x100,
+    /* OR-ed into `what`: the region of a w4a8_moe_forward_g workspace of that group size
+     * (the tiled rows are then Hp = H and Fp = F padded to 128 and to the group). */
+    W4A8_DUMP_GROUP64 = 0x400,
+    W4A8_DUMP_GROUP256 = 0x800
 };
 /* R = w4a8_moe_rows_capacity(T,E,k).  Tiled INT8 rows: rows are grouped in blocks of
  * RB = w4a8_moe_act_block_rows(T,E,k) rows (16 for decode-shaped layers, whose mean

@@ -373,14 +373,17 @@ def round_to_bf16(x: np.ndarray) -> np.ndarray:
 # --------------------------------------------------------------------------- #
 class QuantExpert:
     """Quantised weights of one expert: up [2F][Hp] (gate|up rows) and down [H][Fp]
-    (asymmetric INT4, or the symmetric variant)."""
+    (asymmetric INT4, or the symmetric variant), `group` weights per scale along K."""
 
-    def __init__(self, w_up: np.ndarray, w_down: np.ndarray, symmetric: bool = False, clip999: bool = False):
+    def __init__(self, w_up: np.ndarray, w_down: np.ndarray, symmetric: bool = False, clip999: bool = False,
+                 group: int = GROUP):
+        self.group = group
         if symmetric:
-            quant = quantize_weights_symmetric
+            def quant(w):
+                return quantize_weights_symmetric(w, group)
         else:
             def quant(w):
-                return quantize_weights(w, clip999)
+                return quantize_weights(w, clip999, group)
         self.up = quant(w_up)
         self.down = quant(w_down)
 
@@ -393,7 +396,7 @@ def expert_forward(xq, xs, qe: QuantExpert, F: int, stages: dict | None = None):
     cu, su, zu = qe.up
     y_up = w4a8_linear(xq, xs, cu, su, zu)  # [M][2F]
     h = swiglu(y_up, F).astype(np.float32)  # R14: h enters requant as fp32
-    qh, sh = quantize_act(h)  # [P1] §4.3 step 3: the next op's input is quantised per token
+    qh, sh = quantize_act(h, qe.group)  # [P1] §4.3 step 3: the next op's input is quantised per token
     cd, sd, zd = qe.down
     y2 = w4a8_linear(qh, sh, cd, sd, zd)
     if stages is not None:
@@ -413,7 +416,8 @@ def moe_forward(x, ids, w, experts: dict, E: int, F: int, stages: dict | None = 
     x = np.asarray(x, dtype=np.float32)
     T, H = x.shape
     k = ids.shape[1]
-    xq, xs = quantize_act(x)
+    group = next(iter(experts.values())).group if experts else GROUP
+    xq, xs = quantize_act(x, group)
     counts, offs, perm, inv = permute(ids, E)
     y2 = np.zeros((T * k, H), dtype=np.float64)
     for e in range(E):
@@ -429,7 +433,8 @@ def moe_forward(x, ids, w, experts: dict, E: int, F: int, stages: dict | None = 
 
 def token_forward(t: int, x, ids, w, experts: dict, F: int) -> np.ndarray:
     """The layer's output (bf16-rounded) for one token only (used to sample large layers)."""
-    xq, xs = quantize_act(np.asarray(x, dtype=np.float32)[t:t + 1])
+    group = experts[int(ids[t, 0])].group
+    xq, xs = quantize_act(np.asarray(x, dtype=np.float32)[t:t + 1], group)
     out = 0.0
     for j in range(ids.shape[1]):
         y2 = expert_forward(xq, xs, experts[int(ids[t, j])], F)[0]

@@ -45,15 +45,22 @@ def packed_tiles(N: int, layout: int) -> int:
     return -(-(N // 2) // 64) if layout == 1 else -(-N // 128)
 
 
-def decode_packed(buf: np.ndarray, E: int, N: int, K: int, layout: int):
-    """Tiled packed buffer -> (codes uint8 [E][N][Kp], scale f16 [E][N][G], zp f16 [E][N][G])."""
-    G = -(-K // 128)
-    Kp = G * 128
+def decode_packed(buf: np.ndarray, E: int, N: int, K: int, layout: int, group: int = 128):
+    """Tiled packed buffer -> (codes uint8 [E][N][Kp], scale f16 [E][N][Gq], zp f16 [E][N][Gq]).
+
+    One block per 128-wide plane: codes, then per row the fp16 scale and zero point of
+    the plane's group (group 64: of its two groups, the second pair 512 bytes after
+    the first; group 256: both planes of a group carry the pair, checked equal)."""
+    m = max(128, group)
+    Kp = -(-K // m) * m
+    G = Kp // 128
+    Gq = Kp // group
+    blk_bytes = BLOCK + 512 if group == 64 else BLOCK
     NT = packed_tiles(N, layout)
-    blocks = np.asarray(buf, dtype=np.uint8)[HEADER:HEADER + E * NT * G * BLOCK].reshape(E, NT, G, BLOCK)
+    blocks = np.asarray(buf, dtype=np.uint8)[HEADER:HEADER + E * NT * G * blk_bytes].reshape(E, NT, G, blk_bytes)
     codes = np.zeros((E, N, Kp), np.uint8)
-    scale = np.zeros((E, N, G), np.float16)
-    zp = np.zeros((E, N, G), np.float16)
+    scale = np.zeros((E, N, Gq), np.float16)
+    zp = np.zeros((E, N, Gq), np.float16)
     r = np.arange(128)
     if layout == 1:
         F = N // 2
@@ -79,11 +86,18 @@ def decode_packed(buf: np.ndarray, E: int, N: int, K: int, layout: int):
                     for b in range(4):
                         rows[:, :, 8 * i + b] = (x >> (8 * b)) & 0xF
                         rows[:, :, 8 * i + 4 + b] = (x >> (8 * b + 4)) & 0xF
-            sc = blk[:, 8192:8448].copy().view(np.float16).reshape(E, 128)
-            z = blk[:, 8448:8704].copy().view(np.float16).reshape(E, 128)
             codes[:, src[valid], g * 128:(g + 1) * 128] = rows[:, valid]
-            scale[:, src[valid], g] = sc[:, valid]
-            zp[:, src[valid], g] = z[:, valid]
+            for sub in range(2 if group == 64 else 1):
+                o = 8192 + 512 * sub
+                sc = blk[:, o:o + 256].copy().view(np.float16).reshape(E, 128)
+                z = blk[:, o + 256:o + 512].copy().view(np.float16).reshape(E, 128)
+                q = g * 128 // group + sub
+                if group == 256 and g % 2 == 1:  # the group's second plane repeats its pair
+                    assert np.array_equal(sc[:, valid].view(np.uint16), scale[:, src[valid], q].view(np.uint16))
+                    assert np.array_equal(z[:, valid].view(np.uint16), zp[:, src[valid], q].view(np.uint16))
+                    continue
+                scale[:, src[valid], q] = sc[:, valid]
+                zp[:, src[valid], q] = z[:, valid]
     return codes, scale, zp
 
 

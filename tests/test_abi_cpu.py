@@ -53,7 +53,16 @@ def test_packed_bytes_accounting(lib):
     assert lib.w4a8_packed_bytes(8, 2048, 2048, 1 | 0x100) == lib.w4a8_packed_bytes(8, 2048, 2048, 1)
     assert lib.w4a8_packed_bytes(1, 256, 512, 0x200) == lib.w4a8_packed_bytes(1, 256, 512, 0)
     assert lib.w4a8_packed_bytes(1, 256, 512, 0x300) == 0  # two scheme flags
-    assert lib.w4a8_packed_bytes(1, 256, 512, 0x400) == 0  # unknown flag
+    assert lib.w4a8_packed_bytes(1, 256, 512, 0x1000) == 0  # unknown flag
+    # group sizes: group 64 blocks carry two scale / zero-point pairs per row (9216 bytes),
+    # group 256 pads K to 256 and repeats its pair in both planes (8704 bytes)
+    assert lib.w4a8_packed_bytes(1, 256, 512, 0x400) == 256 + 2 * 4 * 9216
+    assert lib.w4a8_packed_bytes(1, 256, 512, 0x800) == 256 + 2 * 4 * 8704
+    assert lib.w4a8_packed_bytes(1, 128, 300, 0x800) == 256 + 4 * 8704  # K 300 -> 512
+    assert lib.w4a8_packed_bytes(1, 128, 300, 0x400) == 256 + 3 * 9216  # K 300 -> 384
+    assert lib.w4a8_packed_bytes(1, 256, 512, 0x400 | 0x800) == 0  # two group sizes
+    assert lib.w4a8_packed_bytes(1, 256, 512, 0x200 | 0x400) == 0  # percentile range needs group 128
+    assert lib.w4a8_packed_bytes(1, 256, 512, 0x100 | 0x800) == 256 + 2 * 4 * 8704  # symmetric, group 256
     assert lib.w4a8_packed_bytes(0, 128, 128, 0) == 0
     # per weight: 0.5 byte of codes + 4 bytes per 128-group of scale and zero point
     blk = 8704
@@ -157,3 +166,19 @@ def test_w4a16_workspaces_and_validation(lib):
     assert lib.w4a16_gemm(fake, 4, vp((1 << 20) + 16), 256, 512, fake, fake, 1 << 40, None) == EALIGN
     assert lib.w4a16_moe_forward(fake, fake, 8, 256, 128, fake, 4, fake, fake, 2, fake, fake, 16, None) == ENOSPACE
     assert lib.w4a16_moe_forward(fake, fake, 8, 256, 128, fake, 4, fake, fake, 9, fake, fake, 1 << 40, None) == EINVAL
+
+
+def test_group_size_entry_points_validate(lib):
+    vp = ctypes.c_void_p
+    fake = vp(1 << 20)
+    assert lib.w4a8_gemm_workspace_bytes_g(16, 256, 300, 256) >= 4 * 16 * 128  # K 300 -> 4 planes
+    assert lib.w4a8_gemm_workspace_bytes_g(16, 256, 300, 96) == 0  # not a group size
+    assert lib.w4a8_gemm_g(fake, fake, 4, fake, 256, 512, 32, fake, None, fake, 1 << 40, None) == EINVAL
+    assert lib.w4a8_moe_workspace_bytes_g(64, 8, 2, 300, 200, 256) > lib.w4a8_moe_workspace_bytes(64, 8, 2, 300, 200)
+    assert lib.w4a8_moe_workspace_bytes_g(64, 8, 2, 300, 200, 128) == lib.w4a8_moe_workspace_bytes(64, 8, 2, 300, 200)
+    assert lib.w4a8_moe_forward_g(fake, fake, 8, 256, 128, 100, fake, 4, fake, fake, 2, fake, fake, 1 << 40,
+                                  None) == EINVAL
+    # dump regions of a group-256 workspace: rows padded to whole groups (H 300 -> 512)
+    R = lib.w4a8_moe_rows_capacity(64, 8, 2)
+    _, nb = B.w4a8_debug_region(64, 8, 2, 300, 200, B.DUMP["act1"] | B.DUMP_GROUP[256])
+    assert nb == 4 * R * 128

@@ -439,11 +439,16 @@ def _tiny_layer(seed=0, T=9, E=4, k=2, H=256, F=128):
     return x, ids, w, experts
 
 
-def test_moe_forward_equals_per_token_dequantized_formulation():
+@pytest.mark.parametrize("group", [128, 64, 256])
+def test_moe_forward_equals_per_token_dequantized_formulation(group):
     T, E, k, H, F = 9, 4, 2, 256, 128
     x, ids, w, experts = _tiny_layer(T=T, E=E, k=k, H=H, F=F)
+    if group != 128:  # the same weights quantised with another group size
+        experts = {e: O.QuantExpert(synth.expert_weight(0, e, "up", 2 * F, H), synth.expert_weight(0, e, "down", H, F),
+                                    group=group) for e in experts}
+        assert experts[0].up[1].shape == (2 * F, H // group)
     out = O.moe_forward(x, ids, w, experts, E, F)
-    xq, xs = O.quantize_act(x)
+    xq, xs = O.quantize_act(x, group)
     for t in range(T):
         acc = np.zeros(H)
         a = xq[t].astype(np.float64) * float(xs[t])
@@ -453,7 +458,7 @@ def test_moe_forward_equals_per_token_dequantized_formulation():
             wd = O.dequantize_weights(*qe.down)
             yu = wu @ a
             hh = (yu[:F] / (1 + np.exp(-yu[:F])) * yu[F:]).astype(np.float32)
-            qh, sh = O.quantize_act(hh[None, :])
+            qh, sh = O.quantize_act(hh[None, :], group)
             acc += float(w[t, j]) * (wd @ (qh[0].astype(np.float64) * float(sh[0])))
         # the layer's output is rounded to bf16: within half a bf16 ulp of the fp64 value
         assert np.all(np.abs(out[t] - acc) <= np.abs(acc) * 2.0 ** -8 + 1e-30)

@@ -20,12 +20,16 @@ W4A8_LAYOUT_PLAIN = 0
 W4A8_LAYOUT_GATEUP = 1
 W4A8_PACK_SYMMETRIC = 0x100  # OR into the layout: symmetric INT4 (scale = max|w|/7, codes q + 8, zero point 8)
 W4A8_PACK_CLIP999 = 0x200  # OR into the layout: asymmetric INT4 over the 0.1th..99.9th percentile range
+W4A8_PACK_GROUP64 = 0x400  # OR into the layout: one scale and zero point per 64 weights along K
+W4A8_PACK_GROUP256 = 0x800  # OR into the layout: one scale and zero point per 256 weights along K
+GROUP_FLAG = {64: W4A8_PACK_GROUP64, 128: 0, 256: W4A8_PACK_GROUP256}
 
 DUMP = {
     "counts": 0, "offs": 1, "perm": 2, "inv": 3, "poffs": 4, "act1": 5, "s1": 6,
     "h": 7, "act2": 8, "s2": 9, "y2": 10, "err": 11,
 }
 W4A8_DUMP_W4A16 = 0x100  # OR into a dump id: the region of a w4a16_moe_forward workspace
+DUMP_GROUP = {64: 0x400, 128: 0, 256: 0x800}  # OR into a dump id: a w4a8_moe_forward_g workspace
 
 _c_int, _c_size, _vp = ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p
 _SIGS = {
@@ -49,6 +53,11 @@ _SIGS = {
     "w4a8_gemm_workspace_bytes": ([_c_int] * 3, _c_size),
     "w4a8_gemm": ([_vp, _vp, _c_int, _vp, _c_int, _c_int, _vp, _vp, _vp, _c_size, _vp], _c_int),
     "w4a8_gemm_noalloc": ([_vp, _vp, _c_int, _vp, _c_int, _c_int, _vp, _vp, _vp], _c_int),
+    "w4a8_gemm_workspace_bytes_g": ([_c_int] * 4, _c_size),
+    "w4a8_gemm_g": ([_vp, _vp, _c_int, _vp, _c_int, _c_int, _c_int, _vp, _vp, _vp, _c_size, _vp], _c_int),
+    "w4a8_moe_workspace_bytes_g": ([_c_int] * 6, _c_size),
+    "w4a8_moe_forward_g": ([_vp, _vp, _c_int, _c_int, _c_int, _c_int, _vp, _c_int, _vp, _vp, _c_int, _vp, _vp, _c_size,
+                            _vp], _c_int),
     "w4a8_gemm_noalloc_last_error": ([_vp], _c_int),
     "w4a8_moe_forward_logits_host": ([_vp, _vp, _c_int, _c_int, _c_int, _vp, _c_int, _vp, _c_int, _vp, _vp,
                                       _c_size, _vp], _c_int),
@@ -126,9 +135,11 @@ def _need(cond, msg):
         raise W4A8Error(msg)
 
 
-def padded_k(K: int) -> int:
-    """K rounded up to a whole number of 128-wide groups (the layout's row length)."""
-    return (K + 127) // 128 * 128
+def padded_k(K: int, group: int = 128) -> int:
+    """K rounded up to a whole number of 128-wide planes and of groups (the layout's
+    row length)."""
+    m = max(128, group)
+    return (K + m - 1) // m * m
 
 
 # --------------------------------------------------------------------------- #
@@ -213,13 +224,14 @@ def w4a8_moe_act_block_rows(T, E, k) -> int:
     return lib().w4a8_moe_act_block_rows(T, E, k)
 
 
-def _moe_buffers(packed_up, packed_down, E, H, F, ws, host_ws=False):
+def _moe_buffers(packed_up, packed_down, E, H, F, ws, host_ws=False, group=128):
     _dev(packed_up, torch.uint8, "packed_up")
     _dev(packed_down, torch.uint8, "packed_down")
     _dev(ws, torch.uint8, "ws")
-    _need(packed_up.numel() >= w4a8_packed_bytes(E, 2 * F, H, W4A8_LAYOUT_GATEUP),
+    _need(group in GROUP_FLAG, f"group must be 64, 128 or 256, got {group}")
+    _need(packed_up.numel() >= w4a8_packed_bytes(E, 2 * F, H, W4A8_LAYOUT_GATEUP | GROUP_FLAG[group]),
           "packed_up is smaller than the packed gate|up weights of this layer")
-    _need(packed_down.numel() >= w4a8_packed_bytes(E, H, F, W4A8_LAYOUT_PLAIN),
+    _need(packed_down.numel() >= w4a8_packed_bytes(E, H, F, W4A8_LAYOUT_PLAIN | GROUP_FLAG[group]),
           "packed_down is smaller than the packed down weights of this layer")
 
 
@@ -236,6 +248,25 @@ def w4a8_moe_forward(packed_up, packed_down, E, H, F, x, ids, w, out, ws):
     _need(tuple(out.shape) == (T, H), f"out must be [T={T}][H={H}], got {tuple(out.shape)}")
     _check(lib().w4a8_moe_forward(_ptr(packed_up), _ptr(packed_down), E, H, F, _ptr(x), T, _ptr(ids), _ptr(w), k,
                                   _ptr(out), _ptr(ws), ws.numel(), _stream()), "w4a8_moe_forward")
+
+
+def w4a8_moe_workspace_bytes_g(T, E, k, H, F, group) -> int:
+    return lib().w4a8_moe_workspace_bytes_g(T, E, k, H, F, group)
+
+
+def w4a8_moe_forward_g(packed_up, packed_down, E, H, F, group, x, ids, w, out, ws):
+    """w4a8_moe_forward for experts packed with group size 64, 128 or 256."""
+    _dev(x, torch.bfloat16, "x")
+    _dev(ids, torch.int32, "ids")
+    _dev(w, torch.float32, "w")
+    _dev(out, torch.bfloat16, "out")
+    _moe_buffers(packed_up, packed_down, E, H, F, ws, group=group)
+    T, k = ids.shape
+    _need(tuple(x.shape) == (T, H), f"x must be [T={T}][H={H}], got {tuple(x.shape)}")
+    _need(tuple(w.shape) == (T, k), f"w must be [T={T}][k={k}], got {tuple(w.shape)}")
+    _need(tuple(out.shape) == (T, H), f"out must be [T={T}][H={H}], got {tuple(out.shape)}")
+    _check(lib().w4a8_moe_forward_g(_ptr(packed_up), _ptr(packed_down), E, H, F, group, _ptr(x), T, _ptr(ids),
+                                    _ptr(w), k, _ptr(out), _ptr(ws), ws.numel(), _stream()), "w4a8_moe_forward_g")
 
 
 def w4a16_moe_workspace_bytes(T, E, k, H, F) -> int:
@@ -293,9 +324,10 @@ def w4a8_gemm_workspace_bytes(M, N, K) -> int:
     return lib().w4a8_gemm_workspace_bytes(M, N, K)
 
 
-def _gemm_buffers(qa, sa, packed, N, K, y, partials):
+def _gemm_buffers(qa, sa, packed, N, K, y, partials, group=128):
     """Check every buffer of a dense GEMM against its shape before the call: the
     kernels trust the sizes they are given."""
+    _need(group in GROUP_FLAG, f"group must be 64, 128 or 256, got {group}")
     _dev(qa, torch.int8, "qa")
     _dev(sa, torch.float32, "sa")
     _dev(y, torch.float32, "y")
@@ -306,11 +338,12 @@ def _gemm_buffers(qa, sa, packed, N, K, y, partials):
     _need(tuple(qa.shape) == (M, Kp), f"qa must be [M][{Kp}] for K = {K}, got {tuple(qa.shape)}")
     _need(sa.numel() >= M, f"sa needs {M} entries, has {sa.numel()}")
     _need(y.numel() >= M * N, f"y needs {M * N} elements, has {y.numel()}")
-    _need(packed.numel() >= w4a8_packed_bytes(1, N, K, W4A8_LAYOUT_PLAIN),
+    _need(packed.numel() >= w4a8_packed_bytes(1, N, K, W4A8_LAYOUT_PLAIN | GROUP_FLAG[group]),
           "packed is smaller than the packed weights of an N x K matrix")
     if partials is not None:
         _dev(partials, torch.int32, "partials")
-        _need(partials.numel() >= M * N * (Kp // 128), f"partials needs {M * N * (Kp // 128)} elements")
+        ng = padded_k(K, group) // group
+        _need(partials.numel() >= M * N * ng, f"partials needs {M * N * ng} elements")
     return M
 
 
@@ -320,6 +353,19 @@ def w4a8_gemm(qa, sa, packed, N, K, y, ws, partials=None):
     _dev(ws, torch.uint8, "ws")
     _check(lib().w4a8_gemm(_ptr(qa), _ptr(sa), M, _ptr(packed), N, K, _ptr(y), _ptr(partials), _ptr(ws), ws.numel(),
                            _stream()), "w4a8_gemm")
+
+
+def w4a8_gemm_workspace_bytes_g(M, N, K, group) -> int:
+    return lib().w4a8_gemm_workspace_bytes_g(M, N, K, group)
+
+
+def w4a8_gemm_g(qa, sa, packed, N, K, group, y, ws, partials=None):
+    """w4a8_gemm for weights packed with group size 64, 128 or 256; partials int32
+    [M][N][padded_k(K, group) / group] or None."""
+    M = _gemm_buffers(qa, sa, packed, N, K, y, partials, group)
+    _dev(ws, torch.uint8, "ws")
+    _check(lib().w4a8_gemm_g(_ptr(qa), _ptr(sa), M, _ptr(packed), N, K, group, _ptr(y), _ptr(partials), _ptr(ws),
+                             ws.numel(), _stream()), "w4a8_gemm_g")
 
 
 def w4a8_gemm_noalloc(qa, sa, packed, N, K, y, partials=None):

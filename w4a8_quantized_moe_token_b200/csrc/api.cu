@@ -59,14 +59,17 @@ struct MoeLayout {
 
 // w4a16: the W4A16 layer's workspace, in which ACT1 and ACT2 hold bf16 token rows
 // (act16_offset, 16-row blocks) and the INT8 scales and the fp32 h are absent
-bool moe_layout(int T, int E, int k, int H, int F, bool host_io, MoeLayout* L, bool w4a16 = false) {
+// group: weights per scale of the packed weights (64, 128, 256): the token rows are
+// padded to whole groups
+bool moe_layout(int T, int E, int k, int H, int F, bool host_io, MoeLayout* L, bool w4a16 = false, int group = 128) {
     if (T < 0 || E < 1 || E > kMaxExperts || k < 1 || k > 32 || k > E || H < 1 || F < 1) return false;
     if ((long long)T * k >= (1ll << 31)) return false;
+    if (group != 64 && group != 128 && group != 256) return false;
     L->nslots = T * k;
     L->nchunk = ceil_div(L->nslots, kPermChunk);
     L->R = rows_capacity(T, E, k);
-    L->Hp = round_up(H, kGroup);
-    L->Fp = round_up(F, kGroup);
+    L->Hp = k_padded_for(H, group);
+    L->Fp = k_padded_for(F, group);
     L->G1 = L->Hp / kGroup;
     L->G2 = L->Fp / kGroup;
     const size_t R = (size_t)L->R;
@@ -173,7 +176,7 @@ T* at(void* base, const MoeLayout& L, Region r) {
 // the forward on device buffers, workspace already validated
 int moe_forward_impl(const void* packed_up, const void* packed_down, int E, int H, int F, const uint16_t* x, int T,
                      const int32_t* ids, const float* w, int k, uint16_t* out, void* ws, const MoeLayout& L,
-                     cudaStream_t st) {
+                     cudaStream_t st, int group = 128) {
     uint32_t* err = at<uint32_t>(ws, L, R_ERR);
     W4A8_TRY(cudaMemsetAsync(err, 0, 16, st));
     if (T == 0) return W4A8_OK;
@@ -202,7 +205,7 @@ int moe_forward_impl(const void* packed_up, const void* packed_down, int E, int 
     }
     {
         ProfScope p(W4A8_KERNEL_ACT_QUANT, 1, st);
-        W4A8_TRY(launch_act_scatter(x, T, H, k, inv, offs, poffs, E, rb, act1, s1, st));
+        W4A8_TRY(launch_act_scatter(x, T, H, L.Hp, k, inv, offs, poffs, E, rb, act1, s1, st));
     }
 
     GemmArgs up{};
@@ -221,6 +224,7 @@ int moe_forward_impl(const void* packed_up, const void* packed_down, int E, int 
     up.nvalid = F;
     up.partials = nullptr;
     up.err = err;
+    up.group = group;
     apply_debug(up);
     {
         ProfScope p(W4A8_KERNEL_GEMM_UP, 1, st);
@@ -228,7 +232,7 @@ int moe_forward_impl(const void* packed_up, const void* packed_down, int E, int 
     }
     {
         ProfScope p(W4A8_KERNEL_REQUANT, 1, st);
-        W4A8_TRY(launch_requant(h, L.Fp, F, row_src, poffs, E, L.R, rb, act2, s2, st));
+        W4A8_TRY(launch_requant(h, L.Fp, F, L.Fp, row_src, poffs, E, L.R, rb, act2, s2, st));
     }
 
     GemmArgs dn = up;
@@ -320,8 +324,8 @@ int moe_forward_w4a16_impl(const void* packed_up, const void* packed_down, int E
 }
 
 int check_moe_args(const void* packed_up, const void* packed_down, int E, int H, int F, int T, int k, void* ws,
-                   size_t ws_bytes, bool host_io, MoeLayout* L, bool w4a16 = false) {
-    if (!moe_layout(T, E, k, H, F, host_io, L, w4a16)) {
+                   size_t ws_bytes, bool host_io, MoeLayout* L, bool w4a16 = false, int group = 128) {
+    if (!moe_layout(T, E, k, H, F, host_io, L, w4a16, group)) {
         if (E > kMaxExperts || k > 32) return W4A8_EUNSUPPORTED;
         return W4A8_EINVAL;
     }
@@ -352,21 +356,47 @@ W4A8_EXPORT const char* w4a8_status_string(int status) {
     }
 }
 
-W4A8_EXPORT size_t w4a8_packed_bytes(int E, int N, int K, int layout) {
-    if (E < 1 || N < 1 || K < 1) return 0;
+namespace w4a8 {
+namespace {
+// Split the packer's `layout` argument into the row layout, the quantisation scheme
+// (0 asymmetric, 1 symmetric, 2 percentile range) and the group size; false for an
+// unknown flag or combination (two schemes, two group sizes, the percentile range
+// with a group other than 128).
+bool parse_layout(int layout, int* base, int* scheme, int* group) {
     const int flags = layout & ~0xFF;
-    if (flags != 0 && flags != W4A8_PACK_SYMMETRIC && flags != W4A8_PACK_CLIP999) return 0;
-    layout &= 0xFF;  // the scheme flag does not change the size
-    if (layout != W4A8_LAYOUT_PLAIN && layout != W4A8_LAYOUT_GATEUP) return 0;
-    if (layout == W4A8_LAYOUT_GATEUP && (N & 1)) return 0;
-    const size_t G = (size_t)ceil_div(K, kGroup);
-    return (size_t)kHeaderBytes + (size_t)E * packed_tiles(N, layout) * G * kBlockBytes;
+    if (flags & ~(W4A8_PACK_SYMMETRIC | W4A8_PACK_CLIP999 | W4A8_PACK_GROUP64 | W4A8_PACK_GROUP256)) return false;
+    if ((flags & W4A8_PACK_SYMMETRIC) && (flags & W4A8_PACK_CLIP999)) return false;
+    if ((flags & W4A8_PACK_GROUP64) && (flags & W4A8_PACK_GROUP256)) return false;
+    *base = layout & 0xFF;
+    if (*base != W4A8_LAYOUT_PLAIN && *base != W4A8_LAYOUT_GATEUP) return false;
+    *scheme = (flags & W4A8_PACK_SYMMETRIC) ? 1 : (flags & W4A8_PACK_CLIP999) ? 2 : 0;
+    *group = (flags & W4A8_PACK_GROUP64) ? 64 : (flags & W4A8_PACK_GROUP256) ? 256 : 128;
+    return !(*scheme == 2 && *group != 128);
+}
+
+size_t packed_bytes_of(int E, int N, int K, int base, int group) {
+    if (E < 1 || N < 1 || K < 1) return 0;
+    if (base == W4A8_LAYOUT_GATEUP && (N & 1)) return 0;
+    const size_t G = (size_t)k_padded_for(K, group) / kGroup;
+    return (size_t)kHeaderBytes + (size_t)E * packed_tiles(N, base) * G * block_bytes_for(group);
+}
+
+bool valid_group(int group) { return group == 64 || group == 128 || group == 256; }
+}  // namespace
+}  // namespace w4a8
+
+W4A8_EXPORT size_t w4a8_packed_bytes(int E, int N, int K, int layout) {
+    int base, scheme, group;
+    if (!parse_layout(layout, &base, &scheme, &group)) return 0;
+    return packed_bytes_of(E, N, K, base, group);
 }
 
 W4A8_EXPORT int w4a8_pack_weights(const void* w_bf16, int E, int N, int K, int layout, void* packed,
                                   size_t packed_bytes, uint8_t* codes_opt, uint16_t* scale_f16_opt,
                                   uint16_t* zp_f16_opt, void* stream) {
-    const size_t need = w4a8_packed_bytes(E, N, K, layout);
+    int base, scheme, group;
+    if (!parse_layout(layout, &base, &scheme, &group)) return W4A8_EINVAL;
+    const size_t need = packed_bytes_of(E, N, K, base, group);
     if (need == 0 || w_bf16 == nullptr || packed == nullptr) return W4A8_EINVAL;
     if (E > 65535) return W4A8_EUNSUPPORTED;
     if (!aligned(w_bf16, 16) || !aligned(packed, kAlign)) return W4A8_EALIGN;
@@ -374,8 +404,7 @@ W4A8_EXPORT int w4a8_pack_weights(const void* w_bf16, int E, int N, int K, int l
         (zp_f16_opt && !aligned(zp_f16_opt, 2)))
         return W4A8_EALIGN;
     if (packed_bytes < need) return W4A8_ENOSPACE;
-    const int scheme = (layout & W4A8_PACK_SYMMETRIC) ? 1 : (layout & W4A8_PACK_CLIP999) ? 2 : 0;
-    return to_status(launch_pack(static_cast<const uint16_t*>(w_bf16), E, N, K, layout & 0xFF, scheme,
+    return to_status(launch_pack(static_cast<const uint16_t*>(w_bf16), E, N, K, base, scheme, group,
                                  static_cast<uint8_t*>(packed), codes_opt, scale_f16_opt, zp_f16_opt,
                                  static_cast<cudaStream_t>(stream)));
 }
@@ -475,6 +504,28 @@ W4A8_EXPORT int w4a8_moe_forward(const void* packed_up, const void* packed_down,
                             static_cast<uint16_t*>(out_bf16), ws, L, static_cast<cudaStream_t>(stream));
 }
 
+W4A8_EXPORT size_t w4a8_moe_workspace_bytes_g(int T, int E, int k, int H, int F, int group) {
+    MoeLayout L;
+    if (!moe_layout(T, E, k, H, F, false, &L, false, group)) return 0;
+    return L.off[R_COUNT];
+}
+
+W4A8_EXPORT int w4a8_moe_forward_g(const void* packed_up, const void* packed_down, int E, int H, int F, int group,
+                                   const void* x_bf16, int T, const int32_t* ids, const float* w, int k,
+                                   void* out_bf16, void* ws, size_t ws_bytes, void* stream) {
+    if (!valid_group(group)) return W4A8_EINVAL;
+    MoeLayout L;
+    const int st = check_moe_args(packed_up, packed_down, E, H, F, T, k, ws, ws_bytes, false, &L, false, group);
+    if (st != W4A8_OK) return st;
+    if (T > 0) {
+        if (x_bf16 == nullptr || ids == nullptr || w == nullptr || out_bf16 == nullptr) return W4A8_EINVAL;
+        if (!aligned(x_bf16, 16) || !aligned(ids, 16) || !aligned(w, 16) || !aligned(out_bf16, 16))
+            return W4A8_EALIGN;
+    }
+    return moe_forward_impl(packed_up, packed_down, E, H, F, static_cast<const uint16_t*>(x_bf16), T, ids, w, k,
+                            static_cast<uint16_t*>(out_bf16), ws, L, static_cast<cudaStream_t>(stream), group);
+}
+
 W4A8_EXPORT size_t w4a16_moe_workspace_bytes(int T, int E, int k, int H, int F) {
     MoeLayout L;
     if (!moe_layout(T, E, k, H, F, false, &L, true)) return 0;
@@ -551,10 +602,10 @@ struct GemmLayout {
     size_t err, nmt, mttab, act, total;
     int Mp, G;
 };
-bool gemm_layout(int M, int N, int K, GemmLayout* L, bool bf16 = false) {
-    if (M < 0 || N < 1 || K < 1) return false;
+bool gemm_layout(int M, int N, int K, GemmLayout* L, bool bf16 = false, int group = 128) {
+    if (M < 0 || N < 1 || K < 1 || !valid_group(group)) return false;
     L->Mp = round_up(M, kRowPad);
-    L->G = ceil_div(K, kGroup);
+    L->G = k_padded_for(K, group) / kGroup;  // 128-wide planes
     size_t o = 0;
     L->err = o; o += align_up(16);
     L->nmt = o; o += align_up(4);
@@ -572,10 +623,16 @@ W4A8_EXPORT size_t w4a8_gemm_workspace_bytes(int M, int N, int K) {
     return L.total;
 }
 
-W4A8_EXPORT int w4a8_gemm(const int8_t* qa, const float* sa, int M, const void* packed, int N, int K, float* y,
-                          int32_t* partials_opt, void* ws, size_t ws_bytes, void* stream) {
+W4A8_EXPORT size_t w4a8_gemm_workspace_bytes_g(int M, int N, int K, int group) {
     GemmLayout L;
-    if (!gemm_layout(M, N, K, &L)) return W4A8_EINVAL;
+    if (!gemm_layout(M, N, K, &L, false, group)) return 0;
+    return L.total;
+}
+
+W4A8_EXPORT int w4a8_gemm_g(const int8_t* qa, const float* sa, int M, const void* packed, int N, int K, int group,
+                            float* y, int32_t* partials_opt, void* ws, size_t ws_bytes, void* stream) {
+    GemmLayout L;
+    if (!gemm_layout(M, N, K, &L, false, group)) return W4A8_EINVAL;
     if (packed == nullptr || ws == nullptr) return W4A8_EINVAL;
     if (!aligned(packed, kAlign) || !aligned(ws, kAlign)) return W4A8_EALIGN;
     if (ws_bytes < L.total) return W4A8_ENOSPACE;
@@ -593,7 +650,7 @@ W4A8_EXPORT int w4a8_gemm(const int8_t* qa, const float* sa, int M, const void* 
     ProfScope prof(W4A8_KERNEL_GEMM_DENSE, 2, s);
     const int tile = gemm_tile_tokens(M);
     const int rb = act_block_rows(tile, L.Mp);
-    W4A8_TRY(launch_dense_prep(qa, M, L.G * kGroup, tile, rb, act, mt_tab, n_mtiles, s));
+    W4A8_TRY(launch_dense_prep(qa, M, round_up(K, kGroup), L.G * kGroup, tile, rb, act, mt_tab, n_mtiles, s));
     GemmArgs a{};
     a.wblocks = static_cast<const uint8_t*>(packed) + kHeaderBytes;
     a.NT = packed_tiles(N, W4A8_LAYOUT_PLAIN);
@@ -610,9 +667,15 @@ W4A8_EXPORT int w4a8_gemm(const int8_t* qa, const float* sa, int M, const void* 
     a.nvalid = N;
     a.partials = partials_opt;
     a.err = err;
+    a.group = group;
     apply_debug(a);
     W4A8_TRY(launch_gemm(a, tile, sm_count(), s));
     return W4A8_OK;
+}
+
+W4A8_EXPORT int w4a8_gemm(const int8_t* qa, const float* sa, int M, const void* packed, int N, int K, float* y,
+                          int32_t* partials_opt, void* ws, size_t ws_bytes, void* stream) {
+    return w4a8_gemm_g(qa, sa, M, packed, N, K, 128, y, partials_opt, ws, ws_bytes, stream);
 }
 
 W4A8_EXPORT size_t w4a16_gemm_workspace_bytes(int M, int N, int K) {
@@ -661,8 +724,10 @@ W4A8_EXPORT int w4a16_gemm(const void* x_bf16, int M, const void* packed, int N,
 W4A8_EXPORT int w4a8_debug_region(int T, int E, int k, int H, int F, int what, size_t* offset, size_t* bytes) {
     MoeLayout L;
     const bool w4a16 = (what & W4A8_DUMP_W4A16) != 0;
-    what &= ~W4A8_DUMP_W4A16;
-    if (!moe_layout(T, E, k, H, F, false, &L, w4a16) || offset == nullptr || bytes == nullptr) return W4A8_EINVAL;
+    const int group = (what & W4A8_DUMP_GROUP64) ? 64 : (what & W4A8_DUMP_GROUP256) ? 256 : 128;
+    what &= ~(W4A8_DUMP_W4A16 | W4A8_DUMP_GROUP64 | W4A8_DUMP_GROUP256);
+    if (!moe_layout(T, E, k, H, F, false, &L, w4a16, group) || offset == nullptr || bytes == nullptr)
+        return W4A8_EINVAL;
     static const Region map[] = {R_COUNTS, R_OFFS, R_PERM, R_INV, R_POFFS, R_ACT1,
                                  R_S1,     R_H,    R_ACT2, R_S2,  R_Y2,    R_ERR};
     if (what < 0 || what >= (int)(sizeof(map) / sizeof(map[0]))) return W4A8_EINVAL;

@@ -9,7 +9,7 @@
 // kernel must run at HBM speed.  Every synchronisation between the roles (mbarrier
 // wait / arrive, tcgen05 commit, tensor-memory store + wait) costs a few hundred
 // cycles, which is as long as one 8.7 KB weight block takes to arrive at full
-// bandwidth; so one pipeline step here carries GPS = 4 consecutive K groups of a tile
+// bandwidth; so one pipeline step here carries 4 consecutive K groups of a tile
 // (35 KB of weights, 16 MMAs), paying the synchronisation once per 4 groups.
 //
 // Roles (one persistent CTA per SM, 20 warps):
@@ -35,6 +35,12 @@
 // (|P| < 2^22), so the bits read back as fp32 are exactly 1.5 * 2^23 + P, and one packed
 // fp32 subtraction yields P without an int -> float conversion.  The epilogue only
 // reads the accumulators.
+//
+// Other group sizes (the «Kimi 2.7 Moe» page, section 4.3, tried 64, 128 and 256): the
+// pipeline still moves 128-wide K planes, but accumulators, scales, zero points and
+// code sums S follow the groups -- two per plane for group 64 (2 MMAs each), one per
+// two planes for group 256 (8 MMAs into one accumulator; |P| <= 256 * 128 * 15 stays
+// below 2^22).  A second instance serves the W4A16 comparison (see DecCfg).
 #include "w4a8_common.cuh"
 #include "w4a8_internal.h"
 
@@ -45,21 +51,26 @@ namespace {
 constexpr uint32_t kMagicBits = 0x4B400000u;  // 1.5 * 2^23 (what the reset MMA writes)
 constexpr float kMagicF = 12582912.0f;
 
-// Pipeline shape per operand kind.  W4A8: INT8 token rows (128 bytes per row and K
-// group), 4 groups per step.  W4A16: bf16 token rows (256 bytes per row and group);
-// a group's converted weights take 64 tensor-memory columns instead of 32, so a step
-// carries 2 groups and the rings are deeper (6 stages) to keep as many weight bytes
-// in flight.
-template <bool kBf16>
+// Pipeline shape per operand kind and group size.  A step carries PPS 128-wide K
+// planes (one packed weight block each) and the GQ quantisation groups they hold.
+// W4A8, group 128: INT8 token rows (128 bytes per row and plane), 4 planes per step.
+// Group 256: the same, 2 groups per step.  Group 64: 2 planes (4 groups) per step,
+// whose accumulators take as many columns as 4 planes of group 128, and 6 stages.
+// W4A16 (group 128): bf16 token rows (256 bytes per row and plane); a plane's
+// converted weights take 64 tensor-memory columns instead of 32, so a step carries
+// 2 planes and the rings are deeper (6 stages) to keep as many weight bytes in flight.
+template <bool kBf16, int GRP>
 struct DecCfg {
-    static constexpr int GPS = kBf16 ? 2 : 4;     // K groups per pipeline step
-    static constexpr int NS = kBf16 ? 6 : 4;      // shared-memory stages
-    static constexpr int NA = 2;                  // tensor-memory A slots
-    static constexpr int ND = NS;                 // tensor-memory accumulators (GPS x BN columns each)
-    static constexpr int NSC = kBf16 ? 8 : 6;     // scale ring slots (>= NA + ND)
-    static constexpr int kRowBytes = kBf16 ? 256 : 128;  // token row bytes per K group
-    static constexpr int kGCols = kBf16 ? 64 : 32;       // A columns per K group
-    static constexpr int kMmaK = kBf16 ? 16 : 32;        // K per MMA instruction
+    static_assert(!kBf16 || GRP == 128, "W4A16 uses group 128");
+    static constexpr int PPS = (kBf16 || GRP == 64) ? 2 : 4;  // K planes per pipeline step
+    static constexpr int GQ = PPS * 128 / GRP;                // quantisation groups per step
+    static constexpr int NS = (kBf16 || GRP == 64) ? 6 : 4;   // shared-memory stages
+    static constexpr int NA = 2;                              // tensor-memory A slots
+    static constexpr int ND = NS;                             // accumulators (GQ x BN columns each)
+    static constexpr int NSC = NS + NA;                       // scale ring slots (>= NA + ND)
+    static constexpr int kRowBytes = kBf16 ? 256 : 128;       // token row bytes per K plane
+    static constexpr int kGCols = kBf16 ? 64 : 32;            // A columns per K plane
+    static constexpr int kBlk = block_bytes_for(GRP);         // packed weight block
 };
 
 constexpr int BN = 16;    // tokens per tile (one 16-row block)
@@ -73,30 +84,30 @@ constexpr int kRegLaunch = 96;  // 65536 / 640, rounded down to the allocation u
 constexpr int kRegConv = 88, kRegCtrl = 48, kRegEpi = 128;
 static_assert(128 * (2 * kRegConv + kRegCtrl + 2 * kRegEpi) <= kRegLaunch * kThreads, "register split");
 
-template <bool kBf16>
+template <bool kBf16, int GRP>
 struct DecLayout {
-    using C = DecCfg<kBf16>;
-    static constexpr int GPS = C::GPS, NS = C::NS, NA = C::NA, ND = C::ND, NSC = C::NSC;
-    static constexpr int kAStage = GPS * kBlockBytes;        // weight blocks of one step
-    static constexpr int kBStage = GPS * BN * C::kRowBytes;  // token rows of one step
-    static constexpr int kACols = GPS * C::kGCols;
-    static constexpr int kDCols = GPS * BN;
+    using C = DecCfg<kBf16, GRP>;
+    static constexpr int PPS = C::PPS, GQ = C::GQ, NS = C::NS, NA = C::NA, ND = C::ND, NSC = C::NSC;
+    static constexpr int kAStage = PPS * C::kBlk;            // weight blocks of one step
+    static constexpr int kBStage = PPS * BN * C::kRowBytes;  // token rows of one step
+    static constexpr int kACols = PPS * C::kGCols;
+    static constexpr int kDCols = GQ * BN;
     static constexpr uint32_t kACol0 = 0;
     static constexpr uint32_t kDCol0 = NA * kACols;
     static_assert(kDCol0 + ND * kDCols <= kTmemCols, "tensor memory over-subscribed");
     static_assert(NSC >= NA + ND, "scale ring too small");
     static_assert(NS % 2 == 0, "the two producers own the stages of one parity each");
-    static_assert(GPS % 2 == 0, "the two MMA warps split the groups of a step");
+    static_assert(GQ % 2 == 0, "the two MMA warps split the groups of a step");
     // one "MMA of step j done" barrier per j % NS serves the stage ring, the A slots and
     // the accumulators: their rings must step together
     static_assert(ND == NS && NS % NA == 0, "shared completion ring");
     // shared memory carve-up (offsets from a 1024-aligned base)
     static constexpr int kOffB = 0;
     static constexpr int kOffA = kOffB + NS * kBStage;
-    static constexpr int kOffSc = kOffA + NS * kAStage;          // ring: fp32 scale       [NSC][GPS][128]
-    static constexpr int kOffZp = kOffSc + NSC * GPS * 128 * 4;  // ring: fp32 zero point  [NSC][GPS][128]
-    static constexpr int kOffS = kOffZp + NSC * GPS * 128 * 4;   // ring: token group sums [NSC][GPS][BN]
-    static constexpr int kOffX = kOffS + NSC * GPS * BN * 4;     // epilogue exchange: [2][128][BN] fp32
+    static constexpr int kOffSc = kOffA + NS * kAStage;         // ring: fp32 scale       [NSC][GQ][128]
+    static constexpr int kOffZp = kOffSc + NSC * GQ * 128 * 4;  // ring: fp32 zero point  [NSC][GQ][128]
+    static constexpr int kOffS = kOffZp + NSC * GQ * 128 * 4;   // ring: token group sums [NSC][GQ][BN]
+    static constexpr int kOffX = kOffS + NSC * GQ * BN * 4;     // epilogue exchange: [2][128][BN] fp32
     static constexpr int kOffReset = kOffX + 2 * 128 * BN * 4;   // the accumulator-reset operands
     static constexpr int kOffBar = kOffReset + 2 * kResetTileBytes;
     // full[NS] empty[NS] conv[NA] (unused: NA + ND) dempty[ND] side[NSC] final[2]
@@ -205,13 +216,14 @@ __device__ __forceinline__ void unpack2(uint64_t p, float& lo, float& hi) {
 
 __device__ __forceinline__ float silu_mul(float g, float u) { return __fdividef(g, 1.0f + __expf(-g)) * u; }
 
-template <bool kBf16>
+template <bool kBf16, int GRP>
 __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs a) {
-    using L = DecLayout<kBf16>;
-    constexpr int GPS = L::GPS, NS = L::NS, NA = L::NA, ND = L::ND, NSC = L::NSC;
+    using L = DecLayout<kBf16, GRP>;
+    constexpr int PPS = L::PPS, GQ = L::GQ, NS = L::NS, NA = L::NA, ND = L::ND, NSC = L::NSC;
     constexpr int kAStage = L::kAStage, kBStage = L::kBStage, kACols = L::kACols, kDCols = L::kDCols;
     constexpr uint32_t kACol0 = L::kACol0, kDCol0 = L::kDCol0;
-    constexpr int kRowBytes = DecCfg<kBf16>::kRowBytes, kGCols = DecCfg<kBf16>::kGCols;
+    constexpr int kRowBytes = DecCfg<kBf16, GRP>::kRowBytes, kGCols = DecCfg<kBf16, GRP>::kGCols;
+    constexpr int kBlk = DecCfg<kBf16, GRP>::kBlk;
     constexpr int kOffA = L::kOffA, kOffB = L::kOffB, kOffSc = L::kOffSc, kOffZp = L::kOffZp, kOffS = L::kOffS;
     constexpr int kOffX = L::kOffX, kOffReset = L::kOffReset, kOffBar = L::kOffBar, kOffMisc = L::kOffMisc;
     extern __shared__ uint8_t smem_raw[];
@@ -267,8 +279,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
 
     const int total = a.NT * __ldg(a.n_mtiles);
-    const int G = a.G;
-    const int steps_per_item = (G + GPS - 1) / GPS;
+    const int G = a.G;                 // 128-wide K planes (packed blocks) per tile
+    const int Gq = G * kGroup / GRP;   // quantisation groups per row
+    const int steps_per_item = (G + PPS - 1) / PPS;
 
     if (warp >= kCtrlWarp0) {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegCtrl));
@@ -281,19 +294,19 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
                 bool ok = true, rdy = false;  // rdy: an early test found this step's stage free
                 for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
                     const Item it = decode_item(u, a);
-                    const uint8_t* wsrc = a.wblocks + (size_t)(it.e * a.NT + it.nt) * G * kBlockBytes;
+                    const uint8_t* wsrc = a.wblocks + (size_t)(it.e * a.NT + it.nt) * G * kBlk;
                     const int8_t* bsrc = a.act + (size_t)(it.row0 / BN) * a.act_rb_stride;
                     for (int t = 0; t < steps_per_item; ++t, ++j) {
                         if ((int)(j & 1u) != pi) continue;
                         last = j + 1;
-                        const int g0 = t * GPS, ng = min(GPS, G - g0);
+                        const int g0 = t * PPS, ng = min(PPS, G - g0);
                         const int s = j % NS;
                         if (!rdy && !wait_bar(EMPTY_BAR(s), ((j / NS) & 1u) ^ 1u, abort_flag, a.err, a.wait_limit)) { ok = false; break; }
                         rdy = mbar_test(EMPTY_BAR((j + 2) % NS), (((j + 2) / NS) & 1u) ^ 1u);
                         // test hook: leave the first step's stage empty, so that its consumers time out
                         if (j == 0 && blockIdx.x == 0 && (a.debug & kDebugSkipFirstCopy)) continue;
-                        mbar_arrive_expect_tx(FULL_BAR(s), (uint32_t)ng * (kBlockBytes + BN * kRowBytes));
-                        bulk_g2s(sA + s * kAStage, wsrc + (size_t)g0 * kBlockBytes, ng * kBlockBytes, FULL_BAR(s));
+                        mbar_arrive_expect_tx(FULL_BAR(s), (uint32_t)ng * (kBlk + BN * kRowBytes));
+                        bulk_g2s(sA + s * kAStage, wsrc + (size_t)g0 * kBlk, ng * kBlk, FULL_BAR(s));
                         bulk_g2s(sB + s * kBStage, bsrc + (size_t)g0 * BN * kRowBytes, ng * BN * kRowBytes, FULL_BAR(s));
                     }
                 }
@@ -317,7 +330,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
                 const uint32_t idesc = kBf16 ? idesc_bf16(128, BN) : idesc_i8(128, BN, false);
                 for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
                     for (int t = 0; t < steps_per_item; ++t, ++j) {
-                        const int ng = min(GPS, G - t * GPS);
+                        const int nq = min(PPS, G - t * PPS) * kGroup / GRP;  // groups of this step
                         const int s = j % NS, x = j % NA, b = j % ND;
                         if (!conv_rdy && !wait_bar(CONV_BAR(x), (j / NA) & 1u, abort_flag, a.err, a.wait_limit)) { ok = false; break; }
                         if (!acc_rdy && !wait_bar(DEMPTY_BAR(b), ((j / ND) & 1u) ^ 1u, abort_flag, a.err, a.wait_limit)) { ok = false; break; }
@@ -328,17 +341,17 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
                         // W4A8: reset this warp's groups' INT32 accumulators to the magic
                         // pattern, then add the partials.  W4A16: the first MMA of a group
                         // overwrites its fp32 accumulator.
-                        if (!kBf16 && mi * (GPS / 2) < ng)
-                            mma_reset_acc(tmem_base + kDCol0 + (uint32_t)(b * kDCols + mi * (GPS / 2) * BN), sReset,
-                                          (GPS / 2) * BN);
+                        if (!kBf16 && mi * (GQ / 2) < nq)
+                            mma_reset_acc(tmem_base + kDCol0 + (uint32_t)(b * kDCols + mi * (GQ / 2) * BN), sReset,
+                                          (GQ / 2) * BN);
 #pragma unroll
-                        for (int gh = 0; gh < GPS / 2; ++gh) {
-                            const int gq = mi * (GPS / 2) + gh;
-                            if (gq < ng) {
+                        for (int gh = 0; gh < GQ / 2; ++gh) {
+                            const int gq = mi * (GQ / 2) + gh;
+                            if (gq < nq) {
                                 const uint32_t dt = tmem_base + kDCol0 + (uint32_t)(b * kDCols + gq * BN);
-                                const uint32_t at = tmem_base + kACol0 + (uint32_t)(x * kACols + gq * kGCols);
-                                const uint32_t sb = sB + s * kBStage + gq * BN * kRowBytes;
                                 if constexpr (kBf16) {
+                                    const uint32_t at = tmem_base + kACol0 + (uint32_t)(x * kACols + gq * kGCols);
+                                    const uint32_t sb = sB + s * kBStage + gq * BN * kRowBytes;
                                     // K = 16 per MMA: steps 0-3 in the group's first 64-column
                                     // plane of token rows, 4-7 in the second
 #pragma unroll
@@ -347,9 +360,15 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
                                                     smem_desc_sw128(sb + (kk >> 2) * BN * 128 + (kk & 3) * 32), idesc,
                                                     kk > 0 ? 1u : 0u);
                                 } else {
+                                    // the group's K range inside the step, 32 per MMA: plane
+                                    // ko / 128 of the token rows, A columns ko / 4
 #pragma unroll
-                                    for (int kk = 0; kk < 4; ++kk)
-                                        mma_i8_ts(dt, at + kk * 8, smem_desc_sw128(sb + kk * 32), idesc, 1u);
+                                    for (int kk = 0; kk < GRP / 32; ++kk) {
+                                        const int ko = gq * GRP + kk * 32;
+                                        mma_i8_ts(dt, tmem_base + kACol0 + (uint32_t)(x * kACols + ko / 4),
+                                                  smem_desc_sw128(sB + s * kBStage + (ko >> 7) * BN * 128 + (ko & 127)),
+                                                  idesc, 1u);
+                                    }
                                 }
                             }
                         }
@@ -371,15 +390,19 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegConv));
         const int cg = warp >> 2;
         const int r = threadIdx.x & 127;
-        // group sums: this thread adds half (64 bytes) of token m's row in group gs
-        const int gs = r >> 5, m = (r & 31) >> 1, half = r & 1;
+        // group sums: GQ groups x BN tokens x SP parts; this thread adds part `part` of
+        // token m's codes in group gs (with group 128: half a row, 64 bytes)
+        constexpr int SP = 128 / (GQ * BN);
+        static_assert(SP * GQ * BN == 128 && (SP == 2 || SP == 4), "group-sum split");
+        const int gs = r / (BN * SP), m = (r / SP) % BN, part = r % SP;
         uint32_t m28;
         asm volatile("mov.u32 %0, 0x10000000;" : "=r"(m28));  // x * 2^28 >> 32 = x >> 4, on the FMA pipe
         const int nsteps = ((total - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x) * steps_per_item;
         bool full_rdy = false;  // an early test of this step's stage
         for (int j = cg; j < nsteps; j += 2) {
             const int t = j % steps_per_item;
-            const int ng = min(GPS, G - t * GPS);
+            const int ng = min(PPS, G - t * PPS);  // planes of this step
+            const int nq = ng * kGroup / GRP;      // groups of this step
             const int s = j % NS, x = j % NA, slot = j % NSC;
             if (!full_rdy && !wait_bar(FULL_BAR(s), (j / NS) & 1u, abort_flag, a.err, a.wait_limit)) break;
             // A slot x was last read by the MMAs of step j - NA
@@ -388,12 +411,30 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
             if (j >= NA && !wait_bar(EMPTY_BAR((j - NA) % NS), ((j - NA) / NS) & 1u, abort_flag, a.err, a.wait_limit))
                 break;
             full_rdy = mbar_test(FULL_BAR((j + 2) % NS), ((j + 2) / NS) & 1u);  // this group's next step
-            for (int gq = 0; gq < ng; ++gq) {
-                const uint8_t* blk = smA + s * kAStage + gq * kBlockBytes;
+            for (int gq = 0; gq < ng; ++gq) {  // plane gq of the step
+                const uint8_t* blk = smA + s * kAStage + gq * kBlk;
                 uint4 w[4];
 #pragma unroll
                 for (int c = 0; c < 4; ++c) w[c] = *reinterpret_cast<const uint4*>(blk + code_chunk_offset(r, c));
-                sc_ring[(slot * GPS + gq) * 128 + r] = __half2float(reinterpret_cast<const __half*>(blk + kScaleOff)[r]);
+                // the scale and zero point of each group the plane starts (group 64: two,
+                // the second 512 bytes after the first; group 256: one on even planes)
+                const __half* shp = reinterpret_cast<const __half*>(blk + kScaleOff);
+                const __half* zhp = reinterpret_cast<const __half*>(blk + kZpOff);
+                if constexpr (GRP == 64) {
+#pragma unroll
+                    for (int sub = 0; sub < 2; ++sub) {
+                        sc_ring[(slot * GQ + 2 * gq + sub) * 128 + r] = __half2float(shp[r + sub * 256]);
+                        zp_ring[(slot * GQ + 2 * gq + sub) * 128 + r] = __half2float(zhp[r + sub * 256]);
+                    }
+                } else if constexpr (GRP == 256) {
+                    if ((gq & 1) == 0) {
+                        sc_ring[(slot * GQ + gq / 2) * 128 + r] = __half2float(shp[r]);
+                        zp_ring[(slot * GQ + gq / 2) * 128 + r] = __half2float(zhp[r]);
+                    }
+                } else {
+                    sc_ring[(slot * GQ + gq) * 128 + r] = __half2float(shp[r]);
+                    if (!kBf16) zp_ring[(slot * GQ + gq) * 128 + r] = __half2float(zhp[r]);
+                }
                 if constexpr (kBf16) {
                     // (code - zp) as bf16, exactly: the byte permute puts each code under
                     // the bf16 bits 0x43, giving 128 + code, and one packed bf16 FMA
@@ -421,26 +462,25 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
                         }
                         tmem_st32(tmem_base + lane_base + kACol0 + (uint32_t)(x * kACols + gq * kGCols + hh * 32), v);
                     }
-                    continue;
-                }
-                zp_ring[(slot * GPS + gq) * 128 + r] = __half2float(reinterpret_cast<const __half*>(blk + kZpOff)[r]);
-                uint32_t v[32];
+                } else {
+                    uint32_t v[32];
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const uint32_t xw[4] = {w[c].x, w[c].y, w[c].z, w[c].w};
+                    for (int c = 0; c < 4; ++c) {
+                        const uint32_t xw[4] = {w[c].x, w[c].y, w[c].z, w[c].w};
 #pragma unroll
-                    for (int qq = 0; qq < 4; ++qq) {
-                        const int i = 4 * c + qq;  // word i holds K = 8i .. 8i+7 of the group
-                        v[2 * i] = xw[qq] & 0x0F0F0F0Fu;
-                        v[2 * i + 1] = __umulhi(xw[qq], m28) & 0x0F0F0F0Fu;
+                        for (int qq = 0; qq < 4; ++qq) {
+                            const int i = 4 * c + qq;  // word i holds K = 8i .. 8i+7 of the plane
+                            v[2 * i] = xw[qq] & 0x0F0F0F0Fu;
+                            v[2 * i + 1] = __umulhi(xw[qq], m28) & 0x0F0F0F0Fu;
+                        }
                     }
+                    tmem_st32(tmem_base + lane_base + kACol0 + (uint32_t)(x * kACols + gq * 32), v);
                 }
-                tmem_st32(tmem_base + lane_base + kACol0 + (uint32_t)(x * kACols + gq * 32), v);
             }
-            if (!kBf16 && gs < ng) {
+            if (GRP == 128 && !kBf16 && gs < nq) {
                 // S[gs][m] = sum of token m's 128 INT8 codes of group gs (the swizzle only
                 // permutes the 16-byte chunks inside the row, so the row sum is unaffected)
-                const uint4* rowp = reinterpret_cast<const uint4*>(smB + s * kBStage + gs * BN * kRowBytes + m * 128 + half * 64);
+                const uint4* rowp = reinterpret_cast<const uint4*>(smB + s * kBStage + gs * BN * kRowBytes + m * 128 + part * 64);
                 int sum = 0;
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
@@ -451,7 +491,24 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
                     sum = __dp4a((int)b4.w, 0x01010101, sum);
                 }
                 sum += __shfl_xor_sync(0xffffffffu, sum, 1);
-                if (half == 0) s_ring[(slot * GPS + gs) * BN + m] = (float)sum;
+                if (part == 0) s_ring[(slot * GQ + gs) * BN + m] = (float)sum;
+            } else if (GRP != 128 && gs < nq) {
+                // S[gs][m] over the group's K range, SP parts of GRP / SP codes each: logical
+                // 16-byte chunk c of token row m sits at chunk position c ^ (m & 7)
+                int sum = 0;
+#pragma unroll
+                for (int c = 0; c < GRP / SP / 16; ++c) {
+                    const int k = gs * GRP + part * (GRP / SP) + 16 * c;  // K offset in the step
+                    const uint4 b4 = *reinterpret_cast<const uint4*>(smB + s * kBStage + (k >> 7) * BN * 128 + m * 128 +
+                                                                     ((((k & 127) >> 4) ^ (m & 7)) << 4));
+                    sum = __dp4a((int)b4.x, 0x01010101, sum);
+                    sum = __dp4a((int)b4.y, 0x01010101, sum);
+                    sum = __dp4a((int)b4.z, 0x01010101, sum);
+                    sum = __dp4a((int)b4.w, 0x01010101, sum);
+                }
+#pragma unroll
+                for (int o = 1; o < SP; o <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+                if (part == 0) s_ring[(slot * GQ + gs) * BN + m] = (float)sum;
             }
             tmem_st_wait();
             tc_fence_before();
@@ -482,16 +539,16 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
             const uint64_t m2 = splat2(kMagicF);
             const int n_out = (a.mode == 1) ? -1 : it.nt * kTileRows + r;
             for (int t = 0; t < steps_per_item; ++t, ++j) {
-                const int ng = min(GPS, G - t * GPS);
+                const int nq = min(PPS, G - t * PPS) * kGroup / GRP;  // groups of this step
                 const int b = j % ND, slot = j % NSC;
                 if (!acc_rdy && !wait_bar(EMPTY_BAR(j % NS), (j / NS) & 1u, abort_flag, a.err, a.wait_limit)) { ok = false; break; }
                 acc_rdy = mbar_test(EMPTY_BAR((j + 1) % NS), ((j + 1) / NS) & 1u);
                 tc_fence_after();
                 const uint32_t taddr = tmem_base + lane_base + kDCol0 + (uint32_t)(b * kDCols);
-                uint32_t v[GPS / 2][BN];
+                uint32_t v[GQ / 2][BN];
 #pragma unroll
-                for (int gh = 0; gh < GPS / 2; ++gh)
-                    if (eh * (GPS / 2) + gh < ng) tmem_ld16(taddr + (eh * (GPS / 2) + gh) * BN, v[gh]);
+                for (int gh = 0; gh < GQ / 2; ++gh)
+                    if (eh * (GQ / 2) + gh < nq) tmem_ld16(taddr + (eh * (GQ / 2) + gh) * BN, v[gh]);
                 tmem_ld_wait();
                 tc_fence_before();
                 __syncwarp();
@@ -499,18 +556,18 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
                 if (!side_rdy && !wait_bar(SIDE_BAR(slot), (j / NSC) & 1u, abort_flag, a.err, a.wait_limit)) { ok = false; break; }
                 side_rdy = mbar_test(SIDE_BAR((j + 1) % NSC), ((j + 1) / NSC) & 1u);
 #pragma unroll
-                for (int gh = 0; gh < GPS / 2; ++gh) {
-                    const int gq = eh * (GPS / 2) + gh;
-                    if (kBf16 && gq < ng) {
+                for (int gh = 0; gh < GQ / 2; ++gh) {
+                    const int gq = eh * (GQ / 2) + gh;
+                    if (kBf16 && gq < nq) {
                         // fp32 partials: acc += scale * D
-                        const uint64_t sc2 = splat2(sc_ring[(slot * GPS + gq) * 128 + r]);
+                        const uint64_t sc2 = splat2(sc_ring[(slot * GQ + gq) * 128 + r]);
 #pragma unroll
                         for (int i = 0; i < BN; i += 2) fold2_f32(acc2[i / 2], sc2, v[gh][i], v[gh][i + 1]);
-                    } else if (!kBf16 && gq < ng) {
-                        const float zpf = zp_ring[(slot * GPS + gq) * 128 + r];
-                        const uint64_t sc2 = splat2(sc_ring[(slot * GPS + gq) * 128 + r]);
+                    } else if (!kBf16 && gq < nq) {
+                        const float zpf = zp_ring[(slot * GQ + gq) * 128 + r];
+                        const uint64_t sc2 = splat2(sc_ring[(slot * GQ + gq) * 128 + r]);
                         const uint64_t nzp2 = splat2(-zpf);
-                        const float4* sp = reinterpret_cast<const float4*>(s_ring + (slot * GPS + gq) * BN);
+                        const float4* sp = reinterpret_cast<const float4*>(s_ring + (slot * GQ + gq) * BN);
                         float sg[BN];
 #pragma unroll
                         for (int i = 0; i < BN / 4; ++i) {
@@ -518,8 +575,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
                             sg[4 * i] = f4.x; sg[4 * i + 1] = f4.y; sg[4 * i + 2] = f4.z; sg[4 * i + 3] = f4.w;
                         }
                         if (a.partials != nullptr && n_out < a.nvalid) {
-                            int32_t* pp = a.partials + ((size_t)it.row0 * a.nvalid + n_out) * G + t * GPS + gq;
-                            const size_t pstride = (size_t)a.nvalid * G;
+                            int32_t* pp = a.partials + ((size_t)it.row0 * a.nvalid + n_out) * Gq + t * GQ + gq;
+                            const size_t pstride = (size_t)a.nvalid * Gq;
 #pragma unroll
                             for (int i = 0; i < BN; ++i)
                                 if (i < it.nrows)
@@ -623,34 +680,37 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
 int gemm_decode_tile_tokens() { return BN; }
 
 namespace {
-template <bool kBf16>
+template <bool kBf16, int GRP>
 cudaError_t launch_decode(const GemmArgs& a, int num_ctas, cudaStream_t stream) {
-    constexpr int kSmem = DecLayout<kBf16>::kSmemBytes;
+    constexpr int kSmem = DecLayout<kBf16, GRP>::kSmemBytes;
     static int attr_done[64] = {0};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64 || !attr_done[dev]) {
         // the register split assumes kRegLaunch registers per thread at launch
         cudaFuncAttributes fa;
-        cudaError_t e = cudaFuncGetAttributes(&fa, gemm_decode_kernel<kBf16>);
+        cudaError_t e = cudaFuncGetAttributes(&fa, gemm_decode_kernel<kBf16, GRP>);
         if (e != cudaSuccess) return e;
         if (fa.numRegs != kRegLaunch) return cudaErrorInvalidConfiguration;
-        e = cudaFuncSetAttribute(gemm_decode_kernel<kBf16>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+        e = cudaFuncSetAttribute(gemm_decode_kernel<kBf16, GRP>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
         if (e != cudaSuccess) return e;
         if (dev >= 0 && dev < 64) attr_done[dev] = 1;
     }
-    gemm_decode_kernel<kBf16><<<num_ctas, kThreads, kSmem, stream>>>(a);
+    gemm_decode_kernel<kBf16, GRP><<<num_ctas, kThreads, kSmem, stream>>>(a);
     return cudaGetLastError();
 }
 }  // namespace
 
 cudaError_t launch_gemm_decode(const GemmArgs& a, int num_ctas, cudaStream_t stream) {
-    return launch_decode<false>(a, num_ctas, stream);
+    if (a.group == 64) return launch_decode<false, 64>(a, num_ctas, stream);
+    if (a.group == 256) return launch_decode<false, 256>(a, num_ctas, stream);
+    return launch_decode<false, 128>(a, num_ctas, stream);
 }
 
 cudaError_t launch_gemm_w4a16(const GemmArgs& a, int num_ctas, cudaStream_t stream) {
-    if (a.partials != nullptr || (a.mode == 1 && a.out16 == nullptr)) return cudaErrorInvalidValue;
-    return launch_decode<true>(a, num_ctas, stream);
+    if (a.partials != nullptr || (a.mode == 1 && a.out16 == nullptr) || (a.group != 0 && a.group != 128))
+        return cudaErrorInvalidValue;
+    return launch_decode<true, 128>(a, num_ctas, stream);
 }
 
 }  // namespace w4a8

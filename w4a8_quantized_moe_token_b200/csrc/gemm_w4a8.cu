@@ -57,9 +57,11 @@ constexpr float kMagicF = 12582912.0f;
 //   NS    : shared-memory stages        NA : tensor-memory A slots
 //   ND    : INT32 accumulators          NEPI: epilogue warpgroups (split the columns)
 //   NCG   : converter warpgroups (they take alternate steps)
-template <int BN_, int NS_, int NA_, int ND_, int NEPI_, int NCG_>
+//   GRP   : weights per scale along K (64, 128 or 256; a step is always one 128-wide plane)
+template <int BN_, int NS_, int NA_, int ND_, int NEPI_, int NCG_, int GRP_ = 128>
 struct Cfg {
-    static constexpr int BN = BN_, NS = NS_, NA = NA_, ND = ND_, NEPI = NEPI_, NCG = NCG_;
+    static constexpr int BN = BN_, NS = NS_, NA = NA_, ND = ND_, NEPI = NEPI_, NCG = NCG_, GRP = GRP_;
+    static constexpr int kBlk = block_bytes_for(GRP);  // packed weight block of one plane
     static constexpr int kNSC = 16;       // scale ring slots (>= NA + ND + 4)
     static constexpr int kCW = BN / NEPI;  // accumulator columns per epilogue thread
     // warpgroups: NCG converter groups, NEPI epilogue groups, 1 control group
@@ -88,7 +90,7 @@ struct Cfg {
     // shared memory carve-up
     static constexpr int kOffB = 0;  // 1024-aligned (128-byte swizzle atoms)
     static constexpr int kOffA = kOffB + NS * kBStageBytes;
-    static constexpr int kOffSc = kOffA + NS * kBlockBytes;  // ring: fp32 scale per row
+    static constexpr int kOffSc = kOffA + NS * kBlk;  // ring: fp32 scale per row and group
     static constexpr int kOffReset = kOffSc + kNSC * kTileRows * 4;  // the accumulator-reset operands
     // output staging tile: fp32 [BN tokens][128 channels] (plain output) or
     // [BN tokens][kStageH] (SwiGLU output, 64 channels + padding against bank conflicts)
@@ -191,6 +193,9 @@ __device__ __forceinline__ float silu_mul(float g, float u) { return __fdividef(
 template <class C, bool kPartials>
 __global__ void __launch_bounds__(C::kThreads, 1) gemm_w4a8_kernel(const GemmArgs a) {
     constexpr int BN = C::BN, NS = C::NS, NA = C::NA, ND = C::ND, kNSC = C::kNSC, kCW = C::kCW;
+    constexpr int GRP = C::GRP, kBlk = C::kBlk;
+    // groups per plane (group 64) and planes per group (group 256)
+    constexpr int kGPP = GRP < kGroup ? kGroup / GRP : 1, kPPG = GRP > kGroup ? GRP / kGroup : 1;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
     const uint32_t base_addr = (raw_addr + 1023u) & ~1023u;
@@ -243,7 +248,8 @@ __global__ void __launch_bounds__(C::kThreads, 1) gemm_w4a8_kernel(const GemmArg
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
 
     const int total = a.NT * __ldg(a.n_mtiles);
-    const int G = a.G;
+    const int G = a.G;                // 128-wide K planes (steps) per tile
+    const int Gq = G * kGroup / GRP;  // quantisation groups per tile
 
     // each role first moves its warpgroup's register budget (converter and control
     // groups give registers to the epilogue groups), then runs
@@ -261,7 +267,7 @@ __global__ void __launch_bounds__(C::kThreads, 1) gemm_w4a8_kernel(const GemmArg
             for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
                 const Item it = decode_item<BN>(u, a);
                 const uint32_t bbytes = (uint32_t)round_up(it.nrows, 16) * 128u;
-                const uint8_t* wsrc = a.wblocks + (size_t)(it.e * a.NT + it.nt) * G * kBlockBytes;
+                const uint8_t* wsrc = a.wblocks + (size_t)(it.e * a.NT + it.nt) * G * kBlk;
                 const int8_t* asrc = a.act + (size_t)it.row0 * 128;
                 for (int g = 0; g < G; ++g, ++j) {
                     if ((int)(j & 1u) != pi) continue;
@@ -271,8 +277,8 @@ __global__ void __launch_bounds__(C::kThreads, 1) gemm_w4a8_kernel(const GemmArg
                     rdy = mbar_test(EMPTY_BAR((j + 2) % NS), (((j + 2) / NS) & 1u) ^ 1u);
                     // test hook: leave the first step's stage empty, so that its consumers time out
                     if (j == 0 && blockIdx.x == 0 && (a.debug & kDebugSkipFirstCopy)) continue;
-                    mbar_arrive_expect_tx(FULL_BAR(s), kBlockBytes + bbytes);
-                    bulk_g2s(sA + s * kBlockBytes, wsrc + (size_t)g * kBlockBytes, kBlockBytes, FULL_BAR(s));
+                    mbar_arrive_expect_tx(FULL_BAR(s), kBlk + bbytes);
+                    bulk_g2s(sA + s * kBlk, wsrc + (size_t)g * kBlk, kBlk, FULL_BAR(s));
                     bulk_g2s(sB + s * C::kBStageBytes, asrc + (size_t)g * a.act_plane, bbytes, FULL_BAR(s));
                 }
             }
@@ -296,7 +302,11 @@ __global__ void __launch_bounds__(C::kThreads, 1) gemm_w4a8_kernel(const GemmArg
             __syncwarp();
             if (lane == 0) {
                 mbar_arrive(CONV_BAR(jp % NA));
-                mbar_arrive(SCFULL_BAR(jp % kNSC));
+                // the scales of the groups that start in plane jp
+                if (kPPG == 1 || jp % kPPG == 0) {
+#pragma unroll
+                    for (int sub = 0; sub < kGPP; ++sub) mbar_arrive(SCFULL_BAR((jp * kGPP / kPPG + sub) % kNSC));
+                }
             }
         };
         bool full_rdy = false, aslot_rdy = false;  // early tests of this step's barriers
@@ -310,22 +320,33 @@ __global__ void __launch_bounds__(C::kThreads, 1) gemm_w4a8_kernel(const GemmArg
                 full_rdy = mbar_test(FULL_BAR(jn % NS), (jn / NS) & 1u);
                 aslot_rdy = mbar_test(AEMPTY_BAR(jn % NA), ((jn / NA) & 1u) ^ 1u);
             }
-            const uint8_t* blk = smA + s * kBlockBytes;
+            const uint8_t* blk = smA + s * kBlk;
             uint4 w[4];
 #pragma unroll
             for (int c = 0; c < 4; ++c) w[c] = *reinterpret_cast<const uint4*>(blk + code_chunk_offset(r, c));
-            const int zp = (int)__half2float(reinterpret_cast<const __half*>(blk + kZpOff)[r]);
-            sc_ring[(j % kNSC) * kTileRows + r] = __half2float(reinterpret_cast<const __half*>(blk + kScaleOff)[r]);
+            // zero point of each half plane (one group 64 per half; else the plane's group)
+            int zp[2];
+            zp[0] = (int)__half2float(reinterpret_cast<const __half*>(blk + kZpOff)[r]);
+            zp[1] = kGPP == 2 ? (int)__half2float(reinterpret_cast<const __half*>(blk + kZpOff + 512)[r]) : zp[0];
+            // the scales of the groups that start in this plane
+            if (kPPG == 1 || j % kPPG == 0) {
+#pragma unroll
+                for (int sub = 0; sub < kGPP; ++sub)
+                    sc_ring[((j * kGPP / kPPG + sub) % kNSC) * kTileRows + r] =
+                        __half2float(reinterpret_cast<const __half*>(blk + kScaleOff + sub * 512)[r]);
+            }
             uint32_t v[32];
             {
                 // signed INT8 (code - zp): byte-wise (code + 128 - zp) ^ 128, no carries
-                const uint32_t nz = (uint32_t)(0x80 - zp) * 0x01010101u;
+                const uint32_t nz0 = (uint32_t)(0x80 - zp[0]) * 0x01010101u;
+                const uint32_t nz1 = (uint32_t)(0x80 - zp[1]) * 0x01010101u;
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     const uint32_t xw[4] = {w[c].x, w[c].y, w[c].z, w[c].w};
+                    const uint32_t nz = c < 2 ? nz0 : nz1;  // chunks 0-1: K 0..63, 2-3: K 64..127
 #pragma unroll
                     for (int qq = 0; qq < 4; ++qq) {
-                        const int i = 4 * c + qq;  // word i holds K = 8i .. 8i+7 of the group
+                        const int i = 4 * c + qq;  // word i holds K = 8i .. 8i+7 of the plane
                         v[2 * i] = ((xw[qq] & 0x0F0F0F0Fu) + nz) ^ 0x80808080u;
                         v[2 * i + 1] = (((xw[qq] >> 4) & 0x0F0F0F0Fu) + nz) ^ 0x80808080u;
                     }
@@ -349,6 +370,41 @@ __global__ void __launch_bounds__(C::kThreads, 1) gemm_w4a8_kernel(const GemmArg
                 const int ncols = round_up(it.nrows, 16);
                 const uint32_t idesc = idesc_i8(128, ncols);
                 for (int g = 0; g < G; ++g, ++j) {
+                    if constexpr (GRP != kGroup) {
+                        // group 64: two accumulators per plane; group 256: the two planes of a
+                        // group go to the same warp and accumulator.  Plain waits.
+                        if ((int)((j / kPPG) & 1u) != mi) continue;
+                        const int s = j % NS, x = j % NA;
+                        const bool starts = kPPG == 1 || j % kPPG == 0;  // a group starts in this plane
+                        if (!wait_bar(CONV_BAR(x), (j / NA) & 1u, abort_flag, a.err, a.wait_limit)) { ok = false; break; }
+                        if (starts) {
+#pragma unroll
+                            for (int sub = 0; sub < kGPP; ++sub) {
+                                const uint32_t qg = j * kGPP / kPPG + sub;
+                                if (ok && !wait_bar(DEMPTY_BAR(qg % ND), ((qg / ND) & 1u) ^ 1u, abort_flag, a.err, a.wait_limit))
+                                    ok = false;
+                            }
+                            if (!ok) break;
+                        }
+                        tc_fence_after();
+                        const uint32_t at = tmem_base + C::kACol0 + (uint32_t)x * 32u;
+                        const uint32_t sb = sB + s * C::kBStageBytes;
+                        if (elect_one()) {
+#pragma unroll
+                            for (int kk = 0; kk < 4; ++kk) {
+                                const uint32_t kg = j * (uint32_t)kGroup + kk * 32u;  // K position of the MMA
+                                const uint32_t qg = kg / GRP;                          // its group
+                                const uint32_t dt = tmem_base + C::kDCol0 + (qg % ND) * BN;
+                                if (kg % GRP == 0) mma_reset_acc(dt, sReset, ncols);
+                                mma_i8_ts(dt, at + kk * 8, smem_desc_sw128(sb + kk * 32), idesc, 1u);
+                                if ((kg + 32u) % GRP == 0) tc_commit(DFULL_BAR(qg % ND));
+                            }
+                            tc_commit(EMPTY_BAR(s));
+                            tc_commit(AEMPTY_BAR(x));
+                        }
+                        __syncwarp();
+                        continue;
+                    }
                     if ((int)(j & 1u) != mi) continue;
                     const int s = j % NS, x = j % NA, b = j % ND;
                     if (!conv_rdy && !wait_bar(CONV_BAR(x), (j / NA) & 1u, abort_flag, a.err, a.wait_limit)) { ok = false; break; }
@@ -406,7 +462,54 @@ __global__ void __launch_bounds__(C::kThreads, 1) gemm_w4a8_kernel(const GemmArg
             for (int i = 0; i < kCW / 2; ++i) acc2[i] = 0ull;
             const uint64_t m2 = splat2(kMagicF);
             const int n_out = (a.mode == 1) ? -1 : it.nt * kTileRows + r;
-            for (int g = 0; g < G; ++g, ++j) {
+            if constexpr (GRP != kGroup) {
+                // one pass per quantisation group (j counts groups here); plain waits
+                for (int g = 0; g < Gq; ++g, ++j) {
+                    const int b = j % ND;
+                    if (!wait_bar(SCFULL_BAR(j % kNSC), (j / kNSC) & 1u, abort_flag, a.err, a.wait_limit)) { ok = false; break; }
+                    const uint64_t sc2 = splat2(sc_ring[(j % kNSC) * kTileRows + r]);
+                    if (!wait_bar(DFULL_BAR(b), (j / ND) & 1u, abort_flag, a.err, a.wait_limit)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t taddr = tmem_base + lane_base + C::kDCol0 + (uint32_t)b * BN + col0;
+                    if constexpr (!kPartials) {
+                        static_assert(kCW == 64, "64 columns per epilogue thread");
+                        uint32_t v[64];
+                        tmem_ld32(taddr, v);
+                        tmem_ld_wait();
+                        tmem_ld32(taddr + 32, v + 32);
+#pragma unroll
+                        for (int i = 0; i < 32; i += 2) fold2_packed(acc2[i / 2], sc2, m2, v[i], v[i + 1]);
+                        tmem_ld_wait();
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(DEMPTY_BAR(b));
+#pragma unroll
+                        for (int i = 32; i < 64; i += 2) fold2_packed(acc2[i / 2], sc2, m2, v[i], v[i + 1]);
+                    } else {
+#pragma unroll
+                        for (int rd = 0; rd < kCW / 16; ++rd) {
+                            const int m0 = col0 + rd * 16;
+                            uint32_t v[16];
+                            tmem_ld16(taddr + rd * 16, v);
+                            tmem_ld_wait();
+                            if (n_out < a.nvalid) {
+                                int32_t* pp = a.partials + ((size_t)(it.row0 + m0) * a.nvalid + n_out) * Gq + g;
+                                const size_t pstride = (size_t)a.nvalid * Gq;
+#pragma unroll
+                                for (int i = 0; i < 16; ++i)
+                                    if (m0 + i < it.nrows) pp[i * pstride] = (int32_t)(v[i] - kMagicBits);
+                            }
+#pragma unroll
+                            for (int i = 0; i < 16; i += 2)
+                                fold2_packed(acc2[(rd * 16 + i) / 2], sc2, m2, v[i], v[i + 1]);
+                        }
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(DEMPTY_BAR(b));
+                    }
+                }
+            }
+            for (int g = 0; g < (GRP == kGroup ? G : 0); ++g, ++j) {
                 const int b = j % ND;
                 // the scales come in blocks of four steps: one wait on the last step of
                 // the block (of each converter group, which work in step order) covers all four
@@ -598,6 +701,9 @@ __global__ void __launch_bounds__(C::kThreads, 1) gemm_w4a8_kernel(const GemmArg
 #undef STAGE_BAR
 
 using CfgLarge = Cfg<128, 6, 4, 3, 2, 1>;  // many tokens per expert
+// the other group sizes (group 64's larger blocks leave room for 4 stages)
+using CfgLarge64 = Cfg<128, 4, 4, 3, 2, 1, 64>;
+using CfgLarge256 = Cfg<128, 6, 4, 3, 2, 1, 256>;
 
 template <class C, bool kPartials>
 cudaError_t launch_cfg(const GemmArgs& a, int num_ctas, cudaStream_t stream) {
@@ -628,6 +734,12 @@ int gemm_tile_tokens(int avg_tokens_per_expert) { return avg_tokens_per_expert <
 cudaError_t launch_gemm(const GemmArgs& a, int tile_tokens, int num_ctas, cudaStream_t stream) {
     if (tile_tokens == 16) return launch_gemm_decode(a, num_ctas, stream);
     // the INT32-partials output (a parity check of the dense entry point) has its own instance
+    if (a.group == 64)
+        return a.partials != nullptr ? launch_cfg<CfgLarge64, true>(a, num_ctas, stream)
+                                     : launch_cfg<CfgLarge64, false>(a, num_ctas, stream);
+    if (a.group == 256)
+        return a.partials != nullptr ? launch_cfg<CfgLarge256, true>(a, num_ctas, stream)
+                                     : launch_cfg<CfgLarge256, false>(a, num_ctas, stream);
     if (a.partials != nullptr) return launch_cfg<CfgLarge, true>(a, num_ctas, stream);
     return launch_cfg<CfgLarge, false>(a, num_ctas, stream);
 }

@@ -32,15 +32,41 @@ __device__ __forceinline__ float warp_sum(float v) {
 }
 
 // ---------------------------------------------------------------------------
-// a1: weight quantisation + packing.  One block per (group g, tile t, matrix e);
-// thread r quantises tiled row r's 128 weights of group g.
+// a1: weight quantisation + packing.  One block per (group gq, tile t, matrix e);
+// thread r quantises tiled row r's GRP weights of group gq, 64 at a time: a first
+// pass over the group finds its range, a second one (re-reading the row from cache)
+// computes the codes and writes them into the group's 128-wide plane blocks.
 // ---------------------------------------------------------------------------
-// sym: 0 asymmetric min/max, 1 symmetric, 2 asymmetric on the 0.1th..99.9th percentile range
+// 64 weights of a row from K index k0 on (zero past K and for rows past N)
+__device__ __forceinline__ void load_w64(const uint16_t* row, int K, int k0, float (&v)[64]) {
+    if (row != nullptr && (K & 7) == 0 && k0 + 64 <= K) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const uint4 p = *reinterpret_cast<const uint4*>(row + k0 + 8 * i);
+            const uint32_t pw[4] = {p.x, p.y, p.z, p.w};
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                v[8 * i + 2 * h] = bf16_to_f32((uint16_t)(pw[h] & 0xFFFFu));
+                v[8 * i + 2 * h + 1] = bf16_to_f32((uint16_t)(pw[h] >> 16));
+            }
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 64; ++i) v[i] = (row != nullptr && k0 + i < K) ? bf16_to_f32(row[k0 + i]) : 0.f;
+    }
+}
+
+// sym: 0 asymmetric min/max, 1 symmetric, 2 asymmetric on the 0.1th..99.9th percentile
+// range (128-value groups only); G = 128-wide planes per row
+template <int GRP>
 __global__ void __launch_bounds__(128) pack_kernel(const uint16_t* __restrict__ w, int N, int K, int layout, int sym,
                                                    int NT, int G, uint8_t* __restrict__ blocks,
                                                    uint8_t* __restrict__ codes_out, uint16_t* __restrict__ scale_out,
                                                    uint16_t* __restrict__ zp_out) {
-    const int g = blockIdx.x, t = blockIdx.y, e = blockIdx.z;
+    constexpr int kChunks = GRP / 64;
+    constexpr int kBB = block_bytes_for(GRP);
+    const int gq = blockIdx.x, t = blockIdx.y, e = blockIdx.z;
+    const int Gq = G * kGroup / GRP;
     const int r = threadIdx.x;
     int src;
     bool valid;
@@ -53,132 +79,134 @@ __global__ void __launch_bounds__(128) pack_kernel(const uint16_t* __restrict__ 
         src = t * kTileRows + r;
         valid = src < N;
     }
-    float v[kGroup];
-    const int k0 = g * kGroup;
-    if (valid) {
-        const uint16_t* row = w + ((size_t)e * N + src) * (size_t)K;
-        if ((K & 7) == 0 && k0 + kGroup <= K) {
-#pragma unroll
-            for (int i = 0; i < kGroup / 8; ++i) {
-                const uint4 p = *reinterpret_cast<const uint4*>(row + k0 + 8 * i);
-                const uint32_t pw[4] = {p.x, p.y, p.z, p.w};
-#pragma unroll
-                for (int h = 0; h < 4; ++h) {
-                    v[8 * i + 2 * h] = bf16_to_f32((uint16_t)(pw[h] & 0xFFFFu));
-                    v[8 * i + 2 * h + 1] = bf16_to_f32((uint16_t)(pw[h] >> 16));
-                }
-            }
-        } else {
-#pragma unroll
-            for (int i = 0; i < kGroup; ++i) v[i] = (k0 + i < K) ? bf16_to_f32(row[k0 + i]) : 0.f;
-        }
-    } else {
-#pragma unroll
-        for (int i = 0; i < kGroup; ++i) v[i] = 0.f;
-    }
+    const uint16_t* row = valid ? w + ((size_t)e * N + src) * (size_t)K : nullptr;
+    float v[64];
     __half sh;
     int zp;
-    uint32_t code[kGroup];
     if (sym != 1) {
         float lo, hi;
-        if (sym == 2) {
-            // the 0.1th and 99.9th percentiles of the group: linear interpolation
-            // between the order statistics around positions 0.127 and 126.873, so
-            // only the two smallest and the two largest values are needed
-            float a0 = v[0], a1 = INFINITY, b0 = v[0], b1 = -INFINITY;  // a0 <= a1 smallest, b0 >= b1 largest
+        // min / max, and the two smallest and two largest values (a0 <= a1, b0 >= b1)
+        float mn0 = INFINITY, mx0 = -INFINITY;
+        float a0 = INFINITY, a1 = INFINITY, b0 = -INFINITY, b1 = -INFINITY;
+#pragma unroll 1
+        for (int c = 0; c < kChunks; ++c) {
+            load_w64(row, K, gq * GRP + c * 64, v);
 #pragma unroll
-            for (int i = 1; i < kGroup; ++i) {
-                a1 = fminf(a1, fmaxf(v[i], a0));
-                a0 = fminf(a0, v[i]);
-                b1 = fmaxf(b1, fminf(v[i], b0));
-                b0 = fmaxf(b0, v[i]);
+            for (int i = 0; i < 64; ++i) {
+                mn0 = fminf(mn0, v[i]);
+                mx0 = fmaxf(mx0, v[i]);
+                if (sym == 2) {
+                    a1 = fminf(a1, fmaxf(v[i], a0));
+                    a0 = fminf(a0, v[i]);
+                    b1 = fmaxf(b1, fminf(v[i], b0));
+                    b0 = fmaxf(b0, v[i]);
+                }
             }
+        }
+        if (sym == 2) {
+            // the 0.1th and 99.9th percentiles of a 128-value group: linear interpolation
+            // between the order statistics around positions 0.127 and 126.873
             lo = __fadd_rn(a0, __fmul_rn(0.127f, __fsub_rn(a1, a0)));
             hi = __fadd_rn(b1, __fmul_rn(0.873f, __fsub_rn(b0, b1)));
         } else {
-            lo = v[0];
-            hi = v[0];
-#pragma unroll
-            for (int i = 1; i < kGroup; ++i) {
-                lo = fminf(lo, v[i]);
-                hi = fmaxf(hi, v[i]);
-            }
+            lo = mn0;
+            hi = mx0;
         }
         // range widened to contain 0
         const float mn = fminf(lo, 0.f), mx = fmaxf(hi, 0.f);
         // scale = (max - min) / (2^4 - 1), stored as fp16; the fp16 value is the one used
         sh = __float2half_rn(__fdiv_rn(__fsub_rn(mx, mn), 15.0f));
         if (__half2float(sh) == 0.f) sh = __float2half_rn(1.0f);
-        const float shf = __half2float(sh);
         // zero_point = round(-min / scale)
-        zp = (int)fminf(fmaxf(rintf(__fdiv_rn(-mn, shf)), 0.f), 15.f);
-        // index = clamp(round(w / scale) + zero_point, 0, 15)
-#pragma unroll
-        for (int i = 0; i < kGroup; ++i) {
-            const int c = (int)rintf(__fdiv_rn(v[i], shf)) + zp;
-            code[i] = (uint32_t)min(max(c, 0), 15);
-        }
+        zp = (int)fminf(fmaxf(rintf(__fdiv_rn(-mn, __half2float(sh))), 0.f), 15.f);
     } else {
-        // symmetric (b = 4): scale = max|w| / (2^3 - 1), q = clamp(round(w / scale), -7, 7),
-        // stored as code q + 8 with zero point 8
+        // symmetric (b = 4): scale = max|w| / (2^3 - 1), stored as code q + 8 with zero point 8
         float amax = 0.f;
+#pragma unroll 1
+        for (int c = 0; c < kChunks; ++c) {
+            load_w64(row, K, gq * GRP + c * 64, v);
 #pragma unroll
-        for (int i = 0; i < kGroup; ++i) amax = fmaxf(amax, fabsf(v[i]));
+            for (int i = 0; i < 64; ++i) amax = fmaxf(amax, fabsf(v[i]));
+        }
         sh = __float2half_rn(__fdiv_rn(amax, 7.0f));
         if (__half2float(sh) == 0.f) sh = __float2half_rn(1.0f);
-        const float shf = __half2float(sh);
         zp = 8;
-#pragma unroll
-        for (int i = 0; i < kGroup; ++i) {
-            const int q = (int)rintf(__fdiv_rn(v[i], shf));
-            code[i] = (uint32_t)(min(max(q, -7), 7) + 8);
-        }
     }
-    // tiled block: word i (K = 8i..8i+7): byte b = code[8i+b] | code[8i+4+b] << 4
-    uint8_t* blk = blocks + ((size_t)(e * NT + t) * G + g) * kBlockBytes;
+    const float shf = __half2float(sh);
+    const size_t tile_blk = (size_t)(e * NT + t) * G;
+#pragma unroll 1
+    for (int c = 0; c < kChunks; ++c) {
+        const int k0 = gq * GRP + c * 64;  // K index of this chunk's first weight
+        load_w64(row, K, k0, v);
+        uint32_t code[64];
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-        uint32_t wd[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const int i = 4 * c + q;
-            uint32_t x = 0;
-#pragma unroll
-            for (int b = 0; b < 4; ++b) x |= (code[8 * i + b] | (code[8 * i + 4 + b] << 4)) << (8 * b);
-            wd[q] = x;
+        for (int i = 0; i < 64; ++i) {
+            if (sym != 1) {
+                // index = clamp(round(w / scale) + zero_point, 0, 15)
+                const int cc = (int)rintf(__fdiv_rn(v[i], shf)) + zp;
+                code[i] = (uint32_t)min(max(cc, 0), 15);
+            } else {
+                // q = clamp(round(w / scale), -7, 7)
+                const int q = (int)rintf(__fdiv_rn(v[i], shf));
+                code[i] = (uint32_t)(min(max(q, -7), 7) + 8);
+            }
         }
-        *reinterpret_cast<uint4*>(blk + code_chunk_offset(r, c)) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
-    }
-    reinterpret_cast<__half*>(blk + kScaleOff)[r] = sh;
-    reinterpret_cast<__half*>(blk + kZpOff)[r] = __float2half_rn((float)zp);
-
-    if (valid) {
-        const int Kp = G * kGroup;
-        if (codes_out != nullptr) {
-            uint8_t* dst = codes_out + ((size_t)e * N + src) * (size_t)(Kp / 2) + (size_t)g * (kGroup / 2);
+        // tiled block of plane k0 / 128: word i of the plane (K = 8i .. 8i+7):
+        // byte b = code[8i+b] | code[8i+4+b] << 4; this chunk is the plane's half k0 / 64 % 2
+        uint8_t* blk = blocks + (tile_blk + (size_t)(k0 / kGroup)) * kBB;
+        const int hh = (k0 / 64) & 1;
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
+        for (int cc = 0; cc < 2; ++cc) {
+            uint32_t wd[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int l = 32 * cc + 8 * q;  // chunk-local index of the word's first code
+                uint32_t x = 0;
+#pragma unroll
+                for (int b = 0; b < 4; ++b) x |= (code[l + b] | (code[l + 4 + b] << 4)) << (8 * b);
+                wd[q] = x;
+            }
+            *reinterpret_cast<uint4*>(blk + code_chunk_offset(r, 2 * hh + cc)) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+        }
+        if (valid && codes_out != nullptr) {
+            // canonical order: byte j = code[2j] | code[2j+1] << 4
+            uint8_t* dst = codes_out + ((size_t)e * N + src) * (size_t)(G * kGroup / 2) + (size_t)k0 / 2;
+#pragma unroll
+            for (int cc = 0; cc < 2; ++cc) {
                 uint32_t wd[4];
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
                     uint32_t x = 0;
 #pragma unroll
                     for (int b = 0; b < 4; ++b) {
-                        const int j = 16 * c + 4 * q + b;  // canonical byte j: code[2j] | code[2j+1] << 4
+                        const int j = 16 * cc + 4 * q + b;
                         x |= (code[2 * j] | (code[2 * j + 1] << 4)) << (8 * b);
                     }
                     wd[q] = x;
                 }
-                *reinterpret_cast<uint4*>(dst + 16 * c) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+                *reinterpret_cast<uint4*>(dst + 16 * cc) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
             }
         }
-        if (scale_out != nullptr) scale_out[((size_t)e * N + src) * G + g] = __half_as_ushort(sh);
-        if (zp_out != nullptr) zp_out[((size_t)e * N + src) * G + g] = __half_as_ushort(__float2half_rn((float)zp));
     }
-    if (e == 0 && t == 0 && g == 0 && r == 0) {
+    // scale and zero point: in the plane block (group 64: the plane's sub-group slot;
+    // group 256: both of the group's planes)
+    const __half zh = __float2half_rn((float)zp);
+#pragma unroll
+    for (int pp = 0; pp < (GRP > kGroup ? GRP / kGroup : 1); ++pp) {
+        const int plane = GRP > kGroup ? gq * (GRP / kGroup) + pp : gq * GRP / kGroup;
+        const int sub = GRP < kGroup ? (gq & 1) : 0;
+        uint8_t* blk = blocks + (tile_blk + (size_t)plane) * kBB + sub * 512;
+        reinterpret_cast<__half*>(blk + kScaleOff)[r] = sh;
+        reinterpret_cast<__half*>(blk + kZpOff)[r] = zh;
+    }
+    if (valid) {
+        if (scale_out != nullptr) scale_out[((size_t)e * N + src) * Gq + gq] = __half_as_ushort(sh);
+        if (zp_out != nullptr) zp_out[((size_t)e * N + src) * Gq + gq] = __half_as_ushort(zh);
+    }
+    if (e == 0 && t == 0 && gq == 0 && r == 0) {
         PackHeader* h = reinterpret_cast<PackHeader*>(blocks - kHeaderBytes);
         h->magic = kPackMagic;
-        h->version = 1;
+        h->version = 2;
         h->layout = (uint32_t)layout | (sym == 1 ? 0x100u : sym == 2 ? 0x200u : 0u);
         h->E = gridDim.z;
         h->N = (uint32_t)N;
@@ -187,7 +215,8 @@ __global__ void __launch_bounds__(128) pack_kernel(const uint16_t* __restrict__ 
         h->G = (uint32_t)G;
         h->NT = (uint32_t)NT;
         h->rows_per_tile = kTileRows;
-        h->block_bytes = kBlockBytes;
+        h->block_bytes = kBB;
+        h->group = GRP;
     }
 }
 
@@ -496,10 +525,9 @@ __device__ __forceinline__ void load_chunk(const float* row, int len, int k0, Ch
 }
 
 template <int kCache, typename TIn>
-__device__ __forceinline__ void quant_row_cta(const TIn* row, int len, int r, int RB, int8_t* __restrict__ act,
-                                              float* __restrict__ s) {
+__device__ __forceinline__ void quant_row_cta(const TIn* row, int len, int Kp, int r, int RB,
+                                              int8_t* __restrict__ act, float* __restrict__ s) {
     __shared__ float red[4];
-    const int Kp = round_up(len, kGroup);
     const int nch = Kp / 16;
     const int G = Kp / kGroup;
     const int t = threadIdx.x;
@@ -565,12 +593,11 @@ __device__ __forceinline__ void quant_row_cta(const TIn* row, int len, int r, in
 // x rows (bf16) -> INT8 rows in expert-grouped order.  CTA t < T quantises token t
 // once (one read of x) and writes the codes to each of its k grouped rows; CTA T + e
 // writes zero codes and scale 0 into the pad rows of expert e.
-__global__ void __launch_bounds__(128) act_scatter_kernel(const uint16_t* __restrict__ x, int T, int H, int k,
+__global__ void __launch_bounds__(128) act_scatter_kernel(const uint16_t* __restrict__ x, int T, int H, int Kp, int k,
                                                           const int* __restrict__ inv,
                                                           const int* __restrict__ offs,
                                                           const int* __restrict__ poffs, int RB,
                                                           int8_t* __restrict__ act, float* __restrict__ s) {
-    const int Kp = round_up(H, kGroup);
     const int nch = Kp / 16;
     const int G = Kp / kGroup;
     const int t = threadIdx.x;
@@ -644,12 +671,12 @@ __global__ void __launch_bounds__(128) act_scatter_kernel(const uint16_t* __rest
 // h rows (fp32, SwiGLU output of the up GEMM) -> INT8 rows for the down GEMM
 // (kCache chunks of 16 per thread stay in registers: 1 covers F <= 2048)
 template <int kCache>
-__global__ void __launch_bounds__(128) requant_kernel(const float* __restrict__ h, int ldh, int F,
+__global__ void __launch_bounds__(128) requant_kernel(const float* __restrict__ h, int ldh, int F, int Kp,
                                                       const int* __restrict__ row_src, const int* __restrict__ poffs,
                                                       int E, int RB, int8_t* __restrict__ act, float* __restrict__ s) {
     const int r = blockIdx.x;
     if (r >= __ldg(poffs + E)) return;
-    quant_row_cta<kCache, float>(row_src[r] < 0 ? nullptr : h + (size_t)r * ldh, F, r, RB, act, s);
+    quant_row_cta<kCache, float>(row_src[r] < 0 ? nullptr : h + (size_t)r * ldh, F, Kp, r, RB, act, s);
 }
 
 // ---------------------------------------------------------------------------
@@ -708,7 +735,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
 
 // dense GEMM: copy INT8 rows into the tiled planes (pad rows zero) and describe
 // them as one "expert" with M rows.
-__global__ void __launch_bounds__(256) dense_prep_kernel(const int8_t* __restrict__ qa, int M, int Kp, int tile_tokens,
+__global__ void __launch_bounds__(256) dense_prep_kernel(const int8_t* __restrict__ qa, int M, int Kq, int Kp, int tile_tokens,
                                                          int RB, int8_t* __restrict__ act, int4* mt_tab, int* n_mtiles) {
     const int Mp = round_up(M, kRowPad);
     const int nch = Kp / 16;
@@ -720,7 +747,7 @@ __global__ void __launch_bounds__(256) dense_prep_kernel(const int8_t* __restric
     const int r = (int)(idx / nch);
     const int ci = (int)(idx % nch);
     uint4 v = make_uint4(0, 0, 0, 0);
-    if (r < M) v = *reinterpret_cast<const uint4*>(qa + (size_t)r * Kp + ci * 16);
+    if (r < M && ci * 16 < Kq) v = *reinterpret_cast<const uint4*>(qa + (size_t)r * Kq + ci * 16);
     *reinterpret_cast<uint4*>(act + act_offset(r, ci * 16, Kp / kGroup, RB)) = v;
 }
 
@@ -791,12 +818,18 @@ __global__ void __launch_bounds__(256) dense_prep_bf16_kernel(const uint16_t* __
 }  // namespace
 
 // ------------------------------- launchers ---------------------------------
-cudaError_t launch_pack(const uint16_t* w, int E, int N, int K, int layout, int scheme, uint8_t* packed,
+cudaError_t launch_pack(const uint16_t* w, int E, int N, int K, int layout, int scheme, int group, uint8_t* packed,
                         uint8_t* codes, uint16_t* scale, uint16_t* zp, cudaStream_t stream) {
-    const int G = ceil_div(K, kGroup);
+    const int G = k_padded_for(K, group) / kGroup;
     const int NT = layout == 1 ? ceil_div(N / 2, kTileRows / 2) : ceil_div(N, kTileRows);
-    dim3 grid(G, NT, E);
-    pack_kernel<<<grid, 128, 0, stream>>>(w, N, K, layout, scheme, NT, G, packed + kHeaderBytes, codes, scale, zp);
+    dim3 grid(G * kGroup / group, NT, E);
+    uint8_t* blocks = packed + kHeaderBytes;
+    if (group == 64)
+        pack_kernel<64><<<grid, 128, 0, stream>>>(w, N, K, layout, scheme, NT, G, blocks, codes, scale, zp);
+    else if (group == 256)
+        pack_kernel<256><<<grid, 128, 0, stream>>>(w, N, K, layout, scheme, NT, G, blocks, codes, scale, zp);
+    else
+        pack_kernel<128><<<grid, 128, 0, stream>>>(w, N, K, layout, scheme, NT, G, blocks, codes, scale, zp);
     return cudaGetLastError();
 }
 
@@ -838,20 +871,20 @@ cudaError_t launch_perm(const int32_t* ids, int nslots, int E, int tile_tokens, 
     return cudaGetLastError();
 }
 
-cudaError_t launch_act_scatter(const uint16_t* x, int T, int H, int k, const int* inv, const int* offs,
+cudaError_t launch_act_scatter(const uint16_t* x, int T, int H, int Kp, int k, const int* inv, const int* offs,
                                const int* poffs, int E, int rb, int8_t* act, float* s, cudaStream_t stream) {
     if (T == 0) return cudaSuccess;
-    act_scatter_kernel<<<T + E, 128, 0, stream>>>(x, T, H, k, inv, offs, poffs, rb, act, s);
+    act_scatter_kernel<<<T + E, 128, 0, stream>>>(x, T, H, Kp, k, inv, offs, poffs, rb, act, s);
     return cudaGetLastError();
 }
 
-cudaError_t launch_requant(const float* h, int ldh, int F, const int* row_src, const int* poffs, int E,
+cudaError_t launch_requant(const float* h, int ldh, int F, int Kp, const int* row_src, const int* poffs, int E,
                            int rows_cap, int rb, int8_t* act, float* s, cudaStream_t stream) {
     if (rows_cap == 0) return cudaSuccess;
     if (F <= 128 * 16)
-        requant_kernel<1><<<rows_cap, 128, 0, stream>>>(h, ldh, F, row_src, poffs, E, rb, act, s);
+        requant_kernel<1><<<rows_cap, 128, 0, stream>>>(h, ldh, F, Kp, row_src, poffs, E, rb, act, s);
     else
-        requant_kernel<kRowCache><<<rows_cap, 128, 0, stream>>>(h, ldh, F, row_src, poffs, E, rb, act, s);
+        requant_kernel<kRowCache><<<rows_cap, 128, 0, stream>>>(h, ldh, F, Kp, row_src, poffs, E, rb, act, s);
     return cudaGetLastError();
 }
 
@@ -862,10 +895,10 @@ cudaError_t launch_combine(const float* y2, int H, const int* inv, const float* 
     return cudaGetLastError();
 }
 
-cudaError_t launch_dense_prep(const int8_t* qa, int M, int Kp, int tile_tokens, int rb, int8_t* act, int4* mt_tab,
+cudaError_t launch_dense_prep(const int8_t* qa, int M, int Kq, int Kp, int tile_tokens, int rb, int8_t* act, int4* mt_tab,
                               int* n_mtiles, cudaStream_t stream) {
     const size_t n = (size_t)round_up(M, kRowPad) * (Kp / 16);
-    dense_prep_kernel<<<(unsigned)((n + 255) / 256 + 1), 256, 0, stream>>>(qa, M, Kp, tile_tokens, rb, act, mt_tab,
+    dense_prep_kernel<<<(unsigned)((n + 255) / 256 + 1), 256, 0, stream>>>(qa, M, Kq, Kp, tile_tokens, rb, act, mt_tab,
                                                                           n_mtiles);
     return cudaGetLastError();
 }

@@ -20,6 +20,17 @@ constexpr int kScaleOff = kCodeBytes;                // fp16 scales of the 128 r
 constexpr int kZpOff = kCodeBytes + kTileRows * 2;   // fp16 zero points of the 128 rows
 constexpr int kBlockBytes = kZpOff + kTileRows * 2;  // 8704 bytes per (tile, group) block
 constexpr int kHeaderBytes = 256;
+// Other group sizes along K (64 and 256; 128 is the default).  The packed blocks stay
+// one per 128-wide K plane (kGroup above is that plane): 8192 bytes of codes, then per
+// row the fp16 scale and zero point of each group the plane holds.  Group 64: two
+// groups, the second pair after the first (block of 9216 bytes); group 256: the plane
+// is half of a group whose scale and zero point both of its planes carry (8704 bytes),
+// so that every block is self-contained.  K is padded to a whole number of groups and
+// of planes.
+__host__ __device__ constexpr int block_bytes_for(int group) { return group == 64 ? kBlockBytes + 512 : kBlockBytes; }
+__host__ __device__ constexpr int k_padded_for(int K, int group) {
+    return (K + (group > 128 ? group : 128) - 1) / (group > 128 ? group : 128) * (group > 128 ? group : 128);
+}
 constexpr uint32_t kPackMagic = 0x38413457u;         // "W4A8"
 constexpr int kRowPad = 16;           // each expert's row segment is padded to 16 rows
 constexpr int kMaxExperts = 1024;
@@ -70,8 +81,9 @@ __host__ __device__ inline uint32_t code_chunk_offset(int r, int c) {
     return (uint32_t)r * 64u + ((uint32_t)((c ^ (r >> 1)) & 3) << 4);
 }
 
+// G counts 128-wide planes (blocks per tile), `group` the weights per scale along K
 struct PackHeader {
-    uint32_t magic, version, layout, E, N, K, Kp, G, NT, rows_per_tile, block_bytes;
+    uint32_t magic, version, layout, E, N, K, Kp, G, NT, rows_per_tile, block_bytes, group;
 };
 
 // ---------------------------------------------------------------------------

@@ -30,6 +30,9 @@ struct GemmArgs {
     // the tiled token rows of out16 (16-row blocks, out16_G K groups) instead of `out`
     uint8_t* out16;
     int out16_G;
+    // weights per scale along K in the packed blocks: 64, 128 (also 0) or 256; G above
+    // counts 128-wide planes, the partials [rows][nvalid][G * 128 / group] groups
+    int group;
 };
 
 // Test hook of the failure-detection path (w4a8_debug_inject): while set on the
@@ -52,7 +55,8 @@ cudaError_t launch_gemm_decode(const GemmArgs& a, int num_ctas, cudaStream_t str
 cudaError_t launch_gemm_w4a16(const GemmArgs& a, int num_ctas, cudaStream_t stream);
 
 // scheme: 0 asymmetric (min/max), 1 symmetric, 2 asymmetric on the 0.1th..99.9th percentiles
-cudaError_t launch_pack(const uint16_t* w, int E, int N, int K, int layout, int scheme, uint8_t* packed,
+// group: weights per scale along K (64, 128 or 256)
+cudaError_t launch_pack(const uint16_t* w, int E, int N, int K, int layout, int scheme, int group, uint8_t* packed,
                         uint8_t* codes, uint16_t* scale, uint16_t* zp, cudaStream_t stream);
 cudaError_t launch_quant_act(const uint16_t* x, int T, int K, int8_t* q, float* s, cudaStream_t stream);
 cudaError_t launch_route_topk(const uint16_t* logits, int T, int E, int k, int32_t* ids, float* w,
@@ -65,13 +69,15 @@ cudaError_t launch_perm(const int32_t* ids, int nslots, int E, int tile_tokens, 
 // capacity of the row-tile table for a layer: sum over experts of ceil(count / tile)
 // <= nslots / tile + E, with tiles of at least 16 rows
 inline int mt_tab_capacity(int nslots, int E) { return nslots / 16 + E + 1; }
-cudaError_t launch_act_scatter(const uint16_t* x, int T, int H, int k, const int* inv, const int* offs,
+// Kp: the padded row length of the tiled rows (a multiple of 128, >= H)
+cudaError_t launch_act_scatter(const uint16_t* x, int T, int H, int Kp, int k, const int* inv, const int* offs,
                                const int* poffs, int E, int rb, int8_t* act, float* s, cudaStream_t stream);
-cudaError_t launch_requant(const float* h, int ldh, int F, const int* row_src, const int* poffs, int E,
+cudaError_t launch_requant(const float* h, int ldh, int F, int Kp, const int* row_src, const int* poffs, int E,
                            int rows_cap, int rb, int8_t* act, float* s, cudaStream_t stream);
 cudaError_t launch_combine(const float* y2, int H, const int* inv, const float* w, int T, int k, uint16_t* out,
                            cudaStream_t stream);
-cudaError_t launch_dense_prep(const int8_t* qa, int M, int Kp, int tile_tokens, int rb, int8_t* act, int4* mt_tab,
+// qa rows of Kq columns into tiled rows of Kp >= Kq columns (the rest zero)
+cudaError_t launch_dense_prep(const int8_t* qa, int M, int Kq, int Kp, int tile_tokens, int rb, int8_t* act, int4* mt_tab,
                               int* n_mtiles, cudaStream_t stream);
 // W4A16 token rows: x bf16 [M][K] -> tiled bf16 rows (16-row blocks, K padded with
 // zeros) described as one "expert" of 16-row tiles
