@@ -2,13 +2,15 @@
 """Benchmark of the W4A8 MoE expert FFN on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload prefill] [--impl ours|reference]
-                    [--weights asym|sym|clip999] [--no-cpu-baseline] [--no-extra]
+                    [--weights asym|sym|clip999] [--group 64|128|256] [--no-cpu-baseline] [--no-extra]
 
 Workloads: dense_gemm, toy_moe, decode, large_decode, prefill (the default: the
 largest MoE layer, 384 experts, top-8, 16384 tokens, hidden 7168, expert ffn 2048,
 INT8-tensor-bound) and kv_int8 (the INT8 KV cache round trip, reported in GB/s).
 --weights selects the packer's scheme (asymmetric INT4, symmetric, or the
-percentile range).  On one GPU the default run also times the two HBM-bound decode
+percentile range); --group the weights per scale along K (128 by default, or 64 /
+256).  Decode-shaped layers with group 128 are also timed with W4A16 experts (the
+same packed weights with bf16 activations), reported under "w4a16" with the ratio.  On one GPU the default run also times the two HBM-bound decode
 layers (large_decode reusing the packed 384-expert weights, and decode) and reports
 each under "extra" with its own step time, roofline and kernel table (--no-extra
 skips them).
@@ -61,9 +63,11 @@ def padded(k):
 
 
 def packed_matrix_bytes(N, K):
-    """4-bit codes + one fp16 scale and one fp16 zero point per 128-group."""
-    Kp = padded(K)
-    return N * Kp // 2 + N * (Kp // 128) * 4
+    """4-bit codes + one fp16 scale and one fp16 zero point per group (the pages'
+    storage: 0.5 B per weight + 4 B per group of GROUP weights)."""
+    m = max(128, GROUP)
+    Kp = (K + m - 1) // m * m
+    return N * Kp // 2 + N * (Kp // GROUP) * 4
 
 
 def moe_accounting(W, ids, w4a16=False):
@@ -93,8 +97,8 @@ def moe_accounting(W, ids, w4a16=False):
     k_bytes = {
         "perm": slots * 4 * 3.0,
         "act_quant": T * H * 2.0 + slots * Hp + slots * 4,
-        "gemm_up": up_w + slots * Hp + slots * F * 4.0,
-        "requant": slots * F * 4.0 + slots * Fp,
+        "gemm_up": up_w + slots * Hp + slots * F * 2.0,  # h written as bf16
+        "requant": slots * F * 2.0 + slots * Fp,
         "gemm_down": dn_w + slots * Fp + slots * H * 4.0,
         "combine": slots * H * 4.0 + T * H * 2.0 + slots * 8,
         "route": T * W.E * 2.0 + slots * 8,
@@ -207,33 +211,34 @@ def dev_bf16(a, device):
 # weight scheme of the packer: asymmetric INT4 (default), symmetric, or asymmetric on the
 # 0.1th..99.9th percentile range
 SCHEME = "asym"
+GROUP = 128  # weights per scale along K (--group)
 
 
 def weights_desc():
-    return {"asym": "int4 g128 asym (fp16 scale+zp)", "sym": "int4 g128 sym (fp16 scale, zero point 8)",
-            "clip999": "int4 g128 asym on the 0.1..99.9 percentile range (fp16 scale+zp)"}[SCHEME]
+    return {"asym": "int4 g%d asym (fp16 scale+zp)", "sym": "int4 g%d sym (fp16 scale, zero point 8)",
+            "clip999": "int4 g%d asym on the 0.1..99.9 percentile range (fp16 scale+zp)"}[SCHEME] % GROUP
 
 
 def scheme_flag(B):
-    return {"asym": 0, "sym": B.W4A8_PACK_SYMMETRIC, "clip999": B.W4A8_PACK_CLIP999}[SCHEME]
+    return {"asym": 0, "sym": B.W4A8_PACK_SYMMETRIC, "clip999": B.W4A8_PACK_CLIP999}[SCHEME] | B.GROUP_FLAG[GROUP]
 
 
 def oracle_quant(O):
     if SCHEME == "sym":
-        return O.quantize_weights_symmetric
-    return lambda w: O.quantize_weights(w, clip999=SCHEME == "clip999")
+        return lambda w: O.quantize_weights_symmetric(w, GROUP)
+    return lambda w: O.quantize_weights(w, clip999=SCHEME == "clip999", group=GROUP)
 
 
 def pack_experts(B, torch, W, seed, device):
     """Pack every expert's up (gate|up) and down weights on the device, one expert at a time."""
     E, H, F = W.E, W.H, W.F
     flag = scheme_flag(B)
-    up = B.empty_aligned(B.w4a8_packed_bytes(E, 2 * F, H, B.W4A8_LAYOUT_GATEUP), device)
-    dn = B.empty_aligned(B.w4a8_packed_bytes(E, H, F, B.W4A8_LAYOUT_PLAIN), device)
+    up = B.empty_aligned(B.w4a8_packed_bytes(E, 2 * F, H, B.W4A8_LAYOUT_GATEUP | flag), device)
+    dn = B.empty_aligned(B.w4a8_packed_bytes(E, H, F, B.W4A8_LAYOUT_PLAIN | flag), device)
     su = (up.numel() - 256) // E
     sd = (dn.numel() - 256) // E
-    tu = B.empty_aligned(B.w4a8_packed_bytes(1, 2 * F, H, 1), device)
-    td = B.empty_aligned(B.w4a8_packed_bytes(1, H, F, 0), device)
+    tu = B.empty_aligned(B.w4a8_packed_bytes(1, 2 * F, H, 1 | flag), device)
+    td = B.empty_aligned(B.w4a8_packed_bytes(1, H, F, 0 | flag), device)
     for which, (buf, tmp, stride, rows, cols, layout) in (("up", (up, tu, su, 2 * F, H, 1)),
                                                            ("down", (dn, td, sd, H, F, 0))):
         for e, w in synth.expert_weights_parallel(seed, E, which, rows, cols):
@@ -270,15 +275,23 @@ class MoeStep:
         self.logits_host = inp.get("logits")
         self.packed_up, self.packed_down = packed if packed is not None else pack_experts(B, torch, W, seed, device)
         self.out = torch.empty((T, H), dtype=torch.bfloat16, device=device)
-        wsb = B.w4a16_moe_workspace_bytes if w4a16 else B.w4a8_moe_workspace_bytes
-        self.ws = B.empty_aligned(wsb(T, E, k, H, F), device)
+        if w4a16:
+            self.ws = B.empty_aligned(B.w4a16_moe_workspace_bytes(T, E, k, H, F), device)
+        else:
+            self.ws = B.empty_aligned(B.w4a8_moe_workspace_bytes_g(T, E, k, H, F, GROUP), device)
         self.acct = moe_accounting(W, self.ids_host, w4a16)
 
     def __call__(self):
         B, W = self.B, self.W
         if self.logits is not None:
             B.w4a8_route_topk(self.logits, W.topk, self.ids, self.w)
-        fwd = B.w4a16_moe_forward if self.w4a16 else B.w4a8_moe_forward
+        if self.w4a16:
+            fwd = B.w4a16_moe_forward
+        elif GROUP != 128:
+            def fwd(*a):
+                B.w4a8_moe_forward_g(*a[:5], GROUP, *a[5:])
+        else:
+            fwd = B.w4a8_moe_forward
         fwd(self.packed_up, self.packed_down, W.E, W.H, W.F, self.x, self.ids, self.w, self.out,
                            self.ws)
 
@@ -290,7 +303,20 @@ class MoeStep:
         pin = lambda a: torch.from_numpy(a).pin_memory()
         x_h = torch.from_numpy(synth.bf16_bits(self.x_host).view(np.int16)).view(torch.bfloat16).pin_memory()
         out_h = torch.empty((T, H), dtype=torch.bfloat16).pin_memory()
-        if self.logits is None:
+        if GROUP != 128:
+            # the group-size entry point takes device buffers: the step's copies are
+            # issued on the same stream around it
+            ids_h, w_h = pin(np.ascontiguousarray(self.ids_host)), pin(np.ascontiguousarray(self.w_host))
+            h2d = x_h.numel() * 2 + ids_h.numel() * 4 + w_h.numel() * 4
+            logits, self.logits = self.logits, None
+
+            def step():
+                self.x.copy_(x_h, non_blocking=True)
+                self.ids.copy_(ids_h, non_blocking=True)
+                self.w.copy_(w_h, non_blocking=True)
+                self()
+                out_h.copy_(self.out, non_blocking=True)
+        elif self.logits is None:
             ids_h, w_h = pin(np.ascontiguousarray(self.ids_host)), pin(np.ascontiguousarray(self.w_host))
             ws = B.empty_aligned(B.w4a8_moe_host_workspace_bytes(T, E, k, H, F), self.device)
             h2d = x_h.numel() * 2 + ids_h.numel() * 4 + w_h.numel() * 4
@@ -317,6 +343,8 @@ class MoeStep:
             b.record()
             b.synchronize()
             total += a.elapsed_time(b)
+        if GROUP != 128:
+            self.logits = logits
         return total / steps, h2d, T * H * 2
 
 
@@ -327,18 +355,18 @@ class GemmStep:
         self.B, self.torch, self.W, self.device = B, torch, W, device
         x, w = synth.dense_gemm_inputs(seed, W.M, W.K, W.N)
         self.x = dev_bf16(x, device)
-        self.packed = B.empty_aligned(B.w4a8_packed_bytes(1, W.N, W.K, 0), device)
+        self.packed = B.empty_aligned(B.w4a8_packed_bytes(1, W.N, W.K, scheme_flag(B)), device)
         B.w4a8_pack_weights(dev_bf16(w, device), scheme_flag(B), self.packed)
         Kp = padded(W.K)
         self.q = torch.empty((W.M, Kp), dtype=torch.int8, device=device)
         self.s = torch.empty(W.M, dtype=torch.float32, device=device)
         self.y = torch.empty((W.M, W.N), dtype=torch.float32, device=device)
-        self.ws = B.empty_aligned(B.w4a8_gemm_workspace_bytes(W.M, W.N, W.K), device)
+        self.ws = B.empty_aligned(B.w4a8_gemm_workspace_bytes_g(W.M, W.N, W.K, GROUP), device)
         self.acct = gemm_accounting(W)
 
     def __call__(self):
         self.B.w4a8_quant_act(self.x, self.q, self.s)
-        self.B.w4a8_gemm(self.q, self.s, self.packed, self.W.N, self.W.K, self.y, self.ws)
+        self.B.w4a8_gemm_g(self.q, self.s, self.packed, self.W.N, self.W.K, GROUP, self.y, self.ws)
 
     def e2e(self, steps, warmup):
         torch = self.torch
@@ -425,7 +453,8 @@ class OracleSample:
                 W = self.W
                 self.experts[e] = self.O.QuantExpert(synth.expert_weight(self.seed, e, "up", 2 * W.F, W.H),
                                                      synth.expert_weight(self.seed, e, "down", W.H, W.F),
-                                                     symmetric=SCHEME == "sym", clip999=SCHEME == "clip999")
+                                                     symmetric=SCHEME == "sym", clip999=SCHEME == "clip999",
+                                                     group=GROUP)
 
     def _time(self, n):
         self._ensure_experts(n)
@@ -678,9 +707,12 @@ def measure_int8_peak(torch, device, n=8192, reps=10):
 
 def time_steps(step, B, torch, device, world, steps, warmup):
     """Warm up, then time `steps` steps with CUDA events on the launching stream (L2
-    flushed before each, outside the timed span), the library's per-kernel event
-    profiler and NVML clock samples over the same region.  Returns (max-over-ranks
-    ms per step, {kernel kind: (launches, total ms)}, clock summary)."""
+    flushed before each, outside the timed span) and NVML clock samples over the same
+    region; then run the same number of steps again under the library's per-kernel
+    event profiler (its events between kernels would break the overlap of one kernel's
+    start with the previous one's end, so the headline steps run without it).
+    Returns (max-over-ranks ms per step, {kernel kind: (launches, total ms)}, clock
+    summary)."""
     for _ in range(warmup):
         step()
     torch.cuda.synchronize()
@@ -688,7 +720,6 @@ def time_steps(step, B, torch, device, world, steps, warmup):
     sampler = ClockSampler(torch.cuda.current_device())
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
-    B.w4a8_profile_start()
     sampler.start()
     if world > 1:
         torch.distributed.barrier()
@@ -702,9 +733,15 @@ def time_steps(step, B, torch, device, world, steps, warmup):
     if world > 1:
         torch.distributed.barrier()
     sampler.stop()
+    ms = sum(a.elapsed_time(b) for a, b in zip(starts, ends)) / steps
+    # the per-kernel table
+    B.w4a8_profile_start()
+    for _ in range(steps):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
     prof = B.w4a8_profile_stop()
     assert B.w4a8_last_device_error(step.ws) == 0, "device error during the timed steps"
-    ms = sum(a.elapsed_time(b) for a, b in zip(starts, ends)) / steps
     return max_over_ranks(ms, torch, device, world), prof, sampler.summary()
 
 
@@ -775,12 +812,17 @@ def main(argv=None):
     ap.add_argument("--cpu-baseline-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true", help="do not also time the decode layers")
+    ap.add_argument("--group", type=int, choices=[64, 128, 256], default=128,
+                    help="weights per scale and zero point along K (the default 128, or 64 / 256)")
     ap.add_argument("--weights", choices=["asym", "sym", "clip999"], default="asym",
                     help="packer scheme: asymmetric INT4 (default), symmetric, or asymmetric on the "
                          "0.1th..99.9th percentile range")
     args = ap.parse_args(argv)
-    global SCHEME
+    global SCHEME, GROUP
     SCHEME = args.weights
+    GROUP = args.group
+    if GROUP != 128 and SCHEME == "clip999":
+        ap.error("the percentile range is defined for groups of 128")
     W = synth.WORKLOADS[args.workload]
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -851,7 +893,7 @@ def main(argv=None):
 
     # decode-shaped layers: the pages' comparison point, the same layer with W4A16
     # experts (bf16 activations, same packed weights and routing)
-    if W.kind == "moe" and W.name != "prefill":
+    if W.kind == "moe" and W.name != "prefill" and GROUP == 128:
         s16 = MoeStep(B, torch, W, args.seed, device, packed=(step.packed_up, step.packed_down), w4a16=True)
         ms16, prof16, cl16 = time_steps(s16, B, torch, device, world, args.steps, args.warmup)
         w16 = moe_summary(W, s16, ms16, prof16, cl16, args.steps, peaks, world)
@@ -875,7 +917,12 @@ def main(argv=None):
                          "d2h_bytes_per_step": d2x}
             ex["config"] = config_of(Wx, "flushed before every timed step (256 MiB write, outside the timed span)")
             # the pages' comparison point: the same layer with W4A16 experts (bf16
-            # activations, same packed weights and routing)
+            # activations, same packed weights and routing; group 128 only)
+            if GROUP != 128:
+                extra[name] = ex
+                del sx
+                torch.cuda.empty_cache()
+                continue
             s16 = MoeStep(B, torch, Wx, args.seed, device, packed=(sx.packed_up, sx.packed_down), w4a16=True)
             ms16, prof16, cl16 = time_steps(s16, B, torch, device, world, args.steps, args.warmup)
             w16 = moe_summary(Wx, s16, ms16, prof16, cl16, args.steps, peaks, world)

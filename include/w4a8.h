@@ -144,7 +144,10 @@ size_t w4a8_moe_workspace_bytes(int T, int E, int k, int H, int F);
 /* The W4A8 MoE expert FFN  (a4..a8):
  *   out[t] = sum_j w[t][j] * Down_e( SwiGLU( Up_e( x[t] ) ) ),  e = ids[t][j],
  * with x quantised per token to INT8, Up/Down W4A8 GEMMs (INT32 per-group
- * partials), h = silu(gate) * up requantised per token to INT8 before Down.
+ * partials), h = silu(gate) * up rounded to bf16 and requantised per token to INT8
+ * before Down (section 4.3, step 4: the GEMM result is handed on in 16-bit
+ * floating point), and the fp32 weighted sum of the experts' Down results rounded
+ * to bf16.
  * Source: the Kimi 2.7T MoE W4A8 article (hotelren.com 5173946), section 4.3: the
  * activations are quantised per token at run time, the INT4 weights are expanded
  * inside the kernel and multiplied in INT8 with INT32 accumulation, the result is
@@ -286,7 +289,7 @@ enum {
     W4A8_DUMP_POFFS = 4,  /* int32 [E+1]    row offsets with every expert padded to 16 */
     W4A8_DUMP_ACT1 = 5,   /* int8, R x Hp: INT8 x rows (tiled, see below)             */
     W4A8_DUMP_S1 = 6,     /* float [R]      token scale of each padded row            */
-    W4A8_DUMP_H = 7,      /* float [R][Fp]  SwiGLU output h (fp32) per padded row      */
+    W4A8_DUMP_H = 7,      /* bf16 [R][Fp]   SwiGLU output h per padded row             */
     W4A8_DUMP_ACT2 = 8,   /* int8, R x Fp: requantised h (tiled, see below)           */
     W4A8_DUMP_S2 = 9,     /* float [R]      scale of the requantised h rows           */
     W4A8_DUMP_Y2 = 10,    /* float [R][H]   down-projection output per padded row     */

@@ -34,7 +34,9 @@ its reason in the design notes):
   R11 softmax routing: top-k experts by logit (ties -> lower id), gate weight = the
       softmax probability over all E experts, not renormalised;
   R12 tokens inside an expert's segment keep their slot order (t * k + j ascending);
-  R14 h enters the requantisation as fp32;
+  R14 h, the SwiGLU of the up projection's result, is rounded once to bf16 and enters
+      the requantisation as that bf16 value ([P1] §4.3 step 4: the GEMM result is
+      handed on in FP16/BF16; step 3: the next op quantises it per token);
   R18 symmetric INT4 variant: q clamped to [-7, 7], stored as code q + 8 with zero point 8;
   R19 percentile-clipped variant: per group the 0.1th and 99.9th percentiles by linear
       interpolation at q * (n - 1), in fp32 with fractions fp32(0.127) and fp32(0.873);
@@ -389,13 +391,14 @@ class QuantExpert:
 
 
 def expert_forward(xq, xs, qe: QuantExpert, F: int, stages: dict | None = None):
-    """One expert on its tokens: up GEMM -> SwiGLU -> requantise -> down GEMM.
+    """One expert on its tokens: up GEMM -> SwiGLU (rounded to bf16, R14) ->
+    requantise -> down GEMM.
 
     xq int8 [M][Hp], xs float32 [M]; returns y2 float64 [M][H].
     """
     cu, su, zu = qe.up
     y_up = w4a8_linear(xq, xs, cu, su, zu)  # [M][2F]
-    h = swiglu(y_up, F).astype(np.float32)  # R14: h enters requant as fp32
+    h = round_to_bf16(swiglu(y_up, F)).astype(np.float32)  # R14: h is handed on in bf16
     qh, sh = quantize_act(h, qe.group)  # [P1] §4.3 step 3: the next op's input is quantised per token
     cd, sd, zd = qe.down
     y2 = w4a8_linear(qh, sh, cd, sd, zd)

@@ -149,3 +149,30 @@ def w4a16_error_bound(x, codes, scale, zp) -> np.ndarray:
     wabs = np.abs(codes.astype(np.float64) - np.repeat(zp.astype(np.float64), group, axis=1)) * \
         np.repeat(scale.astype(np.float64), group, axis=1)
     return (group - 1 + G + 1) * 2.0 ** -23 * (x @ wabs.T)
+
+
+def bf16_ulp(v) -> np.ndarray:
+    """The spacing of bf16 values at |v| (8 significant bits): 2^(e - 7) for |v| in
+    [2^e, 2^(e+1)); the smallest normal spacing for 0 and subnormals."""
+    a = np.abs(np.asarray(v, dtype=np.float64))
+    e = np.floor(np.log2(np.maximum(a, 2.0 ** -126)))
+    return 2.0 ** (e - 7)
+
+
+def assert_bf16_adjacent(got, ref, what="value", max_frac=0.02):
+    """got: the kernel's bf16 values; ref: the oracle's bf16-rounded values of the same
+    quantity.  Both round a value computed on identical inputs (the kernel in fp32,
+    the oracle in fp64, about 1e-6 apart), so they are equal or, where that value
+    lies next to a bf16 rounding boundary, one bf16 step apart; at most max_frac of
+    the elements may differ."""
+    g = np.asarray(got, dtype=np.float64)
+    r = np.asarray(ref, dtype=np.float64)
+    assert g.shape == r.shape, (g.shape, r.shape)
+    if r.size == 0:
+        return
+    assert np.all(np.isfinite(g)), f"{what}: non-finite values"
+    d = np.abs(g - r)
+    step = np.maximum(bf16_ulp(r), bf16_ulp(g))
+    assert np.all(d <= step * (1 + 1e-9)), f"{what}: {int((d > step).sum())} values more than one bf16 step off"
+    frac = float((d > 0).mean())
+    assert frac <= max_frac, f"{what}: {frac:.3%} of the values differ (> {max_frac:.1%})"

@@ -113,7 +113,7 @@ def test_moe_workspace_regions(lib):
     # the documented sizes
     assert regions[B.DUMP["counts"]][1] == 4 * E
     assert regions[B.DUMP["act1"]][1] == (4096 // 128) * R * 128
-    assert regions[B.DUMP["h"]][1] == R * 1408 * 4
+    assert regions[B.DUMP["h"]][1] == R * 1408 * 2  # bf16
     assert regions[B.DUMP["act2"]][1] == (1408 // 128) * R * 128
     assert regions[B.DUMP["y2"]][1] == R * H * 4
     s = sorted(r for r in regions if r[1] > 4)

@@ -22,7 +22,7 @@ import numpy as np
 import pytest
 import torch
 
-from helpers import assert_close
+from helpers import assert_bf16_adjacent, assert_close
 from oracle import w4a8_oracle as O
 from w4a8_quantized_moe_token_b200 import binding as B
 from w4a8_quantized_moe_token_b200 import synth
@@ -137,12 +137,12 @@ def run_and_check(wl_name, packed, extra_tokens):
 
     # a5 + a6: h of the sampled rows on identical INT8 inputs
     rows_t = torch.from_numpy(rows).long().cuda()
-    h = dump("h").view(torch.float32).view(R, Fp)[rows_t].cpu().numpy()
+    h = synth.bf16_from_bits(dump("h").view(torch.int16).view(R, Fp)[rows_t].cpu().numpy().view(np.uint16))
     h_ref = np.zeros((slots.size, F))
     for i, s in enumerate(slots):
         qe = experts[int(flat[s])]
-        h_ref[i] = O.swiglu(O.w4a8_linear(xq[src[i]:src[i] + 1], xs[src[i]:src[i] + 1], *qe.up), F)[0]
-    assert_close(h[:, :F], h_ref, max_rel=1e-4, mae_rel=1e-5, what="h")
+        h_ref[i] = O.round_to_bf16(O.swiglu(O.w4a8_linear(xq[src[i]:src[i] + 1], xs[src[i]:src[i] + 1], *qe.up), F))[0]
+    assert_bf16_adjacent(h[:, :F], h_ref, what="h")
 
     # a6: requantisation of the dumped h, bit-exact
     qh, sh = O.quantize_act(h[:, :F].astype(np.float32))

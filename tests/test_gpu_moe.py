@@ -9,7 +9,7 @@ import numpy as np
 import pytest
 import torch
 
-from helpers import assert_close, untile_act
+from helpers import assert_bf16_adjacent, assert_close, untile_act
 from oracle import w4a8_oracle as O
 from w4a8_quantized_moe_token_b200 import binding as B
 from w4a8_quantized_moe_token_b200 import synth
@@ -122,16 +122,16 @@ def check_stages(L: Layer, out):
     tok = np.arange(T * k) // k
     assert np.array_equal(act1[rows], xq[tok])
     assert np.array_equal(s1[rows], xs[tok])
-    # a5 + a6: h on identical INT8 inputs
+    # a5 + a6: h (bf16) on identical INT8 inputs
     experts = L.experts()
-    h = L.dump("h", np.float32).reshape(R, Fp)
+    h = synth.bf16_from_bits(L.dump("h", np.uint16).reshape(R, Fp))
     h_ref = np.zeros((T * k, F))
     for e, qe in experts.items():
         sl = perm[offs[e]:offs[e + 1]]
         if sl.size:
             t_e = sl // k
-            h_ref[sl] = O.swiglu(O.w4a8_linear(xq[t_e], xs[t_e], *qe.up), F)
-    assert_close(h[rows, :F], h_ref, max_rel=1e-4, mae_rel=1e-5, what="h")
+            h_ref[sl] = O.round_to_bf16(O.swiglu(O.w4a8_linear(xq[t_e], xs[t_e], *qe.up), F))
+    assert_bf16_adjacent(h[rows, :F], h_ref, what="h")
     # a6: requantisation of the dumped h, bit-exact
     act2 = untile_act(L.dump("act2", np.int8), R, Fp, RB)
     s2 = L.dump("s2", np.float32)

@@ -457,7 +457,8 @@ def test_moe_forward_equals_per_token_dequantized_formulation(group):
             wu = O.dequantize_weights(*qe.up)
             wd = O.dequantize_weights(*qe.down)
             yu = wu @ a
-            hh = (yu[:F] / (1 + np.exp(-yu[:F])) * yu[F:]).astype(np.float32)
+            # h is handed on in bf16 ([P1] §4.3 step 4)
+            hh = O.round_to_bf16(yu[:F] / (1 + np.exp(-yu[:F])) * yu[F:]).astype(np.float32)
             qh, sh = O.quantize_act(hh[None, :], group)
             acc += float(w[t, j]) * (wd @ (qh[0].astype(np.float64) * float(sh[0])))
         # the layer's output is rounded to bf16: within half a bf16 ulp of the fp64 value

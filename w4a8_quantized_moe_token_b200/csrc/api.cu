@@ -87,7 +87,7 @@ bool moe_layout(int T, int E, int k, int H, int F, bool host_io, MoeLayout* L, b
     const size_t row_bytes = w4a16 ? 256 : 128;  // token row bytes per K group
     b[R_ACT1] = (size_t)L->G1 * R * row_bytes;
     b[R_S1] = w4a16 ? 0 : R * 4;
-    b[R_H] = w4a16 ? 0 : R * (size_t)L->Fp * 4;
+    b[R_H] = w4a16 ? 0 : R * (size_t)L->Fp * 2;  // bf16
     b[R_ACT2] = (size_t)L->G2 * R * row_bytes;
     b[R_S2] = w4a16 ? 0 : R * 4;
     b[R_Y2] = R * (size_t)H * 4;
@@ -189,7 +189,7 @@ int moe_forward_impl(const void* packed_up, const void* packed_down, int E, int 
     int* inv = at<int>(ws, L, R_INV);
     float* s1 = at<float>(ws, L, R_S1);
     float* s2 = at<float>(ws, L, R_S2);
-    float* h = at<float>(ws, L, R_H);
+    uint16_t* h = at<uint16_t>(ws, L, R_H);
     float* y2 = at<float>(ws, L, R_Y2);
     int8_t* act1 = at<int8_t>(ws, L, R_ACT1);
     int8_t* act2 = at<int8_t>(ws, L, R_ACT2);
@@ -219,7 +219,8 @@ int moe_forward_impl(const void* packed_up, const void* packed_down, int E, int 
     up.mt_tab = mt_tab;
     up.n_mtiles = mtstart + E;
     up.mode = 1;
-    up.out = h;
+    up.out = reinterpret_cast<float*>(h);
+    up.out_bf16 = 1;
     up.ldo = L.Fp;
     up.nvalid = F;
     up.partials = nullptr;
@@ -243,7 +244,8 @@ int moe_forward_impl(const void* packed_up, const void* packed_down, int E, int 
     dn.act_rb_stride = (size_t)L.G2 * rb * 128;
     dn.act_scale = s2;
     dn.mode = 2;
-    dn.out = y2;
+    dn.out = y2;  // fp32
+    dn.out_bf16 = 0;
     dn.ldo = H;
     dn.nvalid = H;
     {
@@ -308,7 +310,7 @@ int moe_forward_w4a16_impl(const void* packed_up, const void* packed_down, int E
     dn.act = reinterpret_cast<const int8_t*>(h16);
     dn.act_rb_stride = (size_t)L.G2 * tile * 256;
     dn.mode = 2;
-    dn.out = y2;
+    dn.out = y2;  // fp32
     dn.ldo = H;
     dn.nvalid = H;
     dn.out16 = nullptr;

@@ -278,6 +278,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
     const int q = warp & 3;
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
 
+    // the set-up above (barriers, tensor memory, reset tiles) overlaps the previous
+    // kernel's tail; from here on this kernel reads its results
+    grid_dep_wait();
     const int total = a.NT * __ldg(a.n_mtiles);
     const int G = a.G;                 // 128-wide K planes (packed blocks) per tile
     const int Gq = G * kGroup / GRP;   // quantisation groups per row
@@ -620,6 +623,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
             float sa[BN];
 #pragma unroll
             for (int i = 0; i < BN; ++i) sa[i] = kBf16 ? 1.f : (i < it.nrows ? __ldg(sap + i) : 0.f);  // W4A16: no token scale
+            // mode 1 with out_bf16: h as bf16 (RNE of the fp32 result)
+            const bool obf = a.out_bf16 != 0 && a.mode == 1;
+            uint16_t* out16 = reinterpret_cast<uint16_t*>(a.out);
             if (a.mode != 1) {
                 const bool valid = n_out < a.nvalid;
                 float* op = a.out + (size_t)it.row0 * a.ldo + (valid ? n_out : 0);
@@ -635,7 +641,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
                 const int f = it.nt * (kTileRows / 2) + (r >> 1);
                 const int odd = r & 1;
                 const bool valid = f < a.nvalid;
-                float* op = a.out + (size_t)(it.row0 + odd) * a.ldo + f;
+                const size_t o0 = (size_t)(it.row0 + odd) * a.ldo + f;
 #pragma unroll
                 for (int i = 0; i < BN; i += 2) {
                     // even lane: own gate_i, needs the partner's up_i; odd lane: own up_{i+1},
@@ -650,9 +656,11 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
                         if (valid && i + odd < it.nrows)
                             *reinterpret_cast<__nv_bfloat16*>(a.out16 + act16_offset(it.row0 + i + odd, f, a.out16_G, BN)) =
                                 __float2bfloat16_rn(silu_mul(g, u));
-                    } else {
-                        if (valid && i + odd < it.nrows) *op = silu_mul(g, u);
-                        op += 2 * (size_t)a.ldo;
+                    } else if (valid && i + odd < it.nrows) {
+                        if (obf)
+                            out16[o0 + (size_t)i * a.ldo] = bf16_bits(silu_mul(g, u));
+                        else
+                            a.out[o0 + (size_t)i * a.ldo] = silu_mul(g, u);
                     }
                 }
             }
@@ -696,8 +704,7 @@ cudaError_t launch_decode(const GemmArgs& a, int num_ctas, cudaStream_t stream) 
         if (e != cudaSuccess) return e;
         if (dev >= 0 && dev < 64) attr_done[dev] = 1;
     }
-    gemm_decode_kernel<kBf16, GRP><<<num_ctas, kThreads, kSmem, stream>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(gemm_decode_kernel<kBf16, GRP>, num_ctas, kThreads, kSmem, stream, a);
 }
 }  // namespace
 

@@ -95,6 +95,9 @@ struct Cfg {
     // output staging tile: fp32 [BN tokens][128 channels] (plain output) or
     // [BN tokens][kStageH] (SwiGLU output, 64 channels + padding against bank conflicts)
     static constexpr int kStageH = 80;
+    // bf16 outputs (SwiGLU h): rows of kStageH16 bf16 values (64 channels + 16 against
+    // bank conflicts, a 16-byte multiple)
+    static constexpr int kStageH16 = 80;
     static constexpr int kOffStage = kOffReset + 2 * kResetTileBytes;
     static constexpr int kOffSa = kOffStage + BN * kTileRows * 4;  // the tile's token scales
     static constexpr int kOffBar = kOffSa + BN * 4;
@@ -247,6 +250,9 @@ __global__ void __launch_bounds__(C::kThreads, 1) gemm_w4a8_kernel(const GemmArg
     const int q = warp & 3;  // TMEM lane quarter of this warp
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
 
+    // the set-up above (barriers, tensor memory, reset tiles) overlaps the previous
+    // kernel's tail; from here on this kernel reads its results
+    grid_dep_wait();
     const int total = a.NT * __ldg(a.n_mtiles);
     const int G = a.G;                // 128-wide K planes (steps) per tile
     const int Gq = G * kGroup / GRP;  // quantisation groups per tile
@@ -444,8 +450,13 @@ __global__ void __launch_bounds__(C::kThreads, 1) gemm_w4a8_kernel(const GemmArg
         // (one output row per issuing thread), so the epilogue goes on with the next
         // tile while the stores drain; this needs every output row to start on a
         // 16-byte boundary.  Otherwise (a dense output with N % 4 != 0) it stores directly.
-        const bool staged = !kPartials && (a.ldo % 4 == 0) && (a.mode == 1 || a.nvalid % 4 == 0);
+        // (bf16 outputs, mode 1 with out_bf16: rows must start on 16 bytes too)
+        const bool obf = a.out_bf16 != 0 && a.mode == 1;
+        const int oal = obf ? 8 : 4;
+        const bool staged = !kPartials && (a.ldo % oal == 0) && (a.mode == 1 || a.nvalid % oal == 0);
         float* stage = reinterpret_cast<float*>(smem + C::kOffStage);
+        uint16_t* stage16 = reinterpret_cast<uint16_t*>(smem + C::kOffStage);
+        uint16_t* out16 = reinterpret_cast<uint16_t*>(a.out);
         float* sa_s = reinterpret_cast<float*>(smem + C::kOffSa);
         const int et = threadIdx.x - 32 * C::kEpiWarp0;  // epilogue thread 0 .. 128 * NEPI - 1
         bool issued = false;                            // a bulk copy of this thread is in flight
@@ -611,6 +622,7 @@ __global__ void __launch_bounds__(C::kThreads, 1) gemm_w4a8_kernel(const GemmArg
                     // lane finishes token i, the odd lane token i+1
                     const int odd = r & 1;
                     float* srow = stage + (col0 + odd) * C::kStageH + (r >> 1);
+                    uint16_t* srow16 = stage16 + (col0 + odd) * C::kStageH16 + (r >> 1);
 #pragma unroll
                     for (int i = 0; i < kCW; i += 2) {
                         const float send = odd ? acc[i] : acc[i + 1];
@@ -618,7 +630,10 @@ __global__ void __launch_bounds__(C::kThreads, 1) gemm_w4a8_kernel(const GemmArg
                         const float si = sa_s[col0 + i + odd];
                         const float g = (odd ? recv : acc[i]) * si;
                         const float uu = (odd ? acc[i + 1] : recv) * si;
-                        srow[i * C::kStageH] = silu_mul(g, uu);
+                        if (obf)
+                            srow16[i * C::kStageH16] = bf16_bits(silu_mul(g, uu));
+                        else
+                            srow[i * C::kStageH] = silu_mul(g, uu);
                     }
                 }
                 fence_proxy_async_smem();
@@ -632,8 +647,11 @@ __global__ void __launch_bounds__(C::kThreads, 1) gemm_w4a8_kernel(const GemmArg
                         const int w = min(kTileRows, a.nvalid - n0);
                         bulk_s2g(a.out + (size_t)(it.row0 + et) * a.ldo + n0,
                                  smem_u32(stage + et * kTileRows), (uint32_t)w * 4u);
-                    } else {
+                    } else if (obf) {
                         // all 64 channels: past F they land in the row's padding
+                        bulk_s2g(out16 + (size_t)(it.row0 + et) * a.ldo + it.nt * (kTileRows / 2),
+                                 smem_u32(stage16 + et * C::kStageH16), (kTileRows / 2) * 2u);
+                    } else {
                         bulk_s2g(a.out + (size_t)(it.row0 + et) * a.ldo + it.nt * (kTileRows / 2),
                                  smem_u32(stage + et * C::kStageH), (kTileRows / 2) * 4u);
                     }
@@ -663,7 +681,7 @@ __global__ void __launch_bounds__(C::kThreads, 1) gemm_w4a8_kernel(const GemmArg
                 const int f = it.nt * (kTileRows / 2) + (r >> 1);
                 const int odd = r & 1;
                 const bool valid = f < a.nvalid;
-                float* op = a.out + (size_t)(it.row0 + col0 + odd) * a.ldo + f;
+                const size_t o0 = (size_t)(it.row0 + col0 + odd) * a.ldo + f;
                 float sa[kCW / 2];
 #pragma unroll
                 for (int i = 0; i < kCW; i += 2) sa[i / 2] = i + odd < ncol ? __ldg(sap + i + odd) : 0.f;
@@ -675,8 +693,13 @@ __global__ void __launch_bounds__(C::kThreads, 1) gemm_w4a8_kernel(const GemmArg
                     const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
                     const float g = (odd ? recv : acc[i]) * sa[i / 2];
                     const float u = (odd ? acc[i + 1] : recv) * sa[i / 2];
-                    if (valid && i + odd < ncol) *op = silu_mul(g, u);
-                    op += 2 * (size_t)a.ldo;
+                    if (valid && i + odd < ncol) {
+                        const size_t o = o0 + (size_t)i * a.ldo;
+                        if (obf)
+                            out16[o] = bf16_bits(silu_mul(g, u));
+                        else
+                            a.out[o] = silu_mul(g, u);
+                    }
                 }
             }
         }
@@ -723,8 +746,7 @@ cudaError_t launch_cfg(const GemmArgs& a, int num_ctas, cudaStream_t stream) {
         if (e != cudaSuccess) return e;
         if (dev >= 0 && dev < 64) attr_done[dev] = 1;
     }
-    gemm_w4a8_kernel<C, kPartials><<<num_ctas, C::kThreads, C::kSmemBytes, stream>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(gemm_w4a8_kernel<C, kPartials>, num_ctas, C::kThreads, C::kSmemBytes, stream, a);
 }
 
 }  // namespace

@@ -225,6 +225,7 @@ __global__ void __launch_bounds__(128) pack_kernel(const uint16_t* __restrict__ 
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) quant_act_kernel(const uint16_t* __restrict__ x, int T, int K, int Kp,
                                                         int8_t* __restrict__ q, float* __restrict__ s) {
+    grid_dep_wait();  // the previous kernel of the forward has completed
     const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (row >= T) return;
@@ -248,6 +249,7 @@ __global__ void __launch_bounds__(256) quant_act_kernel(const uint16_t* __restri
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) route_topk_kernel(const uint16_t* __restrict__ logits, int T, int E, int k,
                                                          int32_t* __restrict__ ids, float* __restrict__ wout) {
+    grid_dep_wait();  // the previous kernel of the forward has completed
     const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (t >= T) return;
@@ -300,6 +302,7 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const uint16_t* __restr
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kPermChunk) perm_hist_kernel(const int32_t* __restrict__ ids, int nslots, int E,
                                                               int* __restrict__ chist, uint32_t* err) {
+    grid_dep_wait();  // the previous kernel of the forward has completed
     __shared__ int h[kMaxExperts];
     for (int e = threadIdx.x; e < E; e += blockDim.x) h[e] = 0;
     __syncthreads();
@@ -344,6 +347,7 @@ __global__ void __launch_bounds__(1024) perm_scan_kernel(int* __restrict__ chist
                                                         int* __restrict__ counts, int* __restrict__ offs,
                                                         int* __restrict__ poffs, int* __restrict__ mtstart,
                                                         int4* __restrict__ mt_tab, int* __restrict__ row_src) {
+    grid_dep_wait();  // the previous kernel of the forward has completed
     __shared__ int sh[32];
     const int e = threadIdx.x;
     int c_e = 0;
@@ -381,6 +385,7 @@ __global__ void __launch_bounds__(kPermChunk) perm_scatter_kernel(const int32_t*
                                                                  const int* __restrict__ offs,
                                                                  const int* __restrict__ poffs, int* __restrict__ perm,
                                                                  int* __restrict__ inv, int* __restrict__ row_src) {
+    grid_dep_wait();  // the previous kernel of the forward has completed
     constexpr int kWarps = kPermChunk / 32;
     __shared__ int wcnt[kWarps][kMaxExperts];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -415,6 +420,7 @@ __global__ void __launch_bounds__(1024) perm_small_kernel(const int32_t* __restr
                                                          int* __restrict__ mtstart, int4* __restrict__ mt_tab,
                                                          int* __restrict__ perm, int* __restrict__ inv,
                                                          int* __restrict__ row_src, uint32_t* err) {
+    grid_dep_wait();  // the previous kernel of the forward has completed
     extern __shared__ int psm[];
     int* s_off = psm;          // [E] counts, then the exclusive offsets
     int* s_poff = psm + E;     // [E] padded offsets
@@ -598,6 +604,7 @@ __global__ void __launch_bounds__(128) act_scatter_kernel(const uint16_t* __rest
                                                           const int* __restrict__ offs,
                                                           const int* __restrict__ poffs, int RB,
                                                           int8_t* __restrict__ act, float* __restrict__ s) {
+    grid_dep_wait();  // the previous kernel of the forward has completed
     const int nch = Kp / 16;
     const int G = Kp / kGroup;
     const int t = threadIdx.x;
@@ -671,12 +678,13 @@ __global__ void __launch_bounds__(128) act_scatter_kernel(const uint16_t* __rest
 // h rows (fp32, SwiGLU output of the up GEMM) -> INT8 rows for the down GEMM
 // (kCache chunks of 16 per thread stay in registers: 1 covers F <= 2048)
 template <int kCache>
-__global__ void __launch_bounds__(128) requant_kernel(const float* __restrict__ h, int ldh, int F, int Kp,
+__global__ void __launch_bounds__(128) requant_kernel(const uint16_t* __restrict__ h, int ldh, int F, int Kp,
                                                       const int* __restrict__ row_src, const int* __restrict__ poffs,
                                                       int E, int RB, int8_t* __restrict__ act, float* __restrict__ s) {
+    grid_dep_wait();  // the previous kernel of the forward has completed
     const int r = blockIdx.x;
     if (r >= __ldg(poffs + E)) return;
-    quant_row_cta<kCache, float>(row_src[r] < 0 ? nullptr : h + (size_t)r * ldh, F, Kp, r, RB, act, s);
+    quant_row_cta<kCache, uint16_t>(row_src[r] < 0 ? nullptr : h + (size_t)r * ldh, F, Kp, r, RB, act, s);
 }
 
 // ---------------------------------------------------------------------------
@@ -685,6 +693,7 @@ __global__ void __launch_bounds__(128) requant_kernel(const float* __restrict__ 
 __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ y2, int H, const int* __restrict__ inv,
                                                       const float* __restrict__ w, int T, int k,
                                                       uint16_t* __restrict__ out) {
+    grid_dep_wait();  // the previous kernel of the forward has completed
     __shared__ int rows[32];
     __shared__ float wts[32];
     const int t = blockIdx.x;
@@ -737,6 +746,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
 // them as one "expert" with M rows.
 __global__ void __launch_bounds__(256) dense_prep_kernel(const int8_t* __restrict__ qa, int M, int Kq, int Kp, int tile_tokens,
                                                          int RB, int8_t* __restrict__ act, int4* mt_tab, int* n_mtiles) {
+    grid_dep_wait();  // the previous kernel of the forward has completed
     const int Mp = round_up(M, kRowPad);
     const int nch = Kp / 16;
     const size_t idx = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -774,6 +784,7 @@ __device__ __forceinline__ uint4 load8_bf16(const uint16_t* row, int len, int k0
 __global__ void __launch_bounds__(128) act_gather_bf16_kernel(const uint16_t* __restrict__ x, int H, int k,
                                                               const int* __restrict__ inv, uint8_t* __restrict__ x16,
                                                               uint8_t* __restrict__ h16, int F) {
+    grid_dep_wait();  // the previous kernel of the forward has completed
     const int Hp = round_up(H, kGroup), G1 = Hp / kGroup;
     const int Fp = round_up(F, kGroup), G2 = Fp / kGroup;
     const int tok = blockIdx.x;
@@ -801,6 +812,7 @@ __global__ void __launch_bounds__(128) act_gather_bf16_kernel(const uint16_t* __
 __global__ void __launch_bounds__(256) dense_prep_bf16_kernel(const uint16_t* __restrict__ x, int M, int K,
                                                               uint8_t* __restrict__ act16, int4* mt_tab,
                                                               int* n_mtiles) {
+    grid_dep_wait();  // the previous kernel of the forward has completed
     const int Kp = round_up(K, kGroup), G = Kp / kGroup;
     const int Mp = round_up(M, kRowPad);
     const int nch = Kp / 8;
@@ -834,14 +846,12 @@ cudaError_t launch_pack(const uint16_t* w, int E, int N, int K, int layout, int 
 }
 
 cudaError_t launch_quant_act(const uint16_t* x, int T, int K, int8_t* q, float* s, cudaStream_t stream) {
-    quant_act_kernel<<<ceil_div(T, 8), 256, 0, stream>>>(x, T, K, round_up(K, kGroup), q, s);
-    return cudaGetLastError();
+    return launch_pdl(quant_act_kernel, ceil_div(T, 8), 256, 0, stream, x, T, K, round_up(K, kGroup), q, s);
 }
 
 cudaError_t launch_route_topk(const uint16_t* logits, int T, int E, int k, int32_t* ids, float* w,
                               cudaStream_t stream) {
-    route_topk_kernel<<<ceil_div(T, 8), 256, 0, stream>>>(logits, T, E, k, ids, w);
-    return cudaGetLastError();
+    return launch_pdl(route_topk_kernel, ceil_div(T, 8), 256, 0, stream, logits, T, E, k, ids, w);
 }
 
 int perm_launch_count(int nslots) { return nslots <= kPermSmallSlots ? 1 : 3; }
@@ -860,61 +870,56 @@ cudaError_t launch_perm(const int32_t* ids, int nslots, int E, int tile_tokens, 
             if (e != cudaSuccess) return e;
             if (dev >= 0 && dev < 64) attr_done[dev] = 1;
         }
-        perm_small_kernel<<<1, 1024, smem, stream>>>(ids, nslots, E, tile_tokens, counts, offs, poffs, mtstart, mt_tab,
-                                                     perm, inv, row_src, err);
-        return cudaGetLastError();
+        return launch_pdl(perm_small_kernel, 1, 1024, smem, stream, ids, nslots, E, tile_tokens, counts, offs, poffs,
+                          mtstart, mt_tab, perm, inv, row_src, err);
     }
-    perm_hist_kernel<<<nchunk, kPermChunk, 0, stream>>>(ids, nslots, E, chist, err);
-    perm_scan_kernel<<<1, 1024, 0, stream>>>(chist, nchunk, E, tile_tokens, counts, offs, poffs, mtstart, mt_tab,
-                                             row_src);
-    perm_scatter_kernel<<<nchunk, kPermChunk, 0, stream>>>(ids, nslots, E, chist, offs, poffs, perm, inv, row_src);
-    return cudaGetLastError();
+    cudaError_t e = launch_pdl(perm_hist_kernel, nchunk, kPermChunk, 0, stream, ids, nslots, E, chist, err);
+    if (e != cudaSuccess) return e;
+    e = launch_pdl(perm_scan_kernel, 1, 1024, 0, stream, chist, nchunk, E, tile_tokens, counts, offs, poffs, mtstart,
+                   mt_tab, row_src);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(perm_scatter_kernel, nchunk, kPermChunk, 0, stream, ids, nslots, E, chist, offs, poffs, perm, inv,
+                      row_src);
 }
 
 cudaError_t launch_act_scatter(const uint16_t* x, int T, int H, int Kp, int k, const int* inv, const int* offs,
                                const int* poffs, int E, int rb, int8_t* act, float* s, cudaStream_t stream) {
     if (T == 0) return cudaSuccess;
-    act_scatter_kernel<<<T + E, 128, 0, stream>>>(x, T, H, Kp, k, inv, offs, poffs, rb, act, s);
-    return cudaGetLastError();
+    return launch_pdl(act_scatter_kernel, T + E, 128, 0, stream, x, T, H, Kp, k, inv, offs, poffs, rb, act, s);
 }
 
-cudaError_t launch_requant(const float* h, int ldh, int F, int Kp, const int* row_src, const int* poffs, int E,
+cudaError_t launch_requant(const uint16_t* h, int ldh, int F, int Kp, const int* row_src, const int* poffs, int E,
                            int rows_cap, int rb, int8_t* act, float* s, cudaStream_t stream) {
     if (rows_cap == 0) return cudaSuccess;
     if (F <= 128 * 16)
-        requant_kernel<1><<<rows_cap, 128, 0, stream>>>(h, ldh, F, Kp, row_src, poffs, E, rb, act, s);
-    else
-        requant_kernel<kRowCache><<<rows_cap, 128, 0, stream>>>(h, ldh, F, Kp, row_src, poffs, E, rb, act, s);
-    return cudaGetLastError();
+        return launch_pdl(requant_kernel<1>, rows_cap, 128, 0, stream, h, ldh, F, Kp, row_src, poffs, E, rb, act, s);
+    return launch_pdl(requant_kernel<kRowCache>, rows_cap, 128, 0, stream, h, ldh, F, Kp, row_src, poffs, E, rb, act, s);
 }
 
 cudaError_t launch_combine(const float* y2, int H, const int* inv, const float* w, int T, int k, uint16_t* out,
                            cudaStream_t stream) {
     if (T == 0) return cudaSuccess;
-    combine_kernel<<<T, 256, 0, stream>>>(y2, H, inv, w, T, k, out);
-    return cudaGetLastError();
+    return launch_pdl(combine_kernel, T, 256, 0, stream, y2, H, inv, w, T, k, out);
 }
 
 cudaError_t launch_dense_prep(const int8_t* qa, int M, int Kq, int Kp, int tile_tokens, int rb, int8_t* act, int4* mt_tab,
                               int* n_mtiles, cudaStream_t stream) {
     const size_t n = (size_t)round_up(M, kRowPad) * (Kp / 16);
-    dense_prep_kernel<<<(unsigned)((n + 255) / 256 + 1), 256, 0, stream>>>(qa, M, Kq, Kp, tile_tokens, rb, act, mt_tab,
-                                                                          n_mtiles);
-    return cudaGetLastError();
+    return launch_pdl(dense_prep_kernel, (unsigned)((n + 255) / 256 + 1), 256, 0, stream, qa, M, Kq, Kp, tile_tokens, rb,
+                      act, mt_tab, n_mtiles);
 }
 
 cudaError_t launch_dense_prep_bf16(const uint16_t* x, int M, int K, uint8_t* act16, int4* mt_tab, int* n_mtiles,
                                    cudaStream_t stream) {
     const size_t n = (size_t)round_up(M, kRowPad) * (round_up(K, kGroup) / 8);
-    dense_prep_bf16_kernel<<<(unsigned)((n + 255) / 256 + 1), 256, 0, stream>>>(x, M, K, act16, mt_tab, n_mtiles);
-    return cudaGetLastError();
+    return launch_pdl(dense_prep_bf16_kernel, (unsigned)((n + 255) / 256 + 1), 256, 0, stream, x, M, K, act16, mt_tab,
+                      n_mtiles);
 }
 
 cudaError_t launch_act_gather_bf16(const uint16_t* x, int T, int H, int k, const int* inv, uint8_t* x16, uint8_t* h16,
                                    int F, cudaStream_t stream) {
     if (T == 0) return cudaSuccess;
-    act_gather_bf16_kernel<<<T, 128, 0, stream>>>(x, H, k, inv, x16, h16, F);
-    return cudaGetLastError();
+    return launch_pdl(act_gather_bf16_kernel, T, 128, 0, stream, x, H, k, inv, x16, h16, F);
 }
 
 }  // namespace w4a8

@@ -357,6 +357,34 @@ __device__ __forceinline__ bool named_bar_or(int id, int nthreads, bool pred) {
 }
 
 // ---------------------------------------------------------------------------
+// Programmatic dependent launch.  The kernels of a forward pass are launched with
+// launch_pdl(): each may start (barrier and tensor-memory set-up) while the previous
+// kernel on the stream drains, and calls grid_dep_wait() before it touches global
+// memory -- reads of the previous kernels' results and every write.  Launched
+// without the attribute, the wait returns at once.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                              Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
+// bf16 bit pattern of an fp32 value, rounded to nearest even
+__device__ __forceinline__ uint16_t bf16_bits(float v) { return __bfloat16_as_ushort(__float2bfloat16_rn(v)); }
+
+// ---------------------------------------------------------------------------
 // quantisation arithmetic (IEEE fp32, round half to even, no contraction)
 // ---------------------------------------------------------------------------
 // symmetric INT8 of one value with scale s > 0

@@ -18,8 +18,8 @@ struct GemmArgs {
     const float* act_scale;   // token scale per row
     const int4* mt_tab;       // per row tile: (expert, first row, rows, 0)
     const int* n_mtiles;      // number of row tiles (device)
-    int mode;                 // 0: y = fp32 [rows][ldo];  1: SwiGLU -> h fp32 [rows][ldo];  2: like 0
-    float* out;
+    int mode;                 // 0: y = fp32 [rows][ldo];  1: SwiGLU -> h [rows][ldo];  2: like 0
+    float* out;               // mode 1 with out_bf16: bf16 values, `out` cast to uint16_t*
     int ldo;
     int nvalid;               // valid output columns (N, or F for mode 1)
     int32_t* partials;        // mode 0 only, optional: exact INT32 partials [rows][nvalid][G]
@@ -33,6 +33,7 @@ struct GemmArgs {
     // weights per scale along K in the packed blocks: 64, 128 (also 0) or 256; G above
     // counts 128-wide planes, the partials [rows][nvalid][G * 128 / group] groups
     int group;
+    int out_bf16;             // mode 1: write h as bf16 (RNE of the fp32 result)
 };
 
 // Test hook of the failure-detection path (w4a8_debug_inject): while set on the
@@ -72,8 +73,10 @@ inline int mt_tab_capacity(int nslots, int E) { return nslots / 16 + E + 1; }
 // Kp: the padded row length of the tiled rows (a multiple of 128, >= H)
 cudaError_t launch_act_scatter(const uint16_t* x, int T, int H, int Kp, int k, const int* inv, const int* offs,
                                const int* poffs, int E, int rb, int8_t* act, float* s, cudaStream_t stream);
-cudaError_t launch_requant(const float* h, int ldh, int F, int Kp, const int* row_src, const int* poffs, int E,
+// h: bf16 SwiGLU output rows of ldh values
+cudaError_t launch_requant(const uint16_t* h, int ldh, int F, int Kp, const int* row_src, const int* poffs, int E,
                            int rows_cap, int rb, int8_t* act, float* s, cudaStream_t stream);
+// y2: fp32 expert outputs [rows][H]
 cudaError_t launch_combine(const float* y2, int H, const int* inv, const float* w, int T, int k, uint16_t* out,
                            cudaStream_t stream);
 // qa rows of Kq columns into tiled rows of Kp >= Kq columns (the rest zero)
