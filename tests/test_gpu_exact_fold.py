@@ -55,11 +55,13 @@ def to_dev_bf16(a):
 
 
 @pytest.mark.parametrize("M,N,K", [(300, 256, 640), (129, 384, 200), (17, 128, 1024), (16, 256, 512), (5, 128, 8192),
-                                   (40, 130, 256)])  # N % 4 != 0: rows not 16-byte aligned, direct stores
+                                   (40, 130, 256),  # N % 4 != 0: rows not 16-byte aligned, direct stores
+                                   (5, 20480, 1024), (16, 38400, 2048)])  # more tiles than CTAs
 def test_dense_gemm_without_partials_is_bit_exact(M, N, K):
     """M > 16: the wide-tile production instance (no partials buffer); M <= 16: the
     decode-tile kernel.  K = 8192 is the largest K (64 groups) for which the exact
-    fold argument holds."""
+    fold argument holds.  With 160 or 300 column tiles every CTA of the decode kernel
+    takes several tiles, so its pipeline rings wrap across tile boundaries."""
     x = synth.activations(M * 7 + K, M, K)
     qa, sa = O.quantize_act(x)
     w = exact_scale_weights(M + N + K, N, K)

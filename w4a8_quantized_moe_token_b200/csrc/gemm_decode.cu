@@ -67,7 +67,11 @@ struct DecCfg {
     static constexpr int NS = (kBf16 || GRP == 64) ? 6 : 4;   // shared-memory stages
     static constexpr int NA = 2;                              // tensor-memory A slots
     static constexpr int ND = NS;                             // accumulators (GQ x BN columns each)
-    static constexpr int NSC = NS + NA;                       // scale ring slots (>= NA + ND)
+    // scale ring slots: the converters write step j's slot once the MMAs of step j - NA
+    // are done, which only proves that the epilogue has loaded the accumulators of step
+    // j - NA - ND -- it may still be reading that step's scales -- so the slot's previous
+    // step must be older: NSC >= NA + ND + 1
+    static constexpr int NSC = NS + NA + 1;
     static constexpr int kRowBytes = kBf16 ? 256 : 128;       // token row bytes per K plane
     static constexpr int kGCols = kBf16 ? 64 : 32;            // A columns per K plane
     static constexpr int kBlk = block_bytes_for(GRP);         // packed weight block
@@ -95,7 +99,7 @@ struct DecLayout {
     static constexpr uint32_t kACol0 = 0;
     static constexpr uint32_t kDCol0 = NA * kACols;
     static_assert(kDCol0 + ND * kDCols <= kTmemCols, "tensor memory over-subscribed");
-    static_assert(NSC >= NA + ND, "scale ring too small");
+    static_assert(NSC >= NA + ND + 1, "scale ring too small");
     static_assert(NS % 2 == 0, "the two producers own the stages of one parity each");
     static_assert(GQ % 2 == 0, "the two MMA warps split the groups of a step");
     // one "MMA of step j done" barrier per j % NS serves the stage ring, the A slots and

@@ -221,7 +221,9 @@ __global__ void __launch_bounds__(128) pack_kernel(const uint16_t* __restrict__ 
 }
 
 // ---------------------------------------------------------------------------
-// a2: per-token INT8, natural layout [T][Kp].  One warp per row.
+// a2: per-token INT8, natural layout [T][Kp].  One warp per row.  With K a multiple
+// of 8 the row is read in 16-byte vectors (8 bf16 per lane and step) and the codes are
+// written 8 bytes at a time; other K take the scalar path.  The codes are the same.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) quant_act_kernel(const uint16_t* __restrict__ x, int T, int K, int Kp,
                                                         int8_t* __restrict__ q, float* __restrict__ s) {
@@ -230,12 +232,41 @@ __global__ void __launch_bounds__(256) quant_act_kernel(const uint16_t* __restri
     const int lane = threadIdx.x & 31;
     if (row >= T) return;
     const uint16_t* xr = x + (size_t)row * K;
+    int8_t* qr = q + (size_t)row * Kp;
     float amax = 0.f;
+    if ((K & 7) == 0) {
+        const uint4* xv = reinterpret_cast<const uint4*>(xr);
+        for (int c = lane; c < K / 8; c += 32) {
+            const uint4 p = __ldg(xv + c);
+            const uint32_t pw[4] = {p.x, p.y, p.z, p.w};
+#pragma unroll
+            for (int h = 0; h < 4; ++h)
+                amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(pw[h] << 16)), fabsf(__uint_as_float(pw[h] & 0xFFFF0000u))));
+        }
+        amax = warp_max(amax);
+        const float sc = __fdiv_rn(amax, 127.0f);
+        const float rinv = __fdiv_rn(1.0f, sc);
+        for (int c = lane; c < Kp / 8; c += 32) {
+            uint32_t out[2] = {0u, 0u};
+            if (c < K / 8 && amax > 0.f) {
+                const uint4 p = __ldg(xv + c);
+                const uint32_t pw[4] = {p.x, p.y, p.z, p.w};
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    const uint32_t lo = (uint32_t)(quant_i8_fast(__uint_as_float(pw[h] << 16), sc, rinv) & 0xFF);
+                    const uint32_t hi = (uint32_t)(quant_i8_fast(__uint_as_float(pw[h] & 0xFFFF0000u), sc, rinv) & 0xFF);
+                    out[h >> 1] |= (lo | (hi << 8)) << (16 * (h & 1));
+                }
+            }
+            *reinterpret_cast<uint2*>(qr + 8 * c) = make_uint2(out[0], out[1]);
+        }
+        if (lane == 0) s[row] = sc;
+        return;
+    }
     for (int k = lane; k < K; k += 32) amax = fmaxf(amax, fabsf(bf16_to_f32(xr[k])));
     amax = warp_max(amax);
     const float sc = __fdiv_rn(amax, 127.0f);
     const float rinv = __fdiv_rn(1.0f, sc);
-    int8_t* qr = q + (size_t)row * Kp;
     for (int k = lane; k < Kp; k += 32) {
         int c = 0;
         if (k < K && amax > 0.f) c = quant_i8_fast(bf16_to_f32(xr[k]), sc, rinv);
