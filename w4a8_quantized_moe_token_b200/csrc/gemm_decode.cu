@@ -540,6 +540,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
         bool ok = true, acc_rdy = false, side_rdy = false;  // early tests of this step's barriers
         for (int u = blockIdx.x; u < total && ok; u += gridDim.x, ++nit) {
             const Item it = decode_item(u, a);
+            // token i's scale in lane i, loaded now so that its latency hides behind the
+            // tile's steps (group 0 stores the tile; W4A16 has no token scale)
+            const float my_sa = (kBf16 || eh != 0 || lane >= BN) ? 1.f
+                                : (lane < it.nrows ? __ldg(a.act_scale + it.row0 + lane) : 0.f);
             uint64_t acc2[BN / 2];  // token pairs, packed fp32x2
 #pragma unroll
             for (int i = 0; i < BN / 2; ++i) acc2[i] = 0ull;
@@ -621,12 +625,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_decode_kernel(const GemmArgs
             __syncwarp();
             if (lane == 0) mbar_arrive(XEMPTY_BAR(xp));
 
-            // token scales: all loads before the stores (the compiler may not move a load
-            // across a store it cannot prove disjoint)
-            const float* sap = a.act_scale + it.row0;
             float sa[BN];
 #pragma unroll
-            for (int i = 0; i < BN; ++i) sa[i] = kBf16 ? 1.f : (i < it.nrows ? __ldg(sap + i) : 0.f);  // W4A16: no token scale
+            for (int i = 0; i < BN; ++i) sa[i] = kBf16 ? 1.f : __shfl_sync(0xffffffffu, my_sa, i);
             // mode 1 with out_bf16: h as bf16 (RNE of the fp32 result)
             const bool obf = a.out_bf16 != 0 && a.mode == 1;
             uint16_t* out16 = reinterpret_cast<uint16_t*>(a.out);
