@@ -248,6 +248,9 @@ def pack_experts(B, torch, W, seed, device):
     return up, dn
 
 
+E2E_STREAMS = 2  # end-to-end steps alternate between this many streams (MoeStep.e2e)
+
+
 class MoeStep:
     """One forward of the MoE layer through w4a8_moe_forward (or, with w4a16=True,
     through the W4A16 comparison layer w4a16_moe_forward on the same packed weights)."""
@@ -297,54 +300,78 @@ class MoeStep:
 
     def e2e(self, steps, warmup):
         """Same metric through the public API with HOST inputs/outputs: per step the
-        pinned-host inputs are copied in and the bf16 output copied back."""
+        pinned-host inputs are copied in and the bf16 output copied back.
+
+        Consecutive steps alternate between two streams with their own workspace and
+        output buffer (double buffering, as a server overlaps requests): step i + 1's
+        input copy and step i - 1's output copy run on the copy engines while step i
+        computes.  Every step's copies are inside the timed span, which runs from the
+        first step's issue to the completion of the last one on both streams."""
         torch, B, W = self.torch, self.B, self.W
         T, E, k, H, F = W.T, W.E, W.topk, W.H, W.F
         pin = lambda a: torch.from_numpy(a).pin_memory()
         x_h = torch.from_numpy(synth.bf16_bits(self.x_host).view(np.int16)).view(torch.bfloat16).pin_memory()
-        out_h = torch.empty((T, H), dtype=torch.bfloat16).pin_memory()
+        ids_h, w_h = pin(np.ascontiguousarray(self.ids_host)), pin(np.ascontiguousarray(self.w_host))
+        lanes = []
+        for _ in range(2):
+            lane = {"stream": torch.cuda.Stream(self.device),
+                    "out_h": torch.empty((T, H), dtype=torch.bfloat16).pin_memory()}
+            if GROUP != 128:
+                # the group-size entry point takes device buffers: the step's copies are
+                # issued on the same stream around it
+                lane["x"] = torch.empty_like(self.x)
+                lane["ids"] = torch.empty_like(self.ids)
+                lane["w"] = torch.empty_like(self.w)
+                lane["out"] = torch.empty_like(self.out)
+                lane["ws"] = B.empty_aligned(B.w4a8_moe_workspace_bytes_g(T, E, k, H, F, GROUP), self.device)
+            else:
+                lane["ws"] = B.empty_aligned(B.w4a8_moe_host_workspace_bytes(T, E, k, H, F), self.device)
+            lanes.append(lane)
         if GROUP != 128:
-            # the group-size entry point takes device buffers: the step's copies are
-            # issued on the same stream around it
-            ids_h, w_h = pin(np.ascontiguousarray(self.ids_host)), pin(np.ascontiguousarray(self.w_host))
             h2d = x_h.numel() * 2 + ids_h.numel() * 4 + w_h.numel() * 4
-            logits, self.logits = self.logits, None
 
-            def step():
-                self.x.copy_(x_h, non_blocking=True)
-                self.ids.copy_(ids_h, non_blocking=True)
-                self.w.copy_(w_h, non_blocking=True)
-                self()
-                out_h.copy_(self.out, non_blocking=True)
+            def run(lane):
+                lane["x"].copy_(x_h, non_blocking=True)
+                lane["ids"].copy_(ids_h, non_blocking=True)
+                lane["w"].copy_(w_h, non_blocking=True)
+                B.w4a8_moe_forward_g(self.packed_up, self.packed_down, E, H, F, GROUP, lane["x"], lane["ids"],
+                                     lane["w"], lane["out"], lane["ws"])
+                lane["out_h"].copy_(lane["out"], non_blocking=True)
         elif self.logits is None:
-            ids_h, w_h = pin(np.ascontiguousarray(self.ids_host)), pin(np.ascontiguousarray(self.w_host))
-            ws = B.empty_aligned(B.w4a8_moe_host_workspace_bytes(T, E, k, H, F), self.device)
             h2d = x_h.numel() * 2 + ids_h.numel() * 4 + w_h.numel() * 4
 
-            def step():
-                B.w4a8_moe_forward_host(self.packed_up, self.packed_down, E, H, F, x_h, ids_h, w_h, out_h, ws)
+            def run(lane):
+                B.w4a8_moe_forward_host(self.packed_up, self.packed_down, E, H, F, x_h, ids_h, w_h, lane["out_h"],
+                                        lane["ws"])
         else:
             # routed on the device from the router logits: one C-ABI call with host buffers
             lg_h = torch.from_numpy(synth.bf16_bits(self.logits_host).view(np.int16)).view(torch.bfloat16).pin_memory()
-            ws = B.empty_aligned(B.w4a8_moe_host_workspace_bytes(T, E, k, H, F), self.device)
             h2d = x_h.numel() * 2 + lg_h.numel() * 2
 
-            def step():
-                B.w4a8_moe_forward_logits_host(self.packed_up, self.packed_down, E, H, F, x_h, lg_h, k, out_h, ws)
-        for _ in range(warmup):
-            step()
-        torch.cuda.synchronize()
-        total = 0.0
-        for _ in range(steps):
+            def run(lane):
+                B.w4a8_moe_forward_logits_host(self.packed_up, self.packed_down, E, H, F, x_h, lg_h, k,
+                                               lane["out_h"], lane["ws"])
+
+        def steps_on_lanes(n):
+            main = torch.cuda.current_stream(self.device)
             a = torch.cuda.Event(enable_timing=True)
             b = torch.cuda.Event(enable_timing=True)
-            a.record()
-            step()
-            b.record()
+            a.record(main)
+            for lane in lanes:
+                lane["stream"].wait_event(a)
+            for i in range(n):
+                lane = lanes[i % 2]
+                with torch.cuda.stream(lane["stream"]):
+                    run(lane)
+            for lane in lanes:
+                main.wait_stream(lane["stream"])
+            b.record(main)
             b.synchronize()
-            total += a.elapsed_time(b)
-        if GROUP != 128:
-            self.logits = logits
+            return a.elapsed_time(b)
+
+        steps_on_lanes(max(warmup, 2))
+        torch.cuda.synchronize()
+        total = steps_on_lanes(steps)
         return total / steps, h2d, T * H * 2
 
 
@@ -886,7 +913,7 @@ def main(argv=None):
         "kernels": summ["kernels"],
         "gpu_launches": summ["gpu_launches"],
         "e2e": {"value": whole_job_rate(tokens // world, world, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h},
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "streams": E2E_STREAMS},
         "clocks": summ["clocks"],
         "int8_peak": i8,
     }
@@ -914,7 +941,7 @@ def main(argv=None):
             ex = moe_summary(Wx, sx, msx, profx, clx, args.steps, peaks, world)
             e2x, h2x, d2x = sx.e2e(args.steps, args.warmup)
             ex["e2e"] = {"value": Wx.T / (e2x / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2x,
-                         "d2h_bytes_per_step": d2x}
+                         "d2h_bytes_per_step": d2x, "ms_per_step": e2x, "streams": E2E_STREAMS}
             ex["config"] = config_of(Wx, "flushed before every timed step (256 MiB write, outside the timed span)")
             # the pages' comparison point: the same layer with W4A16 experts (bf16
             # activations, same packed weights and routing; group 128 only)
