@@ -388,6 +388,7 @@ class GemmStep:
         self.q = torch.empty((W.M, Kp), dtype=torch.int8, device=device)
         self.s = torch.empty(W.M, dtype=torch.float32, device=device)
         self.y = torch.empty((W.M, W.N), dtype=torch.float32, device=device)
+        self.out = self.y
         self.ws = B.empty_aligned(B.w4a8_gemm_workspace_bytes_g(W.M, W.N, W.K, GROUP), device)
         self.acct = gemm_accounting(W)
 
@@ -732,6 +733,36 @@ def measure_int8_peak(torch, device, n=8192, reps=10):
     return info
 
 
+def capture_step(step, torch, device):
+    """The step as one CUDA graph (every launch of the forward replayed without host
+    gaps, as a serving loop runs it), if it captures and its replay reproduces the
+    eager output bit for bit; else the eager step.  Returns (callable, note)."""
+    out = getattr(step, "out", None)
+    if out is None:
+        return step, "eager (no output to verify)"
+    try:
+        side = torch.cuda.Stream(device)
+        side.wait_stream(torch.cuda.current_stream(device))
+        with torch.cuda.stream(side):
+            step()
+        torch.cuda.current_stream(device).wait_stream(side)
+        torch.cuda.synchronize(device)
+        ref = out.clone()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step()
+        out.zero_()
+        g.replay()
+        torch.cuda.synchronize(device)
+        if not torch.equal(out, ref):
+            return step, "eager (graph replay differed from the eager step)"
+        step.graph = g  # keep it alive
+        return g.replay, "cuda graph"
+    except Exception as e:  # noqa: BLE001 -- any capture failure falls back to eager launches
+        torch.cuda.synchronize(device)
+        return step, f"eager (capture failed: {type(e).__name__})"
+
+
 def time_steps(step, B, torch, device, world, steps, warmup):
     """Warm up, then time `steps` steps with CUDA events on the launching stream (L2
     flushed before each, outside the timed span) and NVML clock samples over the same
@@ -743,6 +774,7 @@ def time_steps(step, B, torch, device, world, steps, warmup):
     for _ in range(warmup):
         step()
     torch.cuda.synchronize()
+    run, step.graph_note = capture_step(step, torch, device)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
     sampler = ClockSampler(torch.cuda.current_device())
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
@@ -754,7 +786,7 @@ def time_steps(step, B, torch, device, world, steps, warmup):
     for i in range(steps):
         flush.zero_()
         starts[i].record()
-        step()
+        run()
         ends[i].record()
     torch.cuda.synchronize()
     if world > 1:
@@ -904,7 +936,8 @@ def main(argv=None):
         "vs_baseline": None,
         "dtype": "int8",
         "data": "synthetic",
-        "config": config_of(W, "flushed before every timed step (256 MiB write, outside the timed span)"),
+        "config": dict(config_of(W, "flushed before every timed step (256 MiB write, outside the timed span)"),
+                       launch=step.graph_note),
         "tops": summ["tops"],
         "weight_gbs": summ["weight_gbs"],
         "touched_experts": summ["touched_experts"],
@@ -926,6 +959,7 @@ def main(argv=None):
         w16 = moe_summary(W, s16, ms16, prof16, cl16, args.steps, peaks, world)
         line["w4a16"] = {k: w16[k] for k in ("value", "unit", "ms_per_step", "weight_gbs", "roofline", "kernels",
                                              "gpu_launches", "clocks")}
+        line["w4a16"]["launch"] = s16.graph_note
         line["w4a8_over_w4a16"] = summ["value"] / w16["value"]
         del s16
 
@@ -942,7 +976,8 @@ def main(argv=None):
             e2x, h2x, d2x = sx.e2e(args.steps, args.warmup)
             ex["e2e"] = {"value": Wx.T / (e2x / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2x,
                          "d2h_bytes_per_step": d2x, "ms_per_step": e2x, "streams": E2E_STREAMS}
-            ex["config"] = config_of(Wx, "flushed before every timed step (256 MiB write, outside the timed span)")
+            ex["config"] = dict(config_of(Wx, "flushed before every timed step (256 MiB write, outside the timed span)"),
+                                launch=sx.graph_note)
             # the pages' comparison point: the same layer with W4A16 experts (bf16
             # activations, same packed weights and routing; group 128 only)
             if GROUP != 128:
@@ -955,6 +990,7 @@ def main(argv=None):
             w16 = moe_summary(Wx, s16, ms16, prof16, cl16, args.steps, peaks, world)
             ex["w4a16"] = {k: w16[k] for k in ("value", "unit", "ms_per_step", "weight_gbs", "roofline", "kernels",
                                                "gpu_launches", "clocks")}
+            ex["w4a16"]["launch"] = s16.graph_note
             ex["w4a8_over_w4a16"] = ex["value"] / w16["value"]
             extra[name] = ex
             del sx, s16
