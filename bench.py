@@ -76,7 +76,8 @@ def moe_accounting(W, ids, w4a16=False):
     T, k, H, F = W.T, W.topk, W.H, W.F
     touched = int(np.unique(ids).size)
     slots = T * k
-    Hp, Fp = padded(H), padded(F)
+    m = max(128, GROUP)  # token rows are padded to whole groups (and 128-wide planes)
+    Hp, Fp = (H + m - 1) // m * m, (F + m - 1) // m * m
     up_w = touched * packed_matrix_bytes(2 * F, H)
     dn_w = touched * packed_matrix_bytes(H, F)
     k_ops = {
